@@ -1,0 +1,368 @@
+"""Pins for the CPU oracle, each against something other than the oracle itself.
+
+* Philox4x32-10 against the published known-answer vectors (tests/golden).
+* bf16 rounding against torch's float32 -> bfloat16 conversion.
+* Stick-breaking exit probabilities (gist.science summary, section 2, equation
+  for p_k with w_{N_V} = 1) against the closed form sum_k p_k = 1.
+* The mixture (section 2, equation for pi_mix) sums to one over the vocabulary.
+* The backbone against an independent LLaMA implementation
+  (transformers.LlamaForCausalLM, float64): the dense model is the special case
+  of zero intermediate routing mass (section 5), and every intermediate exit is
+  checked through the same model's hidden states.
+* The piggybacked decode (section 2, "Inferenz: Piggybacking") against an
+  undeferred full-depth forward: KV caches equal after the flush.
+* Exact sampling: chi-square of (exit, token) draws against p_k * pi_k(v).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import nvium_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def tiny_model(mode=O.ROUTER_NORMAL, random_gains=True, seed=0):
+    w = W.make_weights(W.TINY, seed=seed, random_gains=random_gains)
+    return O.OracleModel(W.TINY, w, mode), w
+
+
+# --------------------------------------------------------------------------
+def test_philox_known_answers():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "philox4x32_10_kat.txt")) if not l.startswith("#")]
+    assert len(rows) == 3
+    for r in rows:
+        v = [int(x, 16) for x in r]
+        out = O.philox4x32_10(v[:4], v[4:6])
+        assert [int(o) for o in out] == v[6:]
+
+
+def test_philox_vectorised_matches_scalar():
+    rng = np.random.default_rng(5)
+    ctr = rng.integers(0, 2**32, size=(4, 64), dtype=np.uint64)
+    key = rng.integers(0, 2**32, size=(2, 64), dtype=np.uint64)
+    vec = O.philox4x32_10(list(ctr), list(key))
+    for i in range(0, 64, 13):
+        one = O.philox4x32_10([int(c[i]) for c in ctr], [int(k[i]) for k in key])
+        assert [int(x[i]) for x in vec] == [int(x) for x in one]
+
+
+def test_uniform_is_exact_in_fp32_and_open_interval():
+    x = np.array([0, 1, 511, 512, 2**31, 2**32 - 1, 0xDEADBEEF], dtype=np.uint64)
+    u = O.uniform01(x)
+    assert np.all(u > 0) and np.all(u < 1)
+    assert np.array_equal(u.astype(np.float32).astype(np.float64), u)
+    assert u[0] == 2.0 ** -24 and u[-2] == 1 - 2.0 ** -24
+
+
+def test_bf16_round_matches_torch():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(100000) * 3,
+                        rng.standard_normal(1000) * 1e-3,
+                        # exact ties between two bf16 neighbours
+                        (np.arange(1, 200) * 2 + 1) * 2.0 ** -8 + 1.0]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.bf16_round(x.astype(np.float64)), ref)
+
+
+# --------------------------------------------------------------------------
+def test_stick_breaking_sums_to_one():
+    rng = np.random.default_rng(2)
+    for n in (1, 2, 3, 7):
+        w = rng.random((1000, n))
+        p = O.exit_probs(w)
+        assert np.all(p >= 0)
+        np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-12)
+        # log-space form agrees with the direct product
+        z = np.log(w) - np.log1p(-w)
+        np.testing.assert_allclose(np.exp(O.log_exit_probs(z)), p, rtol=1e-10, atol=1e-14)
+    # p_1 = w_1 and p_k for a hand example
+    p = O.exit_probs(np.array([0.5, 0.5, 0.5]))
+    np.testing.assert_allclose(p, [0.5, 0.25, 0.125, 0.125])
+
+
+def test_force_last_log_exit_probs():
+    lp = O.log_exit_probs(np.array([[3.0, -2.0, 0.1]]), O.ROUTER_FORCE_LAST)
+    assert np.all(np.isneginf(lp[0, :3])) and lp[0, 3] == 0.0
+
+
+def test_mixture_logprob_logspace_vs_direct():
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((50, 3)) * 2
+    logpi = np.log(rng.dirichlet(np.ones(6), size=(50, 4)))[..., 0]
+    direct = np.log(np.sum(O.exit_probs(1 / (1 + np.exp(-z))) * np.exp(logpi), axis=-1))
+    np.testing.assert_allclose(O.mixture_logprob(O.log_exit_probs(z), logpi), direct, rtol=1e-12)
+
+
+def test_mixture_sums_to_one_on_tiny_vocab():
+    model, _ = tiny_model()
+    prompt = W.make_prompts(W.WORKLOADS["T"])[0][:12]
+    _, states, _ = model.forward_sequence(prompt)
+    for pos in (0, 5, 11):
+        p, pi = O.step_distribution(model, [states[k][pos:pos + 1] for k in range(4)])
+        np.testing.assert_allclose(p.sum(), 1.0, atol=1e-12)
+        mix = (p[:, None] * pi).sum(0)
+        np.testing.assert_allclose(mix.sum(), 1.0, atol=1e-12)
+        assert 0.0 < p[0] < 1.0
+
+
+def test_rope_relative_position_and_identity():
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((1, 2, 32))
+    k = rng.standard_normal((1, 2, 32))
+    np.testing.assert_allclose(O.rope(q, np.array([0]), 1e4), q)
+    d1 = np.einsum("nhd,nhd->nh", O.rope(q, np.array([17]), 1e4), O.rope(k, np.array([5]), 1e4))
+    d2 = np.einsum("nhd,nhd->nh", O.rope(q, np.array([112]), 1e4), O.rope(k, np.array([100]), 1e4))
+    np.testing.assert_allclose(d1, d2, rtol=1e-10)
+
+
+# --------------------------------------------------------------------------
+# independent LLaMA (transformers, float64)
+# --------------------------------------------------------------------------
+
+def _hf_llama(cfg, w):
+    from transformers import LlamaConfig, LlamaForCausalLM
+    hc = LlamaConfig(vocab_size=cfg.vocab, hidden_size=cfg.d_model, intermediate_size=cfg.d_ff,
+                     num_hidden_layers=cfg.n_layers, num_attention_heads=cfg.n_heads,
+                     num_key_value_heads=cfg.n_heads, head_dim=cfg.head_dim,
+                     rms_norm_eps=cfg.rms_eps, rope_theta=cfg.rope_theta,
+                     max_position_embeddings=4096, tie_word_embeddings=False,
+                     attention_bias=False, mlp_bias=False, hidden_act="silu")
+    hc._attn_implementation = "eager"
+    torch.manual_seed(0)
+    m = LlamaForCausalLM(hc).to(torch.float64).eval()
+    t = lambda a: torch.from_numpy(W.as_f32(a).astype(np.float64))
+    with torch.no_grad():
+        m.model.embed_tokens.weight.copy_(t(w["tok_emb"]))
+        for i, L in enumerate(w["layers"]):
+            ly = m.model.layers[i]
+            ly.input_layernorm.weight.copy_(t(L["attn_norm"]))
+            ly.self_attn.q_proj.weight.copy_(t(L["wq"]))
+            ly.self_attn.k_proj.weight.copy_(t(L["wk"]))
+            ly.self_attn.v_proj.weight.copy_(t(L["wv"]))
+            ly.self_attn.o_proj.weight.copy_(t(L["wo"]))
+            ly.post_attention_layernorm.weight.copy_(t(L["mlp_norm"]))
+            ly.mlp.gate_proj.weight.copy_(t(L["wg"]))
+            ly.mlp.up_proj.weight.copy_(t(L["wu"]))
+            ly.mlp.down_proj.weight.copy_(t(L["wd"]))
+        m.model.norm.weight.copy_(t(w["exits"][-1]["norm"]))
+        m.lm_head.weight.copy_(t(w["exits"][-1]["head"]))
+    return m
+
+
+HF_TOL = 2e-6
+
+
+@pytest.fixture(scope="module")
+def hf_tiny():
+    model, w = tiny_model(random_gains=True)
+    return model, w, _hf_llama(W.TINY, w)
+
+
+def test_dense_equals_hf_llama(hf_tiny):
+    model, w, hf = hf_tiny
+    toks = W.make_prompts(W.WORKLOADS["T"])[0]
+    ours = O.dense_logprobs(model, toks)
+    with torch.no_grad():
+        ref = torch.log_softmax(hf(torch.from_numpy(toks.astype(np.int64))[None]).logits[0], -1).numpy()
+    # transformers computes RMSNorm and the RoPE tables in float32 internally,
+    # so agreement is at the 1e-7 level; a wrong sign, index or term is >1e-3.
+    np.testing.assert_allclose(ours, ref, atol=HF_TOL, rtol=0)
+
+
+def test_mixture_scoring_against_hf_hidden_states(hf_tiny):
+    """Every exit's head, the routers and the mixture, recomputed from the
+    independent model's per-layer hidden states with torch routines."""
+    model, w, hf = hf_tiny
+    cfg = W.TINY
+    toks = W.make_prompts(W.WORKLOADS["T"])[0][None, :24]
+    logp, nll = O.score_mixture(model, toks)
+    with torch.no_grad():
+        out = hf(torch.from_numpy(toks[:, :-1].astype(np.int64)), output_hidden_states=True)
+    tgt = torch.from_numpy(toks[0, 1:].astype(np.int64))
+    t = lambda a: torch.from_numpy(W.as_f32(a).astype(np.float64))
+    probs = torch.zeros(toks.shape[1] - 1, dtype=torch.float64)
+    surv = torch.ones(toks.shape[1] - 1, dtype=torch.float64)
+    for k, layer in enumerate(cfg.exit_layers):
+        hs = out.hidden_states[layer][0]          # residual after `layer` layers
+        if layer == cfg.n_layers:
+            # the last exit is the model's own final norm + LM head
+            pik = torch.softmax(out.logits[0], -1)
+        else:
+            nk = torch.nn.functional.rms_norm(hs, (cfg.d_model,), t(w["exits"][k]["norm"]), cfg.rms_eps)
+            pik = torch.softmax(nk @ t(w["exits"][k]["head"]).T, -1)
+        if k < cfg.n_exits - 1:
+            wk = torch.sigmoid(nk @ t(w["exits"][k]["router_w"]) + w["exits"][k]["router_b"])
+            pk = wk * surv
+            surv = surv * (1 - wk)
+        else:
+            pk = surv
+        probs += pk * pik[torch.arange(len(tgt)), tgt]
+    np.testing.assert_allclose(logp[0], torch.log(probs).numpy(), atol=HF_TOL, rtol=0)
+    assert abs(nll + float(torch.log(probs).mean())) < HF_TOL
+
+
+def test_force_last_scoring_equals_dense():
+    model, _ = tiny_model(O.ROUTER_FORCE_LAST)
+    toks = W.make_prompts(W.WORKLOADS["T"])[0][None, :20]
+    logp, _ = O.score_mixture(model, toks)
+    dense = O.dense_logprobs(model, toks[0, :-1])
+    np.testing.assert_array_equal(logp[0], dense[np.arange(19), toks[0, 1:]])
+
+
+def test_bf16_model_matches_hf_in_fp64_when_rounding_off():
+    """The bf16 code path minus its rounding points is the plain LLaMA; with
+    the rounding points the change is at the bf16 scale, not more."""
+    cfg = W.ModelConfig("mini-bf16", 2, 64, 4, 16, 128, 512, (1, 2), W.BF16)
+    w = W.make_weights(cfg, seed=3, random_gains=True)
+    model = O.OracleModel(cfg, w, O.ROUTER_FORCE_LAST)
+    toks = W.zipf_ids(16, cfg.vocab, np.random.default_rng(0))
+    hf = _hf_llama(cfg, w)
+    with torch.no_grad():
+        ref = torch.log_softmax(hf(torch.from_numpy(toks.astype(np.int64))[None]).logits[0], -1).numpy()
+    model.bf16 = False
+    np.testing.assert_allclose(O.dense_logprobs(model, toks), ref, atol=HF_TOL, rtol=0)
+    model.bf16 = True
+    d = np.abs(O.dense_logprobs(model, toks) - ref).max()
+    assert 1e-6 < d < 5e-2
+
+
+# --------------------------------------------------------------------------
+# piggybacked decode == undeferred full depth
+# --------------------------------------------------------------------------
+
+def _check_invariants(dec, b):
+    cfg = dec.model.cfg
+    lens = dec.caches[b].lens
+    t = dec.t[b]
+    # len non-increasing in m, every layer up to the first exit complete
+    assert all(lens[i] >= lens[i + 1] for i in range(cfg.n_layers - 1))
+    assert all(lens[i] == t for i in range(cfg.exit_layers[0]))
+    # pending set = suffix [len_L, t)
+    assert sorted(dec.pending[b]) == list(range(lens[-1], t))
+
+
+@pytest.mark.parametrize("pattern", ["all1", "alternate", "random", "routed", "last"])
+def test_deferred_kv_equals_full_depth(pattern):
+    cfg = W.TINY
+    model, _ = tiny_model()
+    prompts = [W.make_prompts(W.WORKLOADS["T"])[0][:9], W.make_prompts(W.WORKLOADS["T"], seed=7)[0][:14]]
+    steps = 20
+    dec = O.OracleDecoder(model, prompts, steps)
+    rng = np.random.default_rng(11)
+    for s in range(steps):
+        if pattern == "all1":
+            ex = [1, 1]
+        elif pattern == "alternate":
+            ex = [1 + (s % 2) * 3, 4 - (s % 2) * 2]
+        elif pattern == "random":
+            ex = list(rng.integers(1, 5, size=2))
+        elif pattern == "last":
+            ex = [4, 4]
+        else:
+            ex = None
+        dec.step(1234, forced_exits=ex)
+        for b in range(2):
+            _check_invariants(dec, b)
+    dec.flush()
+    for b in range(2):
+        t = dec.t[b]
+        assert dec.caches[b].lens == [t] * cfg.n_layers
+        _, _, full = model.forward_sequence(dec.tokens[b][:t])
+        for m in range(cfg.n_layers):
+            np.testing.assert_allclose(dec.caches[b].K[m][:t], full.K[m][:t], rtol=1e-10, atol=1e-13)
+            np.testing.assert_allclose(dec.caches[b].V[m][:t], full.V[m][:t], rtol=1e-10, atol=1e-13)
+
+
+def test_decode_step_law_matches_full_depth_states():
+    """The h a new token reaches each junction with, under deferral, is the
+    full-depth forward's h: the step's (u, w) and scores use it."""
+    model, _ = tiny_model()
+    p = W.make_prompts(W.WORKLOADS["T"])[0][:10]
+    dec = O.OracleDecoder(model, [p], 8)
+    for s in range(6):
+        dec.step(99, forced_exits=[1 + (s % 3)])
+    t = dec.t[0]
+    rec = dec.step_seq(0, 4321, forced_exit=4)
+    _, states, _ = model.forward_sequence(dec.tokens[0][: t + 1])
+    for (k, u, w) in rec.junctions:
+        np.testing.assert_allclose(w, model.router_prob(k - 1, states[k - 1][t]).item(), rtol=1e-10)
+        assert u == float(O.exit_uniform(4321, 0, t, k))
+    lg = model.head_logits(3, states[3][t:t + 1])[0]
+    np.testing.assert_allclose(rec.scores, lg + O.gumbel_noise(4321, 0, t, W.TINY.vocab), rtol=1e-10)
+
+
+# --------------------------------------------------------------------------
+# exact sampling
+# --------------------------------------------------------------------------
+
+def _chisq_merged(counts, expected, min_expected=5.0):
+    from scipy import stats
+    counts = np.asarray(counts, dtype=np.float64).ravel()
+    expected = np.asarray(expected, dtype=np.float64).ravel()
+    order = np.argsort(expected)
+    c, e = counts[order], expected[order]
+    small = np.cumsum(e) < min_expected * 4
+    big = ~small
+    cc = np.concatenate([c[big], [c[small].sum()]]) if small.any() else c
+    ee = np.concatenate([e[big], [e[small].sum()]]) if small.any() else e
+    assert np.all(ee >= min_expected)
+    return stats.chisquare(cc, ee * cc.sum() / ee.sum()).pvalue
+
+
+def test_sequential_stop_frequencies_match_pk():
+    w = np.array([0.3, 0.5, 0.2])
+    seeds = np.arange(200000, dtype=np.uint64)
+    u = np.stack([O.exit_uniform(seeds, 0, 7, k) for k in (1, 2, 3)], -1)
+    ex = O.sample_exit(u, w)
+    counts = np.bincount(ex, minlength=5)[1:]
+    assert _chisq_merged(counts, O.exit_probs(w) * len(seeds)) > 0.01
+
+
+def test_exact_sampler_joint_frequencies():
+    """(exit, token) from sequential stopping + Gumbel-max, 2e5 seeds, against
+    p_k * pi_k(v); the token marginal against pi_mix."""
+    model, _ = tiny_model()
+    cfg = W.TINY
+    prompt = W.make_prompts(W.WORKLOADS["T"])[0][:16]
+    _, states, _ = model.forward_sequence(prompt)
+    t = len(prompt) - 1
+    js = [states[k][t:t + 1] for k in range(4)]
+    p, pi = O.step_distribution(model, js)
+    w = np.array([model.router_prob(k, js[k]).item() for k in range(3)])
+    logits = np.stack([model.head_logits(k, js[k])[0] for k in range(4)])
+    N, chunk = 200000, 25000
+    joint = np.zeros((4, cfg.vocab))
+    for c0 in range(0, N, chunk):
+        seeds = np.arange(c0, c0 + chunk, dtype=np.uint64) + np.uint64(10**6)
+        u = np.stack([O.exit_uniform(seeds, 0, t, k) for k in (1, 2, 3)], -1)
+        ex = O.sample_exit(u, w) - 1
+        tok = O.gumbel_argmax(logits[ex], O.gumbel_noise(seeds, 0, t, cfg.vocab))
+        np.add.at(joint, (ex, tok), 1)
+    assert _chisq_merged(joint, p[:, None] * pi * N) > 0.01
+    assert _chisq_merged(joint.sum(0), (p[:, None] * pi).sum(0) * N) > 0.01
+    assert _chisq_merged(joint.sum(1), p * N) > 0.01
+
+
+def test_decoder_step_uses_the_vectorised_sampler():
+    model, _ = tiny_model()
+    prompt = W.make_prompts(W.WORKLOADS["T"])[0][:16]
+    _, states, _ = model.forward_sequence(prompt)
+    t = len(prompt) - 1
+    js = [states[k][t:t + 1] for k in range(4)]
+    w = np.array([model.router_prob(k, js[k]).item() for k in range(3)])
+    logits = np.stack([model.head_logits(k, js[k])[0] for k in range(4)])
+    for seed in (1, 2, 3, 1234, 2**40 + 5):
+        dec = O.OracleDecoder(model, [prompt], 1)
+        rec = dec.step(seed)[0]
+        u = np.array([float(O.exit_uniform(seed, 0, t, k)) for k in (1, 2, 3)])
+        ex = int(O.sample_exit(u, w))
+        tok = int(O.gumbel_argmax(logits[ex - 1], O.gumbel_noise(seed, 0, t, W.TINY.vocab)))
+        assert (rec.exit, rec.token) == (ex, tok)
+
+
+def test_gumbel_argmax_ties_to_lowest_id():
+    assert int(O.gumbel_argmax(np.array([1.0, 3.0, 3.0, 2.0]), np.zeros(4))) == 1
