@@ -1,0 +1,59 @@
+// GEMM dispatch (see gemm.cuh).
+#include <cstdlib>
+#include <cstring>
+
+#include "gemm.cuh"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+namespace nv {
+
+struct GemmPlanCache {
+  TcPlanCache* tc = nullptr;
+};
+
+GemmPlanCache* gemm_plans_create() {
+  GemmPlanCache* c = new GemmPlanCache();
+  c->tc = tc_plans_create();
+  return c;
+}
+void gemm_plans_destroy(GemmPlanCache* c) {
+  if (!c) return;
+  tc_plans_destroy(c->tc);
+  delete c;
+}
+
+int* gemm_status_ptr(GemmPlanCache* c) { return c ? tc_status_ptr(c->tc) : nullptr; }
+
+int gemm_default_kind() {
+  const char* e = std::getenv("NVIUM_GEMM");
+  if (e && std::strcmp(e, "simt") == 0) return GEMM_SIMT;
+  return GEMM_TC;
+}
+
+nv_status gemm_prepare(int kind, bool bf16) {
+  if (kind == GEMM_TC && bf16) return tc_prepare();
+  return NV_OK;
+}
+
+size_t gemm_workspace_elems(int kind, size_t rows, size_t N) {
+  size_t e = rows * N;
+  if (kind == GEMM_TC) {
+    const size_t t = tc_workspace_elems(N);
+    if (t > e) e = t;
+  }
+  return e;
+}
+
+nv_status gemm_run(GemmPlanCache* plans, int kind, bool bf16, const void* X, int ldx, const void* W, int N, int K,
+                   const int* nrows, int max_rows, float* Y, bool allow_split, int* split_grid, size_t* split_stride,
+                   cudaStream_t st) {
+  if (kind == GEMM_TC && bf16)
+    return tc_gemm_run(plans->tc, X, ldx, W, N, K, nrows, max_rows, Y, allow_split, split_grid, split_stride, st);
+  launch_gemm_simt(bf16, X, ldx, W, N, K, nrows, max_rows, Y, st);
+  *split_grid = 0;
+  *split_stride = 0;
+  return NV_OK;
+}
+
+}  // namespace nv

@@ -1,0 +1,979 @@
+// libnvium kernels: planner + RMSNorm, SIMT GEMM and epilogues, paged
+// attention, exit junction and the fused exit-head sampler, scoring.
+//
+// Method: "N-vium: Mixture-of-Exits Transformer for Accelerated Exact
+// Generation" (arXiv 2605.13190).  Section 2 "Architektur" gives the exit
+// probability p_k and the mixture pi_mix; section 2 "Inferenz: Piggybacking"
+// gives the deferral of the layers above an exit and their batching with
+// later tokens; the backbone is LLaMA-2 (section 4).
+#include <math_constants.h>
+
+#include "kernels.cuh"
+
+namespace nv {
+
+// ---------------------------------------------------------------------------
+// reductions (fixed shuffle / tree order: results are deterministic)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Sum over the block (NT threads); every thread gets the total.
+template <int NT>
+__device__ float block_sum(float v) {
+  __shared__ float s[NT / 32];
+  __shared__ float tot;
+  v = warp_sum(v);
+  if ((threadIdx.x & 31) == 0) s[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = 0.f;
+    for (int i = 0; i < NT / 32; ++i) a += s[i];
+    tot = a;
+  }
+  __syncthreads();
+  const float r = tot;
+  __syncthreads();
+  return r;
+}
+
+// Exclusive prefix sum of one int per thread over the block; *total = sum.
+template <int NT>
+__device__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int ws[NT / 32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) ws[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int s = lane < NT / 32 ? ws[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < NT / 32) ws[lane] = s;
+  }
+  __syncthreads();
+  const int excl = x - v + (w ? ws[w - 1] : 0);
+  *total = ws[NT / 32 - 1];
+  __syncthreads();
+  return excl;
+}
+
+// Largest b with start[b] <= r (start non-decreasing, start[0] = 0).
+__device__ __forceinline__ int find_seq(const int* start, int B, int r) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// RMSNorm of one row by one warp: out = rnd(g * h / sqrt(mean(h^2) + eps)).
+template <typename T>
+__device__ __forceinline__ void warp_norm_row(const float* __restrict__ h, const T* __restrict__ g,
+                                              T* __restrict__ out, int d, float eps) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+  for (int i = lane; i < d; i += 32) ss = fmaf(h[i], h[i], ss);
+  ss = warp_sum(ss);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  for (int i = lane; i < d; i += 32) out[i] = cvt<T>(h[i] * inv * ld(g + i));
+}
+
+// ---------------------------------------------------------------------------
+// RoPE table: (cos, sin) of pos * theta^(-2i/hd), computed in double.
+// ---------------------------------------------------------------------------
+__global__ void k_rope_table(float2* cs, int max_seq, int hd, double theta) {
+  const int half = hd / 2;
+  const long long n = (long long)max_seq * half;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int pos = (int)(idx / half), i = (int)(idx % half);
+    const double ang = (double)pos * pow(theta, -2.0 * (double)i / (double)hd);
+    cs[idx] = make_float2((float)cos(ang), (float)sin(ang));
+  }
+}
+void launch_rope_table(float2* cs, int max_seq, int hd, double theta, cudaStream_t st) {
+  k_rope_table<<<256, 256, 0, st>>>(cs, max_seq, hd, theta);
+}
+
+// ---------------------------------------------------------------------------
+// embedding and RMSNorm over an explicit row set (prefill / scoring)
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_embed_rows(const T* __restrict__ emb, const int* __restrict__ tok, RowSet rs, int d) {
+  const int R = *rs.nrows;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    const T* e = emb + (size_t)tok[r] * d;
+    float* h = rs.h + (size_t)rs.row_hrow[r] * d;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) h[i] = ld(e + i);
+  }
+}
+void launch_embed_rows(bool bf16, const void* emb, const int* tok_row, RowSet rs, int d, cudaStream_t st) {
+  const int grid = rs.max_rows < 4096 ? rs.max_rows : 4096;
+  if (bf16) k_embed_rows<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)emb, tok_row, rs, d);
+  else k_embed_rows<float><<<grid, 256, 0, st>>>((const float*)emb, tok_row, rs, d);
+}
+
+template <typename T>
+__global__ void k_rmsnorm_rows(RowSet rs, const T* __restrict__ g, T* __restrict__ act, int d, float eps) {
+  const int R = *rs.nrows;
+  const int wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb)
+    warp_norm_row<T>(rs.h + (size_t)rs.row_hrow[r] * d, g, act + (size_t)r * d, d, eps);
+}
+void launch_rmsnorm_rows(bool bf16, RowSet rs, const void* gain, void* act, int d, float eps, cudaStream_t st) {
+  int grid = (rs.max_rows + 7) / 8;
+  if (grid > 2048) grid = 2048;
+  if (bf16)
+    k_rmsnorm_rows<__nv_bfloat16><<<grid, 256, 0, st>>>(rs, (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
+  else k_rmsnorm_rows<float><<<grid, 256, 0, st>>>(rs, (const float*)gain, (float*)act, d, eps);
+}
+
+// ---------------------------------------------------------------------------
+// Work-list planner fused with the attention RMSNorm (decode and flush).
+//
+// Rows of layer m for sequence b (section 2 "Inferenz: Piggybacking", lazy
+// reading): when b's new token is still active at m, its deferred positions
+// [len[b][m], t_b) followed by the new position t_b; when the sequence must
+// complete early (its deferred store is full) the deferred positions alone;
+// in flush mode every deferred position [len[b][m], t_b).  Every CTA computes
+// the same prefix sums in shared memory; CTA 0 publishes the list.
+// ---------------------------------------------------------------------------
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) k_plan_norm(PlanArgs a, const T* __restrict__ gain, T* __restrict__ act,
+                                                  int d, float eps) {
+  extern __shared__ int s_start[];  // [B+1]
+  __shared__ long long s_kv[NT / 32];
+  const int B = a.B, tid = threadIdx.x;
+  const int ipt = (B + NT - 1) / NT;
+  const int b0 = tid * ipt;
+  int local = 0;
+  long long kvr = 0;
+  for (int i = 0; i < ipt; ++i) {
+    const int b = b0 + i;
+    if (b >= B) break;
+    const int tb = a.t[b], lb = a.lens[b * a.L + a.layer];
+    int cnt = 0;
+    if (a.mode == 1) {
+      cnt = tb - lb;
+    } else {
+      const int ac = a.active[b];
+      if (ac || a.force[b]) cnt = tb - lb + (ac ? 1 : 0);
+    }
+    if (cnt < 0) cnt = 0;
+    s_start[b + 1] = cnt;
+    local += cnt;
+    if (cnt > 0) kvr += (long long)(lb + cnt) * a.kv_pos_bytes;
+  }
+  int total;
+  int run = block_exclusive_scan<NT>(local, &total);
+  for (int i = 0; i < ipt; ++i) {
+    const int b = b0 + i;
+    if (b >= B) break;
+    run += s_start[b + 1];
+    s_start[b + 1] = run;
+  }
+  if (tid == 0) s_start[0] = 0;
+  __syncthreads();
+  if (total > a.max_rows) {
+    if (blockIdx.x == 0 && tid == 0) {
+      dev_fail(a.status, DEV_ERR_ROWS);
+      *a.nrows = 0;
+    }
+    return;
+  }
+  if (blockIdx.x == 0) {
+    for (int b = tid; b <= B; b += NT) a.seq_start[b] = s_start[b];
+    for (int r = tid; r < total; r += NT) {
+      const int b = find_seq(s_start, B, r);
+      const int pos = a.lens[b * a.L + a.layer] + (r - s_start[b]);
+      a.row_b[r] = b;
+      a.row_pos[r] = pos;
+      a.row_hrow[r] = b * a.cap + pos % a.cap;
+    }
+    // bytes the layer must move: weights once, K/V of positions 0..last per sequence
+    kvr = warp_sum_ll(kvr);
+    if ((tid & 31) == 0) s_kv[tid >> 5] = kvr;
+    __syncthreads();
+    if (tid == 0) {
+      *a.nrows = total;
+      if (total > 0 && a.counters) {
+        long long kv = 0;
+        for (int i = 0; i < NT / 32; ++i) kv += s_kv[i];
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_ROWS], (unsigned long long)total);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_LAYERS_RUN], 1ull);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_WEIGHT_BYTES], (unsigned long long)a.weight_bytes);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_KV_READ_BYTES], (unsigned long long)kv);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_KV_WRITE_BYTES],
+                  (unsigned long long)((long long)total * a.kv_pos_bytes));
+      }
+    }
+  }
+  const int wpb = NT / 32;
+  for (int r = blockIdx.x * wpb + (tid >> 5); r < total; r += gridDim.x * wpb) {
+    const int b = find_seq(s_start, B, r);
+    const int pos = a.lens[b * a.L + a.layer] + (r - s_start[b]);
+    const int hrow = b * a.cap + pos % a.cap;
+    warp_norm_row<T>(a.h + (size_t)hrow * d, gain, act + (size_t)r * d, d, eps);
+  }
+}
+void launch_plan_norm(bool bf16, const PlanArgs& a, const void* gain, void* act, int d, float eps, int grid,
+                      cudaStream_t st) {
+  const size_t sm = (size_t)(a.B + 1) * sizeof(int);
+  if (bf16)
+    k_plan_norm<__nv_bfloat16, 256><<<grid, 256, sm, st>>>(a, (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
+  else k_plan_norm<float, 256><<<grid, 256, sm, st>>>(a, (const float*)gain, (float*)act, d, eps);
+}
+
+// ---------------------------------------------------------------------------
+// SIMT GEMM, Y[r][n] = sum_k X[r][k] W[n][k] (fp32 accumulate, k ascending).
+// The fp32 model's contraction (tensor-core tf32 would lose the 1e-4 bound).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) k_gemm_simt(const T* __restrict__ X, int ldx, const T* __restrict__ W,
+                                                   int N, int K, const int* __restrict__ nrows, float* __restrict__ Y) {
+  __shared__ float Xs[16][68];
+  __shared__ float Ws[16][68];
+  const int R = *nrows;
+  const int n0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int lr = threadIdx.x >> 2, lk = (threadIdx.x & 3) * 4;
+  for (int r0 = blockIdx.y * 64; r0 < R; r0 += gridDim.y * 64) {
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int k0 = 0; k0 < K; k0 += 16) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int k = k0 + lk + j;
+        const int r = r0 + lr, n = n0 + lr;
+        Xs[lk + j][lr] = (r < R && k < K) ? ld(X + (size_t)r * ldx + k) : 0.f;
+        Ws[lk + j][lr] = (n < N && k < K) ? ld(W + (size_t)n * K + k) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          av[i] = Xs[kk][ty * 4 + i];
+          bv[i] = Ws[kk][tx * 4 + i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = r0 + ty * 4 + i;
+      if (r >= R) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = n0 + tx * 4 + j;
+        if (n < N) Y[(size_t)r * N + n] = acc[i][j];
+      }
+    }
+  }
+}
+void launch_gemm_simt(bool bf16, const void* X, int ldx, const void* W, int N, int K, const int* nrows,
+                      int max_rows, float* Y, cudaStream_t st) {
+  int gy = (max_rows + 63) / 64;
+  if (gy > 64) gy = 64;
+  dim3 grid((N + 63) / 64, gy);
+  if (bf16)
+    k_gemm_simt<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)X, ldx, (const __nv_bfloat16*)W, N, K,
+                                                     nrows, Y);
+  else k_gemm_simt<float><<<grid, 256, 0, st>>>((const float*)X, ldx, (const float*)W, N, K, nrows, Y);
+}
+
+// ---------------------------------------------------------------------------
+// GEMM epilogues (split partial sums added in fixed order)
+//   EPI_QKV:    RoPE on q and k (rotate-half pairs), q -> q_out, k and v ->
+//               the paged KV cache at the row's position.
+//   EPI_RESID:  h[row] += y.
+//   EPI_SWIGLU: u = silu(gate) * up, gate/up interleaved in blocks of G rows.
+//   EPI_STORE:  out = y.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float epi_sum(const EpiArgs& a, int ns, int r, int n) {
+  float y = 0.f;
+  for (int s = 0; s < ns; ++s) y += a.Y[s * a.split_stride + (size_t)r * a.N + n];
+  return y;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_epilogue(EpiArgs a) {
+  const int R = *a.rs.nrows;
+  const int ns = a.split_grid ? tc_split_count(R, a.N, a.split_K, a.split_grid, TC_MAX_SPLIT) : 1;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const long long tid0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (a.mode == EPI_QKV) {
+    const int half = a.hd / 2;
+    const long long per_row = 3LL * a.H * half;
+    for (long long idx = tid0; idx < (long long)R * per_row; idx += stride) {
+      const int r = (int)(idx / per_row);
+      const int rem = (int)(idx % per_row);
+      const int h3 = rem / half, i = rem % half;
+      const int part = h3 / a.H, head = h3 % a.H;
+      const int c0 = h3 * a.hd + i;
+      float y0 = epi_sum(a, ns, r, c0), y1 = epi_sum(a, ns, r, c0 + half);
+      const int pos = a.rs.row_pos[r];
+      if (part < 2) {
+        const float2 cs = a.rope[(size_t)pos * half + i];
+        const float u0 = y0 * cs.x - y1 * cs.y;
+        const float u1 = y1 * cs.x + y0 * cs.y;
+        y0 = u0;
+        y1 = u1;
+      }
+      if (part == 0) {
+        T* q = (T*)a.q_out + (size_t)r * a.H * a.hd + head * a.hd;
+        q[i] = cvt<T>(y0);
+        q[i + half] = cvt<T>(y1);
+      } else {
+        T* kv = (T*)a.kv.base + a.kv.offset(a.layer, a.rs.row_b[r], pos, head, part - 1);
+        kv[i] = cvt<T>(y0);
+        kv[i + half] = cvt<T>(y1);
+      }
+    }
+  } else if (a.mode == EPI_RESID) {
+    for (long long idx = tid0; idx < (long long)R * a.N; idx += stride) {
+      const int r = (int)(idx / a.N), n = (int)(idx % a.N);
+      a.rs.h[(size_t)a.rs.row_hrow[r] * a.d + n] += epi_sum(a, ns, r, n);
+    }
+  } else if (a.mode == EPI_SWIGLU) {
+    for (long long idx = tid0; idx < (long long)R * a.F; idx += stride) {
+      const int r = (int)(idx / a.F), j = (int)(idx % a.F);
+      const int blk = j / a.G, jj = j % a.G;
+      const float g = epi_sum(a, ns, r, blk * 2 * a.G + jj);
+      const float u = epi_sum(a, ns, r, blk * 2 * a.G + a.G + jj);
+      ((T*)a.u_out)[(size_t)r * a.F + j] = cvt<T>(g / (1.0f + expf(-g)) * u);
+    }
+  } else {
+    for (long long idx = tid0; idx < (long long)R * a.N; idx += stride) {
+      const int r = (int)(idx / a.N), n = (int)(idx % a.N);
+      a.out[(size_t)r * a.N + n] = epi_sum(a, ns, r, n);
+    }
+  }
+}
+void launch_epilogue(bool bf16, const EpiArgs& a, int grid, cudaStream_t st) {
+  if (bf16) k_epilogue<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+  else k_epilogue<float><<<grid, 256, 0, st>>>(a);
+}
+
+// ---------------------------------------------------------------------------
+// Paged attention with per-(sequence, layer) cache lengths.
+//
+// CTA (b, head, z): z = row group * kv_splits + split.  The row group is up to
+// 32 consecutive rows of sequence b (ascending positions p); row p attends
+// causally to keys 0..p of this layer, which are either in the cache already
+// or were written by this layer's QKV epilogue (the deferred rows of the same
+// chunk).  Keys are streamed in tiles of 64 from one page (page_size is a
+// multiple of 64); each tile is loaded once and reused by every row of the
+// group.  Online softmax in fp32; with kv_splits > 1 the unnormalised
+// partials are merged by k_attn_combine in split order.
+// ---------------------------------------------------------------------------
+template <typename T, int HD>
+__global__ void __launch_bounds__(128) k_attention(AttnArgs a) {
+  constexpr int NW = 4, RPW = ATTN_RPC / NW, KT = ATTN_KT, DPL = HD / 32;
+  __shared__ float Ks[KT][HD + 1];
+  __shared__ float Vs[KT][HD];
+  __shared__ float Qs[ATTN_RPC][HD];
+  const int b = blockIdx.x, head = blockIdx.y, z = blockIdx.z;
+  const int rg = z / a.kv_splits, sp = z % a.kv_splits;
+  if (*a.rs.nrows == 0) return;
+  const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
+  const int g0 = s0 + rg * ATTN_RPC;
+  if (g0 >= s1) return;
+  const int g1 = min(s1, g0 + ATTN_RPC), nr = g1 - g0;
+  const int pos_last = a.rs.row_pos[g1 - 1];
+  const int nt = pos_last / KT + 1;
+  const int tps = (nt + a.kv_splits - 1) / a.kv_splits;
+  const int t0 = sp * tps, t1 = min(nt, t0 + tps);
+  const int H = a.H;
+  const T* qg = (const T*)a.q;
+  for (int i = threadIdx.x; i < nr * HD; i += blockDim.x) {
+    const int r = i / HD, dd = i % HD;
+    Qs[r][dd] = ld(qg + (size_t)(g0 + r) * H * HD + head * HD + dd);
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float m[RPW], l[RPW], acc[RPW][DPL];
+  int pos[RPW];
+#pragma unroll
+  for (int j = 0; j < RPW; ++j) {
+    const int ri = w + NW * j;
+    pos[j] = ri < nr ? a.rs.row_pos[g0 + ri] : -1;
+    m[j] = -CUDART_INF_F;
+    l[j] = 0.f;
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) acc[j][c] = 0.f;
+  }
+  const T* kvb = (const T*)a.kv.base;
+  for (int tt = t0; tt < t1; ++tt) {
+    const int k0 = tt * KT;
+    __syncthreads();
+    const T* Kg = kvb + a.kv.offset(a.layer, b, k0, head, 0);
+    const T* Vg = kvb + a.kv.offset(a.layer, b, k0, head, 1);
+    const int nk = min(KT, pos_last + 1 - k0);
+    for (int i = threadIdx.x; i < KT * HD; i += blockDim.x) {
+      const int kk = i / HD, dd = i % HD;
+      const bool ok = kk < nk;
+      Ks[kk][dd] = ok ? ld(Kg + i) : 0.f;
+      Vs[kk][dd] = ok ? ld(Vg + i) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < RPW; ++j) {
+      const int p = pos[j];
+      if (p < k0) continue;
+      const int ri = w + NW * j;
+      float sa = 0.f, sb = 0.f;
+#pragma unroll 8
+      for (int dd = 0; dd < HD; ++dd) {
+        const float qv = Qs[ri][dd];
+        sa = fmaf(qv, Ks[lane][dd], sa);
+        sb = fmaf(qv, Ks[lane + 32][dd], sb);
+      }
+      sa = (k0 + lane <= p) ? sa * a.scale : -CUDART_INF_F;
+      sb = (k0 + lane + 32 <= p) ? sb * a.scale : -CUDART_INF_F;
+      const float mn = fmaxf(m[j], warp_max(fmaxf(sa, sb)));
+      const float corr = expf(m[j] - mn);
+      const float pa = expf(sa - mn), pb = expf(sb - mn);
+      l[j] = l[j] * corr + warp_sum(pa + pb);
+#pragma unroll
+      for (int c = 0; c < DPL; ++c) acc[j][c] *= corr;
+#pragma unroll 4
+      for (int kk = 0; kk < 32; ++kk) {
+        const float wa = __shfl_sync(0xffffffffu, pa, kk);
+        const float wb = __shfl_sync(0xffffffffu, pb, kk);
+#pragma unroll
+        for (int c = 0; c < DPL; ++c) {
+          acc[j][c] = fmaf(wa, Vs[kk][lane + 32 * c], acc[j][c]);
+          acc[j][c] = fmaf(wb, Vs[kk + 32][lane + 32 * c], acc[j][c]);
+        }
+      }
+      m[j] = mn;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < RPW; ++j) {
+    const int ri = w + NW * j;
+    if (ri >= nr) continue;
+    const int r = g0 + ri;
+    if (a.kv_splits == 1) {
+      const float inv = 1.0f / l[j];
+      T* o = (T*)a.o + (size_t)r * H * HD + head * HD;
+#pragma unroll
+      for (int c = 0; c < DPL; ++c) o[lane + 32 * c] = cvt<T>(acc[j][c] * inv);
+    } else {
+      float* pp = a.part + (((size_t)r * H + head) * a.kv_splits + sp) * (HD + 2);
+#pragma unroll
+      for (int c = 0; c < DPL; ++c) pp[lane + 32 * c] = acc[j][c];
+      if (lane == 0) {
+        pp[HD] = m[j];
+        pp[HD + 1] = l[j];
+      }
+    }
+  }
+  if (a.lens && head == 0 && sp == 0 && g1 == s1 && threadIdx.x == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
+}
+
+template <typename T, int HD>
+__global__ void k_attn_combine(AttnArgs a) {
+  constexpr int DPL = HD / 32;
+  const int R = *a.rs.nrows;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int item = blockIdx.x * wpb + (threadIdx.x >> 5); item < R * a.H; item += gridDim.x * wpb) {
+    const int r = item / a.H, head = item % a.H;
+    const float* pp = a.part + ((size_t)r * a.H + head) * a.kv_splits * (HD + 2);
+    float M = -CUDART_INF_F;
+    for (int s = 0; s < a.kv_splits; ++s) M = fmaxf(M, pp[s * (HD + 2) + HD]);
+    float L = 0.f, acc[DPL];
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) acc[c] = 0.f;
+    for (int s = 0; s < a.kv_splits; ++s) {
+      const float ms = pp[s * (HD + 2) + HD];
+      if (ms == -CUDART_INF_F) continue;
+      const float e = expf(ms - M);
+      L += pp[s * (HD + 2) + HD + 1] * e;
+#pragma unroll
+      for (int c = 0; c < DPL; ++c) acc[c] += pp[s * (HD + 2) + lane + 32 * c] * e;
+    }
+    T* o = (T*)a.o + (size_t)r * a.H * HD + head * HD;
+#pragma unroll
+    for (int c = 0; c < DPL; ++c) o[lane + 32 * c] = cvt<T>(acc[c] / L);
+  }
+}
+
+template <typename T, int HD>
+static void attention_t(const AttnArgs& a, cudaStream_t st) {
+  dim3 grid(a.rs.B, a.H, a.row_groups * a.kv_splits);
+  k_attention<T, HD><<<grid, 128, 0, st>>>(a);
+  if (a.kv_splits > 1) {
+    int g = (a.rs.max_rows * a.H + 7) / 8;
+    if (g > 4096) g = 4096;
+    k_attn_combine<T, HD><<<g, 256, 0, st>>>(a);
+  }
+}
+void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st) {
+  if (a.hd == 64) {
+    if (bf16) attention_t<__nv_bfloat16, 64>(a, st); else attention_t<float, 64>(a, st);
+  } else {
+    if (bf16) attention_t<__nv_bfloat16, 32>(a, st); else attention_t<float, 32>(a, st);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decode step begin / end
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_step_begin(StepArgs a) {
+  const int b = blockIdx.x;
+  const int tb = a.t[b];
+  if (threadIdx.x == 0) {
+    a.active[b] = 1;
+    a.exit_id[b] = 0;
+    // a sequence whose deferred store would overflow completes its deferred
+    // rows in this step (the values do not change, only when they are made)
+    const int pending = tb - a.lens[b * a.L + a.L - 1];
+    const int f = (pending + 1 >= a.cap) ? 1 : 0;
+    a.force[b] = f;
+    if (f && a.counters) atomicAdd((unsigned long long*)&a.counters[NV_CTR_FORCED], 1ull);
+    for (int k = 0; k < a.n_exits; ++k) a.stop[k * a.B + b] = 0;
+    if (b == 0) *a.seed_dev = a.seed;
+  }
+  const T* e = (const T*)a.emb + (size_t)a.tok[b] * a.d;
+  float* h = a.hbuf + ((size_t)b * a.cap + tb % a.cap) * a.d;
+  for (int i = threadIdx.x; i < a.d; i += blockDim.x) h[i] = ld(e + i);
+}
+void launch_step_begin(bool bf16, const StepArgs& a, cudaStream_t st) {
+  if (bf16) k_step_begin<__nv_bfloat16><<<a.B, 256, 0, st>>>(a);
+  else k_step_begin<float><<<a.B, 256, 0, st>>>(a);
+}
+
+__global__ void k_step_end(StepArgs a) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b == 0 && a.counters) atomicAdd((unsigned long long*)&a.counters[NV_CTR_STEPS], 1ull);
+  if (b >= a.B) return;
+  const int tokn = a.sampled[b];
+  a.out_tok[b] = tokn;
+  a.out_exit[b] = a.exit_id[b];
+  a.tok[b] = tokn;
+  a.t[b] += 1;
+}
+void launch_step_end(const StepArgs& a, cudaStream_t st) {
+  k_step_end<<<(a.B + 255) / 256, 256, 0, st>>>(a);
+}
+
+// ---------------------------------------------------------------------------
+// Exit junction k (section 2 "Architektur": router w_k, stop/continue).
+// n_k = RMSNorm_k(h) (rounded to the model dtype), z = r_k . n_k + b_k,
+// w_k = sigmoid(z) (0 when routing is forced to the last exit), and the token
+// stops here iff u_k < w_k; the last exit always stops.  u_k is the Philox
+// uniform of counter (b, t, 0, k/4), lane k%4 (k 0-based).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) k_junction(JuncArgs a) {
+  const int b = blockIdx.x;
+  if (!a.active[b]) return;
+  const int tb = a.t[b];
+  const float* h = a.hbuf + ((size_t)b * a.cap + tb % a.cap) * a.d;
+  const T* g = (const T*)a.norm;
+  const bool last = a.k == a.n_exits - 1;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < a.d; i += 256) ss = fmaf(h[i], h[i], ss);
+  ss = block_sum<256>(ss);
+  const float inv = 1.0f / sqrtf(ss / (float)a.d + a.eps);
+  T* out = (T*)a.exit_act + (size_t)b * a.d;
+  const T* rw = (const T*)a.router_w;
+  float z = 0.f;
+  for (int i = threadIdx.x; i < a.d; i += 256) {
+    const float n = rnd<T>(h[i] * inv * ld(g + i));
+    out[i] = cvt<T>(n);
+    if (!last) z = fmaf(n, ld(rw + i), z);
+  }
+  z = block_sum<256>(z);
+  if (threadIdx.x == 0) {
+    bool stop = true;
+    if (!last) {
+      const float w = (a.router_mode == NV_ROUTER_FORCE_LAST) ? 0.f : 1.0f / (1.0f + expf(-(z + a.router_b)));
+      const unsigned long long seed = *a.seed;
+      const uint4 r = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)tb, STREAM_EXIT, (uint32_t)(a.k / 4)),
+                                    (uint32_t)seed, (uint32_t)(seed >> 32));
+      const float u = uniform01(lane_of(r, a.k % 4));
+      stop = u < w;
+    }
+    if (stop) {
+      a.active[b] = 0;
+      a.exit_id[b] = a.k + 1;
+      a.stop[b] = 1;
+      if (a.counters) atomicAdd((unsigned long long*)&a.counters[NV_CTR_EXIT0 + a.k], 1ull);
+    }
+  }
+}
+void launch_junction(bool bf16, const JuncArgs& a, cudaStream_t st) {
+  if (bf16) k_junction<__nv_bfloat16><<<a.B, 256, 0, st>>>(a);
+  else k_junction<float><<<a.B, 256, 0, st>>>(a);
+}
+
+// ---------------------------------------------------------------------------
+// Fused exit-head sampler (exact sampling, section 3; Gumbel-max reading).
+// For the rows that stopped at exit k: logit_v = W_k[v] . n_k with 16-byte
+// coalesced loads of each head row, score_v = logit_v + Gumbel(U_v) with U_v
+// from counter (b, t, 1, v/4) lane v%4, running argmax (ties to the lowest v)
+// and online log-sum-exp of the logits.  Logits never leave the chip; each CTA
+// writes one partial per row, merged by k_head_reduce in CTA order.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
+  constexpr int NW = 8, EPC = 16 / sizeof(T), MAXC = 8;
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* s_list = (int*)smem;                                   // [B]
+  T* s_act = (T*)(smem + (((size_t)a.B * 4 + 15) / 16) * 16);  // [HEAD_RMAX][d]
+  __shared__ float s_part[NW][HEAD_RMAX][HEAD_PART];
+  __shared__ int s_b[HEAD_RMAX], s_t[HEAD_RMAX];
+  const int B = a.B, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  // compact the rows that stopped here, in sequence order
+  const int ipt = (B + 255) / 256;
+  int local = 0;
+  for (int i = 0; i < ipt; ++i) {
+    const int b = tid * ipt + i;
+    if (b < B) local += a.stop[b] ? 1 : 0;
+  }
+  int n;
+  int off = block_exclusive_scan<256>(local, &n);
+  for (int i = 0; i < ipt; ++i) {
+    const int b = tid * ipt + i;
+    if (b < B && a.stop[b]) s_list[off++] = b;
+  }
+  __syncthreads();
+  if (n == 0) return;
+  if (blockIdx.x == 0 && tid == 0 && a.counters)
+    atomicAdd((unsigned long long*)&a.counters[NV_CTR_HEAD_BYTES], (unsigned long long)a.head_bytes);
+  const unsigned long long seed = *a.seed;
+  const int d = a.d, V = a.V;
+  const int nchunk = d / EPC;  // 16-byte chunks per row
+  // this CTA's vocab range, a multiple of 4 rows
+  const int groups = (V + 3) / 4;
+  const int gpc = (groups + gridDim.x - 1) / gridDim.x;
+  const int gbeg = blockIdx.x * gpc, gend = min(groups, gbeg + gpc);
+  for (int p0 = 0; p0 < n; p0 += HEAD_RMAX) {
+    const int nr = min(HEAD_RMAX, n - p0);
+    __syncthreads();
+    for (int i = tid; i < nr * nchunk; i += 256) {
+      const int r = i / nchunk, c = i % nchunk;
+      ((uint4*)s_act)[(size_t)r * nchunk + c] =
+          ((const uint4*)((const T*)a.exit_act + (size_t)s_list[p0 + r] * d))[c];
+    }
+    if (tid < nr) {
+      s_b[tid] = s_list[p0 + tid];
+      s_t[tid] = a.t[s_list[p0 + tid]];
+    }
+    __syncthreads();
+    // lane r keeps row r's running state
+    float best_s = -CUDART_INF_F, best_l = 0.f, mx = -CUDART_INF_F, se = 0.f;
+    int best_v = 0x7fffffff;
+    const int myb = lane < nr ? s_b[lane] : 0, myt = lane < nr ? s_t[lane] : 0;
+    for (int g = gbeg + w; g < gend; g += NW) {
+      uint4 rb = make_uint4(0, 0, 0, 0);
+      if (lane < nr)
+        rb = philox4x32_10(make_uint4((uint32_t)myb, (uint32_t)myt, STREAM_GUMBEL, (uint32_t)g), (uint32_t)seed,
+                           (uint32_t)(seed >> 32));
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        const int v = 4 * g + q;
+        if (v >= V) break;
+        uint4 wv[MAXC];
+        const uint4* wrow = (const uint4*)((const T*)a.head + (size_t)v * d);
+#pragma unroll
+        for (int c = 0; c < MAXC; ++c)
+          if (lane + 32 * c < nchunk) wv[c] = __ldg(wrow + lane + 32 * c);
+        float gm = 0.f;
+        if (lane < nr) gm = -logf(-logf(uniform01(lane_of(rb, q))));
+        for (int r = 0; r < nr; ++r) {
+          const uint4* arow = (const uint4*)s_act + (size_t)r * nchunk;
+          float part = 0.f;
+#pragma unroll
+          for (int c = 0; c < MAXC; ++c) {
+            if (lane + 32 * c < nchunk) {
+              const uint4 av = arow[lane + 32 * c];
+              const T* wp = (const T*)&wv[c];
+              const T* ap = (const T*)&av;
+#pragma unroll
+              for (int e = 0; e < EPC; ++e) part = fmaf(ld(wp + e), ld(ap + e), part);
+            }
+          }
+          const float logit = warp_sum(part);
+          if (lane == r) {
+            const float s = logit + gm;
+            if (s > best_s) {
+              best_s = s;
+              best_v = v;
+              best_l = logit;
+            }
+            if (logit > mx) {
+              se = se * expf(mx - logit) + 1.0f;
+              mx = logit;
+            } else {
+              se += expf(logit - mx);
+            }
+          }
+        }
+      }
+    }
+    if (lane < nr) {
+      s_part[w][lane][0] = best_s;
+      s_part[w][lane][1] = __int_as_float(best_v);
+      s_part[w][lane][2] = best_l;
+      s_part[w][lane][3] = mx;
+      s_part[w][lane][4] = se;
+    }
+    __syncthreads();
+    if (tid < nr) {
+      float bs = -CUDART_INF_F, bl = 0.f, M = -CUDART_INF_F, S = 0.f;
+      int bv = 0x7fffffff;
+      for (int ww = 0; ww < NW; ++ww) {
+        const float s = s_part[ww][tid][0];
+        const int v = __float_as_int(s_part[ww][tid][1]);
+        if (s > bs || (s == bs && v < bv)) {
+          bs = s;
+          bv = v;
+          bl = s_part[ww][tid][2];
+        }
+        const float m2 = s_part[ww][tid][3], s2 = s_part[ww][tid][4];
+        if (m2 == -CUDART_INF_F) continue;
+        if (m2 > M) {
+          S = S * expf(M - m2) + s2;
+          M = m2;
+        } else {
+          S += s2 * expf(m2 - M);
+        }
+      }
+      float* out = a.part + ((size_t)s_b[tid] * a.nblk + blockIdx.x) * HEAD_PART;
+      out[0] = bs;
+      out[1] = __int_as_float(bv);
+      out[2] = bl;
+      out[3] = M;
+      out[4] = S;
+    }
+  }
+}
+void launch_head_sample(bool bf16, const HeadArgs& a, cudaStream_t st) {
+  const size_t esz = bf16 ? 2 : 4;
+  const size_t sm = (((size_t)a.B * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * a.d * esz;
+  if (bf16) k_head_sample<__nv_bfloat16><<<a.nblk, 256, sm, st>>>(a);
+  else k_head_sample<float><<<a.nblk, 256, sm, st>>>(a);
+}
+
+__global__ void k_head_reduce(HeadArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (b >= a.B || !a.stop[b]) return;
+  float bs = -CUDART_INF_F, bl = 0.f, M = -CUDART_INF_F, S = 0.f;
+  int bv = 0x7fffffff;
+  for (int c = lane; c < a.nblk; c += 32) {
+    const float* p = a.part + ((size_t)b * a.nblk + c) * HEAD_PART;
+    const float s = p[0];
+    const int v = __float_as_int(p[1]);
+    if (s > bs || (s == bs && v < bv)) {
+      bs = s;
+      bv = v;
+      bl = p[2];
+    }
+    const float m2 = p[3], s2 = p[4];
+    if (m2 == -CUDART_INF_F) continue;
+    if (m2 > M) {
+      S = S * expf(M - m2) + s2;
+      M = m2;
+    } else {
+      S += s2 * expf(m2 - M);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float s2 = __shfl_xor_sync(0xffffffffu, bs, o);
+    const int v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+    const float l2 = __shfl_xor_sync(0xffffffffu, bl, o);
+    const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
+    const float S2 = __shfl_xor_sync(0xffffffffu, S, o);
+    if (s2 > bs || (s2 == bs && v2 < bv)) {
+      bs = s2;
+      bv = v2;
+      bl = l2;
+    }
+    const float Mn = fmaxf(M, M2);
+    if (Mn != -CUDART_INF_F) {
+      S = (M == -CUDART_INF_F ? 0.f : S * expf(M - Mn)) + (M2 == -CUDART_INF_F ? 0.f : S2 * expf(M2 - Mn));
+      M = Mn;
+    }
+  }
+  if (lane == 0) {
+    a.sampled[b] = bv;
+    if (a.logp) a.logp[b] = bl - (M + logf(S));
+  }
+}
+void launch_head_reduce(const HeadArgs& a, cudaStream_t st) {
+  k_head_reduce<<<(a.B + 7) / 8, 256, 0, st>>>(a);
+}
+
+// ---------------------------------------------------------------------------
+// Scoring (section 2: the mixture and its cross-entropy)
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_exit_rows(RowSet rs, const T* __restrict__ g, const T* __restrict__ rw, float rb, int k,
+                            int n_exits, T* __restrict__ act, float* __restrict__ z, int d, float eps) {
+  const int R = *rs.nrows;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  const bool last = k == n_exits - 1;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb) {
+    const float* h = rs.h + (size_t)rs.row_hrow[r] * d;
+    float ss = 0.f;
+    for (int i = lane; i < d; i += 32) ss = fmaf(h[i], h[i], ss);
+    ss = warp_sum(ss);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    float zz = 0.f;
+    for (int i = lane; i < d; i += 32) {
+      const float n = rnd<T>(h[i] * inv * ld(g + i));
+      act[(size_t)r * d + i] = cvt<T>(n);
+      if (!last) zz = fmaf(n, ld(rw + i), zz);
+    }
+    zz = warp_sum(zz);
+    if (!last && lane == 0) z[(size_t)r * (n_exits - 1) + k] = zz + rb;
+  }
+}
+void launch_exit_rows(bool bf16, RowSet rs, const void* norm, const void* router_w, float router_b, int k,
+                      int n_exits, void* act, float* z, int d, float eps, cudaStream_t st) {
+  int grid = (rs.max_rows + 7) / 8;
+  if (grid > 2048) grid = 2048;
+  if (bf16)
+    k_exit_rows<__nv_bfloat16><<<grid, 256, 0, st>>>(rs, (const __nv_bfloat16*)norm, (const __nv_bfloat16*)router_w,
+                                                     router_b, k, n_exits, (__nv_bfloat16*)act, z, d, eps);
+  else k_exit_rows<float><<<grid, 256, 0, st>>>(rs, (const float*)norm, (const float*)router_w, router_b, k, n_exits,
+                                                (float*)act, z, d, eps);
+}
+
+// log pi_k(target) = logit[target] - LSE(logits), one warp per row.
+__global__ void k_lse_target(const float* __restrict__ Y, int r_begin, int n, int V, const int* __restrict__ target,
+                             float* __restrict__ logpi, int k, int n_exits) {
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
+    const float* y = Y + (size_t)i * V;
+    float m = -CUDART_INF_F;
+    for (int v = lane; v < V; v += 32) m = fmaxf(m, y[v]);
+    m = warp_max(m);
+    float s = 0.f;
+    for (int v = lane; v < V; v += 32) s += expf(y[v] - m);
+    s = warp_sum(s);
+    const int r = r_begin + i;
+    if (lane == 0) logpi[(size_t)r * n_exits + k] = y[target[r]] - (m + logf(s));
+  }
+}
+void launch_lse_target(const float* Y, int r_begin, int n, int V, const int* target, float* logpi, int k,
+                       int n_exits, cudaStream_t st) {
+  int grid = (n + 7) / 8;
+  if (grid > 4096) grid = 4096;
+  if (grid < 1) grid = 1;
+  k_lse_target<<<grid, 256, 0, st>>>(Y, r_begin, n, V, target, logpi, k, n_exits);
+}
+
+__device__ __forceinline__ float log_sigmoid(float z) {
+  // log sigma(z) = -softplus(-z) = min(z, 0) - log1p(exp(-|z|))
+  return fminf(z, 0.f) - log1pf(expf(-fabsf(z)));
+}
+
+// log pi_mix = LSE_k(log p_k + log pi_k), log p_k = log sigma(z_k) + sum_{j<k} log sigma(-z_j).
+__global__ void k_mixture(const float* __restrict__ z, const float* __restrict__ logpi, int R, int n_exits, int mode,
+                          float* __restrict__ logp) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= R) return;
+  float terms[NV_MAX_EXITS];
+  float acc = 0.f, M = -CUDART_INF_F;
+  for (int k = 0; k < n_exits; ++k) {
+    float lp;
+    if (mode == NV_ROUTER_FORCE_LAST) {
+      lp = (k == n_exits - 1) ? 0.f : -CUDART_INF_F;
+    } else if (k < n_exits - 1) {
+      const float zk = z[(size_t)r * (n_exits - 1) + k];
+      lp = log_sigmoid(zk) + acc;
+      acc += log_sigmoid(-zk);
+    } else {
+      lp = acc;
+    }
+    terms[k] = lp + logpi[(size_t)r * n_exits + k];
+    M = fmaxf(M, terms[k]);
+  }
+  float s = 0.f;
+  for (int k = 0; k < n_exits; ++k) s += (terms[k] == -CUDART_INF_F) ? 0.f : expf(terms[k] - M);
+  logp[r] = M + logf(s);
+}
+
+__global__ void k_mean_nll(const float* __restrict__ logp, int R, float* __restrict__ out) {
+  __shared__ double s[256];
+  double a = 0.0;
+  for (int r = threadIdx.x; r < R; r += 256) a += (double)logp[r];
+  s[threadIdx.x] = a;
+  __syncthreads();
+  for (int o = 128; o; o >>= 1) {
+    if (threadIdx.x < o) s[threadIdx.x] += s[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = (float)(-s[0] / (double)R);
+}
+
+__global__ void k_philox(unsigned long long seed, const uint4* ctr, int n, uint4* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = philox4x32_10(ctr[i], (uint32_t)seed, (uint32_t)(seed >> 32));
+}
+void launch_philox(unsigned long long seed, const void* ctr, int n, void* out, cudaStream_t st) {
+  k_philox<<<(n + 255) / 256, 256, 0, st>>>(seed, (const uint4*)ctr, n, (uint4*)out);
+}
+
+cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes) {
+  cudaError_t e = cudaSuccess;
+  if (head_bytes > 48 * 1024) {
+    e = cudaFuncSetAttribute(k_head_sample<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)head_bytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_head_sample<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)head_bytes);
+  }
+  if (e == cudaSuccess && plan_bytes > 48 * 1024) {
+    e = cudaFuncSetAttribute(k_plan_norm<__nv_bfloat16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)plan_bytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_plan_norm<float, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan_bytes);
+  }
+  return e;
+}
+
+void launch_mixture(const float* z, const float* logpi, int R, int n_exits, int mode, float* logp, float* mean_nll,
+                    cudaStream_t st) {
+  k_mixture<<<(R + 255) / 256, 256, 0, st>>>(z, logpi, R, n_exits, mode, logp);
+  if (mean_nll) k_mean_nll<<<1, 256, 0, st>>>(logp, R, mean_nll);
+}
+
+}  // namespace nv

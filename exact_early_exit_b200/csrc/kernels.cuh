@@ -1,0 +1,152 @@
+// Launchers for libnvium's kernels (host side).  Every launcher takes
+// `bf16` to pick the element type of weights / activations / KV cache.
+#pragma once
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace nv {
+
+constexpr int ATTN_KT = 64;    // keys per attention tile; page_size must be a multiple
+constexpr int ATTN_RPC = 32;   // rows per attention CTA (row group)
+constexpr int HEAD_RMAX = 32;  // rows per pass of the exit-head sampler
+constexpr int HEAD_PART = 5;   // floats per head partial: score, id, logit, max, sumexp
+
+void launch_rope_table(float2* cs, int max_seq, int hd, double theta, cudaStream_t st);
+
+void launch_embed_rows(bool bf16, const void* emb, const int* tok_row, RowSet rs, int d, cudaStream_t st);
+void launch_rmsnorm_rows(bool bf16, RowSet rs, const void* gain, void* act, int d, float eps, cudaStream_t st);
+
+struct PlanArgs {
+  int B, L, cap, layer, mode;  // mode 0: decode step (lazy rule), 1: flush
+  const int* t;
+  const int* active;
+  const int* force;
+  const int* lens;       // [B][L]
+  int* row_b;
+  int* row_pos;
+  int* row_hrow;
+  int* seq_start;        // [B+1]
+  int* nrows;
+  int max_rows;
+  int* status;
+  long long* counters;
+  long long weight_bytes;   // this layer's weight bytes
+  long long kv_pos_bytes;   // K+V bytes of one position of one layer
+  const float* h;           // residual ring [B][cap][d]
+};
+void launch_plan_norm(bool bf16, const PlanArgs& a, const void* gain, void* act, int d, float eps,
+                      int grid, cudaStream_t st);
+
+// Y[r][n] = sum_k X[r][k] W[n][k], fp32 out, rows r < *nrows.
+void launch_gemm_simt(bool bf16, const void* X, int ldx, const void* W, int N, int K, const int* nrows,
+                      int max_rows, float* Y, cudaStream_t st);
+
+struct EpiArgs {
+  int mode;
+  const float* Y;        // [nsplit][rows][N] partial sums
+  int split_grid;        // 0: one slice; else the GEMM grid (see tc_split_count)
+  int split_K;           // the GEMM's K (for tc_split_count)
+  size_t split_stride;   // elements between partial-sum slices
+  int N;
+  RowSet rs;
+  int d;
+  // EPI_QKV
+  int H, hd;
+  const float2* rope;    // [max_seq][hd/2] (cos, sin)
+  void* q_out;           // [max_rows][H*hd]
+  KVView kv;
+  int layer;
+  // EPI_SWIGLU
+  int F, G;
+  void* u_out;           // [max_rows][F]
+  // EPI_STORE
+  float* out;
+};
+void launch_epilogue(bool bf16, const EpiArgs& a, int grid, cudaStream_t st);
+
+struct AttnArgs {
+  RowSet rs;
+  const void* q;
+  void* o;
+  KVView kv;
+  int layer, H, hd;
+  int kv_splits, row_groups;
+  float scale;
+  float* part;     // [max_rows][H][kv_splits][hd+2] when kv_splits > 1
+  int* lens;       // when set: lens[b*L+layer] = last row position + 1
+  int L;
+};
+void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
+
+struct StepArgs {
+  int B, L, cap, d, n_exits;
+  int* t;
+  int* tok;
+  int* active;
+  int* exit_id;
+  int* force;
+  int* stop;             // [n_exits][B]
+  const int* lens;
+  float* hbuf;
+  const void* emb;
+  unsigned long long* seed_dev;
+  unsigned long long seed;
+  long long* counters;
+  // step end
+  const int* sampled;
+  int* out_tok;
+  int* out_exit;
+};
+void launch_step_begin(bool bf16, const StepArgs& a, cudaStream_t st);
+void launch_step_end(const StepArgs& a, cudaStream_t st);
+
+struct JuncArgs {
+  int B, cap, d, k, n_exits, router_mode;
+  float eps;
+  const int* t;
+  int* active;
+  int* exit_id;
+  int* stop;             // [B] flags of this exit
+  const float* hbuf;
+  const void* norm;
+  const void* router_w;
+  float router_b;
+  void* exit_act;        // [B][d]
+  const unsigned long long* seed;
+  long long* counters;
+};
+void launch_junction(bool bf16, const JuncArgs& a, cudaStream_t st);
+
+struct HeadArgs {
+  int B, d, V, k;
+  const int* t;
+  const int* stop;       // [B] flags of this exit
+  const void* exit_act;  // [B][d]
+  const void* head;      // [V][d]
+  const unsigned long long* seed;
+  float* part;           // [B][nblk][HEAD_PART]
+  int nblk;
+  long long* counters;
+  long long head_bytes;
+  // reduce
+  int* sampled;
+  float* logp;
+};
+void launch_head_sample(bool bf16, const HeadArgs& a, cudaStream_t st);
+void launch_head_reduce(const HeadArgs& a, cudaStream_t st);
+
+// scoring
+void launch_exit_rows(bool bf16, RowSet rs, const void* norm, const void* router_w, float router_b, int k,
+                      int n_exits, void* act, float* z, int d, float eps, cudaStream_t st);
+void launch_lse_target(const float* Y, int r_begin, int n, int V, const int* target, float* logpi, int k,
+                       int n_exits, cudaStream_t st);
+void launch_philox(unsigned long long seed, const void* ctr, int n, void* out, cudaStream_t st);
+
+// Opt-in shared memory for the head sampler and the planner.
+cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes);
+
+void launch_mixture(const float* z, const float* logpi, int R, int n_exits, int mode, float* logp,
+                    float* mean_nll, cudaStream_t st);
+
+}  // namespace nv

@@ -1,0 +1,1136 @@
+// libnvium C ABI: model packing, decode state, and the host-side order of
+// kernel launches for prefill, decode steps, flush and scoring.
+//
+// The decode step follows section 2 "Inferenz: Piggybacking" of the N-vium
+// summary (arXiv 2605.13190): per layer one packed pass over the new tokens
+// still active at that depth and the deferred rows of their sequences.  All
+// control flow inside a step is on the device (row counts, stop decisions),
+// so a step is one CUDA graph replay.
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+namespace nv {
+static thread_local std::string g_err;
+void set_error(const std::string& msg) { g_err = msg; }
+}  // namespace nv
+
+using namespace nv;
+
+namespace {
+
+template <typename T>
+nv_status dalloc(T** p, size_t count) {
+  *p = nullptr;
+  if (count == 0) count = 1;
+  cudaError_t e = cudaMalloc((void**)p, count * sizeof(T));
+  if (e != cudaSuccess) {
+    set_error(std::string("cudaMalloc of ") + std::to_string(count * sizeof(T)) + " bytes: " + cudaGetErrorString(e));
+    cudaGetLastError();
+    return NV_ERR_OOM;
+  }
+  return NV_OK;
+}
+nv_status dalloc_bytes(void** p, size_t bytes) { return dalloc((unsigned char**)p, bytes); }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// grow-only device buffer
+struct Buf {
+  void* p = nullptr;
+  size_t bytes = 0;
+  nv_status need(size_t n) {
+    if (n <= bytes) return NV_OK;
+    if (p) cudaFree(p);
+    p = nullptr;
+    bytes = 0;
+    NV_TRY(dalloc_bytes(&p, n));
+    bytes = n;
+    return NV_OK;
+  }
+  void release() {
+    if (p) cudaFree(p);
+    p = nullptr;
+    bytes = 0;
+  }
+  template <typename T> T* as() const { return (T*)p; }
+};
+
+}  // namespace
+
+struct nv_model {
+  nv_config cfg;
+  bool bf16 = false;
+  size_t esz = 4;
+  int d = 0, H = 0, hd = 0, HQ = 0, F = 0, V = 0, L = 0, NE = 0, G = 0;
+  void* pool = nullptr;
+  void* tok_emb = nullptr;
+  std::vector<LayerDev> layers;
+  std::vector<ExitDev> exits;
+  std::vector<int> exit_at;  // layer (0-based) -> exit index, or -1
+  float2* rope = nullptr;
+  long long layer_weight_bytes = 0;
+  int gemm_kind = GEMM_SIMT;
+  GemmPlanCache* gemm_plans = nullptr;
+  // scoring scratch
+  Buf sc_h, sc_act, sc_q, sc_o, sc_Y, sc_kv, sc_part, sc_z, sc_logpi, sc_logp, sc_i32, sc_nll;
+};
+
+struct nv_state {
+  nv_model* m = nullptr;
+  int B = 0, cap = 0, max_seq = 0, ps = 0, pps = 0, max_rows = 0;
+  // paged KV
+  void* kv = nullptr;
+  size_t kv_layer_stride = 0;
+  int n_pages = 0;
+  int* page_table = nullptr;
+  std::vector<int> h_page_table;
+  int next_free_page = 0;
+  // per-sequence device state
+  int *t = nullptr, *tok = nullptr, *lens = nullptr, *active = nullptr, *exit_id = nullptr, *force = nullptr;
+  int *stop = nullptr, *sampled = nullptr, *out_tok = nullptr, *out_exit = nullptr;
+  int *prompt_len = nullptr, *prompt_last = nullptr;
+  float* logp = nullptr;
+  float* hbuf = nullptr;
+  // work list and activations
+  int *row_b = nullptr, *row_pos = nullptr, *row_hrow = nullptr, *seq_start = nullptr, *nrows = nullptr;
+  void *act = nullptr, *q = nullptr, *o = nullptr, *exit_act = nullptr;
+  float *Y = nullptr, *attn_part = nullptr, *head_part = nullptr;
+  size_t Y_elems = 0;
+  int head_nblk = 0, kv_splits = 1, row_groups = 1;
+  unsigned long long* seed_dev = nullptr;
+  long long* counters = nullptr;
+  int* status = nullptr;
+  // host mirrors
+  std::vector<int> h_prompt_len, h_t;
+  bool prefilled = false;
+  cudaGraphExec_t graph = nullptr;
+  cudaStream_t cap_stream = nullptr;
+  std::vector<void*> allocs;
+  // prefill scratch
+  Buf pf_rows, pf_h, pf_tok;
+};
+
+namespace {
+
+RowSet state_rowset(nv_state* s) {
+  RowSet rs;
+  rs.nrows = s->nrows;
+  rs.row_b = s->row_b;
+  rs.row_pos = s->row_pos;
+  rs.row_hrow = s->row_hrow;
+  rs.seq_start = s->seq_start;
+  rs.h = s->hbuf;
+  rs.max_rows = s->max_rows;
+  rs.B = s->B;
+  return rs;
+}
+
+KVView state_kv(nv_state* s) {
+  KVView kv;
+  kv.base = s->kv;
+  kv.layer_stride = s->kv_layer_stride;
+  kv.page_table = s->page_table;
+  kv.pages_per_seq = s->pps;
+  kv.page_size = s->ps;
+  kv.H = s->m->H;
+  kv.hd = s->m->hd;
+  return kv;
+}
+
+struct LayerIO {
+  RowSet rs;
+  KVView kv;
+  int kv_layer;        // layer index used inside the KV view
+  void* act;           // [rows][max(d,F)]
+  void* q;
+  void* o;
+  float* Y;
+  float* attn_part;
+  int kv_splits, row_groups;
+  int* lens;           // nullable: per-(seq, layer) lengths to advance
+  int L;
+  int epi_grid;
+};
+
+// Everything of layer `layer` after the attention RMSNorm (act holds the
+// normed rows): QKV + RoPE + KV write, attention, O + residual, MLP norm,
+// gate/up + SwiGLU, down + residual.
+nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st) {
+  const LayerDev& Lw = M->layers[layer];
+  const bool bf = M->bf16;
+  int sgrid = 0;
+  size_t sstride = 0;
+  EpiArgs e{};
+  e.rs = io.rs;
+  e.d = M->d;
+  e.H = M->H;
+  e.hd = M->hd;
+  e.rope = M->rope;
+  e.kv = io.kv;
+  e.layer = io.kv_layer;
+  e.F = M->F;
+  e.G = M->G;
+  // QKV
+  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.act, M->d, Lw.w_qkv, 3 * M->HQ, M->d, io.rs.nrows,
+                  io.rs.max_rows, io.Y, true, &sgrid, &sstride, st));
+  e.mode = EPI_QKV;
+  e.Y = io.Y;
+  e.split_grid = sgrid;
+  e.split_K = M->d;
+  e.split_stride = sstride;
+  e.N = 3 * M->HQ;
+  e.q_out = io.q;
+  launch_epilogue(bf, e, io.epi_grid, st);
+  // attention
+  AttnArgs a{};
+  a.rs = io.rs;
+  a.q = io.q;
+  a.o = io.o;
+  a.kv = io.kv;
+  a.layer = io.kv_layer;
+  a.H = M->H;
+  a.hd = M->hd;
+  a.kv_splits = io.kv_splits;
+  a.row_groups = io.row_groups;
+  a.scale = 1.0f / sqrtf((float)M->hd);
+  a.part = io.attn_part;
+  a.lens = io.lens;
+  a.L = io.L;
+  launch_attention(bf, a, st);
+  // output projection + residual
+  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.o, M->HQ, Lw.w_o, M->d, M->HQ, io.rs.nrows, io.rs.max_rows,
+                  io.Y, true, &sgrid, &sstride, st));
+  e.mode = EPI_RESID;
+  e.split_grid = sgrid;
+  e.split_K = M->HQ;
+  e.split_stride = sstride;
+  e.N = M->d;
+  launch_epilogue(bf, e, io.epi_grid, st);
+  // MLP
+  launch_rmsnorm_rows(bf, io.rs, Lw.mlp_norm, io.act, M->d, M->cfg.rms_eps, st);
+  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.act, M->d, Lw.w_gu, 2 * M->F, M->d, io.rs.nrows,
+                  io.rs.max_rows, io.Y, true, &sgrid, &sstride, st));
+  e.mode = EPI_SWIGLU;
+  e.split_grid = sgrid;
+  e.split_K = M->d;
+  e.split_stride = sstride;
+  e.N = 2 * M->F;
+  e.u_out = io.act;
+  launch_epilogue(bf, e, io.epi_grid, st);
+  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.act, M->F, Lw.w_d, M->d, M->F, io.rs.nrows, io.rs.max_rows,
+                  io.Y, true, &sgrid, &sstride, st));
+  e.mode = EPI_RESID;
+  e.split_grid = sgrid;
+  e.split_K = M->F;
+  e.split_stride = sstride;
+  e.N = M->d;
+  launch_epilogue(bf, e, io.epi_grid, st);
+  return NV_OK;
+}
+
+LayerIO state_io(nv_state* s) {
+  LayerIO io{};
+  io.rs = state_rowset(s);
+  io.kv = state_kv(s);
+  io.act = s->act;
+  io.q = s->q;
+  io.o = s->o;
+  io.Y = s->Y;
+  io.attn_part = s->attn_part;
+  io.kv_splits = s->kv_splits;
+  io.row_groups = s->row_groups;
+  io.lens = s->lens;
+  io.L = s->m->L;
+  io.epi_grid = 1184;
+  return io;
+}
+
+PlanArgs state_plan(nv_state* s, int layer, int mode) {
+  nv_model* M = s->m;
+  PlanArgs p{};
+  p.B = s->B;
+  p.L = M->L;
+  p.cap = s->cap;
+  p.layer = layer;
+  p.mode = mode;
+  p.t = s->t;
+  p.active = s->active;
+  p.force = s->force;
+  p.lens = s->lens;
+  p.row_b = s->row_b;
+  p.row_pos = s->row_pos;
+  p.row_hrow = s->row_hrow;
+  p.seq_start = s->seq_start;
+  p.nrows = s->nrows;
+  p.max_rows = s->max_rows;
+  p.status = s->status;
+  p.counters = s->counters;
+  p.weight_bytes = M->layer_weight_bytes;
+  p.kv_pos_bytes = (long long)2 * M->HQ * (long long)M->esz;
+  p.h = s->hbuf;
+  return p;
+}
+
+int plan_grid(nv_state* s) {
+  int g = (s->B * 2 + 7) / 8;
+  if (g < 1) g = 1;
+  if (g > 148) g = 148;
+  return g;
+}
+
+// Launches of one decode step after step_begin (captured into a graph).
+nv_status record_step(nv_state* s, cudaStream_t st) {
+  nv_model* M = s->m;
+  const bool bf = M->bf16;
+  LayerIO io = state_io(s);
+  for (int layer = 0; layer < M->L; ++layer) {
+    PlanArgs p = state_plan(s, layer, 0);
+    launch_plan_norm(bf, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
+    NV_TRY(layer_body(M, layer, io, st));
+    const int k = M->exit_at[layer];
+    if (k >= 0) {
+      JuncArgs j{};
+      j.B = s->B;
+      j.cap = s->cap;
+      j.d = M->d;
+      j.k = k;
+      j.n_exits = M->NE;
+      j.router_mode = M->cfg.router_mode;
+      j.eps = M->cfg.rms_eps;
+      j.t = s->t;
+      j.active = s->active;
+      j.exit_id = s->exit_id;
+      j.stop = s->stop + (size_t)k * s->B;
+      j.hbuf = s->hbuf;
+      j.norm = M->exits[k].norm;
+      j.router_w = M->exits[k].router_w;
+      j.router_b = M->exits[k].router_b;
+      j.exit_act = s->exit_act;
+      j.seed = s->seed_dev;
+      j.counters = s->counters;
+      launch_junction(bf, j, st);
+      HeadArgs h{};
+      h.B = s->B;
+      h.d = M->d;
+      h.V = M->V;
+      h.k = k;
+      h.t = s->t;
+      h.stop = j.stop;
+      h.exit_act = s->exit_act;
+      h.head = M->exits[k].head;
+      h.seed = s->seed_dev;
+      h.part = s->head_part;
+      h.nblk = s->head_nblk;
+      h.counters = s->counters;
+      h.head_bytes = (long long)M->V * M->d * (long long)M->esz;
+      h.sampled = s->sampled;
+      h.logp = s->logp;
+      launch_head_sample(bf, h, st);
+      launch_head_reduce(h, st);
+    }
+  }
+  StepArgs sa{};
+  sa.B = s->B;
+  sa.t = s->t;
+  sa.tok = s->tok;
+  sa.exit_id = s->exit_id;
+  sa.counters = s->counters;
+  sa.sampled = s->sampled;
+  sa.out_tok = s->out_tok;
+  sa.out_exit = s->out_exit;
+  launch_step_end(sa, st);
+  return NV_OK;
+}
+
+nv_status check_status(nv_state* s) {
+  int v = 0;
+  NV_CUDA_TRY(cudaMemcpy(&v, s->status, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v == DEV_OK) {
+    int* g = gemm_status_ptr(s->m->gemm_plans);
+    if (g) NV_CUDA_TRY(cudaMemcpy(&v, g, sizeof(int), cudaMemcpyDeviceToHost));
+  }
+  if (v == DEV_OK) return NV_OK;
+  const char* what = v == DEV_ERR_ROWS ? "a per-layer work list exceeded its capacity"
+                     : v == DEV_ERR_KV ? "a KV position beyond the page table"
+                     : v == DEV_ERR_TIMEOUT ? "a bounded device wait ran out"
+                                            : "unknown device error";
+  set_error(std::string("device reported: ") + what);
+  return v == DEV_ERR_TIMEOUT ? NV_ERR_TIMEOUT : NV_ERR_CAPACITY;
+}
+
+// Give sequence b physical pages for positions [0, upto).
+nv_status ensure_pages(nv_state* s, int b, int upto, bool* changed) {
+  const int need = (upto + s->ps - 1) / s->ps;
+  if (need > s->pps) {
+    set_error("sequence length exceeds max_seq");
+    return NV_ERR_CAPACITY;
+  }
+  for (int i = 0; i < need; ++i) {
+    int& e = s->h_page_table[(size_t)b * s->pps + i];
+    if (e < 0) {
+      if (s->next_free_page >= s->n_pages) {
+        set_error("KV page pool exhausted");
+        return NV_ERR_CAPACITY;
+      }
+      e = s->next_free_page++;
+      *changed = true;
+    }
+  }
+  return NV_OK;
+}
+
+nv_status upload_page_table(nv_state* s, cudaStream_t st) {
+  NV_CUDA_TRY(cudaMemcpyAsync(s->page_table, s->h_page_table.data(), s->h_page_table.size() * sizeof(int),
+                              cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  return NV_OK;
+}
+
+nv_status validate_config(const nv_config* c) {
+  auto bad = [](const char* m) {
+    set_error(std::string("invalid config: ") + m);
+    return NV_ERR_INVALID_ARG;
+  };
+  if (!c) return bad("null");
+  if (c->n_layers < 1 || c->n_layers > NV_MAX_LAYERS) return bad("n_layers");
+  if (c->n_exits < 1 || c->n_exits > NV_MAX_EXITS) return bad("n_exits");
+  if (c->d_model < 32 || c->n_heads < 1 || c->d_ff < 1 || c->vocab < 4) return bad("sizes");
+  if (c->head_dim != 32 && c->head_dim != 64) return bad("head_dim must be 32 or 64");
+  if (c->dtype != NV_F32 && c->dtype != NV_BF16) return bad("dtype");
+  const int epc = c->dtype == NV_BF16 ? 8 : 4;
+  if (c->d_model % epc || c->d_ff % epc || (c->n_heads * c->head_dim) % epc)
+    return bad("d_model, d_ff and n_heads*head_dim must be multiples of 16 bytes");
+  if (c->d_model / epc > 256) return bad("d_model too large for the exit-head kernel");
+  int prev = 0;
+  for (int k = 0; k < c->n_exits; ++k) {
+    if (c->exit_layers[k] <= prev || c->exit_layers[k] > c->n_layers) return bad("exit_layers must increase");
+    prev = c->exit_layers[k];
+  }
+  if (prev != c->n_layers) return bad("last exit must follow the last layer");
+  if (c->max_batch < 1 || c->max_batch > 16384) return bad("max_batch");
+  if (c->max_seq < 2) return bad("max_seq");
+  if (c->page_size < ATTN_KT || c->page_size % ATTN_KT) return bad("page_size must be a multiple of 64");
+  if (c->max_pending < 2) return bad("max_pending must be >= 2");
+  if (c->router_mode != NV_ROUTER_NORMAL && c->router_mode != NV_ROUTER_FORCE_LAST) return bad("router_mode");
+  if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return bad("rms_eps / rope_theta");
+  return NV_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* nv_last_error(void) { return g_err.c_str(); }
+
+nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
+  if (!out) {
+    set_error("out is null");
+    return NV_ERR_INVALID_ARG;
+  }
+  *out = nullptr;
+  NV_TRY(validate_config(cfg));
+  if (!w || !w->tok_emb || !w->layers || !w->exits) {
+    set_error("weights: null pointer");
+    return NV_ERR_INVALID_ARG;
+  }
+  nv_model* M = new nv_model();
+  M->cfg = *cfg;
+  M->bf16 = cfg->dtype == NV_BF16;
+  M->esz = M->bf16 ? 2 : 4;
+  M->d = cfg->d_model;
+  M->H = cfg->n_heads;
+  M->hd = cfg->head_dim;
+  M->HQ = M->H * M->hd;
+  M->F = cfg->d_ff;
+  M->V = cfg->vocab;
+  M->L = cfg->n_layers;
+  M->NE = cfg->n_exits;
+  M->G = (M->F % 64 == 0) ? 64 : M->F;
+  M->exit_at.assign(M->L, -1);
+  for (int k = 0; k < M->NE; ++k) M->exit_at[cfg->exit_layers[k] - 1] = k;
+  const size_t esz = M->esz, d = M->d, HQ = M->HQ, F = M->F, V = M->V;
+  for (int i = 0; i < M->L; ++i) {
+    const nv_layer_weights& lw = w->layers[i];
+    if (!lw.attn_norm || !lw.wq || !lw.wk || !lw.wv || !lw.wo || !lw.mlp_norm || !lw.wg || !lw.wu || !lw.wd) {
+      set_error("weights: null layer tensor");
+      delete M;
+      return NV_ERR_INVALID_ARG;
+    }
+  }
+  for (int k = 0; k < M->NE; ++k) {
+    if (!w->exits[k].norm || !w->exits[k].head || (k < M->NE - 1 && !w->exits[k].router_w)) {
+      set_error("weights: null exit tensor");
+      delete M;
+      return NV_ERR_INVALID_ARG;
+    }
+  }
+  // pool layout
+  const size_t A = 256;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, A);
+    return o;
+  };
+  const size_t o_emb = take(V * d * esz);
+  std::vector<size_t> o_l(M->L * 6);
+  for (int i = 0; i < M->L; ++i) {
+    o_l[i * 6 + 0] = take(d * esz);
+    o_l[i * 6 + 1] = take(3 * HQ * d * esz);
+    o_l[i * 6 + 2] = take(d * HQ * esz);
+    o_l[i * 6 + 3] = take(d * esz);
+    o_l[i * 6 + 4] = take(2 * F * d * esz);
+    o_l[i * 6 + 5] = take(d * F * esz);
+  }
+  // heads: identical pointers share one packed copy
+  std::vector<size_t> o_e(M->NE * 3);
+  for (int k = 0; k < M->NE; ++k) {
+    o_e[k * 3 + 0] = take(d * esz);
+    int same = -1;
+    for (int j = 0; j < k; ++j)
+      if (w->exits[j].head == w->exits[k].head) same = j;
+    o_e[k * 3 + 1] = same >= 0 ? o_e[same * 3 + 1] : take(V * d * esz);
+    o_e[k * 3 + 2] = take(d * esz);
+  }
+  const size_t o_rope = take((size_t)cfg->max_seq * (M->hd / 2) * sizeof(float2));
+  nv_status st = dalloc_bytes(&M->pool, off);
+  if (st != NV_OK) {
+    delete M;
+    return st;
+  }
+  unsigned char* P = (unsigned char*)M->pool;
+  auto cp = [&](size_t o, const void* src, size_t bytes) -> nv_status {
+    NV_CUDA_TRY(cudaMemcpy(P + o, src, bytes, cudaMemcpyDefault));
+    return NV_OK;
+  };
+#define NV_CP(o, src, bytes)         \
+  do {                               \
+    nv_status _s = cp(o, src, bytes); \
+    if (_s != NV_OK) {               \
+      nv_destroy(M);                 \
+      return _s;                     \
+    }                                \
+  } while (0)
+  NV_CP(o_emb, w->tok_emb, V * d * esz);
+  M->tok_emb = P + o_emb;
+  M->layers.resize(M->L);
+  for (int i = 0; i < M->L; ++i) {
+    const nv_layer_weights& lw = w->layers[i];
+    const size_t qkv = o_l[i * 6 + 1], gu = o_l[i * 6 + 4];
+    NV_CP(o_l[i * 6 + 0], lw.attn_norm, d * esz);
+    NV_CP(qkv, lw.wq, HQ * d * esz);
+    NV_CP(qkv + HQ * d * esz, lw.wk, HQ * d * esz);
+    NV_CP(qkv + 2 * HQ * d * esz, lw.wv, HQ * d * esz);
+    NV_CP(o_l[i * 6 + 2], lw.wo, d * HQ * esz);
+    NV_CP(o_l[i * 6 + 3], lw.mlp_norm, d * esz);
+    // gate/up interleaved in blocks of G rows: [g0..gG-1, u0..uG-1, gG.., ...]
+    const size_t blk = (size_t)M->G * d * esz, nblk = F / M->G;
+    cudaError_t e1 = cudaMemcpy2D(P + gu, 2 * blk, lw.wg, blk, blk, nblk, cudaMemcpyDefault);
+    cudaError_t e2 = cudaMemcpy2D(P + gu + blk, 2 * blk, lw.wu, blk, blk, nblk, cudaMemcpyDefault);
+    if (e1 != cudaSuccess || e2 != cudaSuccess) {
+      set_error(std::string("packing gate/up: ") + cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
+      nv_destroy(M);
+      return NV_ERR_CUDA;
+    }
+    NV_CP(o_l[i * 6 + 5], lw.wd, d * F * esz);
+    M->layers[i] = LayerDev{P + o_l[i * 6 + 0], P + qkv, P + o_l[i * 6 + 2], P + o_l[i * 6 + 3], P + gu,
+                            P + o_l[i * 6 + 5]};
+  }
+  M->exits.resize(M->NE);
+  for (int k = 0; k < M->NE; ++k) {
+    const nv_exit_weights& ew = w->exits[k];
+    NV_CP(o_e[k * 3 + 0], ew.norm, d * esz);
+    NV_CP(o_e[k * 3 + 1], ew.head, V * d * esz);
+    if (k < M->NE - 1) NV_CP(o_e[k * 3 + 2], ew.router_w, d * esz);
+    M->exits[k] = ExitDev{P + o_e[k * 3 + 0], P + o_e[k * 3 + 1], P + o_e[k * 3 + 2], ew.router_b};
+  }
+#undef NV_CP
+  M->rope = (float2*)(P + o_rope);
+  launch_rope_table(M->rope, cfg->max_seq, M->hd, (double)cfg->rope_theta, 0);
+  M->layer_weight_bytes = (long long)(4 * HQ * d + 3 * F * d) * (long long)esz;
+  M->gemm_kind = M->bf16 ? gemm_default_kind() : GEMM_SIMT;
+  M->gemm_plans = gemm_plans_create();
+  // kernels that need more than 48 KB of dynamic shared memory
+  nv_status gs = gemm_prepare(M->gemm_kind, M->bf16);
+  if (gs != NV_OK) {
+    nv_destroy(M);
+    return gs;
+  }
+  {
+    const size_t head_sm = (((size_t)cfg->max_batch * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * d * esz;
+    cudaError_t e2 = kernels_set_smem_limits(head_sm, (size_t)(cfg->max_batch + 1) * 4);
+    if (e2 != cudaSuccess) {
+      set_error(std::string("shared memory limits: ") + cudaGetErrorString(e2));
+      nv_destroy(M);
+      return NV_ERR_UNSUPPORTED;
+    }
+  }
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    set_error(std::string("nv_create: ") + cudaGetErrorString(e));
+    nv_destroy(M);
+    return NV_ERR_CUDA;
+  }
+  *out = M;
+  return NV_OK;
+}
+
+nv_status nv_destroy(nv_model* M) {
+  if (!M) return NV_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  if (M->pool) cudaFree(M->pool);
+  gemm_plans_destroy(M->gemm_plans);
+  for (Buf* b : {&M->sc_h, &M->sc_act, &M->sc_q, &M->sc_o, &M->sc_Y, &M->sc_kv, &M->sc_part, &M->sc_z,
+                 &M->sc_logpi, &M->sc_logp, &M->sc_i32, &M->sc_nll})
+    b->release();
+  delete M;
+  return NV_OK;
+}
+
+nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
+  if (!M || !out) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  *out = nullptr;
+  if (B < 1 || B > M->cfg.max_batch) {
+    set_error("B must be in [1, max_batch]");
+    return NV_ERR_INVALID_ARG;
+  }
+  nv_state* s = new nv_state();
+  s->m = M;
+  s->B = B;
+  s->cap = M->cfg.max_pending;
+  s->max_seq = M->cfg.max_seq;
+  s->ps = M->cfg.page_size;
+  s->pps = (s->max_seq + s->ps - 1) / s->ps;
+  s->max_rows = B * (s->cap + 1);
+  s->n_pages = B * s->pps;
+  s->h_page_table.assign((size_t)B * s->pps, -1);
+  const size_t esz = M->esz, d = M->d, HQ = M->HQ, F = M->F;
+  const size_t page_elems = (size_t)2 * M->H * s->ps * M->hd;
+  s->kv_layer_stride = (size_t)s->n_pages * page_elems;
+  // attention parallelism: split the key range when few (sequence, head) pairs
+  int ks = (2 * 148 + B * M->H - 1) / (B * M->H);
+  s->kv_splits = ks < 1 ? 1 : (ks > 16 ? 16 : ks);
+  s->row_groups = (s->cap + 1 + ATTN_RPC - 1) / ATTN_RPC;
+  s->head_nblk = 296;
+  const size_t wide = d > F ? d : F;
+  s->Y_elems = gemm_workspace_elems(M->gemm_kind, (size_t)s->max_rows, (size_t)(3 * HQ > 2 * F ? 3 * HQ : 2 * F));
+  nv_status st = NV_OK;
+  auto A = [&](void** p, size_t bytes) {
+    if (st != NV_OK) return;
+    st = dalloc_bytes(p, bytes);
+    if (st == NV_OK) s->allocs.push_back(*p);
+  };
+  A(&s->kv, (size_t)M->L * s->kv_layer_stride * esz);
+  A((void**)&s->page_table, s->h_page_table.size() * 4);
+  for (int** p : {&s->t, &s->tok, &s->active, &s->exit_id, &s->force, &s->sampled, &s->out_tok, &s->out_exit,
+                  &s->prompt_len, &s->prompt_last})
+    A((void**)p, (size_t)B * 4);
+  A((void**)&s->lens, (size_t)B * M->L * 4);
+  A((void**)&s->stop, (size_t)B * M->NE * 4);
+  A((void**)&s->logp, (size_t)B * 4);
+  A((void**)&s->hbuf, (size_t)B * s->cap * d * 4);
+  for (int** p : {&s->row_b, &s->row_pos, &s->row_hrow}) A((void**)p, (size_t)s->max_rows * 4);
+  A((void**)&s->seq_start, (size_t)(B + 1) * 4);
+  A((void**)&s->nrows, 4);
+  A(&s->act, (size_t)s->max_rows * wide * esz);
+  A(&s->q, (size_t)s->max_rows * HQ * esz);
+  A(&s->o, (size_t)s->max_rows * HQ * esz);
+  A(&s->exit_act, (size_t)B * d * esz);
+  A((void**)&s->Y, s->Y_elems * 4);
+  A((void**)&s->attn_part, (size_t)s->max_rows * M->H * s->kv_splits * (M->hd + 2) * 4);
+  A((void**)&s->head_part, (size_t)B * s->head_nblk * HEAD_PART * 4);
+  A((void**)&s->seed_dev, 8);
+  A((void**)&s->counters, NV_CTR_COUNT * 8);
+  A((void**)&s->status, 4);
+  if (st != NV_OK) {
+    nv_state_destroy(s);
+    return st;
+  }
+  cudaMemset(s->counters, 0, NV_CTR_COUNT * 8);
+  cudaMemset(s->status, 0, 4);
+  cudaMemset(s->nrows, 0, 4);
+  cudaMemset(s->lens, 0, (size_t)B * M->L * 4);
+  cudaMemset(s->t, 0, (size_t)B * 4);
+  cudaMemset(s->page_table, 0xff, s->h_page_table.size() * 4);
+  cudaError_t e = cudaStreamCreateWithFlags(&s->cap_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    set_error(std::string("nv_state_create: ") + cudaGetErrorString(e));
+    nv_state_destroy(s);
+    return NV_ERR_CUDA;
+  }
+  s->h_t.assign(B, 0);
+  *out = s;
+  return NV_OK;
+}
+
+nv_status nv_state_destroy(nv_state* s) {
+  if (!s) return NV_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  if (s->graph) cudaGraphExecDestroy(s->graph);
+  if (s->cap_stream) cudaStreamDestroy(s->cap_stream);
+  for (void* p : s->allocs) cudaFree(p);
+  s->pf_rows.release();
+  s->pf_h.release();
+  s->pf_tok.release();
+  delete s;
+  return NV_OK;
+}
+
+nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, void* stream) {
+  if (!s || !tokens || !lens) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  nv_model* M = s->m;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = s->B;
+  size_t total = 0;
+  for (int b = 0; b < B; ++b) {
+    if (lens[b] < 1 || lens[b] >= s->max_seq) {
+      set_error("prompt length must be in [1, max_seq)");
+      return NV_ERR_INVALID_ARG;
+    }
+    total += lens[b];
+  }
+  std::vector<int> htok(total);
+  NV_CUDA_TRY(cudaMemcpy(htok.data(), tokens, total * 4, cudaMemcpyDefault));
+  for (size_t i = 0; i < total; ++i)
+    if (htok[i] < 0 || htok[i] >= M->V) {
+      set_error("token id out of range");
+      return NV_ERR_INVALID_ARG;
+    }
+  // pages for every prompt position and the first decode position
+  std::fill(s->h_page_table.begin(), s->h_page_table.end(), -1);
+  s->next_free_page = 0;
+  bool changed = false;
+  for (int b = 0; b < B; ++b) NV_TRY(ensure_pages(s, b, lens[b], &changed));
+  NV_TRY(upload_page_table(s, st));
+  // rows: positions 0..P_b-2, in chunks of at most `chunk` rows (a sequence
+  // may straddle chunks: a chunk's rows see the earlier chunks' KV at every
+  // layer because chunks run through all layers in order)
+  const int chunk = 8192;
+  std::vector<int> rb, rp, rtok;
+  std::vector<size_t> offs(B + 1, 0);
+  for (int b = 0; b < B; ++b) offs[b + 1] = offs[b] + lens[b];
+  for (int b = 0; b < B; ++b)
+    for (int p = 0; p + 1 < lens[b]; ++p) {
+      rb.push_back(b);
+      rp.push_back(p);
+      rtok.push_back(htok[offs[b] + p]);
+    }
+  const int R = (int)rb.size();
+  const size_t wide = M->d > M->F ? M->d : M->F;
+  // per-chunk buffers: h, act, q, o, Y, attention partials, row arrays
+  const int cr = R < chunk ? (R > 0 ? R : 1) : chunk;
+  Buf h, act, q, o, Y, rows;
+  nv_status stt = NV_OK;
+  if ((stt = h.need((size_t)cr * M->d * 4)) != NV_OK) return stt;
+  if ((stt = act.need((size_t)cr * wide * M->esz)) != NV_OK) return stt;
+  if ((stt = q.need((size_t)cr * M->HQ * M->esz)) != NV_OK) return stt;
+  if ((stt = o.need((size_t)cr * M->HQ * M->esz)) != NV_OK) return stt;
+  if ((stt = Y.need(gemm_workspace_elems(M->gemm_kind, cr, 3 * M->HQ > 2 * M->F ? 3 * M->HQ : 2 * M->F) * 4)) != NV_OK)
+    return stt;
+  if ((stt = rows.need(((size_t)cr * 5 + B + 2) * 4)) != NV_OK) return stt;
+  int* d_b = rows.as<int>();
+  int* d_pos = d_b + cr;
+  int* d_hrow = d_pos + cr;
+  int* d_tok = d_hrow + cr;
+  int* d_seq = d_tok + cr;
+  int* d_n = d_seq + (B + 1);
+  std::vector<int> hrow(cr), seq(B + 1);
+  for (int i = 0; i < cr; ++i) hrow[i] = i;
+  for (int c0 = 0; c0 < R; c0 += chunk) {
+    const int n = std::min(chunk, R - c0);
+    std::fill(seq.begin(), seq.end(), 0);
+    for (int i = 0; i < n; ++i) seq[rb[c0 + i] + 1]++;
+    for (int b = 0; b < B; ++b) seq[b + 1] += seq[b];
+    NV_CUDA_TRY(cudaMemcpyAsync(d_b, rb.data() + c0, n * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_pos, rp.data() + c0, n * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_hrow, hrow.data(), n * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_tok, rtok.data() + c0, n * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_seq, seq.data(), (B + 1) * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_n, &n, 4, cudaMemcpyHostToDevice, st));
+    LayerIO io{};
+    io.rs = RowSet{d_n, d_b, d_pos, d_hrow, d_seq, h.as<float>(), cr, B};
+    io.kv = state_kv(s);
+    io.act = act.p;
+    io.q = q.p;
+    io.o = o.p;
+    io.Y = Y.as<float>();
+    io.attn_part = nullptr;
+    io.kv_splits = 1;
+    int maxrows_seq = 0;
+    for (int b = 0; b < B; ++b) maxrows_seq = std::max(maxrows_seq, seq[b + 1] - seq[b]);
+    io.row_groups = (maxrows_seq + ATTN_RPC - 1) / ATTN_RPC;
+    io.lens = nullptr;
+    io.L = M->L;
+    io.epi_grid = 2048;
+    launch_embed_rows(M->bf16, M->tok_emb, d_tok, io.rs, M->d, st);
+    for (int layer = 0; layer < M->L; ++layer) {
+      launch_rmsnorm_rows(M->bf16, io.rs, M->layers[layer].attn_norm, io.act, M->d, M->cfg.rms_eps, st);
+      NV_TRY(layer_body(M, layer, io, st));
+    }
+    NV_CUDA_TRY(cudaStreamSynchronize(st));  // the host row arrays are reused by the next chunk
+  }
+  // decode state after the prompt
+  std::vector<int> t0(B), tk(B), ln((size_t)B * M->L);
+  for (int b = 0; b < B; ++b) {
+    t0[b] = lens[b] - 1;
+    tk[b] = htok[offs[b] + lens[b] - 1];
+    for (int m = 0; m < M->L; ++m) ln[(size_t)b * M->L + m] = lens[b] - 1;
+  }
+  NV_CUDA_TRY(cudaMemcpyAsync(s->t, t0.data(), B * 4, cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaMemcpyAsync(s->tok, tk.data(), B * 4, cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaMemcpyAsync(s->lens, ln.data(), ln.size() * 4, cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaMemcpyAsync(s->prompt_len, t0.data(), B * 4, cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaMemcpyAsync(s->prompt_last, tk.data(), B * 4, cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  h.release();
+  act.release();
+  q.release();
+  o.release();
+  Y.release();
+  rows.release();
+  s->h_prompt_len.assign(lens, lens + B);
+  s->h_t = t0;
+  s->prefilled = true;
+  return check_status(s);
+}
+
+nv_status nv_rewind(nv_state* s, void* stream) {
+  if (!s) return NV_ERR_INVALID_ARG;
+  if (!s->prefilled) {
+    set_error("nv_rewind before nv_prefill");
+    return NV_ERR_STATE;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = s->B, L = s->m->L;
+  std::vector<int> t0(B), ln((size_t)B * L);
+  for (int b = 0; b < B; ++b) {
+    t0[b] = s->h_prompt_len[b] - 1;
+    for (int m = 0; m < L; ++m) ln[(size_t)b * L + m] = t0[b];
+  }
+  NV_CUDA_TRY(cudaMemcpyAsync(s->t, s->prompt_len, B * 4, cudaMemcpyDeviceToDevice, st));
+  NV_CUDA_TRY(cudaMemcpyAsync(s->tok, s->prompt_last, B * 4, cudaMemcpyDeviceToDevice, st));
+  // lens[b][m] = prompt_len[b] for all m
+  NV_CUDA_TRY(cudaMemcpyAsync(s->lens, ln.data(), ln.size() * 4, cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  s->h_t = t0;
+  return NV_OK;
+}
+
+nv_status nv_decode_step(nv_state* s, uint64_t seed, int32_t* tokens_out, int32_t* exits_out, float* logp_out,
+                         void* stream) {
+  if (!s || !tokens_out || !exits_out) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  if (!s->prefilled) {
+    set_error("nv_decode_step before nv_prefill");
+    return NV_ERR_STATE;
+  }
+  nv_model* M = s->m;
+  cudaStream_t st = (cudaStream_t)stream;
+  // pages for the positions this step writes (every sequence advances by one)
+  bool changed = false;
+  for (int b = 0; b < s->B; ++b) {
+    if (s->h_t[b] + 1 >= s->max_seq) {
+      set_error("sequence reached max_seq");
+      return NV_ERR_CAPACITY;
+    }
+    NV_TRY(ensure_pages(s, b, s->h_t[b] + 1, &changed));
+  }
+  if (changed) NV_TRY(upload_page_table(s, st));
+  StepArgs sa{};
+  sa.B = s->B;
+  sa.L = M->L;
+  sa.cap = s->cap;
+  sa.d = M->d;
+  sa.n_exits = M->NE;
+  sa.t = s->t;
+  sa.tok = s->tok;
+  sa.active = s->active;
+  sa.exit_id = s->exit_id;
+  sa.force = s->force;
+  sa.stop = s->stop;
+  sa.lens = s->lens;
+  sa.hbuf = s->hbuf;
+  sa.emb = M->tok_emb;
+  sa.seed_dev = s->seed_dev;
+  sa.seed = seed;
+  sa.counters = s->counters;
+  launch_step_begin(M->bf16, sa, st);
+  if (!s->graph) {
+    cudaGraph_t g = nullptr;
+    NV_CUDA_TRY(cudaStreamBeginCapture(s->cap_stream, cudaStreamCaptureModeThreadLocal));
+    nv_status rs = record_step(s, s->cap_stream);
+    cudaError_t e = cudaStreamEndCapture(s->cap_stream, &g);
+    if (rs != NV_OK) {
+      if (g) cudaGraphDestroy(g);
+      return rs;
+    }
+    if (e != cudaSuccess) {
+      set_error(std::string("capturing the decode step: ") + cudaGetErrorString(e));
+      return NV_ERR_CUDA;
+    }
+    e = cudaGraphInstantiate(&s->graph, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) {
+      set_error(std::string("instantiating the decode step: ") + cudaGetErrorString(e));
+      s->graph = nullptr;
+      return NV_ERR_CUDA;
+    }
+  }
+  NV_CUDA_TRY(cudaGraphLaunch(s->graph, st));
+  NV_CUDA_TRY(cudaMemcpyAsync(tokens_out, s->out_tok, s->B * 4, cudaMemcpyDefault, st));
+  NV_CUDA_TRY(cudaMemcpyAsync(exits_out, s->out_exit, s->B * 4, cudaMemcpyDefault, st));
+  if (logp_out) NV_CUDA_TRY(cudaMemcpyAsync(logp_out, s->logp, s->B * 4, cudaMemcpyDefault, st));
+  for (int b = 0; b < s->B; ++b) s->h_t[b] += 1;
+  return NV_OK;
+}
+
+nv_status nv_flush_deferred(nv_state* s, void* stream) {
+  if (!s) return NV_ERR_INVALID_ARG;
+  if (!s->prefilled) {
+    set_error("nv_flush_deferred before nv_prefill");
+    return NV_ERR_STATE;
+  }
+  nv_model* M = s->m;
+  cudaStream_t st = (cudaStream_t)stream;
+  LayerIO io = state_io(s);
+  for (int layer = M->cfg.exit_layers[0]; layer < M->L; ++layer) {
+    PlanArgs p = state_plan(s, layer, 1);
+    launch_plan_norm(M->bf16, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
+    NV_TRY(layer_body(M, layer, io, st));
+  }
+  NV_CUDA_TRY(cudaGetLastError());
+  return NV_OK;
+}
+
+nv_status nv_read_kv(nv_state* s, int b, int layer, void* k_out, void* v_out, int* len_out, void* stream) {
+  if (!s || !k_out || !v_out || !len_out) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  nv_model* M = s->m;
+  if (b < 0 || b >= s->B || layer < 0 || layer >= M->L) {
+    set_error("b or layer out of range");
+    return NV_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  int len = 0;
+  NV_CUDA_TRY(cudaMemcpy(&len, s->lens + (size_t)b * M->L + layer, 4, cudaMemcpyDeviceToHost));
+  *len_out = len;
+  const size_t row = (size_t)M->hd * M->esz;
+  for (int pos = 0; pos < len; pos += s->ps) {
+    const int page = s->h_page_table[(size_t)b * s->pps + pos / s->ps];
+    if (page < 0) {
+      set_error("KV position without a page");
+      return NV_ERR_STATE;
+    }
+    const int n = std::min(s->ps, len - pos);
+    for (int kv = 0; kv < 2; ++kv)
+      for (int h = 0; h < M->H; ++h) {
+        const unsigned char* src = (const unsigned char*)s->kv +
+                                   ((size_t)layer * s->kv_layer_stride +
+                                    (((size_t)page * 2 + kv) * M->H + h) * (size_t)s->ps * M->hd) *
+                                       M->esz;
+        unsigned char* dst = (unsigned char*)(kv ? v_out : k_out) + ((size_t)pos * M->H + h) * row;
+        // n positions of one head: source stride hd, destination stride H*hd
+        NV_CUDA_TRY(cudaMemcpy2DAsync(dst, (size_t)M->H * row, src, row, row, n, cudaMemcpyDefault, st));
+      }
+  }
+  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  return NV_OK;
+}
+
+nv_status nv_read_counters(nv_state* s, int64_t* out, int n) {
+  if (!s || !out || n < 1) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  if (n > NV_CTR_COUNT) n = NV_CTR_COUNT;
+  NV_CUDA_TRY(cudaDeviceSynchronize());
+  NV_CUDA_TRY(cudaMemcpy(out, s->counters, (size_t)n * 8, cudaMemcpyDeviceToHost));
+  return NV_OK;
+}
+
+nv_status nv_reset_counters(nv_state* s) {
+  if (!s) return NV_ERR_INVALID_ARG;
+  NV_CUDA_TRY(cudaDeviceSynchronize());
+  NV_CUDA_TRY(cudaMemset(s->counters, 0, NV_CTR_COUNT * 8));
+  return NV_OK;
+}
+
+nv_status nv_philox4x32_10(uint64_t seed, const uint32_t* ctr, int n, uint32_t* out, void* stream) {
+  if (!ctr || !out || n < 1) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  void* d = nullptr;
+  NV_TRY(dalloc_bytes(&d, (size_t)n * 32));
+  unsigned char* din = (unsigned char*)d;
+  unsigned char* dout = din + (size_t)n * 16;
+  cudaError_t e = cudaMemcpyAsync(din, ctr, (size_t)n * 16, cudaMemcpyDefault, st);
+  if (e == cudaSuccess) {
+    launch_philox(seed, din, n, dout, st);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaMemcpyAsync(out, dout, (size_t)n * 16, cudaMemcpyDefault, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  cudaFree(d);
+  if (e != cudaSuccess) {
+    set_error(std::string("nv_philox4x32_10: ") + cudaGetErrorString(e));
+    return NV_ERR_CUDA;
+  }
+  return NV_OK;
+}
+
+nv_status nv_sync_status(nv_state* s) {
+  if (!s) return NV_ERR_INVALID_ARG;
+  NV_CUDA_TRY(cudaDeviceSynchronize());
+  return check_status(s);
+}
+
+nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll,
+                           void* stream) {
+  if (!M || !tokens || !logp) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  if (B < 1 || S < 2 || S > M->cfg.max_seq) {
+    set_error("need B >= 1 and 2 <= S <= max_seq");
+    return NV_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const int Sm = S - 1;               // positions 0..S-2 predict tokens 1..S-1
+  const long long R64 = (long long)B * Sm;
+  if (R64 > (1LL << 26)) {
+    set_error("B*(S-1) too large");
+    return NV_ERR_CAPACITY;
+  }
+  const int R = (int)R64, NE = M->NE;
+  std::vector<int> htok((size_t)B * S);
+  NV_CUDA_TRY(cudaMemcpy(htok.data(), tokens, htok.size() * 4, cudaMemcpyDefault));
+  for (int v : htok)
+    if (v < 0 || v >= M->V) {
+      set_error("token id out of range");
+      return NV_ERR_INVALID_ARG;
+    }
+  const int ps = ATTN_KT;
+  const int pps = (S + ps - 1) / ps;
+  const size_t wide = M->d > M->F ? M->d : M->F;
+  const int head_chunk = std::min(R, 4096);
+  const size_t y_layers = gemm_workspace_elems(M->gemm_kind, R, 3 * M->HQ > 2 * M->F ? 3 * M->HQ : 2 * M->F);
+  const size_t y_head = gemm_workspace_elems(M->gemm_kind, head_chunk, M->V);
+  NV_TRY(M->sc_h.need((size_t)R * M->d * 4));
+  NV_TRY(M->sc_act.need((size_t)R * wide * M->esz));
+  NV_TRY(M->sc_q.need((size_t)R * M->HQ * M->esz));
+  NV_TRY(M->sc_o.need((size_t)R * M->HQ * M->esz));
+  NV_TRY(M->sc_Y.need(std::max(y_layers, y_head) * 4));
+  NV_TRY(M->sc_kv.need((size_t)B * pps * 2 * M->HQ * ps * M->esz));
+  NV_TRY(M->sc_z.need((size_t)R * (NE > 1 ? NE - 1 : 1) * 4));
+  NV_TRY(M->sc_logpi.need((size_t)R * NE * 4));
+  NV_TRY(M->sc_logp.need((size_t)R * 4));
+  NV_TRY(M->sc_nll.need(4));
+  const int nchunks = (R + head_chunk - 1) / head_chunk;
+  NV_TRY(M->sc_i32.need(((size_t)R * 5 + B + 2 + (size_t)B * pps + nchunks) * 4));
+  int* d_b = M->sc_i32.as<int>();
+  int* d_pos = d_b + R;
+  int* d_hrow = d_pos + R;
+  int* d_tok = d_hrow + R;
+  int* d_tgt = d_tok + R;
+  int* d_seq = d_tgt + R;
+  int* d_n = d_seq + (B + 1);
+  int* d_pt = d_n + 1;
+  int* d_chunk = d_pt + (size_t)B * pps;
+  {
+    std::vector<int> hb(R), hp(R), hr(R), ht(R), hg(R), hs(B + 1), hpt((size_t)B * pps), hc(nchunks);
+    for (int b = 0; b < B; ++b) {
+      hs[b] = b * Sm;
+      for (int p = 0; p < Sm; ++p) {
+        const int r = b * Sm + p;
+        hb[r] = b;
+        hp[r] = p;
+        hr[r] = r;
+        ht[r] = htok[(size_t)b * S + p];
+        hg[r] = htok[(size_t)b * S + p + 1];
+      }
+      for (int i = 0; i < pps; ++i) hpt[(size_t)b * pps + i] = b * pps + i;
+    }
+    hs[B] = R;
+    for (int c = 0; c < nchunks; ++c) hc[c] = std::min(head_chunk, R - c * head_chunk);
+    NV_CUDA_TRY(cudaMemcpyAsync(d_b, hb.data(), R * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_pos, hp.data(), R * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_hrow, hr.data(), R * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_tok, ht.data(), R * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_tgt, hg.data(), R * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_seq, hs.data(), (B + 1) * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_n, &R, 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_pt, hpt.data(), hpt.size() * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaMemcpyAsync(d_chunk, hc.data(), nchunks * 4, cudaMemcpyHostToDevice, st));
+    NV_CUDA_TRY(cudaStreamSynchronize(st));  // host vectors go out of scope
+  }
+  LayerIO io{};
+  io.rs = RowSet{d_n, d_b, d_pos, d_hrow, d_seq, M->sc_h.as<float>(), R, B};
+  io.kv.base = M->sc_kv.p;
+  io.kv.layer_stride = 0;  // one layer's KV at a time
+  io.kv.page_table = d_pt;
+  io.kv.pages_per_seq = pps;
+  io.kv.page_size = ps;
+  io.kv.H = M->H;
+  io.kv.hd = M->hd;
+  io.kv_layer = 0;
+  io.act = M->sc_act.p;
+  io.q = M->sc_q.p;
+  io.o = M->sc_o.p;
+  io.Y = M->sc_Y.as<float>();
+  io.attn_part = nullptr;
+  io.kv_splits = 1;
+  io.row_groups = (Sm + ATTN_RPC - 1) / ATTN_RPC;
+  io.lens = nullptr;
+  io.L = M->L;
+  io.epi_grid = 4096;
+  launch_embed_rows(M->bf16, M->tok_emb, d_tok, io.rs, M->d, st);
+  for (int layer = 0; layer < M->L; ++layer) {
+    launch_rmsnorm_rows(M->bf16, io.rs, M->layers[layer].attn_norm, io.act, M->d, M->cfg.rms_eps, st);
+    NV_TRY(layer_body(M, layer, io, st));
+    const int k = M->exit_at[layer];
+    if (k < 0) continue;
+    launch_exit_rows(M->bf16, io.rs, M->exits[k].norm, M->exits[k].router_w, M->exits[k].router_b, k, NE, io.act,
+                     M->sc_z.as<float>(), M->d, M->cfg.rms_eps, st);
+    for (int c = 0; c < nchunks; ++c) {
+      const int r0 = c * head_chunk;
+      int sgrid = 0;
+      size_t sstride = 0;
+      NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, M->bf16, (const unsigned char*)io.act + (size_t)r0 * M->d * M->esz,
+                      M->d, M->exits[k].head, M->V, M->d, d_chunk + c, head_chunk, io.Y, false, &sgrid, &sstride, st));
+      const float* Yh = io.Y;
+      launch_lse_target(Yh, r0, std::min(head_chunk, R - r0), M->V, d_tgt, M->sc_logpi.as<float>(), k, NE, st);
+    }
+  }
+  launch_mixture(M->sc_z.as<float>(), M->sc_logpi.as<float>(), R, NE, M->cfg.router_mode, M->sc_logp.as<float>(),
+                 M->sc_nll.as<float>(), st);
+  NV_CUDA_TRY(cudaMemcpyAsync(logp, M->sc_logp.p, (size_t)R * 4, cudaMemcpyDefault, st));
+  if (mean_nll) NV_CUDA_TRY(cudaMemcpyAsync(mean_nll, M->sc_nll.p, 4, cudaMemcpyDefault, st));
+  NV_CUDA_TRY(cudaGetLastError());
+  return NV_OK;
+}
+
+}  // extern "C"

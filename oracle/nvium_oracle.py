@@ -243,10 +243,12 @@ class SeqCache:
 class OracleModel:
     """Weights (float32 copies of the stored values; widened to float64 at use)."""
 
-    def __init__(self, cfg, weights: dict, router_mode: int = ROUTER_NORMAL):
+    def __init__(self, cfg, weights: dict, router_mode: int = ROUTER_NORMAL, cache_f64: Optional[bool] = None):
         self.cfg = cfg
         self.mode = router_mode
         self.bf16 = cfg.dtype == _wl.BF16
+        # keep float64 copies of the weights when they fit comfortably
+        self._f64 = {} if (cache_f64 if cache_f64 is not None else cfg.n_params() < 4e8) else None
         f = _wl.as_f32
         self.tok_emb = f(weights["tok_emb"])
         self.layers = [{k: f(v) for k, v in L.items()} for L in weights["layers"]]
@@ -263,10 +265,14 @@ class OracleModel:
     def rnd(self, x):
         return bf16_round(x) if self.bf16 else x
 
-    @staticmethod
-    def mm(x: np.ndarray, w32: np.ndarray) -> np.ndarray:
+    def mm(self, x: np.ndarray, w32: np.ndarray) -> np.ndarray:
         """y = x W^T with x [n, in] float64 and W [out, in]."""
-        return x @ w32.astype(np.float64).T
+        if self._f64 is None:
+            return x @ w32.astype(np.float64).T
+        w = self._f64.get(id(w32))
+        if w is None:
+            w = self._f64[id(w32)] = w32.astype(np.float64)
+        return x @ w.T
 
     def embed(self, tokens) -> np.ndarray:
         return self.tok_emb[np.asarray(tokens, dtype=np.int64)].astype(np.float64)
@@ -277,6 +283,14 @@ class OracleModel:
         Writes the rows' K and V into the cache at layer m, then lets row p
         attend causally to positions 0..p of layer m.  Returns the new residual.
         """
+        return self.layer_rows_multi(m, h, pos, [cache] * len(pos))
+
+    def layer_rows_multi(self, m: int, h: np.ndarray, pos: Sequence[int], caches: List[SeqCache]) -> np.ndarray:
+        """Layer m on rows that may belong to several sequences: row i sits at
+        position pos[i] of the sequence whose cache is caches[i]; each
+        sequence's rows come in ascending position order.  The projections are
+        per-row products (stacked into one matrix product); attention of row i
+        reads only its own sequence's cache."""
         cfg, L = self.cfg, self.layers[m]
         H, hd = cfg.n_heads, cfg.head_dim
         pos = np.asarray(pos, dtype=np.int64)
@@ -289,13 +303,14 @@ class OracleModel:
         q = self.rnd(rope(q, pos, cfg.rope_theta))
         k = self.rnd(rope(k, pos, cfg.rope_theta))
         v = self.rnd(v)
-        cache.K[m][pos] = k
-        cache.V[m][pos] = v
+        for i in range(n):
+            caches[i].K[m][pos[i]] = k[i]
+            caches[i].V[m][pos[i]] = v[i]
         o = np.empty((n, H, hd))
         scale = 1.0 / math.sqrt(hd)
         for i in range(n):
             p = int(pos[i])
-            Kc, Vc = cache.K[m][: p + 1], cache.V[m][: p + 1]          # [p+1, H, hd]
+            Kc, Vc = caches[i].K[m][: p + 1], caches[i].V[m][: p + 1]          # [p+1, H, hd]
             s = np.einsum("hd,jhd->hj", q[i], Kc) * scale
             s = s - s.max(axis=1, keepdims=True)
             e = np.exp(s)
@@ -440,6 +455,7 @@ class OracleDecoder:
         self.model = model
         cfg = model.cfg
         self.B = len(prompts)
+        self.ids = list(range(self.B))   # sequence index b used in the Philox counters
         self.tokens = [list(map(int, p)) for p in prompts]
         self.caches = []
         self.pending = []   # per b: {pos: h}
@@ -475,61 +491,82 @@ class OracleDecoder:
             pend[p] = h[i]
         self.caches[b].lens[layer] = positions[-1] + 1
 
-    def step_seq(self, b: int, seed: int, forced_exit: Optional[int] = None,
-                 forced_token: Optional[int] = None) -> StepRecord:
-        """One decode step of sequence b.  ``forced_exit`` / ``forced_token``
-        make the oracle follow another implementation's choice (teacher
-        forcing) while still recording its own decision and margins."""
+    def step(self, seed: int, forced_exits=None, forced_tokens=None) -> List[StepRecord]:
+        """One decode step of every sequence.  ``forced_exits`` /
+        ``forced_tokens`` ([B]) make the oracle follow another
+        implementation's choices (teacher forcing) while it still records its
+        own decisions and their margins."""
         model, cfg = self.model, self.model.cfg
-        rec = StepRecord()
-        t = self.t[b]
-        cache = self.caches[b]
-        pend = self.pending[b]
-        pend[t] = model.embed([self.tokens[b][t]])[0]
-        exit_k = None
+        B = self.B
+        recs = [StepRecord() for _ in range(B)]
+        active = [True] * B
+        for b in range(B):
+            self.pending[b][self.t[b]] = model.embed([self.tokens[b][self.t[b]]])[0]
         for layer in range(cfg.n_layers):
-            rows = list(range(cache.lens[layer], t + 1))
-            self._run_layer(b, layer, rows)
-            if (layer + 1) in model.exit_at:
-                k0 = model.exit_at[layer + 1]          # 0-based exit index
-                nk = model.exit_state(k0, pend[t])
+            rows = []          # (b, pos) in sequence order, ascending positions
+            for b in range(B):
+                if active[b]:
+                    rows += [(b, p) for p in range(self.caches[b].lens[layer], self.t[b] + 1)]
+            if not rows:
+                break
+            h = np.stack([self.pending[b][p] for b, p in rows])
+            h = model.layer_rows_multi(layer, h, [p for _, p in rows], [self.caches[b] for b, _ in rows])
+            for i, (b, p) in enumerate(rows):
+                self.pending[b][p] = h[i]
+                self.caches[b].lens[layer] = p + 1
+            if (layer + 1) not in model.exit_at:
+                continue
+            k0 = model.exit_at[layer + 1]            # 0-based exit index
+            for b in range(B):
+                if not active[b]:
+                    continue
+                rec, t = recs[b], self.t[b]
+                nk = model.exit_state(k0, self.pending[b][t])
                 if k0 < cfg.n_exits - 1:
                     w = np.asarray(model.router_prob(k0, nk)).item()
-                    u = np.asarray(exit_uniform(seed, b, t, k0 + 1)).item()
+                    u = np.asarray(exit_uniform(seed, self.ids[b], t, k0 + 1)).item()
                     rec.junctions.append((k0 + 1, u, w))
                     own_stop = u < w
                 else:
                     own_stop = True
                 if own_stop and rec.oracle_exit is None:
                     rec.oracle_exit = k0 + 1
-                stop = own_stop if forced_exit is None else (forced_exit == k0 + 1)
-                if stop:
-                    exit_k = k0
+                fe = None if forced_exits is None else int(forced_exits[b])
+                if (own_stop if fe is None else fe == k0 + 1):
+                    active[b] = False
                     lg = model.head_logits(k0, nk)[0]
-                    g = gumbel_noise(seed, b, t, cfg.vocab)
-                    sc = lg + g
+                    sc = lg + gumbel_noise(seed, self.ids[b], t, cfg.vocab)
                     rec.scores = sc
                     rec.oracle_token = int(np.argmax(sc))
-                    tok = rec.oracle_token if forced_token is None else int(forced_token)
+                    tok = rec.oracle_token if forced_tokens is None else int(forced_tokens[b])
                     rec.logp = float(lg[tok] - logsumexp(lg))
                     rec.token = tok
-                    break
-        rec.exit = exit_k + 1
-        if rec.oracle_exit is None:
-            rec.oracle_exit = cfg.n_exits
-        # rows that completed every layer leave the deferred set
-        done = cache.lens[cfg.n_layers - 1]
-        for p in [p for p in pend if p < done]:
-            del pend[p]
-        self.tokens[b].append(rec.token)
-        self.t[b] = t + 1
-        return rec
+                    rec.exit = k0 + 1
+        for b in range(B):
+            rec = recs[b]
+            if rec.oracle_exit is None:
+                rec.oracle_exit = cfg.n_exits
+            done = self.caches[b].lens[cfg.n_layers - 1]
+            for p in [p for p in self.pending[b] if p < done]:
+                del self.pending[b][p]
+            self.tokens[b].append(rec.token)
+            self.t[b] += 1
+        return recs
 
-    def step(self, seed: int, forced_exits=None, forced_tokens=None) -> List[StepRecord]:
-        return [self.step_seq(b, seed,
-                              None if forced_exits is None else int(forced_exits[b]),
-                              None if forced_tokens is None else int(forced_tokens[b]))
-                for b in range(self.B)]
+    def step_seq(self, b: int, seed: int, forced_exit: Optional[int] = None,
+                 forced_token: Optional[int] = None) -> StepRecord:
+        """One decode step of sequence b alone (the others do not move)."""
+        saved = self.B, self.tokens, self.caches, self.pending, self.t, self.ids
+        try:
+            self.B = 1
+            self.tokens, self.caches = [saved[1][b]], [saved[2][b]]
+            self.pending, self.t, self.ids = [saved[3][b]], [saved[4][b]], [saved[5][b]]
+            rec = self.step(seed, None if forced_exit is None else [forced_exit],
+                            None if forced_token is None else [forced_token])[0]
+            saved[4][b] = self.t[0]
+        finally:
+            self.B, self.tokens, self.caches, self.pending, self.t, self.ids = saved
+        return rec
 
     def flush(self):
         """Run every deferred row through the layers it still owes

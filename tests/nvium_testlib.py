@@ -1,0 +1,94 @@
+"""Helpers shared by the GPU parity tests (not a test module)."""
+import numpy as np
+
+import workloads as W
+from oracle import nvium_oracle as O
+
+
+def tolerance(cfg) -> float:
+    """Absolute tolerance on log-probabilities, router margins and Gumbel
+    scores: 1e-4 for the fp32 model, 2e-2 for bf16 models."""
+    return 1e-4 if cfg.dtype == W.F32 else 2e-2
+
+
+def kv_close(gpu, ref, cfg):
+    """KV entries: the tolerance, plus one bf16 step of the value for bf16
+    caches (both sides store rounded values; a rounding flip moves one step)."""
+    tol = tolerance(cfg)
+    rtol = 2.0 ** -7 if cfg.dtype == W.BF16 else 0.0
+    np.testing.assert_allclose(gpu, ref, atol=tol, rtol=rtol)
+
+
+def gpu_kv(state, b, layer, max_len, cfg):
+    K, V, n = state.read_kv(b, layer, max_len)
+    return W.as_f32(K).astype(np.float64), W.as_f32(V).astype(np.float64), n
+
+
+class StepChecker:
+    """Step-synchronous comparison with teacher forcing: exits and tokens
+    must agree except at near-ties (|u_k - w_k| <= tau for an exit,
+    |score gap| <= tau for a token), which are counted."""
+
+    def __init__(self, cfg):
+        self.cfg = cfg
+        self.tau = tolerance(cfg)
+        self.exit_ties = 0
+        self.token_ties = 0
+        self.steps = 0
+        self.max_logp_err = 0.0
+
+    def check(self, recs, tok, ex, lp):
+        for b, rec in enumerate(recs):
+            ge, gt = int(ex[b]), int(tok[b])
+            assert 1 <= ge <= self.cfg.n_exits
+            if ge != rec.oracle_exit:
+                k = min(ge, rec.oracle_exit)
+                uw = [(u, w) for (kk, u, w) in rec.junctions if kk == k]
+                assert uw, (b, ge, rec.oracle_exit)
+                u, w = uw[0]
+                assert abs(u - w) <= self.tau, f"exit mismatch b={b}: gpu {ge} oracle {rec.oracle_exit} u={u} w={w}"
+                self.exit_ties += 1
+            if gt != rec.oracle_token:
+                gap = abs(rec.scores[gt] - rec.scores[rec.oracle_token])
+                assert gap <= self.tau, f"token mismatch b={b}: gpu {gt} oracle {rec.oracle_token} gap={gap}"
+                self.token_ties += 1
+            if lp is not None:
+                err = abs(rec.logp - float(lp[b]))
+                self.max_logp_err = max(self.max_logp_err, err)
+                assert err <= self.tau, f"log-prob b={b}: gpu {lp[b]} oracle {rec.logp}"
+        self.steps += 1
+
+
+def run_decode_parity(nv, cfg, weights, prompts, steps, seed=1234, max_pending=256, router_mode=0,
+                      max_seq=None, check_kv=True):
+    """Decode `steps` steps on the GPU and in the oracle (teacher forced),
+    flush both, compare the caches.  Returns (checker, state, oracle)."""
+    B = len(prompts)
+    lens = np.array([len(p) for p in prompts], dtype=np.int32)
+    max_seq = max_seq or int(lens.max()) + steps + 8
+    model = nv.Model(cfg, weights, max_batch=B, max_seq=max_seq, max_pending=max_pending,
+                     router_mode=router_mode)
+    state = nv.State(model, B)
+    state.prefill(np.concatenate(prompts).astype(np.int32), lens)
+    om = O.OracleModel(cfg, weights, router_mode)
+    dec = O.OracleDecoder(om, prompts, steps)
+    chk = StepChecker(cfg)
+    tok = np.zeros(B, np.int32)
+    ex = np.zeros(B, np.int32)
+    lp = np.zeros(B, np.float32)
+    for s in range(steps):
+        state.decode_step(seed + s, tok, ex, lp)
+        recs = dec.step(seed + s, forced_exits=ex, forced_tokens=tok)
+        chk.check(recs, tok, ex, lp)
+    state.sync_status()
+    if check_kv:
+        state.flush()
+        dec.flush()
+        state.sync_status()
+        for b in range(B):
+            for m in range(cfg.n_layers):
+                K, V, n = gpu_kv(state, b, m, max_seq, cfg)
+                assert n == dec.t[b] == dec.caches[b].lens[m]
+                kv_close(K, dec.caches[b].K[m][:n], cfg)
+                kv_close(V, dec.caches[b].V[m][:n], cfg)
+    return chk, state, dec, model

@@ -1,0 +1,136 @@
+"""GPU parity on the tiny fp32 model (4 layers, d=64, 2 heads, vocab 256,
+exits after layers 1/2/3/4): the CUDA path against the CPU oracle on the same
+seeded inputs, through the C ABI.  Tolerance 1e-4 (fp32)."""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import nvium_oracle as O
+from tests.nvium_testlib import StepChecker, kv_close, run_decode_parity, tolerance
+
+pytestmark = pytest.mark.gpu
+
+nv = pytest.importorskip("exact_early_exit_b200")
+CFG = W.TINY
+
+
+@pytest.fixture(scope="module")
+def weights():
+    return W.make_weights(CFG, seed=0)
+
+
+def test_philox_matches_oracle():
+    rng = np.random.default_rng(0)
+    ctr = rng.integers(0, 2**32, size=(4096, 4), dtype=np.uint64).astype(np.uint32)
+    ctr[0] = 0
+    ctr[1] = 0xFFFFFFFF
+    for seed in (0, 1234, 0xFFFFFFFFFFFFFFFF, 0xA409382229F31D0):
+        out = nv.philox4x32_10(seed, ctr)
+        ref = O.philox4x32_10([ctr[:, i] for i in range(4)], (seed & 0xFFFFFFFF, seed >> 32))
+        np.testing.assert_array_equal(out, np.stack([r.astype(np.uint32) for r in ref], 1))
+
+
+@pytest.mark.parametrize("mode", [O.ROUTER_NORMAL, O.ROUTER_FORCE_LAST])
+def test_scoring_matches_oracle(weights, mode):
+    wl = W.WORKLOADS["T"]
+    toks = np.stack([W.make_prompts(wl, seed=s)[0] for s in (1, 2, 3)]).astype(np.int32)   # [3, 32]
+    model = nv.Model(CFG, weights, max_batch=1, max_seq=64, router_mode=mode)
+    logp = np.zeros((3, 31), np.float32)
+    nll = np.zeros(1, np.float32)
+    model.score_mixture(toks, logp, nll)
+    ref, ref_nll = O.score_mixture(O.OracleModel(CFG, weights, mode), toks)
+    np.testing.assert_allclose(logp, ref, atol=1e-4, rtol=0)
+    assert abs(nll[0] - ref_nll) <= 1e-4
+    if mode == O.ROUTER_FORCE_LAST:
+        dense = O.dense_logprobs(O.OracleModel(CFG, weights, mode), toks[0, :-1])
+        np.testing.assert_allclose(logp[0], dense[np.arange(31), toks[0, 1:]], atol=1e-4, rtol=0)
+
+
+def test_decode_parity_prompt32_steps32(weights):
+    prompts = W.make_prompts(W.WORKLOADS["T"])
+    chk, state, dec, _ = run_decode_parity(nv, CFG, weights, prompts, 32)
+    assert chk.steps == 32
+    # fp32: no near-ties expected
+    assert chk.exit_ties == 0 and chk.token_ties == 0
+    c = state.counters()
+    assert c[nv.CTR["steps"]] == 32
+    assert c[nv.CTR["exit0"]:nv.CTR["exit0"] + 4].sum() == 32
+
+
+def test_decode_parity_batch_ragged(weights):
+    prompts = [W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:n] for s, n in ((1, 5), (2, 1), (3, 17), (4, 64 + 3))]
+    chk, *_ = run_decode_parity(nv, CFG, weights, prompts, 20, max_seq=128)
+    assert chk.steps == 20
+
+
+def test_force_last_decode_is_the_dense_model(weights):
+    prompts = W.make_prompts(W.WORKLOADS["T"])
+    chk, state, dec, _ = run_decode_parity(nv, CFG, weights, prompts, 16, router_mode=O.ROUTER_FORCE_LAST)
+    c = state.counters()
+    assert c[nv.CTR["exit0"] + 3] == 16 and c[nv.CTR["exit0"]:nv.CTR["exit0"] + 3].sum() == 0
+
+
+@pytest.mark.parametrize("bias", [30.0, -30.0])
+def test_extreme_routing_and_overflowing_deferred_store(bias):
+    """All tokens exit at the first junction (bias +30) so rows pile up until
+    the deferred store (max_pending = 4) forces early completion; or none
+    exit early (bias -30)."""
+    w = W.make_weights(CFG, seed=0, router_bias=[bias, bias, bias])
+    prompts = [W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:n] for s, n in ((1, 9), (2, 3))]
+    chk, state, dec, _ = run_decode_parity(nv, CFG, w, prompts, 24, max_pending=4)
+    c = state.counters()
+    if bias > 0:
+        assert c[nv.CTR["exit0"]] == 48
+        assert c[nv.CTR["forced"]] > 0
+    else:
+        assert c[nv.CTR["exit0"] + 3] == 48
+
+
+def test_rewind_replays_identically(weights):
+    prompts = W.make_prompts(W.WORKLOADS["T"])
+    model = nv.Model(CFG, weights, max_batch=1, max_seq=80)
+    st = nv.State(model, 1)
+    st.prefill(prompts[0], [32])
+    outs = []
+    for rep in range(2):
+        seq = []
+        tok = np.zeros(1, np.int32)
+        ex = np.zeros(1, np.int32)
+        for s in range(12):
+            st.decode_step(77 + s, tok, ex)
+            seq.append((int(tok[0]), int(ex[0])))
+        outs.append(seq)
+        st.rewind()
+    assert outs[0] == outs[1]
+
+
+def test_sampler_chi_square():
+    """Exact sampling on the GPU: 4096 copies of one context, 50 seeds, joint
+    (exit, token) frequencies against p_k * pi_k(v) from the oracle."""
+    from scipy import stats
+    w = W.make_weights(CFG, seed=0, router_bias=[-0.3, 0.2, 0.0])
+    prompt = W.make_prompts(W.WORKLOADS["T"])[0][:8]
+    B = 4096
+    model = nv.Model(CFG, w, max_batch=B, max_seq=16, max_pending=4)
+    st = nv.State(model, B)
+    st.prefill(np.tile(prompt, B).astype(np.int32), np.full(B, 8, np.int32))
+    counts = np.zeros((4, CFG.vocab))
+    tok = np.zeros(B, np.int32)
+    ex = np.zeros(B, np.int32)
+    for s in range(50):
+        st.decode_step(1000 + s, tok, ex)
+        np.add.at(counts, (ex - 1, tok), 1)
+        st.rewind()
+    om = O.OracleModel(CFG, w)
+    _, states, _ = om.forward_sequence(prompt)
+    p, pi = O.step_distribution(om, [states[k][7:8] for k in range(4)])
+    exp = p[:, None] * pi * counts.sum()
+    e, c = exp.ravel(), counts.ravel()
+    order = np.argsort(e)
+    e, c = e[order], c[order]
+    small = np.cumsum(e) < 20
+    e = np.concatenate([e[~small], [e[small].sum()]])
+    c = np.concatenate([c[~small], [c[small].sum()]])
+    assert stats.chisquare(c, e * c.sum() / e.sum()).pvalue > 0.01
+    pe = stats.chisquare(counts.sum(1), p * counts.sum()).pvalue
+    assert pe > 0.01
