@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Decode throughput of the N-vium 1.5B 4-exit model on B200.
+
+One bench step = one generation pass of the whole hot path on one batch:
+rewind to the post-prefill state, `decode_steps` decode steps for every
+sequence (mixture-of-exits routing, exact sampling, deferred upper layers
+batched with later tokens), and the final flush of the deferred rows.
+`value` = decoded tokens / time with inputs resident in HBM; `e2e` = the same
+pass through the C ABI from pinned host memory (prompt upload and prefill
+inside, sampled tokens and exits copied back to the host every step).
+
+  python bench.py [--workload X64|X1|S|T] [--steps K] [--warmup W] [--gpus N]
+  python bench.py --impl reference ...     # the CPU oracle on the same config
+
+Multi-GPU (torchrun): every rank decodes its own batch of independent
+sequences (weak scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "decode tokens/s, 1.5B 4-exit model, B=1/B=64 on 1 B200; % of HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+PHILOX_SEED = 1234
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+def rank_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+    rank, world, _ = rank_env()
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seeds(rank: int):
+    """Inputs of rank r: prompt ids seed, prompt length seed, Philox seed."""
+    return 1 + 1000 * rank, 2 + 1000 * rank, PHILOX_SEED + 7919 * rank
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+REASON_FIELDS = ["clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                 "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ",".join(["clocks.sm", "clocks.max.sm", "power.draw"] + REASON_FIELDS)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if not self.proc or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# roofline inputs
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+KERNEL_SOURCES = {
+    "gemm": "exact_early_exit_b200/csrc/gemm_tc.cu",
+    "attention": "exact_early_exit_b200/csrc/kernels.cu",
+    "head": "exact_early_exit_b200/csrc/kernels.cu",
+    "epilogue": "exact_early_exit_b200/csrc/kernels.cu",
+    "plan_norm": "exact_early_exit_b200/csrc/kernels.cu",
+}
+
+
+def source_hash(kind: str) -> str:
+    p = os.path.join(ROOT, KERNEL_SOURCES.get(kind, "exact_early_exit_b200/csrc/kernels.cu"))
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def ncu_traffic(kind: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary of this kernel on this
+    workload, if it was taken from the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"{kind}_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not h or not t or h.group(1) != source_hash(kind):
+        return None
+    return float(t.group(1))
+
+
+# ---------------------------------------------------------------------------
+# the CUDA arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+
+    import exact_early_exit_b200 as nv
+
+    rank, world = dist_init("nccl")
+    _, _, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = W.WORKLOADS[args.workload]
+    cfg = wl.model
+    pseed, lseed, xseed = rank_seeds(rank)
+    lens = W.make_prompt_lengths(wl, seed=lseed)
+    prompts = W.make_prompts(wl, seed=pseed, lengths=lens)
+    B, steps = wl.batch, wl.steps
+    weights = W.make_weights(cfg, seed=0)
+    max_seq = int(lens.max()) + steps + 64
+    model = nv.Model(cfg, weights, max_batch=B, max_seq=max_seq, max_pending=256)
+    del weights
+    st = nv.State(model, B)
+    tok_host = torch.from_numpy(np.concatenate(prompts).astype(np.int32)).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    st.prefill(tok_host, lens)
+
+    tok_d = torch.zeros(B, dtype=torch.int32, device=dev)
+    ex_d = torch.zeros(B, dtype=torch.int32, device=dev)
+
+    def gen_pass(seed):
+        st.rewind()
+        for s in range(steps):
+            st.decode_step(seed + s, tok_d, ex_d)
+        st.flush()
+
+    for i in range(args.warmup):
+        gen_pass(xseed + 100000 * (i + 1))
+    torch.cuda.synchronize()
+    st.sync_status()
+    st.reset_counters()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            gen_pass(xseed)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms_total = e0.elapsed_time(e1)
+    st.sync_status()
+    ctr = st.counters()
+    ms_max = max_over_ranks(ms_total, dev)
+    ms_per_step = ms_max / args.steps
+    tokens_per_step = B * steps
+    value = tokens_per_step * world * args.steps / (ms_max / 1e3)
+    launches = int(ctr[nv.CTR["launches"]])
+
+    # algorithmic bytes of one pass (weights per layer run, K/V attended and
+    # written, exit heads), from the device counters of the timed passes
+    pass_bytes = float(ctr[nv.CTR["weight_bytes"]] + ctr[nv.CTR["kv_read_bytes"]] +
+                       ctr[nv.CTR["kv_write_bytes"]] + ctr[nv.CTR["head_bytes"]]) / args.steps
+    exits = ctr[nv.CTR["exit0"]:nv.CTR["exit0"] + cfg.n_exits].astype(float)
+    exit_mass = (exits / max(exits.sum(), 1)).round(4).tolist()
+
+    # e2e through the C ABI from pinned host memory
+    tok_h = torch.zeros(B, dtype=torch.int32).pin_memory()
+    ex_h = torch.zeros(B, dtype=torch.int32).pin_memory()
+    torch.cuda.synchronize()
+    barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for i in range(args.steps):
+        st.prefill(tok_host, lens)
+        for s in range(steps):
+            st.decode_step(xseed + s, tok_h, ex_h)
+        st.flush()
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3), dev)
+    e2e_value = tokens_per_step * world * args.steps / (e2e_ms / 1e3)
+
+    # per-kernel times: one profiled pass (each launch bracketed by events)
+    stats = (nv.KernelStat * len(nv.KERNEL_KINDS))()
+    st.rewind()
+    for s in range(steps):
+        st.decode_step_profiled(xseed + s, tok_d, ex_d, stats)
+    kern = {k: dict(ms=stats[i].ms, launches=int(stats[i].launches), bytes=int(stats[i].bytes),
+                    flops=int(stats[i].flops)) for i, k in enumerate(nv.KERNEL_KINDS)}
+    total_k_ms = sum(v["ms"] for v in kern.values())
+    dom = max(kern, key=lambda k: kern[k]["ms"])
+    dk = kern[dom]
+    per_launch_ms = dk["ms"] / max(dk["launches"], 1)
+    per_launch_bytes = dk["bytes"] / max(dk["launches"], 1)
+    achieved = per_launch_bytes / (per_launch_ms / 1e3) / 1e9
+    peak, peak_src = measured_peaks()
+    traffic = ncu_traffic(dom, args.workload)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "bytes_per_launch": round(per_launch_bytes), "ms_per_launch": round(per_launch_ms, 5),
+                "peak_source": f"{peak_src} copy bandwidth",
+                "kernel_share": {k: round(v["ms"] / total_k_ms, 4) for k, v in kern.items()},
+                "step_algorithmic_GBps": round(pass_bytes / (ms_per_step / 1e3) / 1e9, 1),
+                "step_frac": round(pass_bytes / (ms_per_step / 1e3) / 1e9 / peak, 4)}
+
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == W.BF16 else "f32",
+           "data": "synthetic",
+           "config": {"workload": wl.name, "model": cfg.name, "global_batch": B * world,
+                      "prompt_len": (f"U[{wl.prompt_len_lo},{wl.prompt_len}]" if wl.prompt_len_lo != wl.prompt_len
+                                     else wl.prompt_len),
+                      "decode_steps": steps, "parallelism": f"dp{world}" if world > 1 else "single",
+                      "step": "rewind + decode_steps decode steps + flush of deferred rows",
+                      "l2": "inputs larger than L2 (weights and KV streamed each step)"},
+           "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                   "h2d_bytes_per_step": int(tok_host.numel() * 4),
+                   "d2h_bytes_per_step": int(steps * B * 8)},
+           "gpu_launches": launches,
+           "roofline": roofline,
+           "realised_exit_mass": exit_mass}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, weights_seed=0, lens=lens, prompts=prompts, xseed=xseed)
+    out["clocks"] = clk.summary()
+    if rank == 0:
+        print(json.dumps(out))
+    st.close()
+    model.close()
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle: baseline sample and the reference arm
+# ---------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_setup(wl, lens, prompts, prefix):
+    from oracle import nvium_oracle as O
+    weights = W.make_weights(wl.model, seed=0)
+    om = O.OracleModel(wl.model, weights)
+    b = int(np.argmin(lens))
+    p = prompts[b][:prefix]
+    dec = O.OracleDecoder(om, [p], 64)
+    dec.ids = [b]
+    return dec, b
+
+
+def cpu_baseline(wl, weights_seed, lens, prompts, xseed, prefix=128, n_steps=2):
+    """The oracle on a bounded sample: one sequence (the batch's shortest
+    prompt, first `prefix` tokens prefilled untimed), `n_steps` decode steps
+    timed; tokens/s of that sample."""
+    dec, b = oracle_setup(wl, lens, prompts, prefix)
+    t0 = time.perf_counter()
+    for s in range(n_steps):
+        dec.step(xseed + s)
+    dt = time.perf_counter() - t0
+    return {"value": round(n_steps / dt, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"sequence {b}, first {min(prefix, len(prompts[b]))} prompt tokens prefilled untimed, "
+                      f"{n_steps} decode steps timed (1 token each), float64 numpy"}
+
+
+def run_reference(args):
+    rank, world, _ = rank_env()
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    pseed, lseed, xseed = rank_seeds(0)
+    lens = W.make_prompt_lengths(wl, seed=lseed)
+    prompts = W.make_prompts(wl, seed=pseed, lengths=lens)
+    dec, b = oracle_setup(wl, lens, prompts, 128)
+    for i in range(args.warmup):
+        dec.step(xseed + 1000 + i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        dec.step(xseed + i)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    cores = blas_threads()
+    sample = (f"sequence {b}, first 128 prompt tokens prefilled untimed; each step = 1 decode step of that "
+              f"sequence (1 token), float64 numpy oracle")
+    out = {"metric": METRIC, "impl": "reference", "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic",
+           "config": {"workload": wl.name, "model": wl.model.name, "global_batch": wl.batch,
+                      "decode_steps": wl.steps},
+           "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["X64", "X1", "S", "T"], default="X64")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

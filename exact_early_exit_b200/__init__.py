@@ -34,8 +34,14 @@ NV_ROUTER_FORCE_LAST = 1
 NV_MAX_EXITS = 8
 
 CTR = dict(steps=0, rows=1, layers_run=2, weight_bytes=3, kv_read_bytes=4, kv_write_bytes=5, head_bytes=6,
-           forced=7, exit0=8)
-NV_CTR_COUNT = 16
+           forced=7, launches=8, exit0=16)
+NV_CTR_COUNT = 24
+KERNEL_KINDS = ("plan_norm", "gemm", "epilogue", "attention", "norm", "junction", "head", "step")
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("ms", ctypes.c_double), ("launches", ctypes.c_int64), ("bytes", ctypes.c_int64),
+                ("flops", ctypes.c_int64)]
 
 
 class NviumError(RuntimeError):
@@ -87,6 +93,7 @@ _SIGS = [
     ("nv_reset_counters", _I, [_P]),
     ("nv_sync_status", _I, [_P]),
     ("nv_philox4x32_10", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
+    ("nv_decode_step_profiled", _I, [_P, ctypes.c_uint64, _P, _P, _P, _P]),
     ("nv_last_error", ctypes.c_char_p, []),
 ]
 
@@ -239,6 +246,15 @@ class State:
     def decode_step(self, seed: int, tokens_out, exits_out, logp_out=None, stream=None):
         _check(lib().nv_decode_step(self.handle, ctypes.c_uint64(seed), _ptr(tokens_out), _ptr(exits_out),
                                     _ptr(logp_out), _stream(stream)))
+
+    def decode_step_profiled(self, seed: int, tokens_out, exits_out, stats=None, stream=None):
+        """One decode step with per-kernel CUDA-event timing; accumulates into
+        and returns `stats` (a KernelStat array indexed like KERNEL_KINDS)."""
+        if stats is None:
+            stats = (KernelStat * len(KERNEL_KINDS))()
+        _check(lib().nv_decode_step_profiled(self.handle, ctypes.c_uint64(seed), _ptr(tokens_out), _ptr(exits_out),
+                                             ctypes.cast(stats, ctypes.c_void_p), _stream(stream)))
+        return stats
 
     def flush(self, stream=None):
         _check(lib().nv_flush_deferred(self.handle, _stream(stream)))

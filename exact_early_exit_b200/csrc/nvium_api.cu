@@ -109,6 +109,7 @@ struct nv_state {
   int* status = nullptr;
   // host mirrors
   std::vector<int> h_prompt_len, h_t;
+  long long launches_per_step = 0, launches_total = 0;
   bool prefilled = false;
   cudaGraphExec_t graph = nullptr;
   cudaStream_t cap_stream = nullptr;
@@ -147,7 +148,6 @@ KVView state_kv(nv_state* s) {
 struct LayerIO {
   RowSet rs;
   KVView kv;
-  int kv_layer;        // layer index used inside the KV view
   void* act;           // [rows][max(d,F)]
   void* q;
   void* o;
@@ -159,14 +159,65 @@ struct LayerIO {
   int epi_grid;
 };
 
+// Per-kernel event timing for nv_decode_step_profiled (null when capturing).
+struct Prof {
+  cudaStream_t st = nullptr;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  struct Rec {
+    int kind;
+    cudaEvent_t a, b;
+    long long bytes, flops;
+  };
+  std::vector<Rec> recs;
+  // host copies of the current layer's work list
+  int R = 0;
+  long long kv_read = 0;
+  cudaEvent_t ev() {
+    if (used == pool.size()) {
+      cudaEvent_t e;
+      cudaEventCreate(&e);
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+  cudaEvent_t open_a = nullptr;
+  void begin() {
+    open_a = ev();
+    cudaEventRecord(open_a, st);
+  }
+  void end(int kind, long long bytes, long long flops) {
+    cudaEvent_t b = ev();
+    cudaEventRecord(b, st);
+    recs.push_back(Rec{kind, open_a, b, bytes, flops});
+  }
+  ~Prof() {
+    for (cudaEvent_t e : pool) cudaEventDestroy(e);
+  }
+};
+
+// Runs `launch` bracketed by events when profiling; counts launches.
+template <typename F>
+void timed(Prof* prof, long long* launches, int nlaunch, int kind, long long bytes, long long flops, F&& launch) {
+  if (prof) prof->begin();
+  launch();
+  if (prof) prof->end(kind, bytes, flops);
+  if (launches) *launches += nlaunch;
+}
+
 // Everything of layer `layer` after the attention RMSNorm (act holds the
 // normed rows): QKV + RoPE + KV write, attention, O + residual, MLP norm,
 // gate/up + SwiGLU, down + residual.
-nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st) {
+nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st, Prof* prof = nullptr,
+                     long long* launches = nullptr) {
   const LayerDev& Lw = M->layers[layer];
   const bool bf = M->bf16;
+  const long long es = (long long)M->esz;
+  const long long R = prof ? prof->R : 0;
+  const long long d = M->d, HQ = M->HQ, F = M->F;
   int sgrid = 0;
   size_t sstride = 0;
+  nv_status gst = NV_OK;
   EpiArgs e{};
   e.rs = io.rs;
   e.d = M->d;
@@ -174,27 +225,38 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st)
   e.hd = M->hd;
   e.rope = M->rope;
   e.kv = io.kv;
-  e.layer = io.kv_layer;
+  e.layer = layer;  // scoring's single-layer scratch has layer_stride 0
   e.F = M->F;
   e.G = M->G;
-  // QKV
-  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.act, M->d, Lw.w_qkv, 3 * M->HQ, M->d, io.rs.nrows,
-                  io.rs.max_rows, io.Y, true, &sgrid, &sstride, st));
-  e.mode = EPI_QKV;
-  e.Y = io.Y;
-  e.split_grid = sgrid;
-  e.split_K = M->d;
-  e.split_stride = sstride;
-  e.N = 3 * M->HQ;
+  // algorithmic bytes of Y = X W^T: W once, X once, Y written once (fp32)
+  auto gemm_bytes = [&](long long N, long long K) { return N * K * es + R * K * es + R * N * 4; };
+  auto gemm = [&](const void* X, long long ldx, const void* W, long long N, long long K) {
+    timed(prof, launches, 1, NV_K_GEMM, gemm_bytes(N, K), 2 * R * N * K, [&] {
+      gst = gemm_run(M->gemm_plans, M->gemm_kind, bf, X, (int)ldx, W, (int)N, (int)K, io.rs.nrows, io.rs.max_rows,
+                     io.Y, true, &sgrid, &sstride, st);
+    });
+    return gst;
+  };
+  auto epi = [&](int mode, long long N, long long K, long long out_bytes) {
+    e.mode = mode;
+    e.Y = io.Y;
+    e.split_grid = sgrid;
+    e.split_K = (int)K;
+    e.split_stride = sstride;
+    e.N = (int)N;
+    timed(prof, launches, 1, NV_K_EPILOGUE, R * N * 4 + out_bytes, 0, [&] { launch_epilogue(bf, e, io.epi_grid, st); });
+  };
+  // QKV, RoPE, KV write
+  NV_TRY(gemm(io.act, d, Lw.w_qkv, 3 * HQ, d));
   e.q_out = io.q;
-  launch_epilogue(bf, e, io.epi_grid, st);
+  epi(EPI_QKV, 3 * HQ, d, R * 3 * HQ * es);
   // attention
   AttnArgs a{};
   a.rs = io.rs;
   a.q = io.q;
   a.o = io.o;
   a.kv = io.kv;
-  a.layer = io.kv_layer;
+  a.layer = layer;
   a.H = M->H;
   a.hd = M->hd;
   a.kv_splits = io.kv_splits;
@@ -203,35 +265,19 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st)
   a.part = io.attn_part;
   a.lens = io.lens;
   a.L = io.L;
-  launch_attention(bf, a, st);
+  timed(prof, launches, io.kv_splits > 1 ? 2 : 1, NV_K_ATTENTION, (prof ? prof->kv_read : 0) + 2 * R * HQ * es, 0,
+        [&] { launch_attention(bf, a, st); });
   // output projection + residual
-  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.o, M->HQ, Lw.w_o, M->d, M->HQ, io.rs.nrows, io.rs.max_rows,
-                  io.Y, true, &sgrid, &sstride, st));
-  e.mode = EPI_RESID;
-  e.split_grid = sgrid;
-  e.split_K = M->HQ;
-  e.split_stride = sstride;
-  e.N = M->d;
-  launch_epilogue(bf, e, io.epi_grid, st);
+  NV_TRY(gemm(io.o, HQ, Lw.w_o, d, HQ));
+  epi(EPI_RESID, d, HQ, R * d * 8);
   // MLP
-  launch_rmsnorm_rows(bf, io.rs, Lw.mlp_norm, io.act, M->d, M->cfg.rms_eps, st);
-  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.act, M->d, Lw.w_gu, 2 * M->F, M->d, io.rs.nrows,
-                  io.rs.max_rows, io.Y, true, &sgrid, &sstride, st));
-  e.mode = EPI_SWIGLU;
-  e.split_grid = sgrid;
-  e.split_K = M->d;
-  e.split_stride = sstride;
-  e.N = 2 * M->F;
+  timed(prof, launches, 1, NV_K_NORM, R * d * (4 + es), 0,
+        [&] { launch_rmsnorm_rows(bf, io.rs, Lw.mlp_norm, io.act, M->d, M->cfg.rms_eps, st); });
+  NV_TRY(gemm(io.act, d, Lw.w_gu, 2 * F, d));
   e.u_out = io.act;
-  launch_epilogue(bf, e, io.epi_grid, st);
-  NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, bf, io.act, M->F, Lw.w_d, M->d, M->F, io.rs.nrows, io.rs.max_rows,
-                  io.Y, true, &sgrid, &sstride, st));
-  e.mode = EPI_RESID;
-  e.split_grid = sgrid;
-  e.split_K = M->F;
-  e.split_stride = sstride;
-  e.N = M->d;
-  launch_epilogue(bf, e, io.epi_grid, st);
+  epi(EPI_SWIGLU, 2 * F, d, R * F * es);
+  NV_TRY(gemm(io.act, F, Lw.w_d, d, F));
+  epi(EPI_RESID, d, F, R * d * 8);
   return NV_OK;
 }
 
@@ -285,15 +331,42 @@ int plan_grid(nv_state* s) {
   return g;
 }
 
-// Launches of one decode step after step_begin (captured into a graph).
-nv_status record_step(nv_state* s, cudaStream_t st) {
+// Read the current layer's row count and attended KV bytes (profiling only).
+nv_status prof_read_plan(nv_state* s, Prof* prof, cudaStream_t st) {
+  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  int R = 0;
+  NV_CUDA_TRY(cudaMemcpy(&R, s->nrows, 4, cudaMemcpyDeviceToHost));
+  prof->R = R;
+  prof->kv_read = 0;
+  if (R > 0) {
+    std::vector<int> start(s->B + 1), pos(R);
+    NV_CUDA_TRY(cudaMemcpy(start.data(), s->seq_start, (s->B + 1) * 4, cudaMemcpyDeviceToHost));
+    NV_CUDA_TRY(cudaMemcpy(pos.data(), s->row_pos, (size_t)R * 4, cudaMemcpyDeviceToHost));
+    for (int b = 0; b < s->B; ++b)
+      if (start[b + 1] > start[b]) prof->kv_read += (long long)(pos[start[b + 1] - 1] + 1) * 2 * s->m->HQ * s->m->esz;
+  }
+  return NV_OK;
+}
+
+// Launches of one decode step after step_begin: captured into a graph, or
+// launched directly with per-kernel events when `prof` is set.
+nv_status record_step(nv_state* s, cudaStream_t st, Prof* prof = nullptr) {
   nv_model* M = s->m;
   const bool bf = M->bf16;
+  const long long es = (long long)M->esz;
+  long long* launches = &s->launches_per_step;
+  *launches = 1;  // step_begin, launched outside the graph
   LayerIO io = state_io(s);
   for (int layer = 0; layer < M->L; ++layer) {
     PlanArgs p = state_plan(s, layer, 0);
-    launch_plan_norm(bf, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
-    NV_TRY(layer_body(M, layer, io, st));
+    timed(prof, launches, 1, NV_K_PLAN_NORM, 0, 0, [&] {
+      launch_plan_norm(bf, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
+    });
+    if (prof) {
+      NV_TRY(prof_read_plan(s, prof, st));
+      prof->recs.back().bytes = (long long)prof->R * M->d * (4 + es);
+    }
+    NV_TRY(layer_body(M, layer, io, st, prof, launches));
     const int k = M->exit_at[layer];
     if (k >= 0) {
       JuncArgs j{};
@@ -315,7 +388,8 @@ nv_status record_step(nv_state* s, cudaStream_t st) {
       j.exit_act = s->exit_act;
       j.seed = s->seed_dev;
       j.counters = s->counters;
-      launch_junction(bf, j, st);
+      timed(prof, launches, 1, NV_K_JUNCTION, (long long)s->B * M->d * (4 + es), 0,
+            [&] { launch_junction(bf, j, st); });
       HeadArgs h{};
       h.B = s->B;
       h.d = M->d;
@@ -329,11 +403,24 @@ nv_status record_step(nv_state* s, cudaStream_t st) {
       h.part = s->head_part;
       h.nblk = s->head_nblk;
       h.counters = s->counters;
-      h.head_bytes = (long long)M->V * M->d * (long long)M->esz;
+      h.head_bytes = (long long)M->V * M->d * es;
       h.sampled = s->sampled;
       h.logp = s->logp;
-      launch_head_sample(bf, h, st);
-      launch_head_reduce(h, st);
+      long long hb = 0, hf = 0;
+      if (prof) {
+        // rows that stop at this exit: known once the junction has run
+        NV_CUDA_TRY(cudaStreamSynchronize(st));
+        std::vector<int> stop(s->B);
+        NV_CUDA_TRY(cudaMemcpy(stop.data(), j.stop, s->B * 4, cudaMemcpyDeviceToHost));
+        long long n = 0;
+        for (int v : stop) n += v;
+        if (n) hb = h.head_bytes + n * M->d * es;
+        hf = 2 * n * (long long)M->V * M->d;
+      }
+      timed(prof, launches, 2, NV_K_HEAD, hb, hf, [&] {
+        launch_head_sample(bf, h, st);
+        launch_head_reduce(h, st);
+      });
     }
   }
   StepArgs sa{};
@@ -345,7 +432,7 @@ nv_status record_step(nv_state* s, cudaStream_t st) {
   sa.sampled = s->sampled;
   sa.out_tok = s->out_tok;
   sa.out_exit = s->out_exit;
-  launch_step_end(sa, st);
+  timed(prof, launches, 1, NV_K_STEP, 0, 0, [&] { launch_step_end(sa, st); });
   return NV_OK;
 }
 
@@ -833,8 +920,11 @@ nv_status nv_rewind(nv_state* s, void* stream) {
   return NV_OK;
 }
 
-nv_status nv_decode_step(nv_state* s, uint64_t seed, int32_t* tokens_out, int32_t* exits_out, float* logp_out,
-                         void* stream) {
+}  // extern "C"
+
+namespace {
+nv_status decode_step_impl(nv_state* s, uint64_t seed, int32_t* tokens_out, int32_t* exits_out, float* logp_out,
+                           cudaStream_t st, Prof* prof) {
   if (!s || !tokens_out || !exits_out) {
     set_error("null argument");
     return NV_ERR_INVALID_ARG;
@@ -844,7 +934,6 @@ nv_status nv_decode_step(nv_state* s, uint64_t seed, int32_t* tokens_out, int32_
     return NV_ERR_STATE;
   }
   nv_model* M = s->m;
-  cudaStream_t st = (cudaStream_t)stream;
   // pages for the positions this step writes (every sequence advances by one)
   bool changed = false;
   for (int b = 0; b < s->B; ++b) {
@@ -873,33 +962,69 @@ nv_status nv_decode_step(nv_state* s, uint64_t seed, int32_t* tokens_out, int32_
   sa.seed_dev = s->seed_dev;
   sa.seed = seed;
   sa.counters = s->counters;
-  launch_step_begin(M->bf16, sa, st);
-  if (!s->graph) {
-    cudaGraph_t g = nullptr;
-    NV_CUDA_TRY(cudaStreamBeginCapture(s->cap_stream, cudaStreamCaptureModeThreadLocal));
-    nv_status rs = record_step(s, s->cap_stream);
-    cudaError_t e = cudaStreamEndCapture(s->cap_stream, &g);
-    if (rs != NV_OK) {
-      if (g) cudaGraphDestroy(g);
-      return rs;
+  timed(prof, nullptr, 1, NV_K_STEP, (long long)s->B * M->d * (4 + (long long)M->esz), 0,
+        [&] { launch_step_begin(M->bf16, sa, st); });
+  if (prof) {
+    NV_TRY(record_step(s, st, prof));
+  } else {
+    if (!s->graph) {
+      cudaGraph_t g = nullptr;
+      NV_CUDA_TRY(cudaStreamBeginCapture(s->cap_stream, cudaStreamCaptureModeThreadLocal));
+      nv_status rs = record_step(s, s->cap_stream);
+      cudaError_t e = cudaStreamEndCapture(s->cap_stream, &g);
+      if (rs != NV_OK) {
+        if (g) cudaGraphDestroy(g);
+        return rs;
+      }
+      if (e != cudaSuccess) {
+        set_error(std::string("capturing the decode step: ") + cudaGetErrorString(e));
+        return NV_ERR_CUDA;
+      }
+      e = cudaGraphInstantiate(&s->graph, g, 0);
+      cudaGraphDestroy(g);
+      if (e != cudaSuccess) {
+        set_error(std::string("instantiating the decode step: ") + cudaGetErrorString(e));
+        s->graph = nullptr;
+        return NV_ERR_CUDA;
+      }
     }
-    if (e != cudaSuccess) {
-      set_error(std::string("capturing the decode step: ") + cudaGetErrorString(e));
-      return NV_ERR_CUDA;
-    }
-    e = cudaGraphInstantiate(&s->graph, g, 0);
-    cudaGraphDestroy(g);
-    if (e != cudaSuccess) {
-      set_error(std::string("instantiating the decode step: ") + cudaGetErrorString(e));
-      s->graph = nullptr;
-      return NV_ERR_CUDA;
-    }
+    NV_CUDA_TRY(cudaGraphLaunch(s->graph, st));
   }
-  NV_CUDA_TRY(cudaGraphLaunch(s->graph, st));
+  s->launches_total += s->launches_per_step;
   NV_CUDA_TRY(cudaMemcpyAsync(tokens_out, s->out_tok, s->B * 4, cudaMemcpyDefault, st));
   NV_CUDA_TRY(cudaMemcpyAsync(exits_out, s->out_exit, s->B * 4, cudaMemcpyDefault, st));
   if (logp_out) NV_CUDA_TRY(cudaMemcpyAsync(logp_out, s->logp, s->B * 4, cudaMemcpyDefault, st));
   for (int b = 0; b < s->B; ++b) s->h_t[b] += 1;
+  return NV_OK;
+}
+}  // namespace
+
+extern "C" {
+
+nv_status nv_decode_step(nv_state* s, uint64_t seed, int32_t* tokens_out, int32_t* exits_out, float* logp_out,
+                         void* stream) {
+  return decode_step_impl(s, seed, tokens_out, exits_out, logp_out, (cudaStream_t)stream, nullptr);
+}
+
+nv_status nv_decode_step_profiled(nv_state* s, uint64_t seed, int32_t* tokens_out, int32_t* exits_out,
+                                  nv_kernel_stat* stats, void* stream) {
+  if (!stats) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  Prof prof;
+  prof.st = (cudaStream_t)stream;
+  NV_TRY(decode_step_impl(s, seed, tokens_out, exits_out, nullptr, prof.st, &prof));
+  NV_CUDA_TRY(cudaStreamSynchronize(prof.st));
+  for (const Prof::Rec& r : prof.recs) {
+    float ms = 0.f;
+    NV_CUDA_TRY(cudaEventElapsedTime(&ms, r.a, r.b));
+    nv_kernel_stat& k = stats[r.kind];
+    k.ms += ms;
+    k.launches += 1;
+    k.bytes += r.bytes;
+    k.flops += r.flops;
+  }
   return NV_OK;
 }
 
@@ -912,11 +1037,14 @@ nv_status nv_flush_deferred(nv_state* s, void* stream) {
   nv_model* M = s->m;
   cudaStream_t st = (cudaStream_t)stream;
   LayerIO io = state_io(s);
+  long long launches = 0;
   for (int layer = M->cfg.exit_layers[0]; layer < M->L; ++layer) {
     PlanArgs p = state_plan(s, layer, 1);
     launch_plan_norm(M->bf16, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
-    NV_TRY(layer_body(M, layer, io, st));
+    ++launches;
+    NV_TRY(layer_body(M, layer, io, st, nullptr, &launches));
   }
+  s->launches_total += launches;
   NV_CUDA_TRY(cudaGetLastError());
   return NV_OK;
 }
@@ -967,6 +1095,7 @@ nv_status nv_read_counters(nv_state* s, int64_t* out, int n) {
   if (n > NV_CTR_COUNT) n = NV_CTR_COUNT;
   NV_CUDA_TRY(cudaDeviceSynchronize());
   NV_CUDA_TRY(cudaMemcpy(out, s->counters, (size_t)n * 8, cudaMemcpyDeviceToHost));
+  if (n > NV_CTR_LAUNCHES) out[NV_CTR_LAUNCHES] = s->launches_total;  // host-side count
   return NV_OK;
 }
 
@@ -974,6 +1103,7 @@ nv_status nv_reset_counters(nv_state* s) {
   if (!s) return NV_ERR_INVALID_ARG;
   NV_CUDA_TRY(cudaDeviceSynchronize());
   NV_CUDA_TRY(cudaMemset(s->counters, 0, NV_CTR_COUNT * 8));
+  s->launches_total = 0;
   return NV_OK;
 }
 
@@ -1096,7 +1226,6 @@ nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, flo
   io.kv.page_size = ps;
   io.kv.H = M->H;
   io.kv.hd = M->hd;
-  io.kv_layer = 0;
   io.act = M->sc_act.p;
   io.q = M->sc_q.p;
   io.o = M->sc_o.p;

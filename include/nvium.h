@@ -183,8 +183,9 @@ enum {
   NV_CTR_KV_WRITE_BYTES = 5, /* KV bytes written                           */
   NV_CTR_HEAD_BYTES = 6,     /* exit-head weight bytes read                */
   NV_CTR_FORCED = 7,         /* sequence-steps with an early completion    */
-  NV_CTR_EXIT0 = 8,          /* 8..8+N_V-1: exits taken, per exit          */
-  NV_CTR_COUNT = 16
+  NV_CTR_LAUNCHES = 8,       /* kernels launched by decode steps and flush */
+  NV_CTR_EXIT0 = 16,         /* 16..16+N_V-1: exits taken, per exit        */
+  NV_CTR_COUNT = 24
 };
 nv_status nv_read_counters(nv_state *s, int64_t *out, int n);
 nv_status nv_reset_counters(nv_state *s);
@@ -196,6 +197,34 @@ nv_status nv_reset_counters(nv_state *s);
  * Synchronous. */
 nv_status nv_philox4x32_10(uint64_t seed, const uint32_t *ctr, int n,
                            uint32_t *out, void *stream);
+
+/* Per-kernel timing of one decode step (a measurement hook, not a second
+ * code path): the step's kernels are launched directly on `stream`, each
+ * bracketed by CUDA events, instead of as one graph replay; the step's
+ * results are identical.  stats[kind] accumulates, for NV_K_* kinds, the
+ * summed event time, the launches, and the algorithmic bytes (the bytes the
+ * kernel must move: weights once, K/V of the attended positions once,
+ * activations in and out) and flops of those launches.  Synchronous. */
+typedef struct nv_kernel_stat {
+  double ms;
+  int64_t launches;
+  int64_t bytes;
+  int64_t flops;
+} nv_kernel_stat;
+enum {
+  NV_K_PLAN_NORM = 0, /* work-list planner + attention RMSNorm    */
+  NV_K_GEMM = 1,      /* packed-row GEMMs (tcgen05 or SIMT)       */
+  NV_K_EPILOGUE = 2,  /* RoPE/KV write, residual, SwiGLU          */
+  NV_K_ATTENTION = 3, /* paged attention (+ split combine)        */
+  NV_K_NORM = 4,      /* MLP RMSNorm                              */
+  NV_K_JUNCTION = 5,  /* exit norm, router, stop draw             */
+  NV_K_HEAD = 6,      /* exit-head sampler (+ reduce)             */
+  NV_K_STEP = 7,      /* step begin / end                         */
+  NV_K_COUNT = 8
+};
+nv_status nv_decode_step_profiled(nv_state *s, uint64_t philox_seed,
+                                  int32_t *tokens_out, int32_t *exits_out,
+                                  nv_kernel_stat *stats, void *stream);
 
 /* Synchronise the state's work and return any device-detected error. */
 nv_status nv_sync_status(nv_state *s);

@@ -92,3 +92,24 @@ def run_decode_parity(nv, cfg, weights, prompts, steps, seed=1234, max_pending=2
                 kv_close(K, dec.caches[b].K[m][:n], cfg)
                 kv_close(V, dec.caches[b].V[m][:n], cfg)
     return chk, state, dec, model
+
+
+def chisq_pvalue(counts, expected, min_expected=5.0):
+    """Chi-square p-value with the smallest-expectation cells merged until
+    every cell expects at least `min_expected` draws."""
+    from scipy import stats
+    c = np.asarray(counts, dtype=np.float64).ravel()
+    e = np.asarray(expected, dtype=np.float64).ravel()
+    keep = e > 0
+    assert c[~keep].sum() == 0, "draws in a cell of probability zero"
+    c, e = c[keep], e[keep]
+    order = np.argsort(e)
+    c, e = c[order], e[order]
+    cut = int(np.sum(e < min_expected))        # cells too small on their own
+    if cut > 0:
+        while cut < len(e) and e[:cut].sum() < min_expected:
+            cut += 1
+        c = np.concatenate([[c[:cut].sum()], c[cut:]])
+        e = np.concatenate([[e[:cut].sum()], e[cut:]])
+    assert np.all(e >= min_expected)
+    return stats.chisquare(c, e * c.sum() / e.sum()).pvalue

@@ -299,18 +299,9 @@ def test_decode_step_law_matches_full_depth_states():
 # exact sampling
 # --------------------------------------------------------------------------
 
-def _chisq_merged(counts, expected, min_expected=5.0):
-    from scipy import stats
-    counts = np.asarray(counts, dtype=np.float64).ravel()
-    expected = np.asarray(expected, dtype=np.float64).ravel()
-    order = np.argsort(expected)
-    c, e = counts[order], expected[order]
-    small = np.cumsum(e) < min_expected * 4
-    big = ~small
-    cc = np.concatenate([c[big], [c[small].sum()]]) if small.any() else c
-    ee = np.concatenate([e[big], [e[small].sum()]]) if small.any() else e
-    assert np.all(ee >= min_expected)
-    return stats.chisquare(cc, ee * cc.sum() / ee.sum()).pvalue
+def _chisq_merged(counts, expected):
+    from tests.nvium_testlib import chisq_pvalue
+    return chisq_pvalue(counts, expected)
 
 
 def test_sequential_stop_frequencies_match_pk():
