@@ -32,6 +32,7 @@ NV_BF16 = 1
 NV_ROUTER_NORMAL = 0
 NV_ROUTER_FORCE_LAST = 1
 NV_MAX_EXITS = 8
+NV_PHILOX_NOALLOC_MAX = 32768
 
 CTR = dict(steps=0, rows=1, layers_run=2, weight_bytes=3, kv_read_bytes=4, kv_write_bytes=5, head_bytes=6,
            forced=7, launches=8, exit0=16)
@@ -94,6 +95,7 @@ _SIGS = [
     ("nv_sync_status", _I, [_P]),
     ("nv_philox4x32_10", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
     ("nv_decode_step_profiled", _I, [_P, ctypes.c_uint64, _P, _P, _P, _P]),
+    ("nv_philox4x32_10_noalloc", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
     ("nv_last_error", ctypes.c_char_p, []),
 ]
 
@@ -297,4 +299,13 @@ def philox4x32_10(seed: int, counters: np.ndarray) -> np.ndarray:
     ctr = np.ascontiguousarray(counters, dtype=np.uint32).reshape(-1, 4)
     out = np.zeros_like(ctr)
     _check(lib().nv_philox4x32_10(ctypes.c_uint64(seed), _ptr(ctr), ctr.shape[0], _ptr(out), None))
+    return out
+
+
+def philox4x32_10_noalloc(seed: int, counters: np.ndarray) -> np.ndarray:
+    """nv_philox4x32_10 without any device allocation (staging through the
+    library's fixed array; at most NV_PHILOX_NOALLOC_MAX counters)."""
+    ctr = np.ascontiguousarray(counters, dtype=np.uint32).reshape(-1, 4)
+    out = np.zeros_like(ctr)
+    _check(lib().nv_philox4x32_10_noalloc(ctypes.c_uint64(seed), _ptr(ctr), ctr.shape[0], _ptr(out), None))
     return out

@@ -198,6 +198,31 @@ nv_status nv_reset_counters(nv_state *s);
 nv_status nv_philox4x32_10(uint64_t seed, const uint32_t *ctr, int n,
                            uint32_t *out, void *stream);
 
+/* The same generator as nv_philox4x32_10, for callers that cannot allocate
+ * device memory.  The paper has no counterpart: this is a service of the
+ * library, not a step of the method.
+ *
+ * Some callers cannot call cudaMalloc: a host framework whose caching
+ * allocator already holds the device's memory (a fresh allocation fails or
+ * fragments it), or a latency-critical loop that cannot afford the
+ * device-wide synchronisation cudaMalloc / cudaFree may imply.
+ * nv_philox4x32_10 allocates a staging buffer on every call; this entry
+ * point allocates nothing.  It stages counters and results through a fixed
+ * array of 2 * NV_PHILOX_NOALLOC_MAX * 16 bytes (1 MiB) in device global
+ * memory, which every GPU that loads the library holds until the process
+ * exits.
+ *
+ * ctr, out: n x 4 uint32 (host or device); 1 <= n <= NV_PHILOX_NOALLOC_MAX,
+ * larger n returns NV_ERR_INVALID_ARG with a message.  The first call on a
+ * device looks up the array's device address once, with that device
+ * current; make that first call before any stream capture.  All calls share
+ * the array and it keeps the last call's contents, so calls that overlap on
+ * the GPU (other streams, other host threads) race; serialise them.
+ * Synchronous. */
+#define NV_PHILOX_NOALLOC_MAX 32768
+nv_status nv_philox4x32_10_noalloc(uint64_t seed, const uint32_t *ctr, int n,
+                                   uint32_t *out, void *stream);
+
 /* Per-kernel timing of one decode step (a measurement hook, not a second
  * code path): the step's kernels are launched directly on `stream`, each
  * bracketed by CUDA events, instead of as one graph replay; the step's
