@@ -531,6 +531,190 @@ __global__ void k_attn_combine(AttnArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode attention: CTA (b, head, chunk) handles keys [chunk*128, chunk*128 +
+// 128) of sequence b at this layer for every row of b whose position reaches
+// the chunk.  One thread issues TMA bulk copies of the chunk's K and V pages
+// (each page of one head is contiguous), completing on an mbarrier, so the
+// whole 2 x 16 KB chunk is in flight at once.  Scores: one lane per key,
+// 16-byte reads of the key row in a per-lane rotated order (conflict-free);
+// P.V: one lane per HD/32 dims.  Unnormalised partials (m, l, acc) per
+// (row, head, chunk) are merged by k_attn_dec_combine in chunk order.
+// Rows of 128 bytes (HD * sizeof(T) == 128) only.
+// ---------------------------------------------------------------------------
+constexpr int DEC_CK = 128;  // keys per chunk (two 64-position pages)
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+template <typename T, int HD>
+__global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
+  static_assert(HD * sizeof(T) == 128, "128-byte rows");
+  constexpr int NW = 4, KPL = DEC_CK / 32, DPL = HD / 32, EPC = 16 / sizeof(T);
+  __shared__ __align__(128) T Ks[DEC_CK * HD];
+  __shared__ __align__(128) T Vs[DEC_CK * HD];
+  __shared__ float Qs[NW][HD];
+  __shared__ __align__(8) uint64_t bar;
+  const int b = blockIdx.x, head = blockIdx.y, chunk = blockIdx.z;
+  if (*a.rs.nrows == 0) return;
+  const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
+  if (s0 >= s1) return;
+  const int pos_last = a.rs.row_pos[s1 - 1];
+  const int k0 = chunk * DEC_CK;
+  if (k0 > pos_last) return;
+  const int nk = min(DEC_CK, pos_last + 1 - k0);
+  const int npages = (nk + a.kv.page_size - 1) / a.kv.page_size;  // page_size == 64 here
+  const uint32_t bytes_per_page = (uint32_t)(a.kv.page_size * HD * sizeof(T));
+  const T* kvb = (const T*)a.kv.base;
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&bar)),
+                 "r"(2u * npages * bytes_per_page)
+                 : "memory");
+    for (int pg = 0; pg < npages; ++pg) {
+      const int pos = k0 + pg * a.kv.page_size;
+      const T* kg = kvb + a.kv.offset(a.layer, b, pos, head, 0);
+      const T* vg = kvb + a.kv.offset(a.layer, b, pos, head, 1);
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_addr(Ks + pg * a.kv.page_size * HD)),
+          "l"(kg), "r"(bytes_per_page), "r"(smem_addr(&bar))
+          : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_addr(Vs + pg * a.kv.page_size * HD)),
+          "l"(vg), "r"(bytes_per_page), "r"(smem_addr(&bar))
+          : "memory");
+    }
+  }
+  __syncthreads();
+  // bounded wait (2 s) for the copies
+  {
+    uint32_t ok = 0;
+    unsigned long long t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(smem_addr(&bar))
+          : "memory");
+      if (ok) break;
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (i == 0) t0 = t;
+      else if (t - t0 > 2000000000ull) {
+        if (threadIdx.x == 0) dev_fail(a.status, DEV_ERR_TIMEOUT);
+        return;
+      }
+    }
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = a.H;
+  const T* qg = (const T*)a.q;
+  // rows of b whose position reaches this chunk: positions are contiguous
+  const int pos0 = a.rs.row_pos[s0];
+  const int first = max(s0, s0 + (k0 - pos0));
+  for (int r = first + w; r < s1; r += NW) {
+    const int p = pos0 + (r - s0);
+    for (int dd = lane; dd < HD; dd += 32) Qs[w][dd] = ld(qg + (size_t)r * H * HD + head * HD + dd);
+    __syncwarp();
+    float sc[KPL];
+    float mx = -CUDART_INF_F;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const int kk = lane + 32 * j;
+      float acc = 0.f;
+      const uint4* krow = (const uint4*)(Ks + kk * HD);
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const int c = (c8 + lane) & 7;
+        const uint4 kv4 = krow[c];
+        const T* kp = (const T*)&kv4;
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc = fmaf(Qs[w][c * EPC + e], ld(kp + e), acc);
+      }
+      sc[j] = (kk < nk && k0 + kk <= p) ? acc * a.scale : -CUDART_INF_F;
+      mx = fmaxf(mx, sc[j]);
+    }
+    mx = warp_max(mx);
+    float l = 0.f;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      sc[j] = expf(sc[j] - mx);
+      l += sc[j];
+    }
+    l = warp_sum(l);
+    float o[DPL];
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) o[d] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const int kbase = 32 * j;
+      if (kbase >= nk) break;
+#pragma unroll 8
+      for (int src = 0; src < 32; ++src) {
+        const float pw = __shfl_sync(0xffffffffu, sc[j], src);
+        if (kbase + src >= nk) break;  // rows past the chunk's keys hold stale data
+        const T* vrow = Vs + (kbase + src) * HD + lane * DPL;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) o[d] = fmaf(pw, ld(vrow + d), o[d]);
+      }
+    }
+    float* pp = a.part + (((size_t)r * H + head) * a.kv_splits + chunk) * (HD + 2);
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) pp[lane * DPL + d] = o[d];
+    if (lane == 0) {
+      pp[HD] = mx;
+      pp[HD + 1] = l;
+    }
+    __syncwarp();
+  }
+  if (a.lens && head == 0 && chunk == 0 && threadIdx.x == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
+}
+
+// Merge the chunk partials of each (row, head): chunks 0 .. pos/128.
+template <typename T, int HD>
+__global__ void k_attn_dec_combine(AttnArgs a) {
+  constexpr int DPL = HD / 32;
+  const int R = *a.rs.nrows;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int item = blockIdx.x * wpb + (threadIdx.x >> 5); item < R * a.H; item += gridDim.x * wpb) {
+    const int r = item / a.H, head = item % a.H;
+    const int nch = a.rs.row_pos[r] / DEC_CK + 1;
+    const float* pp = a.part + ((size_t)r * a.H + head) * a.kv_splits * (HD + 2);
+    float M = -CUDART_INF_F;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, pp[c * (HD + 2) + HD]);
+    float L = 0.f, acc[DPL];
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const float e = expf(pp[c * (HD + 2) + HD] - M);
+      L += pp[c * (HD + 2) + HD + 1] * e;
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) acc[d] += pp[c * (HD + 2) + lane * DPL + d] * e;
+    }
+    T* o = (T*)a.o + (size_t)r * a.H * HD + head * HD;
+    const float inv = 1.0f / L;
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) o[lane * DPL + d] = cvt<T>(acc[d] * inv);
+  }
+}
+
+template <typename T, int HD>
+static void attention_dec_t(const AttnArgs& a, cudaStream_t st) {
+  dim3 grid(a.rs.B, a.H, a.kv_splits);
+  k_attn_dec<T, HD><<<grid, 128, 0, st>>>(a);
+  int g = (a.rs.max_rows * a.H + 7) / 8;
+  if (g > 4096) g = 4096;
+  k_attn_dec_combine<T, HD><<<g, 256, 0, st>>>(a);
+}
+void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st) {
+  if (bf16) attention_dec_t<__nv_bfloat16, 64>(a, st);
+  else attention_dec_t<float, 32>(a, st);
+}
+
 template <typename T, int HD>
 static void attention_t(const AttnArgs& a, cudaStream_t st) {
   dim3 grid(a.rs.B, a.H, a.row_groups * a.kv_splits);

@@ -76,8 +76,14 @@ struct AttnArgs {
   float* part;     // [max_rows][H][kv_splits][hd+2] when kv_splits > 1
   int* lens;       // when set: lens[b*L+layer] = last row position + 1
   int L;
+  int* status;     // device status word (bounded-wait expiry)
 };
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
+// Decode / flush attention: 128-key chunks (grid z = kv_splits = chunks of
+// max_seq), TMA bulk loads of K/V pages, partials merged per row.  Needs
+// head_dim * element size == 128 bytes and page_size == 64.
+constexpr int ATTN_DEC_CK = 128;
+void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st);
 
 struct StepArgs {
   int B, L, cap, d, n_exits;

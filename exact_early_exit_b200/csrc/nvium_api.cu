@@ -104,6 +104,7 @@ struct nv_state {
   float *Y = nullptr, *attn_part = nullptr, *head_part = nullptr;
   size_t Y_elems = 0;
   int head_nblk = 0, kv_splits = 1, row_groups = 1;
+  bool dec_attn = false;
   unsigned long long* seed_dev = nullptr;
   long long* counters = nullptr;
   int* status = nullptr;
@@ -157,6 +158,8 @@ struct LayerIO {
   int* lens;           // nullable: per-(seq, layer) lengths to advance
   int L;
   int epi_grid;
+  bool dec_attn;       // chunked decode attention (else row-group attention)
+  int* status;
 };
 
 // Per-kernel event timing for nv_decode_step_profiled (null when capturing).
@@ -265,8 +268,12 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   a.part = io.attn_part;
   a.lens = io.lens;
   a.L = io.L;
-  timed(prof, launches, io.kv_splits > 1 ? 2 : 1, NV_K_ATTENTION, (prof ? prof->kv_read : 0) + 2 * R * HQ * es, 0,
-        [&] { launch_attention(bf, a, st); });
+  a.status = io.status;
+  timed(prof, launches, (io.kv_splits > 1 || io.dec_attn) ? 2 : 1, NV_K_ATTENTION,
+        (prof ? prof->kv_read : 0) + 2 * R * HQ * es, 0, [&] {
+          if (io.dec_attn) launch_attention_decode(bf, a, st);
+          else launch_attention(bf, a, st);
+        });
   // output projection + residual
   NV_TRY(gemm(io.o, HQ, Lw.w_o, d, HQ));
   epi(EPI_RESID, d, HQ, R * d * 8);
@@ -295,6 +302,8 @@ LayerIO state_io(nv_state* s) {
   io.lens = s->lens;
   io.L = s->m->L;
   io.epi_grid = 1184;
+  io.dec_attn = s->dec_attn;
+  io.status = s->status;
   return io;
 }
 
@@ -707,9 +716,15 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   const size_t esz = M->esz, d = M->d, HQ = M->HQ, F = M->F;
   const size_t page_elems = (size_t)2 * M->H * s->ps * M->hd;
   s->kv_layer_stride = (size_t)s->n_pages * page_elems;
-  // attention parallelism: split the key range when few (sequence, head) pairs
-  int ks = (2 * 148 + B * M->H - 1) / (B * M->H);
-  s->kv_splits = ks < 1 ? 1 : (ks > 16 ? 16 : ks);
+  // attention: 128-key chunks (one CTA each) when rows are 128 bytes and pages
+  // hold 64 or 128 positions; otherwise row groups with a few key splits
+  s->dec_attn = (size_t)M->hd * M->esz == 128 && (s->ps == 64 || s->ps == 128);
+  if (s->dec_attn) {
+    s->kv_splits = (s->max_seq + ATTN_DEC_CK - 1) / ATTN_DEC_CK;
+  } else {
+    int ks = (2 * 148 + B * M->H - 1) / (B * M->H);
+    s->kv_splits = ks < 1 ? 1 : (ks > 16 ? 16 : ks);
+  }
   s->row_groups = (s->cap + 1 + ATTN_RPC - 1) / ATTN_RPC;
   s->head_nblk = 296;
   const size_t wide = d > F ? d : F;

@@ -127,3 +127,12 @@ def test_sampler_chi_square():
     assert chisq_pvalue(counts, p[:, None] * pi * n) > 0.01
     assert chisq_pvalue(counts.sum(1), p * n) > 0.01
     assert chisq_pvalue(counts.sum(0), (p[:, None] * pi).sum(0) * n) > 0.01
+
+
+def test_decode_parity_contexts_spanning_many_chunks(weights):
+    """Contexts of 130..400 positions: several 128-key attention chunks,
+    a ragged last chunk and a chunk that ends exactly on a page."""
+    rng = np.random.default_rng(9)
+    prompts = [rng.integers(0, CFG.vocab, size=n).astype(np.int32) for n in (129, 256, 383)]
+    chk, *_ = run_decode_parity(nv, CFG, weights, prompts, 12, max_seq=420)
+    assert chk.steps == 12
