@@ -178,6 +178,21 @@ def ncu_traffic(kind: str, workload: str):
     return float(t.group(1))
 
 
+def workload_for(args):
+    """The named workload, or a shortened copy for profiling runs."""
+    import dataclasses
+    wl = W.WORKLOADS[args.workload]
+    if args.layers:
+        L = args.layers
+        ne = wl.model.n_exits
+        exits = tuple(max(1, round(L * (k + 1) / ne)) for k in range(ne))
+        model = dataclasses.replace(wl.model, name=f"{wl.model.name}-{L}layers", n_layers=L, exit_layers=exits)
+        wl = dataclasses.replace(wl, model=model, name=f"{wl.name}-{L}layers")
+    if args.decode_steps:
+        wl = dataclasses.replace(wl, steps=args.decode_steps, name=f"{wl.name}-{args.decode_steps}steps")
+    return wl
+
+
 # ---------------------------------------------------------------------------
 # the CUDA arm
 # ---------------------------------------------------------------------------
@@ -190,7 +205,7 @@ def run_ours(args):
     _, _, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl = W.WORKLOADS[args.workload]
+    wl = workload_for(args)
     cfg = wl.model
     pseed, lseed, xseed = rank_seeds(rank)
     lens = W.make_prompt_lengths(wl, seed=lseed)
@@ -391,6 +406,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["X64", "X1", "S", "T"], default="X64")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: the workload's model with this many layers (exits spread evenly)")
+    ap.add_argument("--decode-steps", type=int, default=0, help="profiling only: decode steps per pass")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

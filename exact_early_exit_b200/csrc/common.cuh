@@ -7,6 +7,7 @@
 
 #include <cstddef>
 #include <string>
+#include <utility>
 
 #include "../../include/nvium.h"
 
@@ -141,6 +142,33 @@ struct KVView {
            (((size_t)page * 2 + kv) * H + head) * (size_t)page_size * hd + (size_t)(pos % page_size) * hd;
   }
 };
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch: every kernel of the path is launched with
+// programmatic stream serialisation, so its launch and prologue overlap the
+// previous kernel; each kernel waits (griddepcontrol.wait) before it reads
+// anything a predecessor wrote, on every path, and then lets its own
+// dependents launch.  NVIUM_PDL=0 launches them plainly.
+// ---------------------------------------------------------------------------
+bool pdl_enabled();
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Which part of a fused weight a GEMM output column belongs to.
 enum EpiMode : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_STORE = 3 };

@@ -46,13 +46,39 @@ size_t gemm_workspace_elems(int kind, size_t rows, size_t N) {
 }
 
 nv_status gemm_run(GemmPlanCache* plans, int kind, bool bf16, const void* X, int ldx, const void* W, int N, int K,
-                   const int* nrows, int max_rows, float* Y, bool allow_split, int* split_grid, size_t* split_stride,
-                   cudaStream_t st) {
-  if (kind == GEMM_TC && bf16)
-    return tc_gemm_run(plans->tc, X, ldx, W, N, K, nrows, max_rows, Y, allow_split, split_grid, split_stride, st);
+                   const int* nrows, int max_rows, float* Y, bool allow_split, const EpiArgs* epi, int* tile_counters,
+                   int epi_grid, const void* prefetch, size_t prefetch_bytes, cudaStream_t st,
+                   int* split_grid_out) {
+  if (kind == GEMM_TC && bf16) {
+    if (!allow_split)  // one slice: the epilogue runs inside the GEMM kernel
+      return tc_gemm_run(plans->tc, X, ldx, W, N, K, nrows, max_rows, Y, false, epi, tile_counters, prefetch,
+                         prefetch_bytes, st);
+    // split-K slices: the GEMM writes fp32 partials, the epilogue kernel sums them
+    int grid = 0;
+    NV_TRY(tc_gemm_run(plans->tc, X, ldx, W, N, K, nrows, max_rows, Y, true, nullptr, nullptr, prefetch,
+                       prefetch_bytes, st, &grid));
+    if (split_grid_out) *split_grid_out = grid;
+    if (epi && epi->mode != EPI_STORE) {
+      EpiArgs e = *epi;
+      e.Y = Y;
+      e.split_grid = grid;
+      e.split_K = K;
+      e.split_stride = tc_split_stride(N);
+      e.N = N;
+      launch_epilogue(true, e, epi_grid, st);
+    }
+    return NV_OK;
+  }
   launch_gemm_simt(bf16, X, ldx, W, N, K, nrows, max_rows, Y, st);
-  *split_grid = 0;
-  *split_stride = 0;
+  if (split_grid_out) *split_grid_out = 0;
+  if (epi && epi->mode != EPI_STORE) {
+    EpiArgs e = *epi;
+    e.Y = Y;
+    e.split_grid = 0;
+    e.split_stride = 0;
+    e.N = N;
+    launch_epilogue(bf16, e, epi_grid, st);
+  }
   return NV_OK;
 }
 

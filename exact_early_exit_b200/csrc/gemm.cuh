@@ -42,13 +42,18 @@ __host__ __device__ __forceinline__ int tc_split_count(int R, int N, int K, int 
   return s < 1 ? 1 : s;
 }
 
-// Launch Y = X W^T.  X: [rows][ldx] (rows <= max_rows, count in *nrows on the
-// device), W: [N][K] row-major.  The output is split_count partial slices of
-// `*split_stride` elements; *split_grid is the grid to pass to
-// tc_split_count with TC_MAX_SPLIT (0: always one slice, e.g. when
-// allow_split is false).
+struct EpiArgs;
+// Launch Y = X W^T followed by the layer epilogue `epi` (mode EPI_QKV,
+// EPI_RESID or EPI_SWIGLU; null or EPI_STORE: write fp32 Y).  X: [rows][ldx]
+// (rows <= max_rows, count in *nrows on the device), W: [N][K] row-major.
+// The tcgen05 engine applies the epilogue inside the GEMM kernel (split-K
+// slices in Y, summed by the last CTA of each feature tile, tile_counters
+// zero between launches); the SIMT engine runs the epilogue kernel after it.
+// `prefetch` / `prefetch_bytes`: the next GEMM's weights, pulled into L2 by
+// the tcgen05 engine while it runs (a hint; may be null).
 nv_status gemm_run(GemmPlanCache* plans, int kind, bool bf16, const void* X, int ldx, const void* W, int N, int K,
-                   const int* nrows, int max_rows, float* Y, bool allow_split, int* split_grid, size_t* split_stride,
-                   cudaStream_t st);
+                   const int* nrows, int max_rows, float* Y, bool allow_split, const EpiArgs* epi, int* tile_counters,
+                   int epi_grid, const void* prefetch, size_t prefetch_bytes, cudaStream_t st,
+                   int* split_grid_out = nullptr);
 
 }  // namespace nv

@@ -18,17 +18,21 @@
 //                     fp32 stores (each warp owns 32 features = TMEM lanes).
 // When all rows fit one tile and the feature tiles cannot fill the GPU, the K
 // range is split (tc_split_count); the partial slices are summed in a fixed
-// order by the epilogue kernels.  Every mbarrier wait is bounded: on expiry
+// order by the epilogue kernel that follows.  Without a split, the layer
+// epilogue (RoPE + KV write, residual, SwiGLU) runs in the epilogue warps
+// from a staged tile.  Every mbarrier wait is bounded: on expiry
 // the CTA flags DEV_ERR_TIMEOUT, stops issuing work, frees its TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <tuple>
 
 #include "gemm.cuh"
 #include "gemm_tc.cuh"
+#include "kernels.cuh"
 
 namespace nv {
 namespace {
@@ -42,7 +46,9 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNMAX * BK * 2;
 constexpr int BOX_BYTES = BOXN * BK * 2;
 constexpr int SMEM_TILES = STAGES * (A_BYTES + B_BYTES);
-constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int EPI_ROWS = 32;                    // rows per epilogue staging pass
+constexpr int EPI_BYTES = EPI_ROWS * BM * 4;    // fp32 staging tile [32 rows][128 features]
+constexpr int SMEM_BYTES = SMEM_TILES + 256 /*barriers*/ + EPI_BYTES + 1024 /*align*/;
 constexpr uint32_t TMEM_COLS = 512;  // two 256-column fp32 accumulators
 constexpr int THREADS = 192;
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on any single wait
@@ -54,6 +60,10 @@ struct TcArgs {
   int max_split;
   size_t split_stride;
   int* status;
+  int fused;             // apply `epi` in-kernel (one K slice only; else store fp32 Y)
+  const unsigned char* pf_ptr;  // bytes to pull into L2 for the next GEMM (may be null)
+  unsigned long long pf_bytes;
+  EpiArgs epi;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -161,14 +171,105 @@ __device__ __forceinline__ Item decode_item(int it, int ntn, int splits, int R, 
   return t;
 }
 
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Apply the layer epilogue to a staged tile: S[j][f] = y for row r0 + j and
+// feature n0 + f (f < 128).  Run by the 128 epilogue threads.
+//   EPI_QKV:    the tile holds whole heads of one of q/k/v (n0 % 128 == 0,
+//               head_dim | 128, H*head_dim % 128 == 0): rotate-half RoPE on q
+//               and k pairs, q -> q_out, k and v -> the paged KV cache.
+//   EPI_RESID:  h[row] += y.
+//   EPI_SWIGLU: the tile holds 64 gate rows then the 64 matching up rows.
+__device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, int n0, int r0, int nrows) {
+  const int tid = threadIdx.x;
+  if (e.mode == EPI_QKV) {
+    const int half = e.hd / 2, HQ = e.H * e.hd;
+    const int part = n0 / HQ;
+#pragma unroll 4
+    for (int idx = tid; idx < nrows * (BM / 2); idx += 128) {
+      const int j = idx / (BM / 2), pr = idx % (BM / 2);
+      const int f0 = (pr / half) * e.hd + pr % half;
+      const int nl = n0 % HQ + f0;  // feature within q, k or v
+      const int head = nl / e.hd, i = nl % e.hd;
+      float y0 = S[j * BM + f0], y1 = S[j * BM + f0 + half];
+      const int r = r0 + j;
+      const int pos = e.rs.row_pos[r];
+      if (part < 2) {
+        const float2 cs = e.rope[(size_t)pos * half + i];
+        const float u0 = y0 * cs.x - y1 * cs.y;
+        const float u1 = y1 * cs.x + y0 * cs.y;
+        y0 = u0;
+        y1 = u1;
+      }
+      __nv_bfloat16* dst;
+      if (part == 0) dst = (__nv_bfloat16*)e.q_out + (size_t)r * HQ + head * e.hd;
+      else dst = (__nv_bfloat16*)e.kv.base + e.kv.offset(e.layer, e.rs.row_b[r], pos, head, part - 1);
+      dst[i] = __float2bfloat16_rn(y0);
+      dst[i + half] = __float2bfloat16_rn(y1);
+    }
+  } else if (e.mode == EPI_RESID) {
+    // all row addresses and old values first (independent loads in flight)
+    float* hp[EPI_ROWS];
+    float hv[EPI_ROWS];
+#pragma unroll
+    for (int j = 0; j < EPI_ROWS; ++j)
+      hp[j] = j < nrows ? e.rs.h + (size_t)e.rs.row_hrow[r0 + j] * e.d + n0 + tid : nullptr;
+#pragma unroll
+    for (int j = 0; j < EPI_ROWS; ++j) hv[j] = hp[j] ? *hp[j] : 0.f;
+#pragma unroll
+    for (int j = 0; j < EPI_ROWS; ++j)
+      if (hp[j]) *hp[j] = hv[j] + S[j * BM + tid];
+  } else if (e.mode == EPI_SWIGLU) {
+#pragma unroll 4
+    for (int idx = tid; idx < nrows * (BM / 2); idx += 128) {
+      const int j = idx / (BM / 2), jj = idx % (BM / 2);
+      const float g = S[j * BM + jj], u = S[j * BM + BM / 2 + jj];
+      ((__nv_bfloat16*)e.u_out)[(size_t)(r0 + j) * e.F + (n0 / BM) * (BM / 2) + jj] =
+          __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, TcArgs a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ int s_go;
+  const int ntn = a.N / BM, kblocks = a.K / BK;
+  // Before waiting for the previous kernel: nothing here reads what it
+  // writes.  Pull the weight tiles this CTA will stream when all rows fit
+  // one tile (the decode case), and the next GEMM's share, into L2.
+  if (threadIdx.x == 160) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tx)) : "memory");
+    const int s1 = tc_split_count(1, a.N, a.K, gridDim.x, a.max_split);
+    if ((int)blockIdx.x < ntn * s1) {
+      const Item t = decode_item(blockIdx.x, ntn, s1, 1, kblocks);
+      for (int kb = t.kb0; kb < t.kb1; ++kb)
+        asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                         reinterpret_cast<uint64_t>(&tw)),
+                     "r"(kb * BK), "r"(t.n0)
+                     : "memory");
+    }
+    if (a.pf_ptr && a.pf_bytes) {
+      const unsigned long long share = ((a.pf_bytes / gridDim.x) + 15ull) & ~15ull;
+      const unsigned long long beg = share * blockIdx.x;
+      for (unsigned long long o = beg; o < beg + share && o < a.pf_bytes; o += 65536ull) {
+        unsigned long long n = beg + share - o;
+        if (n > 65536ull) n = 65536ull;
+        if (o + n > a.pf_bytes) n = a.pf_bytes - o;
+        n &= ~15ull;
+        if (n)
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.pf_ptr + o), "r"((uint32_t)n) : "memory");
+      }
+    }
+  }
+  pdl_wait();
+  pdl_launch();
   const int R = *a.nrows;
   if (R <= 0) return;
-  const int ntn = a.N / BM, nrt = (R + BNMAX - 1) / BNMAX, kblocks = a.K / BK;
+  const int nrt = (R + BNMAX - 1) / BNMAX;
   const int splits = tc_split_count(R, a.N, a.K, gridDim.x, a.max_split);
   const int items = ntn * nrt * splits;
   if ((int)blockIdx.x >= items) return;
@@ -180,6 +281,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
+  float* stile = (float*)(smem + SMEM_TILES + 256);  // epilogue staging [EPI_ROWS][BM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -208,8 +310,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 4) {
     if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tx)) : "memory");
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -281,19 +381,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t aphase = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x) {
       const Item t = decode_item(it, ntn, splits, R, kblocks);
-      if (!mbar_wait(tfull + acc, aphase, abort_flag)) break;
-      __syncwarp();
+      // one thread waits, the named barrier releases all four warps together,
+      // so an expired wait makes every epilogue warp leave at the same point
+      if (threadIdx.x == 0) s_go = mbar_wait(tfull + acc, aphase, abort_flag) ? 1 : 0;
+      epi_bar();
+      if (!s_go) break;
       tc_fence_after();
       const int n = t.n0 + warp * 32 + lane;
-      float* Ys = a.Y + (size_t)t.split * a.split_stride;
       const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * BNMAX);
+      const bool direct = a.fused != 0;  // fused launches never split
+      float* Ys = a.Y + (size_t)t.split * a.split_stride;
       for (int c0 = 0; c0 < t.nbox * BOXN; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tbase + (uint32_t)c0, v);
+        if (direct) {
+          // stage [32 rows][128 features], then the layer epilogue
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r = t.r0 + c0 + j;
-          if (r < R) Ys[(size_t)r * a.N + n] = __uint_as_float(v[j]);
+          for (int j = 0; j < 32; ++j) stile[j * BM + warp * 32 + lane] = __uint_as_float(v[j]);
+          epi_bar();
+          tile_epilogue(a.epi, stile, t.n0, t.r0 + c0, min(32, R - (t.r0 + c0)));
+          epi_bar();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int r = t.r0 + c0 + j;
+            if (r < R) Ys[(size_t)r * a.N + n] = __uint_as_float(v[j]);
+          }
         }
       }
       tc_fence_before();
@@ -371,6 +484,8 @@ nv_status tc_prepare() {
   return NV_OK;
 }
 
+size_t tc_split_stride(size_t N) { return (size_t)BNMAX * N; }
+
 size_t tc_workspace_elems(size_t N) { return (size_t)TC_MAX_SPLIT * BNMAX * N; }
 
 static nv_status make_map(TcPlanCache* c, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld_elems,
@@ -409,12 +524,25 @@ static nv_status make_map(TcPlanCache* c, const void* ptr, uint64_t inner, uint6
 }
 
 nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int N, int K, const int* nrows,
-                      int max_rows, float* Y, bool allow_split, int* split_grid, size_t* split_stride,
-                      cudaStream_t st) {
+                      int max_rows, float* Y, bool allow_split, const EpiArgs* epi, int* tile_counters,
+                      const void* prefetch, size_t prefetch_bytes, cudaStream_t st, int* grid_out) {
   if (N % BM || K % BK || K > ldx) {
     set_error("tcgen05 GEMM needs N % 128 == 0 and K % 64 == 0 (N=" + std::to_string(N) + ", K=" +
               std::to_string(K) + ")");
     return NV_ERR_UNSUPPORTED;
+  }
+  if (epi && epi->mode != EPI_STORE) {
+    if (allow_split) {
+      set_error("fused tcgen05 epilogue needs one K slice");
+      return NV_ERR_UNSUPPORTED;
+    }
+    const bool ok = epi->mode == EPI_RESID ||
+                    (epi->mode == EPI_QKV && BM % epi->hd == 0 && (epi->H * epi->hd) % BM == 0) ||
+                    (epi->mode == EPI_SWIGLU && epi->G == BM / 2);
+    if (!ok) {
+      set_error("fused tcgen05 epilogue: unsupported tile layout");
+      return NV_ERR_UNSUPPORTED;
+    }
   }
   CUtensorMap tw, tx;
   NV_TRY(make_map(c, W, (uint64_t)K, (uint64_t)N, (uint64_t)K, BM, &tw));
@@ -433,9 +561,17 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
   a.max_split = allow_split ? TC_MAX_SPLIT : 1;
   a.split_stride = (size_t)BNMAX * N;
   a.status = c->status;
-  k_gemm_tc<<<grid, THREADS, SMEM_BYTES, st>>>(tw, tx, a);
-  *split_grid = allow_split ? grid : 0;
-  *split_stride = a.split_stride;
+  a.fused = (epi && epi->mode != EPI_STORE) ? 1 : 0;
+  a.pf_ptr = (const unsigned char*)prefetch;
+  a.pf_bytes = ((uintptr_t)prefetch & 15) ? 0ull : (unsigned long long)prefetch_bytes;
+  if (epi) a.epi = *epi;
+  else std::memset(&a.epi, 0, sizeof(a.epi));
+  cudaError_t le = launch_k(k_gemm_tc, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tw, tx, a);
+  if (le != cudaSuccess) {
+    set_error(std::string("tcgen05 GEMM launch: ") + cudaGetErrorString(le));
+    return NV_ERR_CUDA;
+  }
+  if (grid_out) *grid_out = grid;
   return NV_OK;
 }
 

@@ -8,9 +8,20 @@
 // later tokens; the backbone is LLaMA-2 (section 4).
 #include <math_constants.h>
 
+#include <cstdlib>
+
 #include "kernels.cuh"
 
 namespace nv {
+
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("NVIUM_PDL");
+    on = (e && e[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
 
 // ---------------------------------------------------------------------------
 // reductions (fixed shuffle / tree order: results are deterministic)
@@ -90,21 +101,75 @@ __device__ __forceinline__ int find_seq(const int* start, int B, int r) {
 }
 
 // RMSNorm of one row by one warp: out = rnd(g * h / sqrt(mean(h^2) + eps)).
+// The row is read once with 16-byte loads and kept in registers (d <= 2048).
+// With Y set, the row is first completed by the residual update
+// h += sum_s Y[s] (split-K slices of a GEMM, summed in slice order) and the
+// new h is written back.
+constexpr int NORM_MAXV = 16;
+template <typename T> __device__ __forceinline__ void store4(T* p, float a, float b, float c, float d);
+template <> __device__ __forceinline__ void store4<float>(float* p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p) = u;
+}
 template <typename T>
-__device__ __forceinline__ void warp_norm_row(const float* __restrict__ h, const T* __restrict__ g,
-                                              T* __restrict__ out, int d, float eps) {
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ void warp_norm_row(float* __restrict__ h, const T* __restrict__ g, T* __restrict__ out,
+                                              int d, float eps, const float* __restrict__ Y = nullptr, int ns = 0,
+                                              size_t sstride = 0) {
+  const int lane = threadIdx.x & 31, nv = d >> 2;
+  float4 x[NORM_MAXV];
   float ss = 0.f;
-  for (int i = lane; i < d; i += 32) ss = fmaf(h[i], h[i], ss);
+#pragma unroll
+  for (int c = 0; c < NORM_MAXV; ++c) {
+    const int j = lane + 32 * c;
+    if (j < nv) {
+      float4 v = reinterpret_cast<const float4*>(h)[j];
+      if (Y) {
+        float4 ys = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < ns; ++sp) {
+          const float4 y = __ldcg(reinterpret_cast<const float4*>(Y + sp * sstride) + j);
+          ys.x += y.x;
+          ys.y += y.y;
+          ys.z += y.z;
+          ys.w += y.w;
+        }
+        v.x += ys.x;
+        v.y += ys.y;
+        v.z += ys.z;
+        v.w += ys.w;
+        reinterpret_cast<float4*>(h)[j] = v;
+      }
+      x[c] = v;
+      ss = fmaf(v.x, v.x, ss);
+      ss = fmaf(v.y, v.y, ss);
+      ss = fmaf(v.z, v.z, ss);
+      ss = fmaf(v.w, v.w, ss);
+    }
+  }
   ss = warp_sum(ss);
   const float inv = 1.0f / sqrtf(ss / (float)d + eps);
-  for (int i = lane; i < d; i += 32) out[i] = cvt<T>(h[i] * inv * ld(g + i));
+#pragma unroll
+  for (int c = 0; c < NORM_MAXV; ++c) {
+    const int j = lane + 32 * c;
+    if (j < nv) {
+      const T* gp = g + 4 * j;
+      store4<T>(out + 4 * j, x[c].x * inv * ld(gp), x[c].y * inv * ld(gp + 1), x[c].z * inv * ld(gp + 2),
+                x[c].w * inv * ld(gp + 3));
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
 // RoPE table: (cos, sin) of pos * theta^(-2i/hd), computed in double.
 // ---------------------------------------------------------------------------
 __global__ void k_rope_table(float2* cs, int max_seq, int hd, double theta) {
+  pdl_wait();
+  pdl_launch();
   const int half = hd / 2;
   const long long n = (long long)max_seq * half;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
@@ -115,7 +180,7 @@ __global__ void k_rope_table(float2* cs, int max_seq, int hd, double theta) {
   }
 }
 void launch_rope_table(float2* cs, int max_seq, int hd, double theta, cudaStream_t st) {
-  k_rope_table<<<256, 256, 0, st>>>(cs, max_seq, hd, theta);
+  launch_k(k_rope_table, 256, 256, 0, st, cs, max_seq, hd, theta);
 }
 
 // ---------------------------------------------------------------------------
@@ -123,6 +188,8 @@ void launch_rope_table(float2* cs, int max_seq, int hd, double theta, cudaStream
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void k_embed_rows(const T* __restrict__ emb, const int* __restrict__ tok, RowSet rs, int d) {
+  pdl_wait();
+  pdl_launch();
   const int R = *rs.nrows;
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     const T* e = emb + (size_t)tok[r] * d;
@@ -132,12 +199,14 @@ __global__ void k_embed_rows(const T* __restrict__ emb, const int* __restrict__ 
 }
 void launch_embed_rows(bool bf16, const void* emb, const int* tok_row, RowSet rs, int d, cudaStream_t st) {
   const int grid = rs.max_rows < 4096 ? rs.max_rows : 4096;
-  if (bf16) k_embed_rows<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)emb, tok_row, rs, d);
-  else k_embed_rows<float><<<grid, 256, 0, st>>>((const float*)emb, tok_row, rs, d);
+  if (bf16) launch_k(k_embed_rows<__nv_bfloat16>, grid, 256, 0, st, (const __nv_bfloat16*)emb, tok_row, rs, d);
+  else launch_k(k_embed_rows<float>, grid, 256, 0, st, (const float*)emb, tok_row, rs, d);
 }
 
 template <typename T>
 __global__ void k_rmsnorm_rows(RowSet rs, const T* __restrict__ g, T* __restrict__ act, int d, float eps) {
+  pdl_wait();
+  pdl_launch();
   const int R = *rs.nrows;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb)
@@ -147,8 +216,33 @@ void launch_rmsnorm_rows(bool bf16, RowSet rs, const void* gain, void* act, int 
   int grid = (rs.max_rows + 7) / 8;
   if (grid > 2048) grid = 2048;
   if (bf16)
-    k_rmsnorm_rows<__nv_bfloat16><<<grid, 256, 0, st>>>(rs, (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
-  else k_rmsnorm_rows<float><<<grid, 256, 0, st>>>(rs, (const float*)gain, (float*)act, d, eps);
+    launch_k(k_rmsnorm_rows<__nv_bfloat16>, grid, 256, 0, st, rs, (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
+  else launch_k(k_rmsnorm_rows<float>, grid, 256, 0, st, rs, (const float*)gain, (float*)act, d, eps);
+}
+
+// Residual update from split-K slices of the output projection, then the MLP
+// RMSNorm, in one pass over each row.
+template <typename T>
+__global__ void k_resid_norm(RowSet rs, const float* __restrict__ Y, int split_grid, int N, int K,
+                             size_t sstride, const T* __restrict__ g, T* __restrict__ act, int d, float eps) {
+  pdl_wait();
+  pdl_launch();
+  const int R = *rs.nrows;
+  const int ns = split_grid ? tc_split_count(R, N, K, split_grid, TC_MAX_SPLIT) : 1;
+  const int wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb)
+    warp_norm_row<T>(rs.h + (size_t)rs.row_hrow[r] * d, g, act + (size_t)r * d, d, eps, Y + (size_t)r * N, ns,
+                     sstride);
+}
+void launch_resid_norm(bool bf16, RowSet rs, const float* Y, int split_grid, int N, int K, size_t sstride,
+                       const void* gain, void* act, int d, float eps, cudaStream_t st) {
+  int grid = (rs.max_rows + 7) / 8;
+  if (grid > 2048) grid = 2048;
+  if (bf16)
+    launch_k(k_resid_norm<__nv_bfloat16>, grid, 256, 0, st, rs, Y, split_grid, N, K, sstride,
+             (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
+  else launch_k(k_resid_norm<float>, grid, 256, 0, st, rs, Y, split_grid, N, K, sstride, (const float*)gain,
+                (float*)act, d, eps);
 }
 
 // ---------------------------------------------------------------------------
@@ -164,6 +258,8 @@ void launch_rmsnorm_rows(bool bf16, RowSet rs, const void* gain, void* act, int 
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT) k_plan_norm(PlanArgs a, const T* __restrict__ gain, T* __restrict__ act,
                                                   int d, float eps) {
+  pdl_wait();
+  pdl_launch();
   extern __shared__ int s_start[];  // [B+1]
   __shared__ long long s_kv[NT / 32];
   const int B = a.B, tid = threadIdx.x;
@@ -236,15 +332,15 @@ __global__ void __launch_bounds__(NT) k_plan_norm(PlanArgs a, const T* __restric
     const int b = find_seq(s_start, B, r);
     const int pos = a.lens[b * a.L + a.layer] + (r - s_start[b]);
     const int hrow = b * a.cap + pos % a.cap;
-    warp_norm_row<T>(a.h + (size_t)hrow * d, gain, act + (size_t)r * d, d, eps);
+    warp_norm_row<T>(const_cast<float*>(a.h) + (size_t)hrow * d, gain, act + (size_t)r * d, d, eps);
   }
 }
 void launch_plan_norm(bool bf16, const PlanArgs& a, const void* gain, void* act, int d, float eps, int grid,
                       cudaStream_t st) {
   const size_t sm = (size_t)(a.B + 1) * sizeof(int);
   if (bf16)
-    k_plan_norm<__nv_bfloat16, 256><<<grid, 256, sm, st>>>(a, (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
-  else k_plan_norm<float, 256><<<grid, 256, sm, st>>>(a, (const float*)gain, (float*)act, d, eps);
+    launch_k(k_plan_norm<__nv_bfloat16, 256>, grid, 256, sm, st, a, (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
+  else launch_k(k_plan_norm<float, 256>, grid, 256, sm, st, a, (const float*)gain, (float*)act, d, eps);
 }
 
 // ---------------------------------------------------------------------------
@@ -254,6 +350,8 @@ void launch_plan_norm(bool bf16, const PlanArgs& a, const void* gain, void* act,
 template <typename T>
 __global__ void __launch_bounds__(256) k_gemm_simt(const T* __restrict__ X, int ldx, const T* __restrict__ W,
                                                    int N, int K, const int* __restrict__ nrows, float* __restrict__ Y) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float Xs[16][68];
   __shared__ float Ws[16][68];
   const int R = *nrows;
@@ -308,9 +406,9 @@ void launch_gemm_simt(bool bf16, const void* X, int ldx, const void* W, int N, i
   if (gy > 64) gy = 64;
   dim3 grid((N + 63) / 64, gy);
   if (bf16)
-    k_gemm_simt<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)X, ldx, (const __nv_bfloat16*)W, N, K,
+    launch_k(k_gemm_simt<__nv_bfloat16>, grid, 256, 0, st, (const __nv_bfloat16*)X, ldx, (const __nv_bfloat16*)W, N, K,
                                                      nrows, Y);
-  else k_gemm_simt<float><<<grid, 256, 0, st>>>((const float*)X, ldx, (const float*)W, N, K, nrows, Y);
+  else launch_k(k_gemm_simt<float>, grid, 256, 0, st, (const float*)X, ldx, (const float*)W, N, K, nrows, Y);
 }
 
 // ---------------------------------------------------------------------------
@@ -329,6 +427,8 @@ __device__ __forceinline__ float epi_sum(const EpiArgs& a, int ns, int r, int n)
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_epilogue(EpiArgs a) {
+  pdl_wait();
+  pdl_launch();
   const int R = *a.rs.nrows;
   const int ns = a.split_grid ? tc_split_count(R, a.N, a.split_K, a.split_grid, TC_MAX_SPLIT) : 1;
   const long long stride = (long long)gridDim.x * blockDim.x;
@@ -382,8 +482,8 @@ __global__ void __launch_bounds__(256) k_epilogue(EpiArgs a) {
   }
 }
 void launch_epilogue(bool bf16, const EpiArgs& a, int grid, cudaStream_t st) {
-  if (bf16) k_epilogue<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
-  else k_epilogue<float><<<grid, 256, 0, st>>>(a);
+  if (bf16) launch_k(k_epilogue<__nv_bfloat16>, grid, 256, 0, st, a);
+  else launch_k(k_epilogue<float>, grid, 256, 0, st, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -400,6 +500,8 @@ void launch_epilogue(bool bf16, const EpiArgs& a, int grid, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 template <typename T, int HD>
 __global__ void __launch_bounds__(128) k_attention(AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
   constexpr int NW = 4, RPW = ATTN_RPC / NW, KT = ATTN_KT, DPL = HD / 32;
   __shared__ float Ks[KT][HD + 1];
   __shared__ float Vs[KT][HD];
@@ -505,6 +607,8 @@ __global__ void __launch_bounds__(128) k_attention(AttnArgs a) {
 
 template <typename T, int HD>
 __global__ void k_attn_combine(AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
   constexpr int DPL = HD / 32;
   const int R = *a.rs.nrows;
   const int lane = threadIdx.x & 31;
@@ -550,6 +654,8 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
 
 template <typename T, int HD>
 __global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
   static_assert(HD * sizeof(T) == 128, "128-byte rows");
   constexpr int NW = 4, KPL = DEC_CK / 32, DPL = HD / 32, EPC = 16 / sizeof(T);
   __shared__ __align__(128) T Ks[DEC_CK * HD];
@@ -677,6 +783,8 @@ __global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
 // Merge the chunk partials of each (row, head): chunks 0 .. pos/128.
 template <typename T, int HD>
 __global__ void k_attn_dec_combine(AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
   constexpr int DPL = HD / 32;
   const int R = *a.rs.nrows;
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
@@ -705,10 +813,10 @@ __global__ void k_attn_dec_combine(AttnArgs a) {
 template <typename T, int HD>
 static void attention_dec_t(const AttnArgs& a, cudaStream_t st) {
   dim3 grid(a.rs.B, a.H, a.kv_splits);
-  k_attn_dec<T, HD><<<grid, 128, 0, st>>>(a);
+  launch_k(k_attn_dec<T, HD>, grid, 128, 0, st, a);
   int g = (a.rs.max_rows * a.H + 7) / 8;
   if (g > 4096) g = 4096;
-  k_attn_dec_combine<T, HD><<<g, 256, 0, st>>>(a);
+  launch_k(k_attn_dec_combine<T, HD>, g, 256, 0, st, a);
 }
 void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st) {
   if (bf16) attention_dec_t<__nv_bfloat16, 64>(a, st);
@@ -718,11 +826,11 @@ void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st) {
 template <typename T, int HD>
 static void attention_t(const AttnArgs& a, cudaStream_t st) {
   dim3 grid(a.rs.B, a.H, a.row_groups * a.kv_splits);
-  k_attention<T, HD><<<grid, 128, 0, st>>>(a);
+  launch_k(k_attention<T, HD>, grid, 128, 0, st, a);
   if (a.kv_splits > 1) {
     int g = (a.rs.max_rows * a.H + 7) / 8;
     if (g > 4096) g = 4096;
-    k_attn_combine<T, HD><<<g, 256, 0, st>>>(a);
+    launch_k(k_attn_combine<T, HD>, g, 256, 0, st, a);
   }
 }
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st) {
@@ -738,6 +846,8 @@ void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void k_step_begin(StepArgs a) {
+  pdl_wait();
+  pdl_launch();
   const int b = blockIdx.x;
   const int tb = a.t[b];
   if (threadIdx.x == 0) {
@@ -757,11 +867,13 @@ __global__ void k_step_begin(StepArgs a) {
   for (int i = threadIdx.x; i < a.d; i += blockDim.x) h[i] = ld(e + i);
 }
 void launch_step_begin(bool bf16, const StepArgs& a, cudaStream_t st) {
-  if (bf16) k_step_begin<__nv_bfloat16><<<a.B, 256, 0, st>>>(a);
-  else k_step_begin<float><<<a.B, 256, 0, st>>>(a);
+  if (bf16) launch_k(k_step_begin<__nv_bfloat16>, a.B, 256, 0, st, a);
+  else launch_k(k_step_begin<float>, a.B, 256, 0, st, a);
 }
 
 __global__ void k_step_end(StepArgs a) {
+  pdl_wait();
+  pdl_launch();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b == 0 && a.counters) atomicAdd((unsigned long long*)&a.counters[NV_CTR_STEPS], 1ull);
   if (b >= a.B) return;
@@ -772,7 +884,7 @@ __global__ void k_step_end(StepArgs a) {
   a.t[b] += 1;
 }
 void launch_step_end(const StepArgs& a, cudaStream_t st) {
-  k_step_end<<<(a.B + 255) / 256, 256, 0, st>>>(a);
+  launch_k(k_step_end, (a.B + 255) / 256, 256, 0, st, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -784,6 +896,8 @@ void launch_step_end(const StepArgs& a, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) k_junction(JuncArgs a) {
+  pdl_wait();
+  pdl_launch();
   const int b = blockIdx.x;
   if (!a.active[b]) return;
   const int tb = a.t[b];
@@ -822,8 +936,8 @@ __global__ void __launch_bounds__(256) k_junction(JuncArgs a) {
   }
 }
 void launch_junction(bool bf16, const JuncArgs& a, cudaStream_t st) {
-  if (bf16) k_junction<__nv_bfloat16><<<a.B, 256, 0, st>>>(a);
-  else k_junction<float><<<a.B, 256, 0, st>>>(a);
+  if (bf16) launch_k(k_junction<__nv_bfloat16>, a.B, 256, 0, st, a);
+  else launch_k(k_junction<float>, a.B, 256, 0, st, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -836,6 +950,8 @@ void launch_junction(bool bf16, const JuncArgs& a, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
+  pdl_wait();
+  pdl_launch();
   constexpr int NW = 8, EPC = 16 / sizeof(T), MAXC = 8;
   extern __shared__ __align__(16) unsigned char smem[];
   int* s_list = (int*)smem;                                   // [B]
@@ -971,11 +1087,13 @@ __global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
 void launch_head_sample(bool bf16, const HeadArgs& a, cudaStream_t st) {
   const size_t esz = bf16 ? 2 : 4;
   const size_t sm = (((size_t)a.B * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * a.d * esz;
-  if (bf16) k_head_sample<__nv_bfloat16><<<a.nblk, 256, sm, st>>>(a);
-  else k_head_sample<float><<<a.nblk, 256, sm, st>>>(a);
+  if (bf16) launch_k(k_head_sample<__nv_bfloat16>, a.nblk, 256, sm, st, a);
+  else launch_k(k_head_sample<float>, a.nblk, 256, sm, st, a);
 }
 
 __global__ void k_head_reduce(HeadArgs a) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (b >= a.B || !a.stop[b]) return;
@@ -1023,7 +1141,7 @@ __global__ void k_head_reduce(HeadArgs a) {
   }
 }
 void launch_head_reduce(const HeadArgs& a, cudaStream_t st) {
-  k_head_reduce<<<(a.B + 7) / 8, 256, 0, st>>>(a);
+  launch_k(k_head_reduce, (a.B + 7) / 8, 256, 0, st, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -1032,6 +1150,8 @@ void launch_head_reduce(const HeadArgs& a, cudaStream_t st) {
 template <typename T>
 __global__ void k_exit_rows(RowSet rs, const T* __restrict__ g, const T* __restrict__ rw, float rb, int k,
                             int n_exits, T* __restrict__ act, float* __restrict__ z, int d, float eps) {
+  pdl_wait();
+  pdl_launch();
   const int R = *rs.nrows;
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   const bool last = k == n_exits - 1;
@@ -1056,15 +1176,17 @@ void launch_exit_rows(bool bf16, RowSet rs, const void* norm, const void* router
   int grid = (rs.max_rows + 7) / 8;
   if (grid > 2048) grid = 2048;
   if (bf16)
-    k_exit_rows<__nv_bfloat16><<<grid, 256, 0, st>>>(rs, (const __nv_bfloat16*)norm, (const __nv_bfloat16*)router_w,
+    launch_k(k_exit_rows<__nv_bfloat16>, grid, 256, 0, st, rs, (const __nv_bfloat16*)norm, (const __nv_bfloat16*)router_w,
                                                      router_b, k, n_exits, (__nv_bfloat16*)act, z, d, eps);
-  else k_exit_rows<float><<<grid, 256, 0, st>>>(rs, (const float*)norm, (const float*)router_w, router_b, k, n_exits,
+  else launch_k(k_exit_rows<float>, grid, 256, 0, st, rs, (const float*)norm, (const float*)router_w, router_b, k, n_exits,
                                                 (float*)act, z, d, eps);
 }
 
 // log pi_k(target) = logit[target] - LSE(logits), one warp per row.
 __global__ void k_lse_target(const float* __restrict__ Y, int r_begin, int n, int V, const int* __restrict__ target,
                              float* __restrict__ logpi, int k, int n_exits) {
+  pdl_wait();
+  pdl_launch();
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
     const float* y = Y + (size_t)i * V;
@@ -1083,7 +1205,7 @@ void launch_lse_target(const float* Y, int r_begin, int n, int V, const int* tar
   int grid = (n + 7) / 8;
   if (grid > 4096) grid = 4096;
   if (grid < 1) grid = 1;
-  k_lse_target<<<grid, 256, 0, st>>>(Y, r_begin, n, V, target, logpi, k, n_exits);
+  launch_k(k_lse_target, grid, 256, 0, st, Y, r_begin, n, V, target, logpi, k, n_exits);
 }
 
 __device__ __forceinline__ float log_sigmoid(float z) {
@@ -1094,6 +1216,8 @@ __device__ __forceinline__ float log_sigmoid(float z) {
 // log pi_mix = LSE_k(log p_k + log pi_k), log p_k = log sigma(z_k) + sum_{j<k} log sigma(-z_j).
 __global__ void k_mixture(const float* __restrict__ z, const float* __restrict__ logpi, int R, int n_exits, int mode,
                           float* __restrict__ logp) {
+  pdl_wait();
+  pdl_launch();
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= R) return;
   float terms[NV_MAX_EXITS];
@@ -1118,6 +1242,8 @@ __global__ void k_mixture(const float* __restrict__ z, const float* __restrict__
 }
 
 __global__ void k_mean_nll(const float* __restrict__ logp, int R, float* __restrict__ out) {
+  pdl_wait();
+  pdl_launch();
   __shared__ double s[256];
   double a = 0.0;
   for (int r = threadIdx.x; r < R; r += 256) a += (double)logp[r];
@@ -1131,11 +1257,13 @@ __global__ void k_mean_nll(const float* __restrict__ logp, int R, float* __restr
 }
 
 __global__ void k_philox(unsigned long long seed, const uint4* ctr, int n, uint4* out) {
+  pdl_wait();
+  pdl_launch();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = philox4x32_10(ctr[i], (uint32_t)seed, (uint32_t)(seed >> 32));
 }
 void launch_philox(unsigned long long seed, const void* ctr, int n, void* out, cudaStream_t st) {
-  k_philox<<<(n + 255) / 256, 256, 0, st>>>(seed, (const uint4*)ctr, n, (uint4*)out);
+  launch_k(k_philox, (n + 255) / 256, 256, 0, st, seed, (const uint4*)ctr, n, (uint4*)out);
 }
 
 cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes) {
@@ -1156,8 +1284,8 @@ cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes) {
 
 void launch_mixture(const float* z, const float* logpi, int R, int n_exits, int mode, float* logp, float* mean_nll,
                     cudaStream_t st) {
-  k_mixture<<<(R + 255) / 256, 256, 0, st>>>(z, logpi, R, n_exits, mode, logp);
-  if (mean_nll) k_mean_nll<<<1, 256, 0, st>>>(logp, R, mean_nll);
+  launch_k(k_mixture, (R + 255) / 256, 256, 0, st, z, logpi, R, n_exits, mode, logp);
+  if (mean_nll) launch_k(k_mean_nll, 1, 256, 0, st, logp, R, mean_nll);
 }
 
 }  // namespace nv

@@ -16,6 +16,10 @@ void launch_rope_table(float2* cs, int max_seq, int hd, double theta, cudaStream
 
 void launch_embed_rows(bool bf16, const void* emb, const int* tok_row, RowSet rs, int d, cudaStream_t st);
 void launch_rmsnorm_rows(bool bf16, RowSet rs, const void* gain, void* act, int d, float eps, cudaStream_t st);
+// h[row] += sum of the split-K slices Y[s][row] (a GEMM's partial sums), then
+// act[row] = RMSNorm(h[row]) * gain.
+void launch_resid_norm(bool bf16, RowSet rs, const float* Y, int split_grid, int N, int K, size_t sstride,
+                       const void* gain, void* act, int d, float eps, cudaStream_t st);
 
 struct PlanArgs {
   int B, L, cap, layer, mode;  // mode 0: decode step (lazy rule), 1: flush

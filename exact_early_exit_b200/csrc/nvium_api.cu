@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "gemm.cuh"
+#include "gemm_tc.cuh"
 #include "kernels.cuh"
 
 namespace nv {
@@ -40,6 +41,9 @@ nv_status dalloc(T** p, size_t count) {
 nv_status dalloc_bytes(void** p, size_t bytes) { return dalloc((unsigned char**)p, bytes); }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kTileCounters = 1024;  // >= N/128 of any split GEMM
+size_t tc_split_stride_elems(int N) { return nv::tc_split_stride((size_t)N); }
 
 // grow-only device buffer
 struct Buf {
@@ -79,7 +83,7 @@ struct nv_model {
   int gemm_kind = GEMM_SIMT;
   GemmPlanCache* gemm_plans = nullptr;
   // scoring scratch
-  Buf sc_h, sc_act, sc_q, sc_o, sc_Y, sc_kv, sc_part, sc_z, sc_logpi, sc_logp, sc_i32, sc_nll;
+  Buf sc_h, sc_act, sc_u, sc_ctr, sc_q, sc_o, sc_Y, sc_kv, sc_part, sc_z, sc_logpi, sc_logp, sc_i32, sc_nll;
 };
 
 struct nv_state {
@@ -100,7 +104,8 @@ struct nv_state {
   float* hbuf = nullptr;
   // work list and activations
   int *row_b = nullptr, *row_pos = nullptr, *row_hrow = nullptr, *seq_start = nullptr, *nrows = nullptr;
-  void *act = nullptr, *q = nullptr, *o = nullptr, *exit_act = nullptr;
+  void *act = nullptr, *u = nullptr, *q = nullptr, *o = nullptr, *exit_act = nullptr;
+  int* tile_counters = nullptr;
   float *Y = nullptr, *attn_part = nullptr, *head_part = nullptr;
   size_t Y_elems = 0;
   int head_nblk = 0, kv_splits = 1, row_groups = 1;
@@ -149,9 +154,11 @@ KVView state_kv(nv_state* s) {
 struct LayerIO {
   RowSet rs;
   KVView kv;
-  void* act;           // [rows][max(d,F)]
+  void* act;           // [rows][d] normed activations
+  void* u;             // [rows][F] SwiGLU output
   void* q;
   void* o;
+  int* tile_counters;  // split-K arrival counters (zeroed)
   float* Y;
   float* attn_part;
   int kv_splits, row_groups;
@@ -159,6 +166,8 @@ struct LayerIO {
   int L;
   int epi_grid;
   bool dec_attn;       // chunked decode attention (else row-group attention)
+  bool prefetch_next;  // the last GEMM of a layer prefetches the next layer's QKV weights
+  bool split_k;        // few rows expected (decode, flush): let the GEMM split K
   int* status;
 };
 
@@ -218,8 +227,6 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   const long long es = (long long)M->esz;
   const long long R = prof ? prof->R : 0;
   const long long d = M->d, HQ = M->HQ, F = M->F;
-  int sgrid = 0;
-  size_t sstride = 0;
   nv_status gst = NV_OK;
   EpiArgs e{};
   e.rs = io.rs;
@@ -231,28 +238,25 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   e.layer = layer;  // scoring's single-layer scratch has layer_stride 0
   e.F = M->F;
   e.G = M->G;
-  // algorithmic bytes of Y = X W^T: W once, X once, Y written once (fp32)
-  auto gemm_bytes = [&](long long N, long long K) { return N * K * es + R * K * es + R * N * 4; };
-  auto gemm = [&](const void* X, long long ldx, const void* W, long long N, long long K) {
-    timed(prof, launches, 1, NV_K_GEMM, gemm_bytes(N, K), 2 * R * N * K, [&] {
-      gst = gemm_run(M->gemm_plans, M->gemm_kind, bf, X, (int)ldx, W, (int)N, (int)K, io.rs.nrows, io.rs.max_rows,
-                     io.Y, true, &sgrid, &sstride, st);
-    });
+  e.q_out = io.q;
+  e.u_out = io.u;
+  // algorithmic bytes of Y = X W^T + epilogue: W once, X once, outputs once
+  // the weights each GEMM pulls into L2 for the one after it
+  const LayerDev* nextL = layer + 1 < M->L ? &M->layers[layer + 1] : nullptr;
+  auto gemm = [&](int mode, const void* X, long long ldx, const void* W, long long N, long long K, long long out_bytes,
+                  const void* pf, long long pf_bytes) {
+    e.mode = mode;
+    e.N = (int)N;
+    timed(prof, launches, M->gemm_kind == GEMM_TC ? 1 : 2, NV_K_GEMM, N * K * es + R * K * es + out_bytes,
+          2 * R * N * K, [&] {
+            gst = gemm_run(M->gemm_plans, M->gemm_kind, bf, X, (int)ldx, W, (int)N, (int)K, io.rs.nrows,
+                           io.rs.max_rows, io.Y, io.split_k, &e, io.tile_counters, io.epi_grid, pf,
+                           pf ? (size_t)pf_bytes : 0, st);
+          });
     return gst;
   };
-  auto epi = [&](int mode, long long N, long long K, long long out_bytes) {
-    e.mode = mode;
-    e.Y = io.Y;
-    e.split_grid = sgrid;
-    e.split_K = (int)K;
-    e.split_stride = sstride;
-    e.N = (int)N;
-    timed(prof, launches, 1, NV_K_EPILOGUE, R * N * 4 + out_bytes, 0, [&] { launch_epilogue(bf, e, io.epi_grid, st); });
-  };
-  // QKV, RoPE, KV write
-  NV_TRY(gemm(io.act, d, Lw.w_qkv, 3 * HQ, d));
-  e.q_out = io.q;
-  epi(EPI_QKV, 3 * HQ, d, R * 3 * HQ * es);
+  // QKV + RoPE + KV write (fused epilogue)
+  NV_TRY(gemm(EPI_QKV, io.act, d, Lw.w_qkv, 3 * HQ, d, R * 3 * HQ * es, Lw.w_o, d * HQ * es));
   // attention
   AttnArgs a{};
   a.rs = io.rs;
@@ -274,17 +278,28 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
           if (io.dec_attn) launch_attention_decode(bf, a, st);
           else launch_attention(bf, a, st);
         });
-  // output projection + residual
-  NV_TRY(gemm(io.o, HQ, Lw.w_o, d, HQ));
-  epi(EPI_RESID, d, HQ, R * d * 8);
-  // MLP
-  timed(prof, launches, 1, NV_K_NORM, R * d * (4 + es), 0,
-        [&] { launch_rmsnorm_rows(bf, io.rs, Lw.mlp_norm, io.act, M->d, M->cfg.rms_eps, st); });
-  NV_TRY(gemm(io.act, d, Lw.w_gu, 2 * F, d));
-  e.u_out = io.act;
-  epi(EPI_SWIGLU, 2 * F, d, R * F * es);
-  NV_TRY(gemm(io.act, F, Lw.w_d, d, F));
-  epi(EPI_RESID, d, F, R * d * 8);
+  // output projection + residual, MLP RMSNorm
+  if (M->gemm_kind == GEMM_TC && io.split_k) {
+    // split-K slices of the projection are summed into h by the norm kernel
+    int sg = 0;
+    timed(prof, launches, 1, NV_K_GEMM, d * HQ * es + R * HQ * es + R * d * 4, 2 * R * d * HQ, [&] {
+      gst = gemm_run(M->gemm_plans, M->gemm_kind, bf, io.o, (int)HQ, Lw.w_o, (int)d, (int)HQ, io.rs.nrows,
+                     io.rs.max_rows, io.Y, true, nullptr, io.tile_counters, io.epi_grid, Lw.w_gu,
+                     (size_t)(2 * F * d * es), st, &sg);
+    });
+    NV_TRY(gst);
+    timed(prof, launches, 1, NV_K_NORM, R * d * (8 + es), 0, [&] {
+      launch_resid_norm(bf, io.rs, io.Y, sg, M->d, M->HQ, tc_split_stride_elems(M->d), Lw.mlp_norm, io.act, M->d,
+                        M->cfg.rms_eps, st);
+    });
+  } else {
+    NV_TRY(gemm(EPI_RESID, io.o, HQ, Lw.w_o, d, HQ, R * d * 8, Lw.w_gu, 2 * F * d * es));
+    timed(prof, launches, 1, NV_K_NORM, R * d * (4 + es), 0,
+          [&] { launch_rmsnorm_rows(bf, io.rs, Lw.mlp_norm, io.act, M->d, M->cfg.rms_eps, st); });
+  }
+  NV_TRY(gemm(EPI_SWIGLU, io.act, d, Lw.w_gu, 2 * F, d, R * F * es, Lw.w_d, d * F * es));
+  NV_TRY(gemm(EPI_RESID, io.u, F, Lw.w_d, d, F, R * d * 8, io.prefetch_next && nextL ? nextL->w_qkv : nullptr,
+              3 * HQ * d * es));
   return NV_OK;
 }
 
@@ -293,6 +308,8 @@ LayerIO state_io(nv_state* s) {
   io.rs = state_rowset(s);
   io.kv = state_kv(s);
   io.act = s->act;
+  io.u = s->u;
+  io.tile_counters = s->tile_counters;
   io.q = s->q;
   io.o = s->o;
   io.Y = s->Y;
@@ -303,6 +320,8 @@ LayerIO state_io(nv_state* s) {
   io.L = s->m->L;
   io.epi_grid = 1184;
   io.dec_attn = s->dec_attn;
+  io.prefetch_next = true;
+  io.split_k = true;
   io.status = s->status;
   return io;
 }
@@ -686,7 +705,7 @@ nv_status nv_destroy(nv_model* M) {
   cudaDeviceSynchronize();
   if (M->pool) cudaFree(M->pool);
   gemm_plans_destroy(M->gemm_plans);
-  for (Buf* b : {&M->sc_h, &M->sc_act, &M->sc_q, &M->sc_o, &M->sc_Y, &M->sc_kv, &M->sc_part, &M->sc_z,
+  for (Buf* b : {&M->sc_h, &M->sc_act, &M->sc_u, &M->sc_ctr, &M->sc_q, &M->sc_o, &M->sc_Y, &M->sc_kv, &M->sc_part, &M->sc_z,
                  &M->sc_logpi, &M->sc_logp, &M->sc_i32, &M->sc_nll})
     b->release();
   delete M;
@@ -748,6 +767,8 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   A((void**)&s->seq_start, (size_t)(B + 1) * 4);
   A((void**)&s->nrows, 4);
   A(&s->act, (size_t)s->max_rows * wide * esz);
+  A(&s->u, (size_t)s->max_rows * F * esz);
+  A((void**)&s->tile_counters, (size_t)kTileCounters * 4);
   A(&s->q, (size_t)s->max_rows * HQ * esz);
   A(&s->o, (size_t)s->max_rows * HQ * esz);
   A(&s->exit_act, (size_t)B * d * esz);
@@ -762,6 +783,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
     return st;
   }
   cudaMemset(s->counters, 0, NV_CTR_COUNT * 8);
+  cudaMemset(s->tile_counters, 0, (size_t)kTileCounters * 4);
   cudaMemset(s->status, 0, 4);
   cudaMemset(s->nrows, 0, 4);
   cudaMemset(s->lens, 0, (size_t)B * M->L * 4);
@@ -838,8 +860,11 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
   const size_t wide = M->d > M->F ? M->d : M->F;
   // per-chunk buffers: h, act, q, o, Y, attention partials, row arrays
   const int cr = R < chunk ? (R > 0 ? R : 1) : chunk;
-  Buf h, act, q, o, Y, rows;
+  Buf h, act, u, q, o, Y, rows, ctr;
   nv_status stt = NV_OK;
+  if ((stt = u.need((size_t)cr * M->F * M->esz)) != NV_OK) return stt;
+  if ((stt = ctr.need((size_t)kTileCounters * 4)) != NV_OK) return stt;
+  NV_CUDA_TRY(cudaMemsetAsync(ctr.p, 0, (size_t)kTileCounters * 4, st));
   if ((stt = h.need((size_t)cr * M->d * 4)) != NV_OK) return stt;
   if ((stt = act.need((size_t)cr * wide * M->esz)) != NV_OK) return stt;
   if ((stt = q.need((size_t)cr * M->HQ * M->esz)) != NV_OK) return stt;
@@ -870,6 +895,8 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
     io.rs = RowSet{d_n, d_b, d_pos, d_hrow, d_seq, h.as<float>(), cr, B};
     io.kv = state_kv(s);
     io.act = act.p;
+    io.u = u.p;
+    io.tile_counters = ctr.as<int>();
     io.q = q.p;
     io.o = o.p;
     io.Y = Y.as<float>();
@@ -903,6 +930,8 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
   NV_CUDA_TRY(cudaStreamSynchronize(st));
   h.release();
   act.release();
+  u.release();
+  ctr.release();
   q.release();
   o.release();
   Y.release();
@@ -1186,6 +1215,11 @@ nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, flo
   const size_t y_head = gemm_workspace_elems(M->gemm_kind, head_chunk, M->V);
   NV_TRY(M->sc_h.need((size_t)R * M->d * 4));
   NV_TRY(M->sc_act.need((size_t)R * wide * M->esz));
+  NV_TRY(M->sc_u.need((size_t)R * M->F * M->esz));
+  if (!M->sc_ctr.p) {
+    NV_TRY(M->sc_ctr.need((size_t)kTileCounters * 4));
+    NV_CUDA_TRY(cudaMemset(M->sc_ctr.p, 0, (size_t)kTileCounters * 4));
+  }
   NV_TRY(M->sc_q.need((size_t)R * M->HQ * M->esz));
   NV_TRY(M->sc_o.need((size_t)R * M->HQ * M->esz));
   NV_TRY(M->sc_Y.need(std::max(y_layers, y_head) * 4));
@@ -1242,6 +1276,8 @@ nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, flo
   io.kv.H = M->H;
   io.kv.hd = M->hd;
   io.act = M->sc_act.p;
+  io.u = M->sc_u.p;
+  io.tile_counters = M->sc_ctr.as<int>();
   io.q = M->sc_q.p;
   io.o = M->sc_o.p;
   io.Y = M->sc_Y.as<float>();
@@ -1261,10 +1297,9 @@ nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, flo
                      M->sc_z.as<float>(), M->d, M->cfg.rms_eps, st);
     for (int c = 0; c < nchunks; ++c) {
       const int r0 = c * head_chunk;
-      int sgrid = 0;
-      size_t sstride = 0;
       NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, M->bf16, (const unsigned char*)io.act + (size_t)r0 * M->d * M->esz,
-                      M->d, M->exits[k].head, M->V, M->d, d_chunk + c, head_chunk, io.Y, false, &sgrid, &sstride, st));
+                      M->d, M->exits[k].head, M->V, M->d, d_chunk + c, head_chunk, io.Y, false, nullptr, nullptr, 0,
+                      nullptr, 0, st));
       const float* Yh = io.Y;
       launch_lse_target(Yh, r0, std::min(head_chunk, R - r0), M->V, d_tgt, M->sc_logpi.as<float>(), k, NE, st);
     }

@@ -55,3 +55,23 @@ def test_simt_and_tcgen05_engines_agree(weights):
         out[eng] = lp
         m.close()
     np.testing.assert_allclose(out["simt"], out["tc"], atol=5e-3, rtol=0)
+
+
+
+def test_prefill_kv_matches_oracle(weights):
+    """Every layer's K and V right after prefill (full-depth rows, before any
+    decode step) against the oracle's prefill caches."""
+    from tests.nvium_testlib import gpu_kv, kv_close
+    wl = W.WORKLOADS["S"]
+    prompts = [p[:n] for p, n in zip(W.make_prompts(wl, seed=4), (70, 5, 129))]
+    lens = np.array([len(p) for p in prompts], np.int32)
+    model = nv.Model(CFG, weights, max_batch=3, max_seq=160)
+    st = nv.State(model, 3)
+    st.prefill(np.concatenate(prompts), lens)
+    dec = O.OracleDecoder(O.OracleModel(CFG, weights), prompts, 4)
+    for b in range(3):
+        for m in range(CFG.n_layers):
+            K, V, n = gpu_kv(st, b, m, 160, CFG)
+            assert n == lens[b] - 1
+            kv_close(K, dec.caches[b].K[m][:n], CFG)
+            kv_close(V, dec.caches[b].V[m][:n], CFG)
