@@ -171,6 +171,6 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // Which part of a fused weight a GEMM output column belongs to.
-enum EpiMode : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_STORE = 3 };
+enum EpiMode : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_STORE = 3, EPI_HEAD = 4 };
 
 }  // namespace nv

@@ -23,6 +23,8 @@ void gemm_plans_destroy(GemmPlanCache* c) {
   delete c;
 }
 
+TcPlanCache* gemm_tc_plans(GemmPlanCache* c) { return c ? c->tc : nullptr; }
+
 int* gemm_status_ptr(GemmPlanCache* c) { return c ? tc_status_ptr(c->tc) : nullptr; }
 
 int gemm_default_kind() {

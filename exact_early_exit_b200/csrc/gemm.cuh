@@ -14,6 +14,8 @@ namespace nv {
 enum GemmKind : int { GEMM_SIMT = 0, GEMM_TC = 1 };
 
 struct GemmPlanCache;  // tensor maps keyed by (pointer, shape)
+struct TcPlanCache;
+TcPlanCache* gemm_tc_plans(GemmPlanCache* c);
 GemmPlanCache* gemm_plans_create();
 void gemm_plans_destroy(GemmPlanCache* c);
 

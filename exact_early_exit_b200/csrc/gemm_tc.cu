@@ -61,6 +61,7 @@ struct TcArgs {
   size_t split_stride;
   int* status;
   int fused;             // apply `epi` in-kernel (one K slice only; else store fp32 Y)
+  const int* skip_if_zero;      // when set and *skip_if_zero == 0 the launch does nothing
   const unsigned char* pf_ptr;  // bytes to pull into L2 for the next GEMM (may be null)
   unsigned long long pf_bytes;
   EpiArgs epi;
@@ -219,6 +220,71 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
 #pragma unroll
     for (int j = 0; j < EPI_ROWS; ++j)
       if (hp[j]) *hp[j] = hv[j] + S[j * BM + tid];
+  } else if (e.mode == EPI_HEAD) {
+    // exact sampling at this exit: score_v = logit_v + Gumbel(U_v), U_v from
+    // Philox counter (b, t, 1, v/4) lane v%4; argmax with ties to the lowest
+    // v, and the log-sum-exp of the logits, over this tile's 128 v
+    __shared__ float red[4][HEAD_PART];
+    const unsigned long long seed = *e.seed;
+    const int lane = tid & 31, w = tid >> 5;
+    for (int j = 0; j < nrows; ++j) {
+      const int b = r0 + j;
+      if (!e.stop[b]) continue;  // same b for every thread: uniform
+      const int v = n0 + tid;
+      const float logit = S[j * BM + tid];
+      const uint4 rb = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)e.t[b], STREAM_GUMBEL, (uint32_t)(v >> 2)),
+                                     (uint32_t)seed, (uint32_t)(seed >> 32));
+      float bs = logit - logf(-logf(uniform01(lane_of(rb, v & 3))));
+      int bv = v;
+      float bl = logit, M = logit, Ssum = 1.0f;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float s2 = __shfl_xor_sync(0xffffffffu, bs, o);
+        const int v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+        const float l2 = __shfl_xor_sync(0xffffffffu, bl, o);
+        const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
+        const float S2 = __shfl_xor_sync(0xffffffffu, Ssum, o);
+        if (s2 > bs || (s2 == bs && v2 < bv)) {
+          bs = s2;
+          bv = v2;
+          bl = l2;
+        }
+        const float Mn = fmaxf(M, M2);
+        Ssum = Ssum * expf(M - Mn) + S2 * expf(M2 - Mn);
+        M = Mn;
+      }
+      if (lane == 0) {
+        red[w][0] = bs;
+        red[w][1] = __int_as_float(bv);
+        red[w][2] = bl;
+        red[w][3] = M;
+        red[w][4] = Ssum;
+      }
+      epi_bar();
+      if (tid == 0) {
+        float fs = red[0][0], fl = red[0][2], fM = red[0][3], fS = red[0][4];
+        int fv = __float_as_int(red[0][1]);
+        for (int q = 1; q < 4; ++q) {
+          const float s2 = red[q][0];
+          const int v2 = __float_as_int(red[q][1]);
+          if (s2 > fs || (s2 == fs && v2 < fv)) {
+            fs = s2;
+            fv = v2;
+            fl = red[q][2];
+          }
+          const float Mn = fmaxf(fM, red[q][3]);
+          fS = fS * expf(fM - Mn) + red[q][4] * expf(red[q][3] - Mn);
+          fM = Mn;
+        }
+        float* out = e.head_part + ((size_t)b * e.nblk + n0 / BM) * HEAD_PART;
+        out[0] = fs;
+        out[1] = __int_as_float(fv);
+        out[2] = fl;
+        out[3] = fM;
+        out[4] = fS;
+      }
+      epi_bar();
+    }
   } else if (e.mode == EPI_SWIGLU) {
 #pragma unroll 4
     for (int idx = tid; idx < nrows * (BM / 2); idx += 128) {
@@ -268,7 +334,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   pdl_wait();
   pdl_launch();
   const int R = *a.nrows;
-  if (R <= 0) return;
+  if (R <= 0 || (a.skip_if_zero && *a.skip_if_zero == 0)) return;
   const int nrt = (R + BNMAX - 1) / BNMAX;
   const int splits = tc_split_count(R, a.N, a.K, gridDim.x, a.max_split);
   const int items = ntn * nrt * splits;
@@ -525,7 +591,8 @@ static nv_status make_map(TcPlanCache* c, const void* ptr, uint64_t inner, uint6
 
 nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int N, int K, const int* nrows,
                       int max_rows, float* Y, bool allow_split, const EpiArgs* epi, int* tile_counters,
-                      const void* prefetch, size_t prefetch_bytes, cudaStream_t st, int* grid_out) {
+                      const void* prefetch, size_t prefetch_bytes, cudaStream_t st, int* grid_out,
+                      const int* skip_if_zero) {
   if (N % BM || K % BK || K > ldx) {
     set_error("tcgen05 GEMM needs N % 128 == 0 and K % 64 == 0 (N=" + std::to_string(N) + ", K=" +
               std::to_string(K) + ")");
@@ -536,7 +603,7 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
       set_error("fused tcgen05 epilogue needs one K slice");
       return NV_ERR_UNSUPPORTED;
     }
-    const bool ok = epi->mode == EPI_RESID ||
+    const bool ok = epi->mode == EPI_RESID || epi->mode == EPI_HEAD ||
                     (epi->mode == EPI_QKV && BM % epi->hd == 0 && (epi->H * epi->hd) % BM == 0) ||
                     (epi->mode == EPI_SWIGLU && epi->G == BM / 2);
     if (!ok) {
@@ -562,6 +629,7 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
   a.split_stride = (size_t)BNMAX * N;
   a.status = c->status;
   a.fused = (epi && epi->mode != EPI_STORE) ? 1 : 0;
+  a.skip_if_zero = skip_if_zero;
   a.pf_ptr = (const unsigned char*)prefetch;
   a.pf_bytes = ((uintptr_t)prefetch & 15) ? 0ull : (unsigned long long)prefetch_bytes;
   if (epi) a.epi = *epi;

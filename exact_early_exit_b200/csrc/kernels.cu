@@ -221,27 +221,70 @@ void launch_rmsnorm_rows(bool bf16, RowSet rs, const void* gain, void* act, int 
 }
 
 // Residual update from split-K slices of the output projection, then the MLP
-// RMSNorm, in one pass over each row.
+// RMSNorm.  One CTA per row, one float4 of the row per thread (d <= 4 *
+// blockDim), every slice's load in flight at once; the row stays in
+// registers between the sum of squares and the scaled write.
 template <typename T>
-__global__ void k_resid_norm(RowSet rs, const float* __restrict__ Y, int split_grid, int N, int K,
-                             size_t sstride, const T* __restrict__ g, T* __restrict__ act, int d, float eps) {
+__global__ void __launch_bounds__(512) k_resid_norm(RowSet rs, const float* __restrict__ Y, int split_grid, int N,
+                                                    int K, size_t sstride, const T* __restrict__ g,
+                                                    T* __restrict__ act, int d, float eps) {
   pdl_wait();
   pdl_launch();
+  __shared__ float s_red[16];
   const int R = *rs.nrows;
   const int ns = split_grid ? tc_split_count(R, N, K, split_grid, TC_MAX_SPLIT) : 1;
-  const int wpb = blockDim.x >> 5;
-  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb)
-    warp_norm_row<T>(rs.h + (size_t)rs.row_hrow[r] * d, g, act + (size_t)r * d, d, eps, Y + (size_t)r * N, ns,
-                     sstride);
+  const int nv = d >> 2, j = threadIdx.x;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4* hp = reinterpret_cast<float4*>(rs.h + (size_t)rs.row_hrow[r] * d);
+    if (j < nv) {
+      const float4* yp = reinterpret_cast<const float4*>(Y + (size_t)r * N) + j;
+      float4 v[TC_MAX_SPLIT];
+#pragma unroll
+      for (int sp = 0; sp < TC_MAX_SPLIT; ++sp)
+        v[sp] = sp < ns ? __ldcg(yp + sp * (sstride / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 ys = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int sp = 0; sp < TC_MAX_SPLIT; ++sp) {
+        ys.x += v[sp].x;
+        ys.y += v[sp].y;
+        ys.z += v[sp].z;
+        ys.w += v[sp].w;
+      }
+      x = hp[j];
+      x.x += ys.x;
+      x.y += ys.y;
+      x.z += ys.z;
+      x.w += ys.w;
+      hp[j] = x;
+    }
+    float ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      float t = threadIdx.x < (blockDim.x >> 5) ? s_red[threadIdx.x] : 0.f;
+      t = warp_sum(t);
+      if (threadIdx.x == 0) s_red[0] = t;
+    }
+    __syncthreads();
+    const float inv = 1.0f / sqrtf(s_red[0] / (float)d + eps);
+    __syncthreads();
+    if (j < nv) {
+      const T* gp = g + 4 * j;
+      store4<T>(act + (size_t)r * d + 4 * j, x.x * inv * ld(gp), x.y * inv * ld(gp + 1), x.z * inv * ld(gp + 2),
+                x.w * inv * ld(gp + 3));
+    }
+  }
 }
 void launch_resid_norm(bool bf16, RowSet rs, const float* Y, int split_grid, int N, int K, size_t sstride,
                        const void* gain, void* act, int d, float eps, cudaStream_t st) {
-  int grid = (rs.max_rows + 7) / 8;
-  if (grid > 2048) grid = 2048;
+  int grid = rs.max_rows < 1184 ? rs.max_rows : 1184;
+  const int threads = ((d / 4 + 31) / 32) * 32;
   if (bf16)
-    launch_k(k_resid_norm<__nv_bfloat16>, grid, 256, 0, st, rs, Y, split_grid, N, K, sstride,
+    launch_k(k_resid_norm<__nv_bfloat16>, grid, threads, 0, st, rs, Y, split_grid, N, K, sstride,
              (const __nv_bfloat16*)gain, (__nv_bfloat16*)act, d, eps);
-  else launch_k(k_resid_norm<float>, grid, 256, 0, st, rs, Y, split_grid, N, K, sstride, (const float*)gain,
+  else launch_k(k_resid_norm<float>, grid, threads, 0, st, rs, Y, split_grid, N, K, sstride, (const float*)gain,
                 (float*)act, d, eps);
 }
 
@@ -419,9 +462,17 @@ void launch_gemm_simt(bool bf16, const void* X, int ldx, const void* W, int N, i
 //   EPI_SWIGLU: u = silu(gate) * up, gate/up interleaved in blocks of G rows.
 //   EPI_STORE:  out = y.
 // ---------------------------------------------------------------------------
+// Sum of the split-K slices of one output, in slice order.  All loads are
+// issued before the first add (the slices sit in L2; a dependent chain of
+// loads would serialise their latency).
 __device__ __forceinline__ float epi_sum(const EpiArgs& a, int ns, int r, int n) {
+  const float* p = a.Y + (size_t)r * a.N + n;
+  float v[TC_MAX_SPLIT];
+#pragma unroll
+  for (int s = 0; s < TC_MAX_SPLIT; ++s) v[s] = s < ns ? __ldcg(p + s * a.split_stride) : 0.f;
   float y = 0.f;
-  for (int s = 0; s < ns; ++s) y += a.Y[s * a.split_stride + (size_t)r * a.N + n];
+#pragma unroll
+  for (int s = 0; s < TC_MAX_SPLIT; ++s) y += v[s];
   return y;
 }
 
@@ -657,10 +708,10 @@ __global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
   pdl_wait();
   pdl_launch();
   static_assert(HD * sizeof(T) == 128, "128-byte rows");
-  constexpr int NW = 4, KPL = DEC_CK / 32, DPL = HD / 32, EPC = 16 / sizeof(T);
+  constexpr int NW = 4, DPL = HD / 32, EPC = 16 / sizeof(T);
+  static_assert(NW * 32 == DEC_CK, "one key per thread");
   __shared__ __align__(128) T Ks[DEC_CK * HD];
   __shared__ __align__(128) T Vs[DEC_CK * HD];
-  __shared__ float Qs[NW][HD];
   __shared__ __align__(8) uint64_t bar;
   const int b = blockIdx.x, head = blockIdx.y, chunk = blockIdx.z;
   if (*a.rs.nrows == 0) return;
@@ -719,63 +770,82 @@ __global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H;
   const T* qg = (const T*)a.q;
-  // rows of b whose position reaches this chunk: positions are contiguous
+  // rows of b whose position reaches this chunk: positions are contiguous.
+  // Each row uses the whole CTA: warp w takes keys [32w, 32w+32) of the
+  // chunk (one key per lane), then the four warps' softmax states merge.
   const int pos0 = a.rs.row_pos[s0];
   const int first = max(s0, s0 + (k0 - pos0));
-  for (int r = first + w; r < s1; r += NW) {
+  __shared__ float Qrow[HD];
+  __shared__ float Wst[NW][HD + 2];
+  const int kk = 32 * w + lane;
+  const uint4* krow = (const uint4*)(Ks + kk * HD);
+  for (int r = first; r < s1; ++r) {
     const int p = pos0 + (r - s0);
-    for (int dd = lane; dd < HD; dd += 32) Qs[w][dd] = ld(qg + (size_t)r * H * HD + head * HD + dd);
-    __syncwarp();
-    float sc[KPL];
-    float mx = -CUDART_INF_F;
-#pragma unroll
-    for (int j = 0; j < KPL; ++j) {
-      const int kk = lane + 32 * j;
+    if (threadIdx.x < HD) Qrow[threadIdx.x] = ld(qg + (size_t)r * H * HD + head * HD + threadIdx.x);
+    __syncthreads();
+    float sc = -CUDART_INF_F;
+    if (kk < nk && k0 + kk <= p) {
       float acc = 0.f;
-      const uint4* krow = (const uint4*)(Ks + kk * HD);
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
         const int c = (c8 + lane) & 7;
         const uint4 kv4 = krow[c];
         const T* kp = (const T*)&kv4;
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) acc = fmaf(Qs[w][c * EPC + e], ld(kp + e), acc);
+        for (int e = 0; e < EPC; ++e) acc = fmaf(Qrow[c * EPC + e], ld(kp + e), acc);
       }
-      sc[j] = (kk < nk && k0 + kk <= p) ? acc * a.scale : -CUDART_INF_F;
-      mx = fmaxf(mx, sc[j]);
+      sc = acc * a.scale;
     }
-    mx = warp_max(mx);
-    float l = 0.f;
-#pragma unroll
-    for (int j = 0; j < KPL; ++j) {
-      sc[j] = expf(sc[j] - mx);
-      l += sc[j];
-    }
-    l = warp_sum(l);
+    const float mw = warp_max(sc);
     float o[DPL];
 #pragma unroll
     for (int d = 0; d < DPL; ++d) o[d] = 0.f;
-#pragma unroll
-    for (int j = 0; j < KPL; ++j) {
-      const int kbase = 32 * j;
-      if (kbase >= nk) break;
+    float lw = 0.f;
+    if (mw != -CUDART_INF_F) {  // this warp's keys reach the row
+      const float pk = expf(sc - mw);
+      lw = warp_sum(pk);
+      const int kmax = min(32, min(nk, p + 1 - k0) - 32 * w);
 #pragma unroll 8
       for (int src = 0; src < 32; ++src) {
-        const float pw = __shfl_sync(0xffffffffu, sc[j], src);
-        if (kbase + src >= nk) break;  // rows past the chunk's keys hold stale data
-        const T* vrow = Vs + (kbase + src) * HD + lane * DPL;
+        const float pw = __shfl_sync(0xffffffffu, pk, src);
+        if (src >= kmax) break;  // rows past the row's keys hold stale data
+        const T* vrow = Vs + (32 * w + src) * HD + lane * DPL;
 #pragma unroll
         for (int d = 0; d < DPL; ++d) o[d] = fmaf(pw, ld(vrow + d), o[d]);
       }
     }
-    float* pp = a.part + (((size_t)r * H + head) * a.kv_splits + chunk) * (HD + 2);
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) pp[lane * DPL + d] = o[d];
+    for (int d = 0; d < DPL; ++d) Wst[w][lane * DPL + d] = o[d];
     if (lane == 0) {
-      pp[HD] = mx;
-      pp[HD + 1] = l;
+      Wst[w][HD] = mw;
+      Wst[w][HD + 1] = lw;
     }
-    __syncwarp();
+    __syncthreads();
+    if (w == 0) {
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int q = 0; q < NW; ++q) M = fmaxf(M, Wst[q][HD]);
+      float L = 0.f, acc[DPL];
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+#pragma unroll
+      for (int q = 0; q < NW; ++q) {
+        const float mq = Wst[q][HD];
+        if (mq == -CUDART_INF_F) continue;
+        const float e = expf(mq - M);
+        L += Wst[q][HD + 1] * e;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) acc[d] += Wst[q][lane * DPL + d] * e;
+      }
+      float* pp = a.part + (((size_t)r * H + head) * a.kv_splits + chunk) * (HD + 2);
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) pp[lane * DPL + d] = acc[d];
+      if (lane == 0) {
+        pp[HD] = M;
+        pp[HD + 1] = L;
+      }
+    }
+    __syncthreads();
   }
   if (a.lens && head == 0 && chunk == 0 && threadIdx.x == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
 }
@@ -860,7 +930,10 @@ __global__ void k_step_begin(StepArgs a) {
     a.force[b] = f;
     if (f && a.counters) atomicAdd((unsigned long long*)&a.counters[NV_CTR_FORCED], 1ull);
     for (int k = 0; k < a.n_exits; ++k) a.stop[k * a.B + b] = 0;
-    if (b == 0) *a.seed_dev = a.seed;
+    if (b == 0) {
+      *a.seed_dev = a.seed;
+      for (int k = 0; k < a.n_exits; ++k) a.nstop[k] = 0;
+    }
   }
   const T* e = (const T*)a.emb + (size_t)a.tok[b] * a.d;
   float* h = a.hbuf + ((size_t)b * a.cap + tb % a.cap) * a.d;
@@ -931,7 +1004,11 @@ __global__ void __launch_bounds__(256) k_junction(JuncArgs a) {
       a.active[b] = 0;
       a.exit_id[b] = a.k + 1;
       a.stop[b] = 1;
-      if (a.counters) atomicAdd((unsigned long long*)&a.counters[NV_CTR_EXIT0 + a.k], 1ull);
+      const int before = atomicAdd(a.nstop, 1);
+      if (a.counters) {
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_EXIT0 + a.k], 1ull);
+        if (before == 0) atomicAdd((unsigned long long*)&a.counters[NV_CTR_HEAD_BYTES], (unsigned long long)a.head_bytes);
+      }
     }
   }
 }
@@ -974,8 +1051,6 @@ __global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
   }
   __syncthreads();
   if (n == 0) return;
-  if (blockIdx.x == 0 && tid == 0 && a.counters)
-    atomicAdd((unsigned long long*)&a.counters[NV_CTR_HEAD_BYTES], (unsigned long long)a.head_bytes);
   const unsigned long long seed = *a.seed;
   const int d = a.d, V = a.V;
   const int nchunk = d / EPC;  // 16-byte chunks per row

@@ -66,6 +66,13 @@ struct EpiArgs {
   void* u_out;           // [max_rows][F]
   // EPI_STORE
   float* out;
+  // EPI_HEAD: rows are sequences b; logits of vocabulary tile n0/128 give one
+  // Gumbel-argmax / log-sum-exp partial per stopped sequence
+  const int* stop;                 // [B] stopped at this exit
+  const int* t;                    // [B] position of the token being processed
+  const unsigned long long* seed;  // Philox key
+  float* head_part;                // [B][nblk][HEAD_PART]
+  int nblk;
 };
 void launch_epilogue(bool bf16, const EpiArgs& a, int grid, cudaStream_t st);
 
@@ -97,6 +104,7 @@ struct StepArgs {
   int* exit_id;
   int* force;
   int* stop;             // [n_exits][B]
+  int* nstop;            // [n_exits]
   const int* lens;
   float* hbuf;
   const void* emb;
@@ -125,6 +133,8 @@ struct JuncArgs {
   void* exit_act;        // [B][d]
   const unsigned long long* seed;
   long long* counters;
+  int* nstop;            // stops at this exit in this step (zeroed at step begin)
+  long long head_bytes;  // counted once per exit that has a stop
 };
 void launch_junction(bool bf16, const JuncArgs& a, cudaStream_t st);
 

@@ -99,6 +99,8 @@ struct nv_state {
   // per-sequence device state
   int *t = nullptr, *tok = nullptr, *lens = nullptr, *active = nullptr, *exit_id = nullptr, *force = nullptr;
   int *stop = nullptr, *sampled = nullptr, *out_tok = nullptr, *out_exit = nullptr;
+  int *nstop = nullptr, *d_B = nullptr;
+  bool tc_head = false;  // exit heads on tensor cores (bf16, B >= 16)
   int *prompt_len = nullptr, *prompt_last = nullptr;
   float* logp = nullptr;
   float* hbuf = nullptr;
@@ -416,6 +418,8 @@ nv_status record_step(nv_state* s, cudaStream_t st, Prof* prof = nullptr) {
       j.exit_act = s->exit_act;
       j.seed = s->seed_dev;
       j.counters = s->counters;
+      j.nstop = s->nstop + k;
+      j.head_bytes = (long long)M->V * M->d * es;
       timed(prof, launches, 1, NV_K_JUNCTION, (long long)s->B * M->d * (4 + es), 0,
             [&] { launch_junction(bf, j, st); });
       HeadArgs h{};
@@ -445,10 +449,28 @@ nv_status record_step(nv_state* s, cudaStream_t st, Prof* prof = nullptr) {
         if (n) hb = h.head_bytes + n * M->d * es;
         hf = 2 * n * (long long)M->V * M->d;
       }
+      nv_status hst = NV_OK;
       timed(prof, launches, 2, NV_K_HEAD, hb, hf, [&] {
-        launch_head_sample(bf, h, st);
+        if (s->tc_head) {
+          // tensor-core head over every sequence's exit state; columns of
+          // sequences that did not stop here are ignored, and nothing runs
+          // when no sequence stopped here
+          EpiArgs he{};
+          he.mode = EPI_HEAD;
+          he.stop = j.stop;
+          he.t = s->t;
+          he.seed = s->seed_dev;
+          he.head_part = s->head_part;
+          he.nblk = M->V / 128;
+          hst = tc_gemm_run(gemm_tc_plans(M->gemm_plans), s->exit_act, M->d, M->exits[k].head, M->V, M->d, s->d_B,
+                            s->B, s->Y, false, &he, nullptr, nullptr, 0, st, nullptr, s->nstop + k);
+          h.nblk = M->V / 128;
+        } else {
+          launch_head_sample(bf, h, st);
+        }
         launch_head_reduce(h, st);
       });
+      NV_TRY(hst);
     }
   }
   StepArgs sa{};
@@ -761,6 +783,8 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
     A((void**)p, (size_t)B * 4);
   A((void**)&s->lens, (size_t)B * M->L * 4);
   A((void**)&s->stop, (size_t)B * M->NE * 4);
+  A((void**)&s->nstop, (size_t)NV_MAX_EXITS * 4);
+  A((void**)&s->d_B, 4);
   A((void**)&s->logp, (size_t)B * 4);
   A((void**)&s->hbuf, (size_t)B * s->cap * d * 4);
   for (int** p : {&s->row_b, &s->row_pos, &s->row_hrow}) A((void**)p, (size_t)s->max_rows * 4);
@@ -784,6 +808,9 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   }
   cudaMemset(s->counters, 0, NV_CTR_COUNT * 8);
   cudaMemset(s->tile_counters, 0, (size_t)kTileCounters * 4);
+  cudaMemset(s->nstop, 0, (size_t)NV_MAX_EXITS * 4);
+  cudaMemcpy(s->d_B, &B, 4, cudaMemcpyHostToDevice);
+  s->tc_head = M->bf16 && M->gemm_kind == GEMM_TC && B >= 16 && M->V % 128 == 0 && M->d % 64 == 0;
   cudaMemset(s->status, 0, 4);
   cudaMemset(s->nrows, 0, 4);
   cudaMemset(s->lens, 0, (size_t)B * M->L * 4);
@@ -1000,6 +1027,7 @@ nv_status decode_step_impl(nv_state* s, uint64_t seed, int32_t* tokens_out, int3
   sa.exit_id = s->exit_id;
   sa.force = s->force;
   sa.stop = s->stop;
+  sa.nstop = s->nstop;
   sa.lens = s->lens;
   sa.hbuf = s->hbuf;
   sa.emb = M->tok_emb;

@@ -75,3 +75,42 @@ def test_prefill_kv_matches_oracle(weights):
             assert n == lens[b] - 1
             kv_close(K, dec.caches[b].K[m][:n], CFG)
             kv_close(V, dec.caches[b].V[m][:n], CFG)
+
+
+def test_decode_parity_b16_tensor_core_head(weights):
+    """16 sequences: the exit heads run as tcgen05 GEMMs with the sampling
+    epilogue (Gumbel-max and log-sum-exp per 128-token tile)."""
+    wl = W.WORKLOADS["S"]
+    rng = np.random.default_rng(12)
+    prompts = [p[:int(n)] for p, n in zip(W.make_prompts(wl, seed=6), rng.integers(3, 40, size=16))]
+    chk, state, dec, _ = run_decode_parity(nv, CFG, weights, prompts, 8)
+    print(f"b16 near ties: exits {chk.exit_ties} tokens {chk.token_ties}, max logp err {chk.max_logp_err:.2e}")
+    assert chk.steps == 8
+
+
+def test_sampler_chi_square_bf16_tensor_core_head():
+    """Exact sampling through the tensor-core head: 4096 copies of one
+    context on a 2-layer bf16 model (vocab 1024), 50 seeds; joint (exit,
+    token) frequencies against p_k * pi_k(v) from the oracle."""
+    from tests.nvium_testlib import chisq_pvalue
+    mini = W.ModelConfig("mini-bf16", 2, 256, 4, 64, 512, 1024, (1, 2), W.BF16)
+    w = W.make_weights(mini, seed=3, router_bias=[0.3])
+    prompt = W.zipf_ids(6, mini.vocab, np.random.default_rng(2))
+    B = 4096
+    model = nv.Model(mini, w, max_batch=B, max_seq=16, max_pending=4)
+    st = nv.State(model, B)
+    st.prefill(np.tile(prompt, B).astype(np.int32), np.full(B, len(prompt), np.int32))
+    counts = np.zeros((2, mini.vocab))
+    tok = np.zeros(B, np.int32)
+    ex = np.zeros(B, np.int32)
+    for s in range(50):
+        st.decode_step(2000 + s, tok, ex)
+        np.add.at(counts, (ex - 1, tok), 1)
+        st.rewind()
+    om = O.OracleModel(mini, w)
+    _, states, _ = om.forward_sequence(prompt)
+    t = len(prompt) - 1
+    p, pi = O.step_distribution(om, [states[k][t:t + 1] for k in range(2)])
+    n = counts.sum()
+    assert chisq_pvalue(counts, p[:, None] * pi * n) > 0.01
+    assert chisq_pvalue(counts.sum(1), p * n) > 0.01
