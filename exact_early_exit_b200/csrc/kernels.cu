@@ -698,9 +698,41 @@ __global__ void k_attn_combine(AttnArgs a) {
 // Rows of 128 bytes (HD * sizeof(T) == 128) only.
 // ---------------------------------------------------------------------------
 constexpr int DEC_CK = 128;  // keys per chunk (two 64-position pages)
+constexpr int DEC_RG = 8;    // rows per register group in k_attn_dec
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Bounded wait of the whole CTA on an mbarrier phase.  Every thread polls;
+// only thread 0 decides that 2 s have passed and says so through `abort`, so
+// all threads leave together (after the closing barrier) either way.
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
+  unsigned long long t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (ok) break;
+    if ((i & 63u) == 0u) {
+      if (threadIdx.x == 0) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (i == 0) t0 = t;
+        else if (t - t0 > 2000000000ull) *abort = 1;
+      }
+      if (*abort) break;
+    }
+  }
+  __syncthreads();
+  if (*abort) {
+    if (threadIdx.x == 0) dev_fail(status, DEV_ERR_TIMEOUT);
+    return false;
+  }
+  return true;
 }
 
 template <typename T, int HD>
@@ -713,6 +745,7 @@ __global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
   __shared__ __align__(128) T Ks[DEC_CK * HD];
   __shared__ __align__(128) T Vs[DEC_CK * HD];
   __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_abort;
   const int b = blockIdx.x, head = blockIdx.y, chunk = blockIdx.z;
   if (*a.rs.nrows == 0) return;
   const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
@@ -725,6 +758,7 @@ __global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
   const uint32_t bytes_per_page = (uint32_t)(a.kv.page_size * HD * sizeof(T));
   const T* kvb = (const T*)a.kv.base;
   if (threadIdx.x == 0) {
+    s_abort = 0;
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bar)) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&bar)),
@@ -747,97 +781,88 @@ __global__ void __launch_bounds__(128) k_attn_dec(AttnArgs a) {
     }
   }
   __syncthreads();
-  // bounded wait (2 s) for the copies
-  {
-    uint32_t ok = 0;
-    unsigned long long t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-          : "=r"(ok)
-          : "r"(smem_addr(&bar))
-          : "memory");
-      if (ok) break;
-      unsigned long long t;
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-      if (i == 0) t0 = t;
-      else if (t - t0 > 2000000000ull) {
-        if (threadIdx.x == 0) dev_fail(a.status, DEV_ERR_TIMEOUT);
-        return;
-      }
-    }
-  }
+  if (!bounded_wait(&bar, 0, &s_abort, a.status)) return;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H;
   const T* qg = (const T*)a.q;
   // rows of b whose position reaches this chunk: positions are contiguous.
-  // Each row uses the whole CTA: warp w takes keys [32w, 32w+32) of the
-  // chunk (one key per lane), then the four warps' softmax states merge.
+  // Warp w takes keys [32w, 32w+32) of the chunk (one key per lane) for up to
+  // DEC_RG rows at a time, keeping each row's softmax state in registers;
+  // the four warps merge once per row group.
   const int pos0 = a.rs.row_pos[s0];
   const int first = max(s0, s0 + (k0 - pos0));
-  __shared__ float Qrow[HD];
-  __shared__ float Wst[NW][HD + 2];
+  __shared__ float Qr[DEC_RG][HD];
+  __shared__ float Wst[NW][DEC_RG][HD + 2];
   const int kk = 32 * w + lane;
   const uint4* krow = (const uint4*)(Ks + kk * HD);
-  for (int r = first; r < s1; ++r) {
-    const int p = pos0 + (r - s0);
-    if (threadIdx.x < HD) Qrow[threadIdx.x] = ld(qg + (size_t)r * H * HD + head * HD + threadIdx.x);
+  for (int g0 = first; g0 < s1; g0 += DEC_RG) {
+    const int ng = min(DEC_RG, s1 - g0);
+    for (int i = threadIdx.x; i < ng * HD; i += blockDim.x)
+      Qr[i / HD][i % HD] = ld(qg + (size_t)(g0 + i / HD) * H * HD + head * HD + i % HD);
     __syncthreads();
-    float sc = -CUDART_INF_F;
-    if (kk < nk && k0 + kk <= p) {
-      float acc = 0.f;
+    // this lane's key, once, as eight 16-byte chunks read in a per-lane
+    // rotated order (conflict-free); kc[c8] holds chunk (c8 + lane) % 8
+    uint4 kc[8];
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const int c = (c8 + lane) & 7;
-        const uint4 kv4 = krow[c];
-        const T* kp = (const T*)&kv4;
+    for (int c8 = 0; c8 < 8; ++c8) kc[c8] = krow[(c8 + lane) & 7];
+#pragma unroll 1
+    for (int j = 0; j < ng; ++j) {
+      const int p = pos0 + (g0 + j - s0);
+      float sc = -CUDART_INF_F;
+      if (kk < nk && k0 + kk <= p) {
+        float acc = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) acc = fmaf(Qrow[c * EPC + e], ld(kp + e), acc);
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const float* qc = &Qr[j][((c8 + lane) & 7) * EPC];
+          const T* kp = (const T*)&kc[c8];
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) acc = fmaf(qc[e], ld(kp + e), acc);
+        }
+        sc = acc * a.scale;
       }
-      sc = acc * a.scale;
-    }
-    const float mw = warp_max(sc);
-    float o[DPL];
+      const float mw = warp_max(sc);
+      float o[DPL];
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) o[d] = 0.f;
-    float lw = 0.f;
-    if (mw != -CUDART_INF_F) {  // this warp's keys reach the row
-      const float pk = expf(sc - mw);
-      lw = warp_sum(pk);
-      const int kmax = min(32, min(nk, p + 1 - k0) - 32 * w);
+      for (int d = 0; d < DPL; ++d) o[d] = 0.f;
+      float lw = 0.f;
+      if (mw != -CUDART_INF_F) {
+        const float pk = expf(sc - mw);
+        lw = warp_sum(pk);
+        const int kmax = min(32, min(nk, p + 1 - k0) - 32 * w);
 #pragma unroll 8
-      for (int src = 0; src < 32; ++src) {
-        const float pw = __shfl_sync(0xffffffffu, pk, src);
-        if (src >= kmax) break;  // rows past the row's keys hold stale data
-        const T* vrow = Vs + (32 * w + src) * HD + lane * DPL;
+        for (int src = 0; src < 32; ++src) {
+          const float pw = __shfl_sync(0xffffffffu, pk, src);
+          if (src >= kmax) break;  // rows past the row's keys hold stale data
+          const T* vrow = Vs + (32 * w + src) * HD + lane * DPL;
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) o[d] = fmaf(pw, ld(vrow + d), o[d]);
+          for (int d = 0; d < DPL; ++d) o[d] = fmaf(pw, ld(vrow + d), o[d]);
+        }
+      }
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) Wst[w][j][lane * DPL + d] = o[d];
+      if (lane == 0) {
+        Wst[w][j][HD] = mw;
+        Wst[w][j][HD + 1] = lw;
       }
     }
-#pragma unroll
-    for (int d = 0; d < DPL; ++d) Wst[w][lane * DPL + d] = o[d];
-    if (lane == 0) {
-      Wst[w][HD] = mw;
-      Wst[w][HD + 1] = lw;
-    }
     __syncthreads();
-    if (w == 0) {
+    for (int j = w; j < ng; j += NW) {
       float M = -CUDART_INF_F;
 #pragma unroll
-      for (int q = 0; q < NW; ++q) M = fmaxf(M, Wst[q][HD]);
+      for (int q = 0; q < NW; ++q) M = fmaxf(M, Wst[q][j][HD]);
       float L = 0.f, acc[DPL];
 #pragma unroll
       for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
 #pragma unroll
       for (int q = 0; q < NW; ++q) {
-        const float mq = Wst[q][HD];
+        const float mq = Wst[q][j][HD];
         if (mq == -CUDART_INF_F) continue;
         const float e = expf(mq - M);
-        L += Wst[q][HD + 1] * e;
+        L += Wst[q][j][HD + 1] * e;
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) acc[d] += Wst[q][lane * DPL + d] * e;
+        for (int d = 0; d < DPL; ++d) acc[d] += Wst[q][j][lane * DPL + d] * e;
       }
-      float* pp = a.part + (((size_t)r * H + head) * a.kv_splits + chunk) * (HD + 2);
+      float* pp = a.part + (((size_t)(g0 + j) * H + head) * a.kv_splits + chunk) * (HD + 2);
 #pragma unroll
       for (int d = 0; d < DPL; ++d) pp[lane * DPL + d] = acc[d];
       if (lane == 0) {
@@ -1339,6 +1364,27 @@ __global__ void k_philox(unsigned long long seed, const uint4* ctr, int n, uint4
 }
 void launch_philox(unsigned long long seed, const void* ctr, int n, void* out, cudaStream_t st) {
   launch_k(k_philox, (n + 255) / 256, 256, 0, st, seed, (const uint4*)ctr, n, (uint4*)out);
+}
+
+// Sets a graph conditional to "some sequence still active or forced to
+// complete its deferred rows"; when set, counts the launches of the block it
+// guards.
+__global__ void k_set_cond(cudaGraphConditionalHandle h, const int* __restrict__ active,
+                           const int* __restrict__ force, int B, long long* counters, const int* block_launches) {
+  pdl_wait();
+  pdl_launch();
+  int any = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) any |= active[b] | force[b];
+  any = __syncthreads_or(any);
+  if (threadIdx.x == 0) {
+    cudaGraphSetConditional(h, any ? 1u : 0u);
+    if (any && counters)
+      atomicAdd((unsigned long long*)&counters[NV_CTR_LAUNCHES], (unsigned long long)*block_launches);
+  }
+}
+void launch_set_cond(cudaGraphConditionalHandle h, const int* active, const int* force, int B, long long* counters,
+                     const int* block_launches, cudaStream_t st) {
+  launch_k(k_set_cond, 1, 256, 0, st, h, active, force, B, counters, block_launches);
 }
 
 cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes) {

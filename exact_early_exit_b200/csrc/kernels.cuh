@@ -161,6 +161,10 @@ void launch_exit_rows(bool bf16, RowSet rs, const void* norm, const void* router
                       int n_exits, void* act, float* z, int d, float eps, cudaStream_t st);
 void launch_lse_target(const float* Y, int r_begin, int n, int V, const int* target, float* logpi, int k,
                        int n_exits, cudaStream_t st);
+// Sets conditional `h` to (any active[b] or force[b]); when set, adds
+// *block_launches to counters[NV_CTR_LAUNCHES].
+void launch_set_cond(cudaGraphConditionalHandle h, const int* active, const int* force, int B, long long* counters,
+                     const int* block_launches, cudaStream_t st);
 void launch_philox(unsigned long long seed, const void* ctr, int n, void* out, cudaStream_t st);
 
 // Opt-in shared memory for the head sampler and the planner.

@@ -99,7 +99,7 @@ struct nv_state {
   // per-sequence device state
   int *t = nullptr, *tok = nullptr, *lens = nullptr, *active = nullptr, *exit_id = nullptr, *force = nullptr;
   int *stop = nullptr, *sampled = nullptr, *out_tok = nullptr, *out_exit = nullptr;
-  int *nstop = nullptr, *d_B = nullptr;
+  int *nstop = nullptr, *d_B = nullptr, *d_block_launches = nullptr;
   bool tc_head = false;  // exit heads on tensor cores (bf16, B >= 16)
   int *prompt_len = nullptr, *prompt_last = nullptr;
   float* logp = nullptr;
@@ -120,7 +120,9 @@ struct nv_state {
   long long launches_per_step = 0, launches_total = 0;
   bool prefilled = false;
   cudaGraphExec_t graph = nullptr;
-  cudaStream_t cap_stream = nullptr;
+  cudaStream_t cap_stream = nullptr, cap_stream2 = nullptr;
+  long long block_launches[NV_MAX_EXITS] = {0};
+  bool cond_graph = false;
   std::vector<void*> allocs;
   // prefill scratch
   Buf pf_rows, pf_h, pf_tok;
@@ -378,16 +380,14 @@ nv_status prof_read_plan(nv_state* s, Prof* prof, cudaStream_t st) {
   return NV_OK;
 }
 
-// Launches of one decode step after step_begin: captured into a graph, or
-// launched directly with per-kernel events when `prof` is set.
-nv_status record_step(nv_state* s, cudaStream_t st, Prof* prof = nullptr) {
+// Layers [l0, l1) of a decode step, with the junction and exit head at every
+// exit layer among them.
+nv_status record_layers(nv_state* s, cudaStream_t st, Prof* prof, long long* launches, int l0, int l1) {
   nv_model* M = s->m;
   const bool bf = M->bf16;
   const long long es = (long long)M->esz;
-  long long* launches = &s->launches_per_step;
-  *launches = 1;  // step_begin, launched outside the graph
   LayerIO io = state_io(s);
-  for (int layer = 0; layer < M->L; ++layer) {
+  for (int layer = l0; layer < l1; ++layer) {
     PlanArgs p = state_plan(s, layer, 0);
     timed(prof, launches, 1, NV_K_PLAN_NORM, 0, 0, [&] {
       launch_plan_norm(bf, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
@@ -398,81 +398,84 @@ nv_status record_step(nv_state* s, cudaStream_t st, Prof* prof = nullptr) {
     }
     NV_TRY(layer_body(M, layer, io, st, prof, launches));
     const int k = M->exit_at[layer];
-    if (k >= 0) {
-      JuncArgs j{};
-      j.B = s->B;
-      j.cap = s->cap;
-      j.d = M->d;
-      j.k = k;
-      j.n_exits = M->NE;
-      j.router_mode = M->cfg.router_mode;
-      j.eps = M->cfg.rms_eps;
-      j.t = s->t;
-      j.active = s->active;
-      j.exit_id = s->exit_id;
-      j.stop = s->stop + (size_t)k * s->B;
-      j.hbuf = s->hbuf;
-      j.norm = M->exits[k].norm;
-      j.router_w = M->exits[k].router_w;
-      j.router_b = M->exits[k].router_b;
-      j.exit_act = s->exit_act;
-      j.seed = s->seed_dev;
-      j.counters = s->counters;
-      j.nstop = s->nstop + k;
-      j.head_bytes = (long long)M->V * M->d * es;
-      timed(prof, launches, 1, NV_K_JUNCTION, (long long)s->B * M->d * (4 + es), 0,
-            [&] { launch_junction(bf, j, st); });
-      HeadArgs h{};
-      h.B = s->B;
-      h.d = M->d;
-      h.V = M->V;
-      h.k = k;
-      h.t = s->t;
-      h.stop = j.stop;
-      h.exit_act = s->exit_act;
-      h.head = M->exits[k].head;
-      h.seed = s->seed_dev;
-      h.part = s->head_part;
-      h.nblk = s->head_nblk;
-      h.counters = s->counters;
-      h.head_bytes = (long long)M->V * M->d * es;
-      h.sampled = s->sampled;
-      h.logp = s->logp;
-      long long hb = 0, hf = 0;
-      if (prof) {
-        // rows that stop at this exit: known once the junction has run
-        NV_CUDA_TRY(cudaStreamSynchronize(st));
-        std::vector<int> stop(s->B);
-        NV_CUDA_TRY(cudaMemcpy(stop.data(), j.stop, s->B * 4, cudaMemcpyDeviceToHost));
-        long long n = 0;
-        for (int v : stop) n += v;
-        if (n) hb = h.head_bytes + n * M->d * es;
-        hf = 2 * n * (long long)M->V * M->d;
-      }
-      nv_status hst = NV_OK;
-      timed(prof, launches, 2, NV_K_HEAD, hb, hf, [&] {
-        if (s->tc_head) {
-          // tensor-core head over every sequence's exit state; columns of
-          // sequences that did not stop here are ignored, and nothing runs
-          // when no sequence stopped here
-          EpiArgs he{};
-          he.mode = EPI_HEAD;
-          he.stop = j.stop;
-          he.t = s->t;
-          he.seed = s->seed_dev;
-          he.head_part = s->head_part;
-          he.nblk = M->V / 128;
-          hst = tc_gemm_run(gemm_tc_plans(M->gemm_plans), s->exit_act, M->d, M->exits[k].head, M->V, M->d, s->d_B,
-                            s->B, s->Y, false, &he, nullptr, nullptr, 0, st, nullptr, s->nstop + k);
-          h.nblk = M->V / 128;
-        } else {
-          launch_head_sample(bf, h, st);
-        }
-        launch_head_reduce(h, st);
-      });
-      NV_TRY(hst);
+    if (k < 0) continue;
+    JuncArgs j{};
+    j.B = s->B;
+    j.cap = s->cap;
+    j.d = M->d;
+    j.k = k;
+    j.n_exits = M->NE;
+    j.router_mode = M->cfg.router_mode;
+    j.eps = M->cfg.rms_eps;
+    j.t = s->t;
+    j.active = s->active;
+    j.exit_id = s->exit_id;
+    j.stop = s->stop + (size_t)k * s->B;
+    j.hbuf = s->hbuf;
+    j.norm = M->exits[k].norm;
+    j.router_w = M->exits[k].router_w;
+    j.router_b = M->exits[k].router_b;
+    j.exit_act = s->exit_act;
+    j.seed = s->seed_dev;
+    j.counters = s->counters;
+    j.nstop = s->nstop + k;
+    j.head_bytes = (long long)M->V * M->d * es;
+    timed(prof, launches, 1, NV_K_JUNCTION, (long long)s->B * M->d * (4 + es), 0,
+          [&] { launch_junction(bf, j, st); });
+    HeadArgs h{};
+    h.B = s->B;
+    h.d = M->d;
+    h.V = M->V;
+    h.k = k;
+    h.t = s->t;
+    h.stop = j.stop;
+    h.exit_act = s->exit_act;
+    h.head = M->exits[k].head;
+    h.seed = s->seed_dev;
+    h.part = s->head_part;
+    h.nblk = s->head_nblk;
+    h.counters = s->counters;
+    h.head_bytes = (long long)M->V * M->d * es;
+    h.sampled = s->sampled;
+    h.logp = s->logp;
+    long long hb = 0, hf = 0;
+    if (prof) {
+      // rows that stop at this exit: known once the junction has run
+      NV_CUDA_TRY(cudaStreamSynchronize(st));
+      std::vector<int> stop(s->B);
+      NV_CUDA_TRY(cudaMemcpy(stop.data(), j.stop, s->B * 4, cudaMemcpyDeviceToHost));
+      long long n = 0;
+      for (int v : stop) n += v;
+      if (n) hb = h.head_bytes + n * M->d * es;
+      hf = 2 * n * (long long)M->V * M->d;
     }
+    nv_status hst = NV_OK;
+    timed(prof, launches, 2, NV_K_HEAD, hb, hf, [&] {
+      if (s->tc_head) {
+        // tensor-core head over every sequence's exit state; columns of
+        // sequences that did not stop here are ignored, and nothing runs
+        // when no sequence stopped here
+        EpiArgs he{};
+        he.mode = EPI_HEAD;
+        he.stop = j.stop;
+        he.t = s->t;
+        he.seed = s->seed_dev;
+        he.head_part = s->head_part;
+        he.nblk = M->V / 128;
+        hst = tc_gemm_run(gemm_tc_plans(M->gemm_plans), s->exit_act, M->d, M->exits[k].head, M->V, M->d, s->d_B,
+                          s->B, s->Y, false, &he, nullptr, nullptr, 0, st, nullptr, s->nstop + k);
+        h.nblk = M->V / 128;
+      } else {
+        launch_head_sample(bf, h, st);
+      }
+      launch_head_reduce(h, st);
+    });
+    NV_TRY(hst);
   }
+  return NV_OK;
+}
+
+void record_step_end(nv_state* s, cudaStream_t st, Prof* prof, long long* launches) {
   StepArgs sa{};
   sa.B = s->B;
   sa.t = s->t;
@@ -483,6 +486,104 @@ nv_status record_step(nv_state* s, cudaStream_t st, Prof* prof = nullptr) {
   sa.out_tok = s->out_tok;
   sa.out_exit = s->out_exit;
   timed(prof, launches, 1, NV_K_STEP, 0, 0, [&] { launch_step_end(sa, st); });
+}
+
+// Launches of one decode step after step_begin, all layers in order: the
+// profiled path (each launch bracketed by events) and the flat graph.
+nv_status record_step(nv_state* s, cudaStream_t st, Prof* prof = nullptr) {
+  long long* launches = &s->launches_per_step;
+  *launches = 1;  // step_begin, launched outside the graph
+  NV_TRY(record_layers(s, st, prof, launches, 0, s->m->L));
+  record_step_end(s, st, prof, launches);
+  return NV_OK;
+}
+
+// The decode-step graph with the layers between two exits in a conditional
+// node: a block runs only if some sequence is still active after the
+// previous junction (or must complete its deferred rows), so layers that no
+// token reaches cost no launches.  Host-side launch count: the unconditional
+// part; each block that runs adds its own count on the device.
+nv_status build_conditional_step_graph(nv_state* s, cudaGraph_t* out) {
+  nv_model* M = s->m;
+  cudaGraph_t g = nullptr;
+  NV_CUDA_TRY(cudaGraphCreate(&g, 0));
+  auto fail = [&](cudaError_t e, const char* what) {
+    set_error(std::string(what) + ": " + cudaGetErrorString(e));
+    cudaGetLastError();
+    cudaGraphDestroy(g);
+    return NV_ERR_CUDA;
+  };
+  std::vector<cudaGraphConditionalHandle> hs(M->NE);
+  for (int k = 1; k < M->NE; ++k) {
+    cudaError_t e = cudaGraphConditionalHandleCreate(&hs[k], g, 0, cudaGraphCondAssignDefault);
+    if (e != cudaSuccess) return fail(e, "cudaGraphConditionalHandleCreate");
+  }
+  cudaStream_t st = s->cap_stream, st2 = s->cap_stream2;
+  cudaError_t e = cudaStreamBeginCaptureToGraph(st, g, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) return fail(e, "cudaStreamBeginCaptureToGraph");
+  long long host_launches = 1;  // step_begin
+  nv_status rs = record_layers(s, st, nullptr, &host_launches, 0, M->cfg.exit_layers[0]);
+  for (int k = 1; k < M->NE && rs == NV_OK; ++k) {
+    long long block = 0;
+    const int l0 = M->cfg.exit_layers[k - 1], l1 = M->cfg.exit_layers[k];
+    // the block's launch count is written to d_block_launches[k] after capture
+    launch_set_cond(hs[k], s->active, s->force, s->B, s->counters, s->d_block_launches + k, st);
+    ++host_launches;
+    cudaStreamCaptureStatus cs;
+    cudaGraph_t capg = nullptr;
+    const cudaGraphNode_t* deps = nullptr;
+    const cudaGraphEdgeData* ed = nullptr;
+    size_t nd = 0;
+    e = cudaStreamGetCaptureInfo_v3(st, &cs, nullptr, &capg, &deps, &ed, &nd);
+    if (e != cudaSuccess) {
+      rs = NV_ERR_CUDA;
+      set_error(std::string("cudaStreamGetCaptureInfo: ") + cudaGetErrorString(e));
+      break;
+    }
+    cudaGraphNodeParams cp = {};
+    cp.type = cudaGraphNodeTypeConditional;
+    cp.conditional.handle = hs[k];
+    cp.conditional.type = cudaGraphCondTypeIf;
+    cp.conditional.size = 1;
+    cudaGraphNode_t node;
+    std::vector<cudaGraphNode_t> dv(deps, deps + nd);
+    e = cudaGraphAddNode(&node, capg, dv.data(), nd, &cp);
+    if (e == cudaSuccess) e = cudaStreamUpdateCaptureDependencies(st, &node, 1, cudaStreamSetCaptureDependencies);
+    if (e != cudaSuccess) {
+      rs = NV_ERR_CUDA;
+      set_error(std::string("adding a conditional node: ") + cudaGetErrorString(e));
+      break;
+    }
+    e = cudaStreamBeginCaptureToGraph(st2, cp.conditional.phGraph_out[0], nullptr, nullptr, 0,
+                                      cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) {
+      rs = NV_ERR_CUDA;
+      set_error(std::string("capturing a conditional body: ") + cudaGetErrorString(e));
+      break;
+    }
+    rs = record_layers(s, st2, nullptr, &block, l0, l1);
+    cudaGraph_t tmp = nullptr;
+    e = cudaStreamEndCapture(st2, &tmp);
+    if (rs == NV_OK && e != cudaSuccess) {
+      rs = NV_ERR_CUDA;
+      set_error(std::string("ending a conditional body: ") + cudaGetErrorString(e));
+    }
+    s->block_launches[k] = block;
+  }
+  record_step_end(s, st, nullptr, &host_launches);
+  cudaGraph_t done = nullptr;
+  e = cudaStreamEndCapture(st, &done);
+  if (rs != NV_OK) {
+    cudaGraphDestroy(g);
+    return rs;
+  }
+  if (e != cudaSuccess) return fail(e, "cudaStreamEndCapture");
+  int counts[NV_MAX_EXITS] = {0};
+  for (int k = 0; k < M->NE; ++k) counts[k] = (int)s->block_launches[k];
+  e = cudaMemcpy(s->d_block_launches, counts, sizeof(counts), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return fail(e, "cudaMemcpy");
+  s->launches_per_step = host_launches;
+  *out = g;
   return NV_OK;
 }
 
@@ -785,6 +886,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   A((void**)&s->stop, (size_t)B * M->NE * 4);
   A((void**)&s->nstop, (size_t)NV_MAX_EXITS * 4);
   A((void**)&s->d_B, 4);
+  A((void**)&s->d_block_launches, NV_MAX_EXITS * 4);
   A((void**)&s->logp, (size_t)B * 4);
   A((void**)&s->hbuf, (size_t)B * s->cap * d * 4);
   for (int** p : {&s->row_b, &s->row_pos, &s->row_hrow}) A((void**)p, (size_t)s->max_rows * 4);
@@ -817,6 +919,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   cudaMemset(s->t, 0, (size_t)B * 4);
   cudaMemset(s->page_table, 0xff, s->h_page_table.size() * 4);
   cudaError_t e = cudaStreamCreateWithFlags(&s->cap_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s->cap_stream2, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     set_error(std::string("nv_state_create: ") + cudaGetErrorString(e));
@@ -833,6 +936,7 @@ nv_status nv_state_destroy(nv_state* s) {
   cudaDeviceSynchronize();
   if (s->graph) cudaGraphExecDestroy(s->graph);
   if (s->cap_stream) cudaStreamDestroy(s->cap_stream);
+  if (s->cap_stream2) cudaStreamDestroy(s->cap_stream2);
   for (void* p : s->allocs) cudaFree(p);
   s->pf_rows.release();
   s->pf_h.release();
@@ -1041,18 +1145,27 @@ nv_status decode_step_impl(nv_state* s, uint64_t seed, int32_t* tokens_out, int3
   } else {
     if (!s->graph) {
       cudaGraph_t g = nullptr;
-      NV_CUDA_TRY(cudaStreamBeginCapture(s->cap_stream, cudaStreamCaptureModeThreadLocal));
-      nv_status rs = record_step(s, s->cap_stream);
-      cudaError_t e = cudaStreamEndCapture(s->cap_stream, &g);
-      if (rs != NV_OK) {
-        if (g) cudaGraphDestroy(g);
-        return rs;
+      const char* cg = std::getenv("NVIUM_COND_GRAPH");
+      const bool try_cond = !(cg && cg[0] == '0') && M->NE > 1;
+      if (!try_cond || build_conditional_step_graph(s, &g) != NV_OK) {
+        // one flat graph of every layer (conditional nodes unavailable or disabled)
+        g = nullptr;
+        NV_CUDA_TRY(cudaStreamBeginCapture(s->cap_stream, cudaStreamCaptureModeThreadLocal));
+        nv_status rs = record_step(s, s->cap_stream);
+        cudaError_t e = cudaStreamEndCapture(s->cap_stream, &g);
+        if (rs != NV_OK) {
+          if (g) cudaGraphDestroy(g);
+          return rs;
+        }
+        if (e != cudaSuccess) {
+          set_error(std::string("capturing the decode step: ") + cudaGetErrorString(e));
+          return NV_ERR_CUDA;
+        }
+        s->cond_graph = false;
+      } else {
+        s->cond_graph = true;
       }
-      if (e != cudaSuccess) {
-        set_error(std::string("capturing the decode step: ") + cudaGetErrorString(e));
-        return NV_ERR_CUDA;
-      }
-      e = cudaGraphInstantiate(&s->graph, g, 0);
+      cudaError_t e = cudaGraphInstantiate(&s->graph, g, 0);
       cudaGraphDestroy(g);
       if (e != cudaSuccess) {
         set_error(std::string("instantiating the decode step: ") + cudaGetErrorString(e));
@@ -1167,7 +1280,8 @@ nv_status nv_read_counters(nv_state* s, int64_t* out, int n) {
   if (n > NV_CTR_COUNT) n = NV_CTR_COUNT;
   NV_CUDA_TRY(cudaDeviceSynchronize());
   NV_CUDA_TRY(cudaMemcpy(out, s->counters, (size_t)n * 8, cudaMemcpyDeviceToHost));
-  if (n > NV_CTR_LAUNCHES) out[NV_CTR_LAUNCHES] = s->launches_total;  // host-side count
+  // launches: the host's count plus the conditional blocks counted on the device
+  if (n > NV_CTR_LAUNCHES) out[NV_CTR_LAUNCHES] += s->launches_total;
   return NV_OK;
 }
 

@@ -136,3 +136,44 @@ def test_decode_parity_contexts_spanning_many_chunks(weights):
     prompts = [rng.integers(0, CFG.vocab, size=n).astype(np.int32) for n in (129, 256, 383)]
     chk, *_ = run_decode_parity(nv, CFG, weights, prompts, 12, max_seq=420)
     assert chk.steps == 12
+
+
+@pytest.mark.parametrize("cfg_name", ["tiny", "mini-bf16"])
+def test_conditional_and_flat_step_graphs_agree(cfg_name):
+    """The decode-step graph skips the layer blocks no token reaches
+    (conditional nodes); the flat graph launches every layer.  Outputs and
+    caches are bit-identical."""
+    import os
+    if cfg_name == "tiny":
+        cfg, w = CFG, W.make_weights(CFG, seed=0)
+    else:
+        cfg = W.ModelConfig("mini-bf16", 4, 256, 4, 64, 512, 1024, (1, 2, 3, 4), W.BF16)
+        w = W.make_weights(cfg, seed=3, router_bias=[0.5, 0.0, -0.5])
+    rng = np.random.default_rng(3)
+    prompts = [rng.integers(0, cfg.vocab, size=n).astype(np.int32) for n in (12, 30, 7)]
+    lens = np.array([len(p) for p in prompts], np.int32)
+    outs = {}
+    for mode in ("1", "0"):
+        os.environ["NVIUM_COND_GRAPH"] = mode
+        try:
+            m = nv.Model(cfg, w, max_batch=3, max_seq=64, max_pending=8)
+            st = nv.State(m, 3)
+            st.prefill(np.concatenate(prompts), lens)
+            tok, ex, lp = np.zeros(3, np.int32), np.zeros(3, np.int32), np.zeros(3, np.float32)
+            seq = []
+            for s in range(16):
+                st.decode_step(77 + s, tok, ex, lp)
+                seq.append(np.concatenate([tok, ex, lp.view(np.int32)]))
+            st.flush()
+            kv = [st.read_kv(b, cfg.n_layers - 1, 64) for b in range(3)]
+            outs[mode] = (np.stack(seq), kv, st.counters())
+            st.close()
+            m.close()
+        finally:
+            os.environ.pop("NVIUM_COND_GRAPH", None)
+    np.testing.assert_array_equal(outs["1"][0], outs["0"][0])
+    for a, b in zip(outs["1"][1], outs["0"][1]):
+        np.testing.assert_array_equal(a[0], b[0])
+        np.testing.assert_array_equal(a[1], b[1])
+    # the conditional graph launches no more kernels than the flat one
+    assert outs["1"][2][nv.CTR["launches"]] <= outs["0"][2][nv.CTR["launches"]]
