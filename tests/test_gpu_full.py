@@ -1,0 +1,142 @@
+"""Parity at the full 1.5B sizes (48 layers, d=1536, 24 heads, vocab 32000,
+exits after layers 12/24/36/48), in the launch configurations the benchmark
+uses.  The oracle cannot replay whole workloads of this size, so it checks
+sampled outputs it can compute one by one, and two properties are checked at
+any size:
+
+* scoring (16 x 2048): causality makes logp[b, t] for t < T depend only on
+  tokens[b, :T+1], so the oracle scores a short prefix of one sequence;
+* decode at B=64 (ragged prompts): the oracle replays the batch's shortest
+  sequence alone (same Philox sequence index), teacher-forced, for a few
+  steps, and its KV after the flush (deep bf16 caches: exceedances of the
+  tolerance are counted, see kv_close_counted);
+* complete KV recovery (the piggybacking summary: deferred rows end with
+  exact caches): after deferred decoding and the flush, every layer's KV
+  equals a dense prefill of the same tokens;
+* zero intermediate mass (the summary's section 5): decode log-probabilities
+  equal the mixture scoring of the generated sequence.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import nvium_oracle as O
+from tests.nvium_testlib import StepChecker, gpu_kv, kv_close_counted, tolerance
+
+pytestmark = pytest.mark.gpu
+
+nv = pytest.importorskip("exact_early_exit_b200")
+CFG = W.X15B
+
+
+@pytest.fixture(scope="module")
+def weights():
+    return W.make_weights(CFG, seed=0)
+
+
+@pytest.fixture(scope="module")
+def oracle_model(weights):
+    return O.OracleModel(CFG, weights, cache_f64=False)
+
+
+def test_scoring_16x2048_prefix_matches_oracle(weights, oracle_model):
+    wl = W.WORKLOADS["XS"]
+    toks = np.stack(W.make_prompts(wl)).astype(np.int32)          # [16, 2048]
+    model = nv.Model(CFG, weights, max_batch=1, max_seq=2048)
+    logp = np.zeros((16, 2047), np.float32)
+    nll = np.zeros(1, np.float32)
+    model.score_mixture(toks, logp, nll)
+    model.close()
+    assert np.all(np.isfinite(logp)) and np.all(logp < 0)
+    assert abs(float(nll[0]) + float(logp.astype(np.float64).mean())) < 1e-3
+    T = 40
+    ref, _ = O.score_mixture(oracle_model, toks[5:6, : T + 1])
+    np.testing.assert_allclose(logp[5, :T], ref[0], atol=tolerance(CFG), rtol=0)
+
+
+def test_decode_b64_sampled_sequence_matches_oracle(weights, oracle_model):
+    wl = W.WORKLOADS["X64"]
+    lens = W.make_prompt_lengths(wl)
+    prompts = W.make_prompts(wl, lengths=lens)
+    B, steps, seed = wl.batch, 4, wl.philox_seed
+    max_seq = int(lens.max()) + wl.steps + 64
+    model = nv.Model(CFG, weights, max_batch=B, max_seq=max_seq)
+    st = nv.State(model, B)
+    st.prefill(np.concatenate(prompts).astype(np.int32), lens)
+    b = int(np.argmin(lens))
+    dec = O.OracleDecoder(oracle_model, [prompts[b]], steps)
+    dec.ids = [b]
+    chk = StepChecker(CFG)
+    tok, ex, lp = np.zeros(B, np.int32), np.zeros(B, np.int32), np.zeros(B, np.float32)
+    for s in range(steps):
+        st.decode_step(seed + s, tok, ex, lp)
+        rec = dec.step(seed + s, forced_exits=[int(ex[b])], forced_tokens=[int(tok[b])])
+        chk.check(rec, tok[b:b + 1], ex[b:b + 1], lp[b:b + 1])
+    st.flush()
+    dec.flush()
+    st.sync_status()
+    for m in (0, 11, 12, 30, 47):
+        K, V, n = gpu_kv(st, b, m, max_seq, CFG)
+        assert n == dec.t[0]
+        # GPU (fp32 accumulation) against the fp64 oracle, 30+ layers deep:
+        # at most 1e-4 of the elements beyond the tolerance, none beyond twice it
+        kv_close_counted(K, dec.caches[0].K[m][:n], CFG, f"K layer {m}", max_frac=1e-4, hard_factor=2.0)
+        kv_close_counted(V, dec.caches[0].V[m][:n], CFG, f"V layer {m}", max_frac=1e-4, hard_factor=2.0)
+    st.close()
+    model.close()
+
+
+def test_decode_b1_deferred_kv_equals_dense_prefill(weights):
+    wl = W.WORKLOADS["X1"]
+    prompt = W.make_prompts(wl)[0]
+    steps = 64
+    max_seq = len(prompt) + steps + 64
+    model = nv.Model(CFG, weights, max_batch=1, max_seq=max_seq)
+    st = nv.State(model, 1)
+    st.prefill(prompt, [len(prompt)])
+    tok, ex = np.zeros(1, np.int32), np.zeros(1, np.int32)
+    gen, exits = [], []
+    for s in range(steps):
+        st.decode_step(wl.philox_seed + s, tok, ex)
+        gen.append(int(tok[0]))
+        exits.append(int(ex[0]))
+    assert len(set(exits)) > 1, "routing should use several exits"
+    st.flush()
+    st.sync_status()
+    # a dense prefill of the same tokens (positions 0..P+steps-2 at full depth)
+    full = np.concatenate([prompt, np.array(gen, np.int32)])
+    st2 = nv.State(model, 1)
+    st2.prefill(full, [len(full)])
+    n_exp = len(full) - 1
+    for m in range(CFG.n_layers):
+        K1, V1, n1 = gpu_kv(st, 0, m, max_seq, CFG)
+        K2, V2, n2 = gpu_kv(st2, 0, m, max_seq, CFG)
+        assert n1 == n2 == n_exp
+        kv_close_counted(K1, K2, CFG, f"K layer {m}")
+        kv_close_counted(V1, V2, CFG, f"V layer {m}")
+    st.close()
+    st2.close()
+    model.close()
+
+
+def test_force_last_decode_logp_equals_scoring(weights):
+    wl = W.WORKLOADS["X1"]
+    prompt = W.make_prompts(wl)[0][:1024]
+    steps = 24
+    model = nv.Model(CFG, weights, max_batch=1, max_seq=len(prompt) + steps + 8,
+                     router_mode=nv.NV_ROUTER_FORCE_LAST)
+    st = nv.State(model, 1)
+    st.prefill(prompt, [len(prompt)])
+    tok, ex, lp = np.zeros(1, np.int32), np.zeros(1, np.int32), np.zeros(1, np.float32)
+    gen, lps = [], []
+    for s in range(steps):
+        st.decode_step(99 + s, tok, ex, lp)
+        assert ex[0] == CFG.n_exits
+        gen.append(int(tok[0]))
+        lps.append(float(lp[0]))
+    full = np.concatenate([prompt, np.array(gen, np.int32)])[None, :]
+    logp = np.zeros((1, full.shape[1] - 1), np.float32)
+    model.score_mixture(full, logp)
+    np.testing.assert_allclose(np.array(lps), logp[0, len(prompt) - 1:], atol=tolerance(CFG), rtol=0)
+    st.close()
+    model.close()
