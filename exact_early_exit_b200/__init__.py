@@ -96,6 +96,7 @@ _SIGS = [
     ("nv_philox4x32_10", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
     ("nv_decode_step_profiled", _I, [_P, ctypes.c_uint64, _P, _P, _P, _P]),
     ("nv_philox4x32_10_noalloc", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
+    ("nv_score_mixture_profiled", _I, [_P, _P, _I, _I, _P, _P, _P, _P]),
     ("nv_last_error", ctypes.c_char_p, []),
 ]
 
@@ -215,6 +216,15 @@ class Model:
         B, S = tokens.shape
         _check(lib().nv_score_mixture(self.handle, _ptr(tokens), B, S, _ptr(logp_out), _ptr(mean_nll_out),
                                       _stream(stream)))
+
+    def score_mixture_profiled(self, tokens, logp_out, mean_nll_out=None, stats=None, stream=None):
+        """score_mixture with per-kernel CUDA-event timing (KernelStat array)."""
+        if stats is None:
+            stats = (KernelStat * len(KERNEL_KINDS))()
+        B, S = tokens.shape
+        _check(lib().nv_score_mixture_profiled(self.handle, _ptr(tokens), B, S, _ptr(logp_out), _ptr(mean_nll_out),
+                                               ctypes.cast(stats, ctypes.c_void_p), _stream(stream)))
+        return stats
 
     def close(self):
         if getattr(self, "handle", None):

@@ -41,14 +41,15 @@ constexpr int BM = 128;      // features per tile (MMA M, TMEM lanes)
 constexpr int BK = 64;       // K per stage: one 128-byte swizzle row of bf16
 constexpr int BNMAX = 256;   // rows per tile (MMA N, TMEM columns)
 constexpr int BOXN = 32;     // rows per X TMA box
-constexpr int STAGES = 4;
+constexpr int STAGES = 4;        // stages at the largest row tile (256 rows)
+constexpr int MAXST = 12;        // stages when the row tile is small
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNMAX * BK * 2;
 constexpr int BOX_BYTES = BOXN * BK * 2;
 constexpr int SMEM_TILES = STAGES * (A_BYTES + B_BYTES);
 constexpr int EPI_ROWS = 32;                    // rows per epilogue staging pass
 constexpr int EPI_BYTES = EPI_ROWS * BM * 4;    // fp32 staging tile [32 rows][128 features]
-constexpr int SMEM_BYTES = SMEM_TILES + 256 /*barriers*/ + EPI_BYTES + 1024 /*align*/;
+constexpr int SMEM_BYTES = SMEM_TILES + 512 /*barriers*/ + EPI_BYTES + 1024 /*align*/;
 constexpr uint32_t TMEM_COLS = 512;  // two 256-column fp32 accumulators
 constexpr int THREADS = 192;
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on any single wait
@@ -341,17 +342,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   if ((int)blockIdx.x >= items) return;
 
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* sA = smem;
-  unsigned char* sB = smem + STAGES * A_BYTES;
+  // Stage ring sized to the row tile this launch needs: a stage is one W tile
+  // (16 KB) plus nbmax X boxes (4 KB each); small row counts (decode) get up
+  // to MAXST stages in flight.
+  const int nbmax = (min(R, BNMAX) + BOXN - 1) / BOXN;
+  const int stage_bytes = A_BYTES + nbmax * BOX_BYTES;
+  const int nst = min(MAXST, SMEM_TILES / stage_bytes);
   uint64_t* full = (uint64_t*)(smem + SMEM_TILES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint64_t* empty = full + MAXST;
+  uint64_t* tfull = empty + MAXST;
   uint64_t* tempty = tfull + 2;
-  float* stile = (float*)(smem + SMEM_TILES + 256);  // epilogue staging [EPI_ROWS][BM]
+  float* stile = (float*)(smem + SMEM_TILES + 512);  // epilogue staging [EPI_ROWS][BM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < nst; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
@@ -379,9 +384,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int issued[STAGES];  // parity of the last load issued into each stage, -1 if none
+      int issued[MAXST];  // parity of the last load issued into each stage, -1 if none
 #pragma unroll
-      for (int s = 0; s < STAGES; ++s) issued[s] = -1;
+      for (int s = 0; s < MAXST; ++s) issued[s] = -1;
       for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
         const Item t = decode_item(it, ntn, splits, R, kblocks);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
@@ -390,11 +395,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           issued[stage] = (int)phase;
+          unsigned char* sa = smem + stage * stage_bytes;
           mbar_expect_tx(full + stage, (uint32_t)(A_BYTES + t.nbox * BOX_BYTES));
-          tma_load_2d(sA + stage * A_BYTES, &tw, full + stage, kb * BK, t.n0);
+          tma_load_2d(sa, &tw, full + stage, kb * BK, t.n0);
           for (int j = 0; j < t.nbox; ++j)
-            tma_load_2d(sB + stage * B_BYTES + j * BOX_BYTES, &tx, full + stage, kb * BK, t.r0 + j * BOXN);
-          if (++stage == STAGES) {
+            tma_load_2d(sa + A_BYTES + j * BOX_BYTES, &tx, full + stage, kb * BK, t.r0 + j * BOXN);
+          if (++stage == nst) {
             stage = 0;
             phase ^= 1u;
           }
@@ -403,7 +409,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (*abort_flag) {
         // let the copies already issued land before the CTA leaves (bounded)
         volatile int never = 0;
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < nst; ++s)
           if (issued[s] >= 0) mbar_wait(full + s, (uint32_t)issued[s], &never, WAIT_NS / 4);
       }
     }
@@ -424,13 +430,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t ad = sw128_desc(smem_u32(sA + stage * A_BYTES));
-          const uint64_t bd = sw128_desc(smem_u32(sB + stage * B_BYTES));
+          const uint64_t ad = sw128_desc(smem_u32(smem + stage * stage_bytes));
+          const uint64_t bd = sw128_desc(smem_u32(smem + stage * stage_bytes + A_BYTES));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (kb > t.kb0 || kk > 0) ? 1u : 0u);
           umma_commit(empty + stage);
-          if (++stage == STAGES) {
+          if (++stage == nst) {
             stage = 0;
             phase ^= 1u;
           }

@@ -1324,8 +1324,11 @@ nv_status nv_sync_status(nv_state* s) {
   return check_status(s);
 }
 
-nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll,
-                           void* stream) {
+}  // extern "C"
+
+namespace {
+nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll, cudaStream_t st,
+                     Prof* prof) {
   if (!M || !tokens || !logp) {
     set_error("null argument");
     return NV_ERR_INVALID_ARG;
@@ -1334,7 +1337,6 @@ nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, flo
     set_error("need B >= 1 and 2 <= S <= max_seq");
     return NV_ERR_INVALID_ARG;
   }
-  cudaStream_t st = (cudaStream_t)stream;
   const int Sm = S - 1;               // positions 0..S-2 predict tokens 1..S-1
   const long long R64 = (long long)B * Sm;
   if (R64 > (1LL << 26)) {
@@ -1429,28 +1431,75 @@ nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, flo
   io.lens = nullptr;
   io.L = M->L;
   io.epi_grid = 4096;
-  launch_embed_rows(M->bf16, M->tok_emb, d_tok, io.rs, M->d, st);
+  const long long es = (long long)M->esz;
+  if (prof) {
+    prof->R = R;
+    // causal attention: row p reads K and V of positions 0..p
+    prof->kv_read = (long long)B * Sm * (Sm + 1) / 2 * 2 * M->HQ * es;
+  }
+  timed(prof, nullptr, 1, NV_K_STEP, 0, 0, [&] { launch_embed_rows(M->bf16, M->tok_emb, d_tok, io.rs, M->d, st); });
   for (int layer = 0; layer < M->L; ++layer) {
-    launch_rmsnorm_rows(M->bf16, io.rs, M->layers[layer].attn_norm, io.act, M->d, M->cfg.rms_eps, st);
-    NV_TRY(layer_body(M, layer, io, st));
+    timed(prof, nullptr, 1, NV_K_NORM, (long long)R * M->d * (4 + es), 0, [&] {
+      launch_rmsnorm_rows(M->bf16, io.rs, M->layers[layer].attn_norm, io.act, M->d, M->cfg.rms_eps, st);
+    });
+    NV_TRY(layer_body(M, layer, io, st, prof, nullptr));
     const int k = M->exit_at[layer];
     if (k < 0) continue;
-    launch_exit_rows(M->bf16, io.rs, M->exits[k].norm, M->exits[k].router_w, M->exits[k].router_b, k, NE, io.act,
-                     M->sc_z.as<float>(), M->d, M->cfg.rms_eps, st);
+    timed(prof, nullptr, 1, NV_K_JUNCTION, (long long)R * M->d * (4 + es), 0, [&] {
+      launch_exit_rows(M->bf16, io.rs, M->exits[k].norm, M->exits[k].router_w, M->exits[k].router_b, k, NE, io.act,
+                       M->sc_z.as<float>(), M->d, M->cfg.rms_eps, st);
+    });
     for (int c = 0; c < nchunks; ++c) {
       const int r0 = c * head_chunk;
-      NV_TRY(gemm_run(M->gemm_plans, M->gemm_kind, M->bf16, (const unsigned char*)io.act + (size_t)r0 * M->d * M->esz,
-                      M->d, M->exits[k].head, M->V, M->d, d_chunk + c, head_chunk, io.Y, false, nullptr, nullptr, 0,
-                      nullptr, 0, st));
-      const float* Yh = io.Y;
-      launch_lse_target(Yh, r0, std::min(head_chunk, R - r0), M->V, d_tgt, M->sc_logpi.as<float>(), k, NE, st);
+      const long long rc = std::min(head_chunk, R - r0);
+      nv_status hst = NV_OK;
+      timed(prof, nullptr, 2, NV_K_HEAD, (long long)M->V * M->d * es + rc * M->d * es + rc * M->V * 4,
+            2 * rc * M->V * M->d, [&] {
+              hst = gemm_run(M->gemm_plans, M->gemm_kind, M->bf16,
+                             (const unsigned char*)io.act + (size_t)r0 * M->d * M->esz, M->d, M->exits[k].head, M->V,
+                             M->d, d_chunk + c, head_chunk, io.Y, false, nullptr, nullptr, 0, nullptr, 0, st);
+              launch_lse_target(io.Y, r0, (int)rc, M->V, d_tgt, M->sc_logpi.as<float>(), k, NE, st);
+            });
+      NV_TRY(hst);
     }
   }
-  launch_mixture(M->sc_z.as<float>(), M->sc_logpi.as<float>(), R, NE, M->cfg.router_mode, M->sc_logp.as<float>(),
-                 M->sc_nll.as<float>(), st);
+  timed(prof, nullptr, 2, NV_K_STEP, 0, 0, [&] {
+    launch_mixture(M->sc_z.as<float>(), M->sc_logpi.as<float>(), R, NE, M->cfg.router_mode, M->sc_logp.as<float>(),
+                   M->sc_nll.as<float>(), st);
+  });
   NV_CUDA_TRY(cudaMemcpyAsync(logp, M->sc_logp.p, (size_t)R * 4, cudaMemcpyDefault, st));
   if (mean_nll) NV_CUDA_TRY(cudaMemcpyAsync(mean_nll, M->sc_nll.p, 4, cudaMemcpyDefault, st));
   NV_CUDA_TRY(cudaGetLastError());
+  return NV_OK;
+}
+}  // namespace
+
+extern "C" {
+
+nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll,
+                           void* stream) {
+  return score_impl(M, tokens, B, S, logp, mean_nll, (cudaStream_t)stream, nullptr);
+}
+
+nv_status nv_score_mixture_profiled(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll,
+                                    nv_kernel_stat* stats, void* stream) {
+  if (!stats) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  Prof prof;
+  prof.st = (cudaStream_t)stream;
+  NV_TRY(score_impl(M, tokens, B, S, logp, mean_nll, prof.st, &prof));
+  NV_CUDA_TRY(cudaStreamSynchronize(prof.st));
+  for (const Prof::Rec& r : prof.recs) {
+    float ms = 0.f;
+    NV_CUDA_TRY(cudaEventElapsedTime(&ms, r.a, r.b));
+    nv_kernel_stat& k = stats[r.kind];
+    k.ms += ms;
+    k.launches += 1;
+    k.bytes += r.bytes;
+    k.flops += r.flops;
+  }
   return NV_OK;
 }
 

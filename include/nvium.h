@@ -251,6 +251,14 @@ nv_status nv_decode_step_profiled(nv_state *s, uint64_t philox_seed,
                                   int32_t *tokens_out, int32_t *exits_out,
                                   nv_kernel_stat *stats, void *stream);
 
+/* nv_score_mixture with the same per-kernel timing (NV_K_GEMM: the layer
+ * GEMMs with their fused epilogues, NV_K_HEAD: exit-head GEMM + log-sum-exp,
+ * NV_K_ATTENTION: causal attention, ...); flops are the GEMMs' 2*rows*N*K.
+ * Results are those of nv_score_mixture.  Synchronous. */
+nv_status nv_score_mixture_profiled(nv_model *m, const int32_t *tokens, int B,
+                                    int S, float *logp, float *mean_nll,
+                                    nv_kernel_stat *stats, void *stream);
+
 /* Synchronise the state's work and return any device-detected error. */
 nv_status nv_sync_status(nv_state *s);
 
