@@ -1,0 +1,302 @@
+// Decode / flush attention for bf16 caches with head_dim 64, on warp-level
+// bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation).
+//
+// What it computes is the causal softmax attention of the LLaMA-2 backbone
+// ("N-vium: Mixture-of-Exits Transformer for Accelerated Exact Generation",
+// section 4): for a row at position p, o = sum_j softmax_j(q . k_j /
+// sqrt(hd)) v_j over keys j <= p.  Rows are the new token of each sequence
+// plus the deferred rows that run this layer in the same step (section 2
+// "Inferenz: Piggybacking": the layers above an exit run later, batched with
+// the next token that reaches them).
+//
+// Work split: one CTA per (sequence, head, 128-key chunk), 4 warps of 32 keys,
+// up to 16 rows per pass (the M of the MMA).  Partials (unnormalised sum,
+// max, sum of weights) go to the same per-(row, head, chunk) slots as the
+// SIMT kernel's, and k_attn_dec_combine merges them.
+//
+// Data movement: the chunk's K and V (two 64-position boxes each) come in by
+// TMA through a 2-D tensor map over the whole KV pool (rows of 64 bf16 =
+// 128 bytes, 128-byte swizzle), so the ldmatrix reads of 8 consecutive keys
+// hit 8 different bank groups.  One thread waits on the transaction barrier;
+// the others wait at the CTA barrier and spend no issue slots.
+//
+// Numerics: q and the cache are bf16 (the bf16 contract of the model), S =
+// q k^T accumulates in fp32; the softmax weights P are fp32 and enter the PV
+// product as a bf16 pair hi + lo (hi = bf16(P), lo = bf16(P - hi)), which
+// keeps ~16 significant bits of P; V is exact in bf16.  So the result matches
+// an fp32 SIMT evaluation to ~1e-5 relative, far inside the path's tolerance.
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace nv {
+namespace {
+
+constexpr int CK = ATTN_DEC_CK;  // keys per CTA
+constexpr int HD = 64;           // head dim (128-byte rows)
+constexpr int RG = 16;           // rows per MMA pass
+constexpr int QLD = HD + 8;      // padded Q row: 144 bytes, conflict-free ldmatrix
+constexpr int OLD = HD + 2;      // per-warp partial row: HD sums, max, weight sum
+constexpr int BOX = 64;          // positions per TMA box (a page holds 64 or 128)
+constexpr int BOX_BYTES = BOX * HD * 2;
+
+struct DecSmem {
+  __nv_bfloat16 K[CK * HD];  // 16 KB, 1024-byte aligned (swizzle atom)
+  __nv_bfloat16 V[CK * HD];  // 16 KB
+  __nv_bfloat16 Q[RG * QLD];
+  float O[4][RG][OLD];
+  uint64_t bar;
+  int abort;
+};
+constexpr size_t DEC_SMEM_BYTES = sizeof(DecSmem) + 1024;  // + alignment slack
+
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(const_cast<void*>(p));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// D += A B, A 16x16 bf16 row-major fragment, B 16x8 bf16 column fragment
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+// byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+__device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, uint64_t* bar, int row) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(saddr(dst)),
+      "l"(map), "r"(saddr(bar)), "r"(0), "r"(row)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(128) k_attn_dec_mma(const __grid_constant__ CUtensorMap kvmap, AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
+  extern __shared__ unsigned char smem_raw[];
+  DecSmem& S = *reinterpret_cast<DecSmem*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  if (*a.rs.nrows == 0) return;
+  const int b = blockIdx.x, head = blockIdx.y, chunk = blockIdx.z;
+  const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
+  if (s0 >= s1) return;
+  const int pos_last = a.rs.row_pos[s1 - 1];
+  const int k0 = chunk * CK;
+  if (k0 > pos_last) return;
+  const int nk = min(CK, pos_last + 1 - k0);
+  const int nbox = (nk + BOX - 1) / BOX;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    S.abort = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&S.bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(&S.bar)),
+                 "r"((uint32_t)(2 * nbox * BOX_BYTES))
+                 : "memory");
+    for (int i = 0; i < nbox; ++i) {
+      const int pos = k0 + i * BOX;
+      tma_box(S.K + i * BOX * HD, &kvmap, &S.bar, (int)(a.kv.offset(a.layer, b, pos, head, 0) / HD));
+      tma_box(S.V + i * BOX * HD, &kvmap, &S.bar, (int)(a.kv.offset(a.layer, b, pos, head, 1) / HD));
+    }
+  }
+  const int H = a.H;
+  const __nv_bfloat16* qg = (const __nv_bfloat16*)a.q;
+  const int pos0 = a.rs.row_pos[s0];
+  const int first = max(s0, s0 + (k0 - pos0));  // rows whose position reaches this chunk
+  const int w = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+  if (tid == 0) {
+    unsigned long long t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+      uint32_t ok;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\tselp.u32 %0, 1, 0, "
+          "p;\n\t}"
+          : "=r"(ok)
+          : "r"(saddr(&S.bar))
+          : "memory");
+      if (ok) break;
+      if ((i & 15u) == 0u) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (i == 0) t0 = t;
+        else if (t - t0 > 2000000000ull) {
+          S.abort = 1;
+          break;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (S.abort) {
+    if (tid == 0) dev_fail(a.status, DEV_ERR_TIMEOUT);
+    return;
+  }
+  // V rows past the last key may hold stale or never-written bytes; P is zero
+  // there, so zero V too (0 * NaN would poison the sums)
+  for (int i = nk * 8 + tid; i < nbox * BOX * 8; i += blockDim.x)
+    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.V) + (i >> 3) * 128 + (i & 7) * 16) =
+        make_uint4(0, 0, 0, 0);
+  for (int g0 = first; g0 < s1; g0 += RG) {
+    const int ng = min(RG, s1 - g0);
+    {  // Q rows of this pass (16 rows x 8 chunks: one chunk per thread), zero padding
+      const int r = tid >> 3, c = tid & 7;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (r < ng) v = *reinterpret_cast<const uint4*>(qg + (size_t)(g0 + r) * H * HD + head * HD + c * 8);
+      *reinterpret_cast<uint4*>(S.Q + r * QLD + c * 8) = v;
+    }
+    __syncthreads();
+
+    // S = Q K^T for this warp's 32 keys: 4 n-tiles of 8 keys, 4 k-steps of 16 dims
+    uint32_t qa[4][4];
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      ldsm_x4(qa[ks], saddr(S.Q + ((lane & 7) + 8 * ((lane >> 3) & 1)) * QLD + (2 * ks + (lane >> 4)) * 8));
+    float sc[4][4];
+    const uint32_t kbase = saddr(S.K), vbase = saddr(S.V);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+      const int r = 32 * w + 8 * nt + (lane & 7);
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) {
+        uint32_t kb[4];
+        ldsm_x4(kb, kbase + swz(r, 4 * kp + (lane >> 3)));
+        mma_bf16(sc[nt], qa[2 * kp], kb[0], kb[1]);
+        mma_bf16(sc[nt], qa[2 * kp + 1], kb[2], kb[3]);
+      }
+    }
+    // causal / length mask, this warp's row maxima and weights
+    const int p_lo = pos0 + (g0 + g - s0), p_hi = p_lo + 8;  // positions of rows g and g + 8
+    const bool v_lo = g < ng, v_hi = g + 8 < ng;
+    float m_lo = -CUDART_INF_F, m_hi = -CUDART_INF_F;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kk = 32 * w + 8 * nt + 2 * tq + (e & 1);
+        const bool hi = e >= 2;
+        const bool ok = kk < nk && (hi ? (v_hi && k0 + kk <= p_hi) : (v_lo && k0 + kk <= p_lo));
+        const float s = ok ? sc[nt][e] * a.scale : -CUDART_INF_F;
+        sc[nt][e] = s;
+        if (hi) m_hi = fmaxf(m_hi, s); else m_lo = fmaxf(m_lo, s);
+      }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      m_lo = fmaxf(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
+      m_hi = fmaxf(m_hi, __shfl_xor_sync(0xffffffffu, m_hi, o));
+    }
+    float l_lo = 0.f, l_hi = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool hi = e >= 2;
+        const float m = hi ? m_hi : m_lo;
+        const float p = m == -CUDART_INF_F ? 0.f : expf(sc[nt][e] - m);
+        sc[nt][e] = p;
+        if (hi) l_hi += p; else l_lo += p;
+      }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, o);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, o);
+    }
+    // O = P V: P as a bf16 hi/lo pair, 2 k-steps of 16 keys, 8 n-tiles of 8 dims
+    float oc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) oc[nt][e] = 0.f;
+#pragma unroll
+    for (int kq = 0; kq < 2; ++kq) {
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const float x0 = sc[2 * kq + h][2 * rr], x1 = sc[2 * kq + h][2 * rr + 1];
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+          ph[2 * h + rr] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+          pl[2 * h + rr] = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+        }
+      const int r = 32 * w + 16 * kq + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t vb[4];
+        ldsm_x4_t(vb, vbase + swz(r, 2 * np + (lane >> 4)));
+        mma_bf16(oc[2 * np], ph, vb[0], vb[1]);
+        mma_bf16(oc[2 * np], pl, vb[0], vb[1]);
+        mma_bf16(oc[2 * np + 1], ph, vb[2], vb[3]);
+        mma_bf16(oc[2 * np + 1], pl, vb[2], vb[3]);
+      }
+    }
+    // per-warp partials to shared memory, then one merge per row
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      *reinterpret_cast<float2*>(&S.O[w][g][8 * nt + 2 * tq]) = make_float2(oc[nt][0], oc[nt][1]);
+      *reinterpret_cast<float2*>(&S.O[w][g + 8][8 * nt + 2 * tq]) = make_float2(oc[nt][2], oc[nt][3]);
+    }
+    if (tq == 0) {
+      S.O[w][g][HD] = m_lo;
+      S.O[w][g][HD + 1] = l_lo;
+      S.O[w][g + 8][HD] = m_hi;
+      S.O[w][g + 8][HD + 1] = l_hi;
+    }
+    __syncthreads();
+    for (int j = w; j < ng; j += 4) {
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) M = fmaxf(M, S.O[q][j][HD]);
+      float L = 0.f, acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float mq = S.O[q][j][HD];
+        if (mq == -CUDART_INF_F) continue;
+        const float e = expf(mq - M);
+        L += S.O[q][j][HD + 1] * e;
+        const float2 v = *reinterpret_cast<const float2*>(&S.O[q][j][2 * lane]);
+        acc0 += v.x * e;
+        acc1 += v.y * e;
+      }
+      float* pp = a.part + (((size_t)(g0 + j) * H + head) * a.kv_splits + chunk) * OLD;
+      *reinterpret_cast<float2*>(pp + 2 * lane) = make_float2(acc0, acc1);
+      if (lane == 0) {
+        pp[HD] = M;
+        pp[HD + 1] = L;
+      }
+    }
+    __syncthreads();
+  }
+  if (a.lens && head == 0 && chunk == 0 && tid == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
+}
+
+}  // namespace
+
+cudaError_t attn_dec_mma_prepare() {
+  return cudaFuncSetAttribute(k_attn_dec_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DEC_SMEM_BYTES);
+}
+
+void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st) {
+  dim3 grid(a.rs.B, a.H, a.kv_splits);
+  launch_k(k_attn_dec_mma, grid, 128, DEC_SMEM_BYTES, st, *kvmap, a);
+}
+
+}  // namespace nv

@@ -556,6 +556,30 @@ nv_status tc_prepare() {
   return NV_OK;
 }
 
+nv_status encode_rows128_map(const void* base, uint64_t rows, uint32_t box_rows, CUtensorMap* out) {
+  auto enc = get_encode();
+  if (!enc) {
+    set_error("cuTensorMapEncodeTiled is unavailable");
+    return NV_ERR_UNSUPPORTED;
+  }
+  if (((uintptr_t)base & 15) || rows == 0 || box_rows == 0 || box_rows > 256) {
+    set_error("row tensor map: bad base or box");
+    return NV_ERR_INVALID_ARG;
+  }
+  cuuint64_t dims[2] = {64, rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled (rows of 128 bytes) failed with code " + std::to_string((int)r));
+    return NV_ERR_CUDA;
+  }
+  return NV_OK;
+}
+
 size_t tc_split_stride(size_t N) { return (size_t)BNMAX * N; }
 
 size_t tc_workspace_elems(size_t N) { return (size_t)TC_MAX_SPLIT * BNMAX * N; }

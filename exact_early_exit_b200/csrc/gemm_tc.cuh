@@ -1,6 +1,8 @@
 // tcgen05 GEMM for bf16 models (sm_100a): Y[r][n] = sum_k X[r][k] W[n][k].
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace nv {
@@ -16,6 +18,9 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
                       int max_rows, float* Y, bool allow_split, const EpiArgs* epi, int* tile_counters,
                       const void* prefetch, size_t prefetch_bytes, cudaStream_t st, int* grid_out = nullptr,
                       const int* skip_if_zero = nullptr);
+// 2-D tensor map over rows of 64 bf16 (128 bytes) with 128-byte swizzle and
+// boxes of box_rows rows (decode attention's view of the KV pool)
+nv_status encode_rows128_map(const void* base, uint64_t rows, uint32_t box_rows, CUtensorMap* out);
 // elements between split-K slices of an N-column output
 size_t tc_split_stride(size_t N);
 }  // namespace nv

@@ -908,7 +908,8 @@ __global__ void k_attn_dec_combine(AttnArgs a) {
 template <typename T, int HD>
 static void attention_dec_t(const AttnArgs& a, cudaStream_t st) {
   dim3 grid(a.rs.B, a.H, a.kv_splits);
-  launch_k(k_attn_dec<T, HD>, grid, 128, 0, st, a);
+  if (a.kv_map && sizeof(T) == 2 && HD == 64) launch_attn_dec_mma(a.kv_map, a, st);
+  else launch_k(k_attn_dec<T, HD>, grid, 128, 0, st, a);
   int g = (a.rs.max_rows * a.H + 7) / 8;
   if (g > 4096) g = 4096;
   launch_k(k_attn_dec_combine<T, HD>, g, 256, 0, st, a);

@@ -2,6 +2,8 @@
 // `bf16` to pick the element type of weights / activations / KV cache.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -88,6 +90,7 @@ struct AttnArgs {
   int* lens;       // when set: lens[b*L+layer] = last row position + 1
   int L;
   int* status;     // device status word (bounded-wait expiry)
+  const CUtensorMap* kv_map;  // host copy of the KV pool's 128-byte-row map (bf16, hd 64), or null
 };
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
 // Decode / flush attention: 128-key chunks (grid z = kv_splits = chunks of
@@ -95,6 +98,10 @@ void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
 // head_dim * element size == 128 bytes and page_size == 64.
 constexpr int ATTN_DEC_CK = 128;
 void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st);
+// bf16 / head_dim 64 decode attention on warp MMAs (attn_dec_mma.cu); needs
+// a.kv_map.  Same partial slots as the SIMT kernel, merged by its combine.
+cudaError_t attn_dec_mma_prepare();
+void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st);
 
 struct StepArgs {
   int B, L, cap, d, n_exits;

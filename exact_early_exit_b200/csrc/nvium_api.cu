@@ -92,6 +92,8 @@ struct nv_state {
   // paged KV
   void* kv = nullptr;
   size_t kv_layer_stride = 0;
+  CUtensorMap kv_map;        // the pool as rows of 128 bytes (bf16, head_dim 64)
+  bool kv_map_ok = false;
   int n_pages = 0;
   int* page_table = nullptr;
   std::vector<int> h_page_table;
@@ -170,6 +172,7 @@ struct LayerIO {
   int L;
   int epi_grid;
   bool dec_attn;       // chunked decode attention (else row-group attention)
+  const CUtensorMap* kv_map;  // nullable: TMA view of the KV pool for the MMA decode attention
   bool prefetch_next;  // the last GEMM of a layer prefetches the next layer's QKV weights
   bool split_k;        // few rows expected (decode, flush): let the GEMM split K
   int* status;
@@ -277,6 +280,7 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   a.lens = io.lens;
   a.L = io.L;
   a.status = io.status;
+  a.kv_map = io.dec_attn ? io.kv_map : nullptr;
   timed(prof, launches, (io.kv_splits > 1 || io.dec_attn) ? 2 : 1, NV_K_ATTENTION,
         (prof ? prof->kv_read : 0) + 2 * R * HQ * es, 0, [&] {
           if (io.dec_attn) launch_attention_decode(bf, a, st);
@@ -324,6 +328,7 @@ LayerIO state_io(nv_state* s) {
   io.L = s->m->L;
   io.epi_grid = 1184;
   io.dec_attn = s->dec_attn;
+  io.kv_map = s->kv_map_ok ? &s->kv_map : nullptr;
   io.prefetch_next = true;
   io.split_k = true;
   io.status = s->status;
@@ -807,6 +812,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
   {
     const size_t head_sm = (((size_t)cfg->max_batch * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * d * esz;
     cudaError_t e2 = kernels_set_smem_limits(head_sm, (size_t)(cfg->max_batch + 1) * 4);
+    if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_dec_mma_prepare();
     if (e2 != cudaSuccess) {
       set_error(std::string("shared memory limits: ") + cudaGetErrorString(e2));
       nv_destroy(M);
@@ -913,6 +919,15 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   cudaMemset(s->nstop, 0, (size_t)NV_MAX_EXITS * 4);
   cudaMemcpy(s->d_B, &B, 4, cudaMemcpyHostToDevice);
   s->tc_head = M->bf16 && M->gemm_kind == GEMM_TC && B >= 16 && M->V % 128 == 0 && M->d % 64 == 0;
+  {
+    // the MMA decode attention reads the pool through a tensor map: rows of
+    // 128 bytes, boxes of 64 positions, row coordinates within int32
+    const uint64_t rows = (uint64_t)M->L * s->kv_layer_stride / 64;
+    const char* ev = std::getenv("NVIUM_DEC_ATTN");
+    const bool want = !(ev && std::string(ev) == "simt");
+    if (want && s->dec_attn && M->bf16 && M->hd == 64 && rows < (1ull << 31))
+      s->kv_map_ok = encode_rows128_map(s->kv, rows, 64, &s->kv_map) == NV_OK;
+  }
   cudaMemset(s->status, 0, 4);
   cudaMemset(s->nrows, 0, 4);
   cudaMemset(s->lens, 0, (size_t)B * M->L * 4);
