@@ -152,7 +152,7 @@ def measured_peaks():
 
 KERNEL_SOURCES = {
     "gemm": "exact_early_exit_b200/csrc/gemm_tc.cu",
-    "attention": "exact_early_exit_b200/csrc/attn_dec_mma.cu",
+    "attention": "exact_early_exit_b200/csrc/attn_mma.cu",
     "head": "exact_early_exit_b200/csrc/kernels.cu",
     "epilogue": "exact_early_exit_b200/csrc/kernels.cu",
     "plan_norm": "exact_early_exit_b200/csrc/kernels.cu",

@@ -1,5 +1,8 @@
-// Decode / flush attention for bf16 caches with head_dim 64, on warp-level
-// bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation).
+// Attention for bf16 caches with head_dim 64 on warp-level bf16 tensor-core
+// MMAs (mma.sync m16n8k16, fp32 accumulation): k_attn_dec_mma for decode and
+// flush (few rows per sequence, keys split in 128-key chunks) and
+// k_attn_fa_mma for prefill and scoring (64-row query tiles streaming 64-key
+// tiles with an online softmax, flash-attention style).
 //
 // What it computes is the causal softmax attention of the LLaMA-2 backbone
 // ("N-vium: Mixture-of-Exits Transformer for Accelerated Exact Generation",
@@ -9,7 +12,7 @@
 // "Inferenz: Piggybacking": the layers above an exit run later, batched with
 // the next token that reaches them).
 //
-// Work split: one CTA per (sequence, head, 128-key chunk), 4 warps of 32 keys,
+// Decode work split: one CTA per (sequence, head, 128-key chunk), 4 warps of 32 keys,
 // up to 16 rows per pass (the M of the MMA).  Partials (unnormalised sum,
 // max, sum of weights) go to the same per-(row, head, chunk) slots as the
 // SIMT kernel's, and k_attn_dec_combine merges them.
@@ -288,15 +291,258 @@ __global__ void __launch_bounds__(128) k_attn_dec_mma(const __grid_constant__ CU
   if (a.lens && head == 0 && chunk == 0 && tid == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
 }
 
+// ---------------------------------------------------------------------------
+// Prefill / scoring: CTA (sequence, head, 64-row query tile), warp w owns
+// query rows 16w .. 16w+15 of the tile.  Key tiles of 64 positions (one TMA
+// box of K and one of V, 128-byte swizzled) stream through a 3-stage ring;
+// each tile is used by all four warps, then refilled.  Per tile and warp:
+// S = Q K^T (32 MMAs), causal mask, online softmax (running max m and sum l
+// per row, O rescaled when m grows), O += P V with P as a bf16 hi/lo pair (64
+// MMAs).  Rows of one sequence have consecutive positions; row p attends to
+// keys 0..p, all in the cache (the QKV epilogue wrote this pass's keys).
+// ---------------------------------------------------------------------------
+constexpr int FQ = 64;   // query rows per CTA
+constexpr int FK = 64;   // keys per tile (one box)
+constexpr int FST = 3;   // ring stages
+
+struct FaSmem {
+  __nv_bfloat16 K[FST][FK * HD];  // 8 KB per stage, 1024-byte aligned
+  __nv_bfloat16 V[FST][FK * HD];
+  __nv_bfloat16 Q[FQ * QLD];
+  uint64_t full[FST];
+  int abort;
+};
+constexpr size_t FA_SMEM_BYTES = sizeof(FaSmem) + 1024;
+
+__device__ __forceinline__ void fa_issue(FaSmem& S, const CUtensorMap* map, const AttnArgs& a, int b, int head,
+                                         int tile, int stage) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(&S.full[stage])),
+               "r"((uint32_t)(2 * BOX_BYTES))
+               : "memory");
+  const int pos = tile * FK;
+  tma_box(S.K[stage], map, &S.full[stage], (int)(a.kv.offset(a.layer, b, pos, head, 0) / HD));
+  tma_box(S.V[stage], map, &S.full[stage], (int)(a.kv.offset(a.layer, b, pos, head, 1) / HD));
+}
+
+// bounded wait on a ring stage by every thread; false once 2 s have passed
+__device__ __forceinline__ bool fa_wait(uint64_t* bar, uint32_t parity) {
+  unsigned long long t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, "
+        "p;\n\t}"
+        : "=r"(ok)
+        : "r"(saddr(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 63u) == 0u) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (i == 0) t0 = t;
+      else if (t - t0 > 2000000000ull) return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(128) k_attn_fa_mma(const __grid_constant__ CUtensorMap kvmap, AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
+  extern __shared__ unsigned char smem_raw[];
+  FaSmem& S = *reinterpret_cast<FaSmem*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  if (*a.rs.nrows == 0) return;
+  const int b = blockIdx.x, head = blockIdx.y;
+  const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
+  const int nrt = (s1 - s0 + FQ - 1) / FQ;
+  const int rt = nrt - 1 - (int)blockIdx.z;  // the longest (latest) row tiles start first
+  if (rt < 0) return;
+  const int g0 = s0 + rt * FQ, g1 = min(s1, g0 + FQ), nr = g1 - g0;
+  const int pos_last = a.rs.row_pos[g1 - 1];
+  const int ntk = pos_last / FK + 1;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    S.abort = 0;
+    for (int st = 0; st < FST; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&S.full[st])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int j = 0; j < FST && j < ntk; ++j) fa_issue(S, &kvmap, a, b, head, j, j);
+  }
+  const int H = a.H;
+  const __nv_bfloat16* qg = (const __nv_bfloat16*)a.q;
+  for (int i = tid; i < FQ * 8; i += 128) {
+    const int r = i >> 3, c = i & 7;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < nr) v = *reinterpret_cast<const uint4*>(qg + (size_t)(g0 + r) * H * HD + head * HD + c * 8);
+    *reinterpret_cast<uint4*>(S.Q + r * QLD + c * 8) = v;
+  }
+  __syncthreads();
+  const int w = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+  const int rl0 = 16 * w + g, rl1 = rl0 + 8;
+  const int p0 = rl0 < nr ? a.rs.row_pos[g0 + rl0] : -1;
+  const int p1 = rl1 < nr ? a.rs.row_pos[g0 + rl1] : -1;
+  const int pw = 16 * w < nr ? a.rs.row_pos[g0 + min(nr - 1, 16 * w + 15)] : -1;  // warp's last position
+  uint32_t qa[4][4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+    ldsm_x4(qa[ks], saddr(S.Q + (16 * w + (lane & 7) + 8 * ((lane >> 3) & 1)) * QLD + (2 * ks + (lane >> 4)) * 8));
+  float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+  float oc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oc[nt][e] = 0.f;
+  int failed_at = -1;
+  for (int j = 0; j < ntk; ++j) {
+    const int stg = j % FST;
+    if (!fa_wait(&S.full[stg], (uint32_t)((j / FST) & 1))) S.abort = 1;
+    const int k0 = j * FK;
+    if (j == ntk - 1 && pos_last + 1 - k0 < FK) {
+      // V rows past the last key may be stale or never written: zero them
+      // (P is 0 there, and 0 * NaN would poison the sums)
+      const int nk = pos_last + 1 - k0;
+      for (int i = nk * 8 + tid; i < FK * 8; i += 128)
+        *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.V[stg]) + (i >> 3) * 128 + (i & 7) * 16) =
+            make_uint4(0, 0, 0, 0);
+      __syncthreads();
+    }
+    if (pw >= k0) {
+      const uint32_t kb_ = saddr(S.K[stg]), vb_ = saddr(S.V[stg]);
+      float sc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+        const int r = 8 * nt + (lane & 7);
+#pragma unroll
+        for (int kp = 0; kp < 2; ++kp) {
+          uint32_t kb[4];
+          ldsm_x4(kb, kb_ + swz(r, 4 * kp + (lane >> 3)));
+          mma_bf16(sc[nt], qa[2 * kp], kb[0], kb[1]);
+          mma_bf16(sc[nt], qa[2 * kp + 1], kb[2], kb[3]);
+        }
+      }
+      float t0 = -CUDART_INF_F, t1 = -CUDART_INF_F;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kk = k0 + 8 * nt + 2 * tq + (e & 1);
+          const bool hi = e >= 2;
+          const float v = kk <= (hi ? p1 : p0) ? sc[nt][e] * a.scale : -CUDART_INF_F;
+          sc[nt][e] = v;
+          if (hi) t1 = fmaxf(t1, v); else t0 = fmaxf(t0, v);
+        }
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+        t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, o));
+      }
+      const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+      const float c0 = n0 == -CUDART_INF_F ? 1.f : expf(m0 - n0);
+      const float c1 = n1 == -CUDART_INF_F ? 1.f : expf(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool hi = e >= 2;
+          const float m = hi ? n1 : n0;
+          const float pr = m == -CUDART_INF_F ? 0.f : expf(sc[nt][e] - m);
+          sc[nt][e] = pr;
+          if (hi) a1 += pr; else a0 += pr;
+        }
+      l0 = l0 * c0 + a0;  // this thread's columns; the quad is summed at the end
+      l1 = l1 * c1 + a1;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        oc[nt][0] *= c0;
+        oc[nt][1] *= c0;
+        oc[nt][2] *= c1;
+        oc[nt][3] *= c1;
+      }
+#pragma unroll
+      for (int kq = 0; kq < 4; ++kq) {
+        uint32_t ph[4], pl[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const float x0 = sc[2 * kq + h][2 * rr], x1 = sc[2 * kq + h][2 * rr + 1];
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+            ph[2 * h + rr] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+            pl[2 * h + rr] = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+          }
+        const int r = 16 * kq + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t vb[4];
+          ldsm_x4_t(vb, vb_ + swz(r, 2 * np + (lane >> 4)));
+          mma_bf16(oc[2 * np], ph, vb[0], vb[1]);
+          mma_bf16(oc[2 * np], pl, vb[0], vb[1]);
+          mma_bf16(oc[2 * np + 1], ph, vb[2], vb[3]);
+          mma_bf16(oc[2 * np + 1], pl, vb[2], vb[3]);
+        }
+      }
+    }
+    __syncthreads();  // every warp is done with this stage
+    if (S.abort) {
+      failed_at = j;
+      break;
+    }
+    if (tid == 0 && j + FST < ntk) fa_issue(S, &kvmap, a, b, head, j + FST, stg);
+  }
+  if (failed_at >= 0) {
+    if (tid == 0) {
+      dev_fail(a.status, DEV_ERR_TIMEOUT);
+      // tiles failed_at .. failed_at + FST - 1 were issued and not consumed:
+      // let those copies land before the CTA leaves (each wait bounded)
+      for (int t = failed_at; t < failed_at + FST && t < ntk; ++t)
+        if (!fa_wait(&S.full[t % FST], (uint32_t)((t / FST) & 1))) break;
+    }
+    return;
+  }
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  __nv_bfloat16* og = (__nv_bfloat16*)a.o;
+  if (rl0 < nr) {
+    const float inv = 1.0f / l0;
+    __nv_bfloat16* orow = og + (size_t)(g0 + rl0) * H * HD + head * HD;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      *reinterpret_cast<__nv_bfloat162*>(orow + 8 * nt + 2 * tq) = __floats2bfloat162_rn(oc[nt][0] * inv, oc[nt][1] * inv);
+  }
+  if (rl1 < nr) {
+    const float inv = 1.0f / l1;
+    __nv_bfloat16* orow = og + (size_t)(g0 + rl1) * H * HD + head * HD;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      *reinterpret_cast<__nv_bfloat162*>(orow + 8 * nt + 2 * tq) = __floats2bfloat162_rn(oc[nt][2] * inv, oc[nt][3] * inv);
+  }
+  if (a.lens && head == 0 && g1 == s1 && tid == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
+}
+
 }  // namespace
 
-cudaError_t attn_dec_mma_prepare() {
-  return cudaFuncSetAttribute(k_attn_dec_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DEC_SMEM_BYTES);
+cudaError_t attn_mma_prepare() {
+  cudaError_t e = cudaFuncSetAttribute(k_attn_dec_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DEC_SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_attn_fa_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FA_SMEM_BYTES);
+  return e;
 }
 
 void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st) {
   dim3 grid(a.rs.B, a.H, a.kv_splits);
   launch_k(k_attn_dec_mma, grid, 128, DEC_SMEM_BYTES, st, *kvmap, a);
+}
+
+void launch_attn_fa_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st) {
+  dim3 grid(a.rs.B, a.H, (a.row_groups * ATTN_RPC + FQ - 1) / FQ);
+  launch_k(k_attn_fa_mma, grid, 128, FA_SMEM_BYTES, st, *kvmap, a);
 }
 
 }  // namespace nv

@@ -930,6 +930,10 @@ static void attention_t(const AttnArgs& a, cudaStream_t st) {
   }
 }
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st) {
+  if (bf16 && a.hd == 64 && a.kv_map && a.kv_splits == 1) {
+    launch_attn_fa_mma(a.kv_map, a, st);
+    return;
+  }
   if (a.hd == 64) {
     if (bf16) attention_t<__nv_bfloat16, 64>(a, st); else attention_t<float, 64>(a, st);
   } else {

@@ -98,10 +98,13 @@ void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
 // head_dim * element size == 128 bytes and page_size == 64.
 constexpr int ATTN_DEC_CK = 128;
 void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st);
-// bf16 / head_dim 64 decode attention on warp MMAs (attn_dec_mma.cu); needs
-// a.kv_map.  Same partial slots as the SIMT kernel, merged by its combine.
-cudaError_t attn_dec_mma_prepare();
+// bf16 / head_dim 64 attention on warp MMAs (attn_mma.cu); both need
+// a.kv_map.  Decode: same partial slots as the SIMT kernel, merged by its
+// combine.  Prefill / scoring (kv_splits == 1): 64-row query tiles, grid z
+// from a.row_groups (units of ATTN_RPC rows).
+cudaError_t attn_mma_prepare();
 void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st);
+void launch_attn_fa_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st);
 
 struct StepArgs {
   int B, L, cap, d, n_exits;

@@ -42,6 +42,13 @@ nv_status dalloc_bytes(void** p, size_t bytes) { return dalloc((unsigned char**)
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// bf16 / head_dim 64 attention runs on the warp-MMA kernels unless
+// NVIUM_ATTN=simt selects the SIMT ones (kept for comparison)
+bool mma_attention_enabled() {
+  const char* ev = std::getenv("NVIUM_ATTN");
+  return !(ev && std::string(ev) == "simt");
+}
+
 constexpr int kTileCounters = 1024;  // >= N/128 of any split GEMM
 size_t tc_split_stride_elems(int N) { return nv::tc_split_stride((size_t)N); }
 
@@ -172,7 +179,7 @@ struct LayerIO {
   int L;
   int epi_grid;
   bool dec_attn;       // chunked decode attention (else row-group attention)
-  const CUtensorMap* kv_map;  // nullable: TMA view of the KV pool for the MMA decode attention
+  const CUtensorMap* kv_map;  // nullable: TMA view of the KV pool for the MMA attention kernels
   bool prefetch_next;  // the last GEMM of a layer prefetches the next layer's QKV weights
   bool split_k;        // few rows expected (decode, flush): let the GEMM split K
   int* status;
@@ -280,7 +287,7 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   a.lens = io.lens;
   a.L = io.L;
   a.status = io.status;
-  a.kv_map = io.dec_attn ? io.kv_map : nullptr;
+  a.kv_map = io.kv_map;
   timed(prof, launches, (io.kv_splits > 1 || io.dec_attn) ? 2 : 1, NV_K_ATTENTION,
         (prof ? prof->kv_read : 0) + 2 * R * HQ * es, 0, [&] {
           if (io.dec_attn) launch_attention_decode(bf, a, st);
@@ -812,7 +819,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
   {
     const size_t head_sm = (((size_t)cfg->max_batch * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * d * esz;
     cudaError_t e2 = kernels_set_smem_limits(head_sm, (size_t)(cfg->max_batch + 1) * 4);
-    if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_dec_mma_prepare();
+    if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_mma_prepare();
     if (e2 != cudaSuccess) {
       set_error(std::string("shared memory limits: ") + cudaGetErrorString(e2));
       nv_destroy(M);
@@ -923,9 +930,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
     // the MMA decode attention reads the pool through a tensor map: rows of
     // 128 bytes, boxes of 64 positions, row coordinates within int32
     const uint64_t rows = (uint64_t)M->L * s->kv_layer_stride / 64;
-    const char* ev = std::getenv("NVIUM_DEC_ATTN");
-    const bool want = !(ev && std::string(ev) == "simt");
-    if (want && s->dec_attn && M->bf16 && M->hd == 64 && rows < (1ull << 31))
+    if (mma_attention_enabled() && s->dec_attn && M->bf16 && M->hd == 64 && rows < (1ull << 31))
       s->kv_map_ok = encode_rows128_map(s->kv, rows, 64, &s->kv_map) == NV_OK;
   }
   cudaMemset(s->status, 0, 4);
@@ -1040,6 +1045,7 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
     LayerIO io{};
     io.rs = RowSet{d_n, d_b, d_pos, d_hrow, d_seq, h.as<float>(), cr, B};
     io.kv = state_kv(s);
+    io.kv_map = s->kv_map_ok ? &s->kv_map : nullptr;
     io.act = act.p;
     io.u = u.p;
     io.tile_counters = ctr.as<int>();
@@ -1434,6 +1440,13 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
   io.kv.page_size = ps;
   io.kv.H = M->H;
   io.kv.hd = M->hd;
+  CUtensorMap sc_map;
+  {
+    const uint64_t rows = (uint64_t)B * pps * 2 * M->HQ * ps / 64;
+    if (mma_attention_enabled() && M->bf16 && M->hd == 64 && ps % 64 == 0 && rows < (1ull << 31) &&
+        encode_rows128_map(M->sc_kv.p, rows, 64, &sc_map) == NV_OK)
+      io.kv_map = &sc_map;
+  }
   io.act = M->sc_act.p;
   io.u = M->sc_u.p;
   io.tile_counters = M->sc_ctr.as<int>();

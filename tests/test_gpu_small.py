@@ -126,12 +126,12 @@ def test_mma_and_simt_decode_attention_agree(weights):
     out = {}
     for eng in ("simt", "mma"):
         if eng == "simt":
-            os.environ["NVIUM_DEC_ATTN"] = "simt"
+            os.environ["NVIUM_ATTN"] = "simt"
         try:
             m = nv.Model(CFG, weights, max_batch=4, max_seq=640)
             st = nv.State(m, 4)
         finally:
-            os.environ.pop("NVIUM_DEC_ATTN", None)
+            os.environ.pop("NVIUM_ATTN", None)
         st.prefill(np.concatenate(prompts).astype(np.int32), lens)
         toks, exs, lps = [], [], []
         tok, ex, lp = np.zeros(4, np.int32), np.zeros(4, np.int32), np.zeros(4, np.float32)
@@ -150,3 +150,24 @@ def test_mma_and_simt_decode_attention_agree(weights):
     # different fp32 summation orders flip bf16 roundings of attention outputs,
     # which propagate through the layers: the bound is the path's tolerance
     np.testing.assert_allclose(l0[same], l1[same], atol=tolerance(CFG), rtol=0)
+
+
+def test_mma_and_simt_scoring_attention_agree(weights):
+    """Flash-style MMA attention (64-row query tiles, 64-key tiles, online
+    softmax) and the SIMT row-group kernel score the same sequences alike:
+    several query and key tiles, ragged tails (700 = 10 x 64 + 60)."""
+    toks = np.stack([W.make_prompts(W.WORKLOADS["S"], seed=s, lengths=[701])[0] for s in (3, 4)]).astype(np.int32)
+    out = {}
+    for eng in ("simt", "mma"):
+        if eng == "simt":
+            os.environ["NVIUM_ATTN"] = "simt"
+        try:
+            m = nv.Model(CFG, weights, max_batch=1, max_seq=704)
+        finally:
+            os.environ.pop("NVIUM_ATTN", None)
+        lp = np.zeros((2, 700), np.float32)
+        m.score_mixture(toks, lp)
+        out[eng] = lp
+        m.close()
+    assert np.all(np.isfinite(out["mma"]))
+    np.testing.assert_allclose(out["mma"], out["simt"], atol=tolerance(CFG), rtol=0)
