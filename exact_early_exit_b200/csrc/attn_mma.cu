@@ -1,6 +1,7 @@
 // Attention for bf16 caches with head_dim 64 on warp-level bf16 tensor-core
 // MMAs (mma.sync m16n8k16, fp32 accumulation): k_attn_dec_mma for decode and
-// flush (few rows per sequence, keys split in 128-key chunks) and
+// flush (few rows per sequence; a CTA streams a sequence's keys for one head,
+// or a range of them when splits are needed to fill the GPU) and
 // k_attn_fa_mma for prefill and scoring (64-row query tiles streaming 64-key
 // tiles with an online softmax, flash-attention style).
 //
@@ -12,16 +13,11 @@
 // "Inferenz: Piggybacking": the layers above an exit run later, batched with
 // the next token that reaches them).
 //
-// Decode work split: one CTA per (sequence, head, 128-key chunk), 4 warps of 32 keys,
-// up to 16 rows per pass (the M of the MMA).  Partials (unnormalised sum,
-// max, sum of weights) go to the same per-(row, head, chunk) slots as the
-// SIMT kernel's, and k_attn_dec_combine merges them.
-//
-// Data movement: the chunk's K and V (two 64-position boxes each) come in by
-// TMA through a 2-D tensor map over the whole KV pool (rows of 64 bf16 =
-// 128 bytes, 128-byte swizzle), so the ldmatrix reads of 8 consecutive keys
-// hit 8 different bank groups.  One thread waits on the transaction barrier;
-// the others wait at the CTA barrier and spend no issue slots.
+// Data movement: K and V arrive in 64-position boxes by TMA through a 2-D
+// tensor map over the whole KV pool (rows of 64 bf16 = 128 bytes, 128-byte
+// swizzle), so the ldmatrix reads of 8 consecutive keys hit 8 different bank
+// groups.  Barrier waits are done by one lane (or thread) while the others
+// wait at a warp or CTA barrier, spending no issue slots.
 //
 // Numerics: q and the cache are bf16 (the bf16 contract of the model), S =
 // q k^T accumulates in fp32; the softmax weights P are fp32 and enter the PV
@@ -44,15 +40,6 @@ constexpr int OLD = HD + 2;      // per-warp partial row: HD sums, max, weight s
 constexpr int BOX = 64;          // positions per TMA box (a page holds 64 or 128)
 constexpr int BOX_BYTES = BOX * HD * 2;
 
-struct DecSmem {
-  __nv_bfloat16 K[CK * HD];  // 16 KB, 1024-byte aligned (swizzle atom)
-  __nv_bfloat16 V[CK * HD];  // 16 KB
-  __nv_bfloat16 Q[RG * QLD];
-  float O[4][RG][OLD];
-  uint64_t bar;
-  int abort;
-};
-constexpr size_t DEC_SMEM_BYTES = sizeof(DecSmem) + 1024;  // + alignment slack
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(const_cast<void*>(p));
@@ -89,206 +76,6 @@ __device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, uint6
       "[%2];" ::"r"(saddr(dst)),
       "l"(map), "r"(saddr(bar)), "r"(0), "r"(row)
       : "memory");
-}
-
-__global__ void __launch_bounds__(128) k_attn_dec_mma(const __grid_constant__ CUtensorMap kvmap, AttnArgs a) {
-  pdl_wait();
-  pdl_launch();
-  extern __shared__ unsigned char smem_raw[];
-  DecSmem& S = *reinterpret_cast<DecSmem*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  if (*a.rs.nrows == 0) return;
-  const int b = blockIdx.x, head = blockIdx.y, chunk = blockIdx.z;
-  const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
-  if (s0 >= s1) return;
-  const int pos_last = a.rs.row_pos[s1 - 1];
-  const int k0 = chunk * CK;
-  if (k0 > pos_last) return;
-  const int nk = min(CK, pos_last + 1 - k0);
-  const int nbox = (nk + BOX - 1) / BOX;
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    S.abort = 0;
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&S.bar)) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(&S.bar)),
-                 "r"((uint32_t)(2 * nbox * BOX_BYTES))
-                 : "memory");
-    for (int i = 0; i < nbox; ++i) {
-      const int pos = k0 + i * BOX;
-      tma_box(S.K + i * BOX * HD, &kvmap, &S.bar, (int)(a.kv.offset(a.layer, b, pos, head, 0) / HD));
-      tma_box(S.V + i * BOX * HD, &kvmap, &S.bar, (int)(a.kv.offset(a.layer, b, pos, head, 1) / HD));
-    }
-  }
-  const int H = a.H;
-  const __nv_bfloat16* qg = (const __nv_bfloat16*)a.q;
-  const int pos0 = a.rs.row_pos[s0];
-  const int first = max(s0, s0 + (k0 - pos0));  // rows whose position reaches this chunk
-  const int w = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
-  if (tid == 0) {
-    unsigned long long t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-      uint32_t ok;
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\tselp.u32 %0, 1, 0, "
-          "p;\n\t}"
-          : "=r"(ok)
-          : "r"(saddr(&S.bar))
-          : "memory");
-      if (ok) break;
-      if ((i & 15u) == 0u) {
-        unsigned long long t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        if (i == 0) t0 = t;
-        else if (t - t0 > 2000000000ull) {
-          S.abort = 1;
-          break;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  if (S.abort) {
-    if (tid == 0) dev_fail(a.status, DEV_ERR_TIMEOUT);
-    return;
-  }
-  // V rows past the last key may hold stale or never-written bytes; P is zero
-  // there, so zero V too (0 * NaN would poison the sums)
-  for (int i = nk * 8 + tid; i < nbox * BOX * 8; i += blockDim.x)
-    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.V) + (i >> 3) * 128 + (i & 7) * 16) =
-        make_uint4(0, 0, 0, 0);
-  for (int g0 = first; g0 < s1; g0 += RG) {
-    const int ng = min(RG, s1 - g0);
-    {  // Q rows of this pass (16 rows x 8 chunks: one chunk per thread), zero padding
-      const int r = tid >> 3, c = tid & 7;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < ng) v = *reinterpret_cast<const uint4*>(qg + (size_t)(g0 + r) * H * HD + head * HD + c * 8);
-      *reinterpret_cast<uint4*>(S.Q + r * QLD + c * 8) = v;
-    }
-    __syncthreads();
-
-    // S = Q K^T for this warp's 32 keys: 4 n-tiles of 8 keys, 4 k-steps of 16 dims
-    uint32_t qa[4][4];
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-      ldsm_x4(qa[ks], saddr(S.Q + ((lane & 7) + 8 * ((lane >> 3) & 1)) * QLD + (2 * ks + (lane >> 4)) * 8));
-    float sc[4][4];
-    const uint32_t kbase = saddr(S.K), vbase = saddr(S.V);
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-      const int r = 32 * w + 8 * nt + (lane & 7);
-#pragma unroll
-      for (int kp = 0; kp < 2; ++kp) {
-        uint32_t kb[4];
-        ldsm_x4(kb, kbase + swz(r, 4 * kp + (lane >> 3)));
-        mma_bf16(sc[nt], qa[2 * kp], kb[0], kb[1]);
-        mma_bf16(sc[nt], qa[2 * kp + 1], kb[2], kb[3]);
-      }
-    }
-    // causal / length mask, this warp's row maxima and weights
-    const int p_lo = pos0 + (g0 + g - s0), p_hi = p_lo + 8;  // positions of rows g and g + 8
-    const bool v_lo = g < ng, v_hi = g + 8 < ng;
-    float m_lo = -CUDART_INF_F, m_hi = -CUDART_INF_F;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kk = 32 * w + 8 * nt + 2 * tq + (e & 1);
-        const bool hi = e >= 2;
-        const bool ok = kk < nk && (hi ? (v_hi && k0 + kk <= p_hi) : (v_lo && k0 + kk <= p_lo));
-        const float s = ok ? sc[nt][e] * a.scale : -CUDART_INF_F;
-        sc[nt][e] = s;
-        if (hi) m_hi = fmaxf(m_hi, s); else m_lo = fmaxf(m_lo, s);
-      }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      m_lo = fmaxf(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
-      m_hi = fmaxf(m_hi, __shfl_xor_sync(0xffffffffu, m_hi, o));
-    }
-    float l_lo = 0.f, l_hi = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool hi = e >= 2;
-        const float m = hi ? m_hi : m_lo;
-        const float p = m == -CUDART_INF_F ? 0.f : expf(sc[nt][e] - m);
-        sc[nt][e] = p;
-        if (hi) l_hi += p; else l_lo += p;
-      }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, o);
-      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, o);
-    }
-    // O = P V: P as a bf16 hi/lo pair, 2 k-steps of 16 keys, 8 n-tiles of 8 dims
-    float oc[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) oc[nt][e] = 0.f;
-#pragma unroll
-    for (int kq = 0; kq < 2; ++kq) {
-      uint32_t ph[4], pl[4];
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const float x0 = sc[2 * kq + h][2 * rr], x1 = sc[2 * kq + h][2 * rr + 1];
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-          ph[2 * h + rr] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-          pl[2 * h + rr] = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-        }
-      const int r = 32 * w + 16 * kq + (lane & 7) + 8 * ((lane >> 3) & 1);
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t vb[4];
-        ldsm_x4_t(vb, vbase + swz(r, 2 * np + (lane >> 4)));
-        mma_bf16(oc[2 * np], ph, vb[0], vb[1]);
-        mma_bf16(oc[2 * np], pl, vb[0], vb[1]);
-        mma_bf16(oc[2 * np + 1], ph, vb[2], vb[3]);
-        mma_bf16(oc[2 * np + 1], pl, vb[2], vb[3]);
-      }
-    }
-    // per-warp partials to shared memory, then one merge per row
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      *reinterpret_cast<float2*>(&S.O[w][g][8 * nt + 2 * tq]) = make_float2(oc[nt][0], oc[nt][1]);
-      *reinterpret_cast<float2*>(&S.O[w][g + 8][8 * nt + 2 * tq]) = make_float2(oc[nt][2], oc[nt][3]);
-    }
-    if (tq == 0) {
-      S.O[w][g][HD] = m_lo;
-      S.O[w][g][HD + 1] = l_lo;
-      S.O[w][g + 8][HD] = m_hi;
-      S.O[w][g + 8][HD + 1] = l_hi;
-    }
-    __syncthreads();
-    for (int j = w; j < ng; j += 4) {
-      float M = -CUDART_INF_F;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) M = fmaxf(M, S.O[q][j][HD]);
-      float L = 0.f, acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float mq = S.O[q][j][HD];
-        if (mq == -CUDART_INF_F) continue;
-        const float e = expf(mq - M);
-        L += S.O[q][j][HD + 1] * e;
-        const float2 v = *reinterpret_cast<const float2*>(&S.O[q][j][2 * lane]);
-        acc0 += v.x * e;
-        acc1 += v.y * e;
-      }
-      float* pp = a.part + (((size_t)(g0 + j) * H + head) * a.kv_splits + chunk) * OLD;
-      *reinterpret_cast<float2*>(pp + 2 * lane) = make_float2(acc0, acc1);
-      if (lane == 0) {
-        pp[HD] = M;
-        pp[HD + 1] = L;
-      }
-    }
-    __syncthreads();
-  }
-  if (a.lens && head == 0 && chunk == 0 && tid == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
 }
 
 // ---------------------------------------------------------------------------
@@ -343,6 +130,316 @@ __device__ __forceinline__ bool fa_wait(uint64_t* bar, uint32_t parity) {
       else if (t - t0 > 2000000000ull) return false;
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Decode / flush: CTA (sequence, head, split).  The split owns a contiguous
+// range of the sequence's 64-key tiles (all of them when there is one
+// split).  Warp 4 streams the range through a DS-stage TMA ring; consumer
+// warp w takes tiles w, w+4, ... for the sequence's rows (16 per pass) with
+// an online softmax, and the four warps merge once per pass.  One split: the
+// CTA writes the normalised output rows; several: unnormalised partials
+// (sum, max, weight sum) per (row, head, split), and the last split CTA of
+// the (sequence, head) to finish (a per-pair arrival counter) merges them in
+// split order, so the result does not depend on which CTA came last.
+// ---------------------------------------------------------------------------
+constexpr int DS = 4;
+constexpr int DEC_THREADS = 160;
+struct DecSmem {
+  __nv_bfloat16 K[DS][BOX * HD];  // 8 KB per stage, 1024-byte aligned
+  __nv_bfloat16 V[DS][BOX * HD];
+  __nv_bfloat16 Q[RG * QLD];
+  uint64_t full[DS], empty[DS];
+  int abort;
+};
+// the per-pass merge buffer [4 warps][16 rows][HD + 2] reuses the idle ring
+static_assert(4 * RG * OLD * 4 <= 2 * DS * BOX * HD * 2, "merge buffer fits in the ring");
+constexpr size_t DEC_SMEM_BYTES = sizeof(DecSmem) + 1024;
+
+// lane 0 waits (bounded), the warp follows
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = fa_wait(bar, parity) ? 1 : 0;
+  __syncwarp();
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Called by every split CTA of (b, head) after its partials are written; the
+// last to arrive merges the splits of each row of b in split order (the same
+// order for any arrival order) and writes the normalised output.
+__device__ __forceinline__ void dec_merge_splits(const AttnArgs& a, int b, int head, int s0, int s1) {
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* c = a.dec_ctr + b * a.H + head;
+    const int last = atomicAdd(c, 1) == (int)gridDim.z - 1;
+    if (last) *c = 0;  // every split has arrived: ready for the next launch
+    s_last = last;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int H = a.H, nsp = gridDim.z, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int r = s0 + (int)(threadIdx.x >> 5); r < s1; r += nw) {
+    const float* pp = a.part + ((size_t)r * H + head) * a.kv_splits * OLD;
+    float M = -CUDART_INF_F;
+    for (int q = 0; q < nsp; ++q) M = fmaxf(M, __ldcg(pp + q * OLD + HD));
+    float L = 0.f, acc0 = 0.f, acc1 = 0.f;
+    for (int q = 0; q < nsp; ++q) {
+      const float mq = __ldcg(pp + q * OLD + HD);
+      if (mq == -CUDART_INF_F) continue;
+      const float e = expf(mq - M);
+      L += __ldcg(pp + q * OLD + HD + 1) * e;
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(pp + q * OLD + 2 * lane));
+      acc0 += v.x * e;
+      acc1 += v.y * e;
+    }
+    const float inv = 1.0f / L;
+    *reinterpret_cast<__nv_bfloat162*>((__nv_bfloat16*)a.o + (size_t)r * H * HD + head * HD + 2 * lane) =
+        __floats2bfloat162_rn(acc0 * inv, acc1 * inv);
+  }
+}
+
+__global__ void __launch_bounds__(DEC_THREADS, 3) k_attn_dec_mma(const __grid_constant__ CUtensorMap kvmap, AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
+  extern __shared__ unsigned char smem_raw[];
+  DecSmem& S = *reinterpret_cast<DecSmem*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  if (*a.rs.nrows == 0) return;
+  const int b = blockIdx.x, head = blockIdx.y, sp = blockIdx.z, nsp = gridDim.z;
+  const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
+  if (s0 >= s1) return;
+  const int pos_last = a.rs.row_pos[s1 - 1];
+  const int ntk = pos_last / BOX + 1;
+  const int tps = (ntk + nsp - 1) / nsp;
+  const int t_beg = min(ntk, sp * tps), t_end = min(ntk, t_beg + tps);
+  const int nt = t_end - t_beg;
+  const int npass = (s1 - s0 + RG - 1) / RG;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
+  if (tid == 0) {
+    S.abort = 0;
+    for (int st = 0; st < DS; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&S.full[st])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&S.empty[st])) : "memory");
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const int H = a.H;
+  const __nv_bfloat16* qg = (const __nv_bfloat16*)a.q;
+  float(*Ob)[RG][OLD] = reinterpret_cast<float(*)[RG][OLD]>(&S.K[0][0]);
+  int q_base = 0;  // ring uses before this pass
+  for (int pass = 0; pass < npass; ++pass) {
+    const int g0 = s0 + pass * RG, ng = min(RG, s1 - g0);
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+    float oc[8][4];
+#pragma unroll
+    for (int nt8 = 0; nt8 < 8; ++nt8)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) oc[nt8][e] = 0.f;
+    if (w == 4) {
+      if (lane == 0) {
+        for (int i = 0; i < nt; ++i) {
+          const int q = q_base + i, st = q % DS;
+          if (q >= DS && !fa_wait(&S.empty[st], (uint32_t)((q / DS - 1) & 1))) {
+            S.abort = 1;
+            break;
+          }
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(&S.full[st])),
+                       "r"((uint32_t)(2 * BOX_BYTES))
+                       : "memory");
+          const int pos = (t_beg + i) * BOX;
+          tma_box(S.K[st], &kvmap, &S.full[st], (int)(a.kv.offset(a.layer, b, pos, head, 0) / HD));
+          tma_box(S.V[st], &kvmap, &S.full[st], (int)(a.kv.offset(a.layer, b, pos, head, 1) / HD));
+        }
+      }
+    } else {
+      {  // this pass's query rows (16 rows x 8 chunks: one chunk per consumer thread)
+        const int r = tid >> 3, c = tid & 7;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < ng) v = *reinterpret_cast<const uint4*>(qg + (size_t)(g0 + r) * H * HD + head * HD + c * 8);
+        *reinterpret_cast<uint4*>(S.Q + r * QLD + c * 8) = v;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      uint32_t qa[4][4];
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        ldsm_x4(qa[ks], saddr(S.Q + ((lane & 7) + 8 * ((lane >> 3) & 1)) * QLD + (2 * ks + (lane >> 4)) * 8));
+      const int p0 = g < ng ? a.rs.row_pos[g0 + g] : -1;
+      const int p1 = g + 8 < ng ? a.rs.row_pos[g0 + g + 8] : -1;
+      for (int i = w; i < nt; i += 4) {
+        const int q = q_base + i, st = q % DS;
+        if (!warp_wait(&S.full[st], (uint32_t)((q / DS) & 1))) {
+          S.abort = 1;
+          break;
+        }
+        const int k0 = (t_beg + i) * BOX;
+        if (k0 + BOX > pos_last + 1) {
+          // V rows past the last key may be stale or never written: zero them
+          // (P is 0 there, and 0 * NaN would poison the sums)
+          for (int e = (pos_last + 1 - k0) * 8 + lane; e < BOX * 8; e += 32)
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.V[st]) + (e >> 3) * 128 + (e & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+        }
+        const uint32_t kb_ = saddr(S.K[st]), vb_ = saddr(S.V[st]);
+        float sc[8][4];
+#pragma unroll
+        for (int n8 = 0; n8 < 8; ++n8) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[n8][e] = 0.f;
+          const int r = 8 * n8 + (lane & 7);
+#pragma unroll
+          for (int kp = 0; kp < 2; ++kp) {
+            uint32_t kb[4];
+            ldsm_x4(kb, kb_ + swz(r, 4 * kp + (lane >> 3)));
+            mma_bf16(sc[n8], qa[2 * kp], kb[0], kb[1]);
+            mma_bf16(sc[n8], qa[2 * kp + 1], kb[2], kb[3]);
+          }
+        }
+        float t0 = -CUDART_INF_F, t1 = -CUDART_INF_F;
+#pragma unroll
+        for (int n8 = 0; n8 < 8; ++n8)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int kk = k0 + 8 * n8 + 2 * tq + (e & 1);
+            const bool hi = e >= 2;
+            const float v = kk <= (hi ? p1 : p0) ? sc[n8][e] * a.scale : -CUDART_INF_F;
+            sc[n8][e] = v;
+            if (hi) t1 = fmaxf(t1, v); else t0 = fmaxf(t0, v);
+          }
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+          t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+          t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, o));
+        }
+        const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+        const float c0 = n0 == -CUDART_INF_F ? 1.f : expf(m0 - n0);
+        const float c1 = n1 == -CUDART_INF_F ? 1.f : expf(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int n8 = 0; n8 < 8; ++n8)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool hi = e >= 2;
+            const float m = hi ? n1 : n0;
+            const float pr = m == -CUDART_INF_F ? 0.f : expf(sc[n8][e] - m);
+            sc[n8][e] = pr;
+            if (hi) a1 += pr; else a0 += pr;
+          }
+        l0 = l0 * c0 + a0;  // this thread's columns; the quad is summed at the merge
+        l1 = l1 * c1 + a1;
+#pragma unroll
+        for (int n8 = 0; n8 < 8; ++n8) {
+          oc[n8][0] *= c0;
+          oc[n8][1] *= c0;
+          oc[n8][2] *= c1;
+          oc[n8][3] *= c1;
+        }
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          uint32_t ph[4], pl[4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const float x0 = sc[2 * kq + h][2 * rr], x1 = sc[2 * kq + h][2 * rr + 1];
+              const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+              ph[2 * h + rr] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+              pl[2 * h + rr] = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+            }
+          const int r = 16 * kq + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+          for (int np = 0; np < 4; ++np) {
+            uint32_t vb[4];
+            ldsm_x4_t(vb, vb_ + swz(r, 2 * np + (lane >> 4)));
+            mma_bf16(oc[2 * np], ph, vb[0], vb[1]);
+            mma_bf16(oc[2 * np], pl, vb[0], vb[1]);
+            mma_bf16(oc[2 * np + 1], ph, vb[2], vb[3]);
+            mma_bf16(oc[2 * np + 1], pl, vb[2], vb[3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(&S.empty[st])) : "memory");
+      }
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+    }
+    __syncthreads();  // pass end: every issued tile has been consumed, the ring is idle
+    if (S.abort) {
+      if (tid == 0) {
+        dev_fail(a.status, DEV_ERR_TIMEOUT);
+        // keep the pair's arrival count consistent for later launches
+        if (nsp > 1 && atomicAdd(a.dec_ctr + b * a.H + head, 1) == nsp - 1) a.dec_ctr[b * a.H + head] = 0;
+      }
+      if (tid == 128) {
+        // let this pass's copies land before the CTA leaves (each wait bounded)
+        for (int i = 0; i < nt; ++i) {
+          const int q = q_base + i;
+          if (!fa_wait(&S.full[q % DS], (uint32_t)((q / DS) & 1))) break;
+        }
+      }
+      return;
+    }
+    if (w < 4) {
+#pragma unroll
+      for (int n8 = 0; n8 < 8; ++n8) {
+        *reinterpret_cast<float2*>(&Ob[w][g][8 * n8 + 2 * tq]) = make_float2(oc[n8][0], oc[n8][1]);
+        *reinterpret_cast<float2*>(&Ob[w][g + 8][8 * n8 + 2 * tq]) = make_float2(oc[n8][2], oc[n8][3]);
+      }
+      if (tq == 0) {
+        Ob[w][g][HD] = m0;
+        Ob[w][g][HD + 1] = l0;
+        Ob[w][g + 8][HD] = m1;
+        Ob[w][g + 8][HD + 1] = l1;
+      }
+    }
+    __syncthreads();
+    if (w < 4) {
+      for (int j = w; j < ng; j += 4) {
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) M = fmaxf(M, Ob[u][j][HD]);
+        float L = 0.f, acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float mu = Ob[u][j][HD];
+          if (mu == -CUDART_INF_F) continue;
+          const float e = expf(mu - M);
+          L += Ob[u][j][HD + 1] * e;
+          const float2 v = *reinterpret_cast<const float2*>(&Ob[u][j][2 * lane]);
+          acc0 += v.x * e;
+          acc1 += v.y * e;
+        }
+        if (nsp == 1) {
+          const float inv = 1.0f / L;
+          *reinterpret_cast<__nv_bfloat162*>((__nv_bfloat16*)a.o + (size_t)(g0 + j) * H * HD + head * HD + 2 * lane) =
+              __floats2bfloat162_rn(acc0 * inv, acc1 * inv);
+        } else {
+          float* pp = a.part + (((size_t)(g0 + j) * H + head) * a.kv_splits + sp) * OLD;
+          *reinterpret_cast<float2*>(pp + 2 * lane) = make_float2(acc0, acc1);
+          if (lane == 0) {
+            pp[HD] = M;
+            pp[HD + 1] = L;
+          }
+        }
+      }
+    }
+    // the ring's next loads overwrite the merge buffer: order these generic
+    // accesses before them
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    q_base += nt;
+  }
+  if (a.lens && head == 0 && sp == 0 && tid == 0) a.lens[b * a.L + a.layer] = pos_last + 1;
+  if (nsp > 1) dec_merge_splits(a, b, head, s0, s1);
 }
 
 __global__ void __launch_bounds__(128) k_attn_fa_mma(const __grid_constant__ CUtensorMap kvmap, AttnArgs a) {
@@ -537,7 +634,7 @@ cudaError_t attn_mma_prepare() {
 
 void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st) {
   dim3 grid(a.rs.B, a.H, a.kv_splits);
-  launch_k(k_attn_dec_mma, grid, 128, DEC_SMEM_BYTES, st, *kvmap, a);
+  launch_k(k_attn_dec_mma, grid, DEC_THREADS, DEC_SMEM_BYTES, st, *kvmap, a);
 }
 
 void launch_attn_fa_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st) {

@@ -907,16 +907,25 @@ __global__ void k_attn_dec_combine(AttnArgs a) {
 
 template <typename T, int HD>
 static void attention_dec_t(const AttnArgs& a, cudaStream_t st) {
-  dim3 grid(a.rs.B, a.H, a.kv_splits);
-  if (a.kv_map && sizeof(T) == 2 && HD == 64) launch_attn_dec_mma(a.kv_map, a, st);
-  else launch_k(k_attn_dec<T, HD>, grid, 128, 0, st, a);
   int g = (a.rs.max_rows * a.H + 7) / 8;
   if (g > 4096) g = 4096;
+  if (a.kv_map && sizeof(T) == 2 && HD == 64) {
+    AttnArgs m = a;
+    m.kv_splits = a.dec_splits;
+    launch_attn_dec_mma(a.kv_map, m, st);
+    return;
+  }
+  dim3 grid(a.rs.B, a.H, a.kv_splits);
+  launch_k(k_attn_dec<T, HD>, grid, 128, 0, st, a);
   launch_k(k_attn_dec_combine<T, HD>, g, 256, 0, st, a);
 }
 void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st) {
   if (bf16) attention_dec_t<__nv_bfloat16, 64>(a, st);
   else attention_dec_t<float, 32>(a, st);
+}
+int attention_decode_launches(bool bf16, const AttnArgs& a) {
+  if (bf16 && a.kv_map) return 1;
+  return 2;
 }
 
 template <typename T, int HD>

@@ -91,6 +91,8 @@ struct AttnArgs {
   int L;
   int* status;     // device status word (bounded-wait expiry)
   const CUtensorMap* kv_map;  // host copy of the KV pool's 128-byte-row map (bf16, hd 64), or null
+  int dec_splits;             // MMA decode attention: key-range splits per (sequence, head)
+  int* dec_ctr;               // [B][H] split arrival counters (zero between launches)
 };
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
 // Decode / flush attention: 128-key chunks (grid z = kv_splits = chunks of
@@ -98,10 +100,14 @@ void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
 // head_dim * element size == 128 bytes and page_size == 64.
 constexpr int ATTN_DEC_CK = 128;
 void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st);
+// kernels launch_attention_decode runs for these arguments (1 or 2)
+int attention_decode_launches(bool bf16, const AttnArgs& a);
 // bf16 / head_dim 64 attention on warp MMAs (attn_mma.cu); both need
-// a.kv_map.  Decode: same partial slots as the SIMT kernel, merged by its
-// combine.  Prefill / scoring (kv_splits == 1): 64-row query tiles, grid z
-// from a.row_groups (units of ATTN_RPC rows).
+// a.kv_map.  Decode: grid z = a.kv_splits key-range splits; with more than
+// one, partials in the row-group kernel's slots, merged by the last split
+// CTA of each (sequence, head) (a.dec_ctr).
+// Prefill / scoring (kv_splits == 1): 64-row query tiles, grid z from
+// a.row_groups (units of ATTN_RPC rows).
 cudaError_t attn_mma_prepare();
 void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st);
 void launch_attn_fa_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st);

@@ -101,6 +101,8 @@ struct nv_state {
   size_t kv_layer_stride = 0;
   CUtensorMap kv_map;        // the pool as rows of 128 bytes (bf16, head_dim 64)
   bool kv_map_ok = false;
+  int dec_splits = 1;        // key-range splits per (sequence, head) of the MMA decode attention
+  int* dec_ctr = nullptr;    // [B][H] split arrival counters of that kernel
   int n_pages = 0;
   int* page_table = nullptr;
   std::vector<int> h_page_table;
@@ -134,7 +136,12 @@ struct nv_state {
   bool cond_graph = false;
   std::vector<void*> allocs;
   // prefill scratch
-  Buf pf_rows, pf_h, pf_tok;
+  // prefill working set, kept between calls (grow-only)
+  Buf pf_rows, pf_h, pf_act, pf_u, pf_q, pf_o, pf_Y, pf_ctr;
+  // page-table uploads go through a pinned copy, reusable once `pt_done` fired
+  int* h_pt_pinned = nullptr;
+  cudaEvent_t pt_done = nullptr;
+  bool pt_pending = false;
 };
 
 namespace {
@@ -180,6 +187,8 @@ struct LayerIO {
   int epi_grid;
   bool dec_attn;       // chunked decode attention (else row-group attention)
   const CUtensorMap* kv_map;  // nullable: TMA view of the KV pool for the MMA attention kernels
+  int dec_splits;             // key-range splits of the MMA decode attention
+  int* dec_ctr;               // its per-(sequence, head) split arrival counters
   bool prefetch_next;  // the last GEMM of a layer prefetches the next layer's QKV weights
   bool split_k;        // few rows expected (decode, flush): let the GEMM split K
   int* status;
@@ -288,7 +297,10 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   a.L = io.L;
   a.status = io.status;
   a.kv_map = io.kv_map;
-  timed(prof, launches, (io.kv_splits > 1 || io.dec_attn) ? 2 : 1, NV_K_ATTENTION,
+  a.dec_splits = io.dec_splits;
+  a.dec_ctr = io.dec_ctr;
+  const int attn_launches = io.dec_attn ? attention_decode_launches(bf, a) : (io.kv_splits > 1 ? 2 : 1);
+  timed(prof, launches, attn_launches, NV_K_ATTENTION,
         (prof ? prof->kv_read : 0) + 2 * R * HQ * es, 0, [&] {
           if (io.dec_attn) launch_attention_decode(bf, a, st);
           else launch_attention(bf, a, st);
@@ -336,6 +348,8 @@ LayerIO state_io(nv_state* s) {
   io.epi_grid = 1184;
   io.dec_attn = s->dec_attn;
   io.kv_map = s->kv_map_ok ? &s->kv_map : nullptr;
+  io.dec_splits = s->dec_splits;
+  io.dec_ctr = s->dec_ctr;
   io.prefetch_next = true;
   io.split_k = true;
   io.status = s->status;
@@ -636,10 +650,16 @@ nv_status ensure_pages(nv_state* s, int b, int upto, bool* changed) {
   return NV_OK;
 }
 
+// Stream-ordered upload of the host page table: copied into a pinned buffer
+// (after the previous upload has read it) and sent asynchronously, so a
+// decode step that opens a page does not stall the host.
 nv_status upload_page_table(nv_state* s, cudaStream_t st) {
-  NV_CUDA_TRY(cudaMemcpyAsync(s->page_table, s->h_page_table.data(), s->h_page_table.size() * sizeof(int),
-                              cudaMemcpyHostToDevice, st));
-  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  const size_t bytes = s->h_page_table.size() * sizeof(int);
+  if (s->pt_pending) NV_CUDA_TRY(cudaEventSynchronize(s->pt_done));
+  std::memcpy(s->h_pt_pinned, s->h_page_table.data(), bytes);
+  NV_CUDA_TRY(cudaMemcpyAsync(s->page_table, s->h_pt_pinned, bytes, cudaMemcpyHostToDevice, st));
+  NV_CUDA_TRY(cudaEventRecord(s->pt_done, st));
+  s->pt_pending = true;
   return NV_OK;
 }
 
@@ -917,6 +937,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   A((void**)&s->seed_dev, 8);
   A((void**)&s->counters, NV_CTR_COUNT * 8);
   A((void**)&s->status, 4);
+  A((void**)&s->dec_ctr, (size_t)B * M->H * 4);
   if (st != NV_OK) {
     nv_state_destroy(s);
     return st;
@@ -932,13 +953,23 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
     const uint64_t rows = (uint64_t)M->L * s->kv_layer_stride / 64;
     if (mma_attention_enabled() && s->dec_attn && M->bf16 && M->hd == 64 && rows < (1ull << 31))
       s->kv_map_ok = encode_rows128_map(s->kv, rows, 64, &s->kv_map) == NV_OK;
+    // enough (sequence, head, split) CTAs for two waves of three per SM, each
+    // split keeping at least two 64-key tiles
+    const int pairs = B * M->H, target = 2 * 3 * 148;
+    int sp = (target + pairs - 1) / pairs;
+    const int max_sp = std::max(1, (s->max_seq / 64) / 2);
+    sp = std::min(sp, std::min(max_sp, s->kv_splits));
+    s->dec_splits = std::max(1, sp);
   }
   cudaMemset(s->status, 0, 4);
+  cudaMemset(s->dec_ctr, 0, (size_t)B * M->H * 4);
   cudaMemset(s->nrows, 0, 4);
   cudaMemset(s->lens, 0, (size_t)B * M->L * 4);
   cudaMemset(s->t, 0, (size_t)B * 4);
   cudaMemset(s->page_table, 0xff, s->h_page_table.size() * 4);
-  cudaError_t e = cudaStreamCreateWithFlags(&s->cap_stream, cudaStreamNonBlocking);
+  cudaError_t e = cudaHostAlloc((void**)&s->h_pt_pinned, s->h_page_table.size() * 4, cudaHostAllocDefault);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s->pt_done, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s->cap_stream, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s->cap_stream2, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -958,9 +989,9 @@ nv_status nv_state_destroy(nv_state* s) {
   if (s->cap_stream) cudaStreamDestroy(s->cap_stream);
   if (s->cap_stream2) cudaStreamDestroy(s->cap_stream2);
   for (void* p : s->allocs) cudaFree(p);
-  s->pf_rows.release();
-  s->pf_h.release();
-  s->pf_tok.release();
+  for (Buf* b : {&s->pf_rows, &s->pf_h, &s->pf_act, &s->pf_u, &s->pf_q, &s->pf_o, &s->pf_Y, &s->pf_ctr}) b->release();
+  if (s->h_pt_pinned) cudaFreeHost(s->h_pt_pinned);
+  if (s->pt_done) cudaEventDestroy(s->pt_done);
   delete s;
   return NV_OK;
 }
@@ -982,7 +1013,18 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
     total += lens[b];
   }
   std::vector<int> htok(total);
-  NV_CUDA_TRY(cudaMemcpy(htok.data(), tokens, total * 4, cudaMemcpyDefault));
+  {
+    cudaPointerAttributes pa{};
+    const bool on_device = cudaPointerGetAttributes(&pa, tokens) == cudaSuccess &&
+                           (pa.type == cudaMemoryTypeDevice || pa.type == cudaMemoryTypeManaged);
+    cudaGetLastError();
+    if (on_device) {
+      NV_CUDA_TRY(cudaMemcpyAsync(htok.data(), tokens, total * 4, cudaMemcpyDeviceToHost, st));
+      NV_CUDA_TRY(cudaStreamSynchronize(st));
+    } else {
+      std::memcpy(htok.data(), tokens, total * 4);
+    }
+  }
   for (size_t i = 0; i < total; ++i)
     if (htok[i] < 0 || htok[i] >= M->V) {
       set_error("token id out of range");
@@ -1011,7 +1053,8 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
   const size_t wide = M->d > M->F ? M->d : M->F;
   // per-chunk buffers: h, act, q, o, Y, attention partials, row arrays
   const int cr = R < chunk ? (R > 0 ? R : 1) : chunk;
-  Buf h, act, u, q, o, Y, rows, ctr;
+  Buf &h = s->pf_h, &act = s->pf_act, &u = s->pf_u, &q = s->pf_q, &o = s->pf_o, &Y = s->pf_Y, &rows = s->pf_rows,
+      &ctr = s->pf_ctr;
   nv_status stt = NV_OK;
   if ((stt = u.need((size_t)cr * M->F * M->esz)) != NV_OK) return stt;
   if ((stt = ctr.need((size_t)kTileCounters * 4)) != NV_OK) return stt;
@@ -1080,14 +1123,6 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
   NV_CUDA_TRY(cudaMemcpyAsync(s->prompt_len, t0.data(), B * 4, cudaMemcpyHostToDevice, st));
   NV_CUDA_TRY(cudaMemcpyAsync(s->prompt_last, tk.data(), B * 4, cudaMemcpyHostToDevice, st));
   NV_CUDA_TRY(cudaStreamSynchronize(st));
-  h.release();
-  act.release();
-  u.release();
-  ctr.release();
-  q.release();
-  o.release();
-  Y.release();
-  rows.release();
   s->h_prompt_len.assign(lens, lens + B);
   s->h_t = t0;
   s->prefilled = true;
