@@ -293,7 +293,7 @@ def run_ours(args):
     per_launch_bytes = dk["bytes"] / max(dk["launches"], 1)
     achieved = per_launch_bytes / (per_launch_ms / 1e3) / 1e9
     peak, peak_src = measured_peaks()
-    traffic = ncu_traffic(dom, args.workload)
+    traffic = ncu_traffic(dom, wl.name)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "bytes_per_launch": round(per_launch_bytes), "ms_per_launch": round(per_launch_ms, 5),

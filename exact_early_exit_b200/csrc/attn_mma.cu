@@ -78,16 +78,6 @@ __device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, uint6
       : "memory");
 }
 
-// ---------------------------------------------------------------------------
-// Prefill / scoring: CTA (sequence, head, 64-row query tile), warp w owns
-// query rows 16w .. 16w+15 of the tile.  Key tiles of 64 positions (one TMA
-// box of K and one of V, 128-byte swizzled) stream through a 3-stage ring;
-// each tile is used by all four warps, then refilled.  Per tile and warp:
-// S = Q K^T (32 MMAs), causal mask, online softmax (running max m and sum l
-// per row, O rescaled when m grows), O += P V with P as a bf16 hi/lo pair (64
-// MMAs).  Rows of one sequence have consecutive positions; row p attends to
-// keys 0..p, all in the cache (the QKV epilogue wrote this pass's keys).
-// ---------------------------------------------------------------------------
 constexpr int FQ = 64;   // query rows per CTA
 constexpr int FK = 64;   // keys per tile (one box)
 constexpr int FST = 3;   // ring stages
@@ -442,16 +432,28 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) k_attn_dec_mma(const __grid_co
   if (nsp > 1) dec_merge_splits(a, b, head, s0, s1);
 }
 
+// ---------------------------------------------------------------------------
+// Prefill / scoring: CTA (sequence, head, 64-row query tile), warp w owns
+// query rows 16w .. 16w+15 of the tile.  Key tiles of 64 positions (one TMA
+// box of K and one of V, 128-byte swizzled) stream through a 3-stage ring;
+// each tile is used by all four warps, then refilled.  Per tile and warp:
+// S = Q K^T (32 MMAs), causal mask, online softmax (running max m and sum l
+// per row, O rescaled when m grows), O += P V with P as a bf16 hi/lo pair (64
+// MMAs).  Rows of one sequence have consecutive positions; row p attends to
+// keys 0..p, all in the cache (the QKV epilogue wrote this pass's keys).
+// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) k_attn_fa_mma(const __grid_constant__ CUtensorMap kvmap, AttnArgs a) {
   pdl_wait();
   pdl_launch();
   extern __shared__ unsigned char smem_raw[];
   FaSmem& S = *reinterpret_cast<FaSmem*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   if (*a.rs.nrows == 0) return;
-  const int b = blockIdx.x, head = blockIdx.y;
+  // grid (row tile, head, sequence): the row tiles of one (sequence, head),
+  // which all read the same keys, run next to each other and share them in L2
+  const int b = blockIdx.z, head = blockIdx.y;
   const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
   const int nrt = (s1 - s0 + FQ - 1) / FQ;
-  const int rt = nrt - 1 - (int)blockIdx.z;  // the longest (latest) row tiles start first
+  const int rt = nrt - 1 - (int)blockIdx.x;  // the longest (latest) row tiles start first
   if (rt < 0) return;
   const int g0 = s0 + rt * FQ, g1 = min(s1, g0 + FQ), nr = g1 - g0;
   const int pos_last = a.rs.row_pos[g1 - 1];
@@ -638,7 +640,7 @@ void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream
 }
 
 void launch_attn_fa_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st) {
-  dim3 grid(a.rs.B, a.H, (a.row_groups * ATTN_RPC + FQ - 1) / FQ);
+  dim3 grid((a.row_groups * ATTN_RPC + FQ - 1) / FQ, a.H, a.rs.B);
   launch_k(k_attn_fa_mma, grid, 128, FA_SMEM_BYTES, st, *kvmap, a);
 }
 

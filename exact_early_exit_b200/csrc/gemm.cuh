@@ -48,9 +48,10 @@ struct EpiArgs;
 // Launch Y = X W^T followed by the layer epilogue `epi` (mode EPI_QKV,
 // EPI_RESID or EPI_SWIGLU; null or EPI_STORE: write fp32 Y).  X: [rows][ldx]
 // (rows <= max_rows, count in *nrows on the device), W: [N][K] row-major.
-// The tcgen05 engine applies the epilogue inside the GEMM kernel (split-K
-// slices in Y, summed by the last CTA of each feature tile, tile_counters
-// zero between launches); the SIMT engine runs the epilogue kernel after it.
+// The tcgen05 engine applies the epilogue inside the GEMM kernel when the K
+// range is not split; with allow_split it may split K (tc_split_count), store
+// fp32 slices in Y and run the epilogue kernel after it, which sums the slices
+// in a fixed order.  The SIMT engine always runs the epilogue kernel after it.
 // `prefetch` / `prefetch_bytes`: the next GEMM's weights, pulled into L2 by
 // the tcgen05 engine while it runs (a hint; may be null).
 nv_status gemm_run(GemmPlanCache* plans, int kind, bool bf16, const void* X, int ldx, const void* W, int N, int K,
