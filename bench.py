@@ -391,7 +391,8 @@ def run_scoring(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e2.elapsed_time(e3), dev) / args.steps
     stats = model.score_mixture_profiled(tok_d, logp_d, nll_d)
-    kern = {k: dict(ms=stats[i].ms, launches=int(stats[i].launches), flops=int(stats[i].flops))
+    kern = {k: dict(ms=stats[i].ms, launches=int(stats[i].launches), kernels=int(stats[i].kernels),
+                    flops=int(stats[i].flops))
             for i, k in enumerate(nv.KERNEL_KINDS)}
     total_k = sum(v["ms"] for v in kern.values())
     gemm_ms = kern["gemm"]["ms"] + kern["head"]["ms"]
@@ -407,7 +408,7 @@ def run_scoring(args):
                       "l2": "inputs larger than L2 (weights and activations streamed each step)"},
            "e2e": {"value": round(tokens * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                    "h2d_bytes_per_step": int(toks.nbytes), "d2h_bytes_per_step": int(B * (S - 1) * 4 + 4)},
-           "gpu_launches": sum(v["launches"] for v in kern.values()) * args.steps,
+           "gpu_launches": sum(v["kernels"] for v in kern.values()) * args.steps,
            "roofline": {"bound": "tensor", "kernel": "gemm (layers + exit heads)", "achieved": round(achieved, 1),
                         "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
                         "peak_source": src, "kernel_share": {k: round(v["ms"] / total_k, 4) for k, v in kern.items()},

@@ -42,7 +42,7 @@ KERNEL_KINDS = ("plan_norm", "gemm", "epilogue", "attention", "norm", "junction"
 
 class KernelStat(ctypes.Structure):
     _fields_ = [("ms", ctypes.c_double), ("launches", ctypes.c_int64), ("bytes", ctypes.c_int64),
-                ("flops", ctypes.c_int64)]
+                ("flops", ctypes.c_int64), ("kernels", ctypes.c_int64)]
 
 
 class NviumError(RuntimeError):

@@ -47,6 +47,12 @@ size_t gemm_workspace_elems(int kind, size_t rows, size_t N) {
   return e;
 }
 
+int gemm_launch_count(int kind, bool bf16, bool allow_split, const EpiArgs* epi) {
+  const int epilogue = (epi && epi->mode != EPI_STORE) ? 1 : 0;
+  if (kind == GEMM_TC && bf16) return allow_split ? 1 + epilogue : 1;
+  return 1 + epilogue;
+}
+
 nv_status gemm_run(GemmPlanCache* plans, int kind, bool bf16, const void* X, int ldx, const void* W, int N, int K,
                    const int* nrows, int max_rows, float* Y, bool allow_split, const EpiArgs* epi, int* tile_counters,
                    int epi_grid, const void* prefetch, size_t prefetch_bytes, cudaStream_t st,

@@ -45,6 +45,8 @@ __host__ __device__ __forceinline__ int tc_split_count(int R, int N, int K, int 
 }
 
 struct EpiArgs;
+// Kernels one gemm_run call with these arguments launches (1 or 2).
+int gemm_launch_count(int kind, bool bf16, bool allow_split, const EpiArgs* epi);
 // Launch Y = X W^T followed by the layer epilogue `epi` (mode EPI_QKV,
 // EPI_RESID or EPI_SWIGLU; null or EPI_STORE: write fp32 Y).  X: [rows][ldx]
 // (rows <= max_rows, count in *nrows on the device), W: [N][K] row-major.

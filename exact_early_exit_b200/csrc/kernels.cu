@@ -361,12 +361,14 @@ __global__ void __launch_bounds__(NT) k_plan_norm(PlanArgs a, const T* __restric
       if (total > 0 && a.counters) {
         long long kv = 0;
         for (int i = 0; i < NT / 32; ++i) kv += s_kv[i];
-        atomicAdd((unsigned long long*)&a.counters[NV_CTR_ROWS], (unsigned long long)total);
-        atomicAdd((unsigned long long*)&a.counters[NV_CTR_LAYERS_RUN], 1ull);
-        atomicAdd((unsigned long long*)&a.counters[NV_CTR_WEIGHT_BYTES], (unsigned long long)a.weight_bytes);
-        atomicAdd((unsigned long long*)&a.counters[NV_CTR_KV_READ_BYTES], (unsigned long long)kv);
+        // the same rows run every layer of the block this plan serves
+        const unsigned long long nl = (unsigned long long)(a.nlayers > 0 ? a.nlayers : 1);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_ROWS], (unsigned long long)total * nl);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_LAYERS_RUN], nl);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_WEIGHT_BYTES], (unsigned long long)a.weight_bytes * nl);
+        atomicAdd((unsigned long long*)&a.counters[NV_CTR_KV_READ_BYTES], (unsigned long long)kv * nl);
         atomicAdd((unsigned long long*)&a.counters[NV_CTR_KV_WRITE_BYTES],
-                  (unsigned long long)((long long)total * a.kv_pos_bytes));
+                  (unsigned long long)((long long)total * a.kv_pos_bytes) * nl);
       }
     }
   }

@@ -37,6 +37,7 @@ struct PlanArgs {
   int max_rows;
   int* status;
   long long* counters;
+  int nlayers;              // layers this plan serves (a block between exits has one row set)
   long long weight_bytes;   // this layer's weight bytes
   long long kv_pos_bytes;   // K+V bytes of one position of one layer
   const float* h;           // residual ring [B][cap][d]

@@ -203,6 +203,7 @@ struct Prof {
     int kind;
     cudaEvent_t a, b;
     long long bytes, flops;
+    int kernels;
   };
   std::vector<Rec> recs;
   // host copies of the current layer's work list
@@ -221,10 +222,10 @@ struct Prof {
     open_a = ev();
     cudaEventRecord(open_a, st);
   }
-  void end(int kind, long long bytes, long long flops) {
+  void end(int kind, long long bytes, long long flops, int kernels) {
     cudaEvent_t b = ev();
     cudaEventRecord(b, st);
-    recs.push_back(Rec{kind, open_a, b, bytes, flops});
+    recs.push_back(Rec{kind, open_a, b, bytes, flops, kernels});
   }
   ~Prof() {
     for (cudaEvent_t e : pool) cudaEventDestroy(e);
@@ -236,15 +237,17 @@ template <typename F>
 void timed(Prof* prof, long long* launches, int nlaunch, int kind, long long bytes, long long flops, F&& launch) {
   if (prof) prof->begin();
   launch();
-  if (prof) prof->end(kind, bytes, flops);
+  if (prof) prof->end(kind, bytes, flops, nlaunch);
   if (launches) *launches += nlaunch;
 }
 
 // Everything of layer `layer` after the attention RMSNorm (act holds the
 // normed rows): QKV + RoPE + KV write, attention, O + residual, MLP norm,
-// gate/up + SwiGLU, down + residual.
+// gate/up + SwiGLU, down + residual.  With `next_norm` (the next layer's
+// attention-norm gain, when it runs the same rows) the down projection's
+// residual is followed by that norm, so act is ready for the next layer.
 nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st, Prof* prof = nullptr,
-                     long long* launches = nullptr) {
+                     long long* launches = nullptr, const void* next_norm = nullptr) {
   const LayerDev& Lw = M->layers[layer];
   const bool bf = M->bf16;
   const long long es = (long long)M->esz;
@@ -270,7 +273,8 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
                   const void* pf, long long pf_bytes) {
     e.mode = mode;
     e.N = (int)N;
-    timed(prof, launches, M->gemm_kind == GEMM_TC ? 1 : 2, NV_K_GEMM, N * K * es + R * K * es + out_bytes,
+    timed(prof, launches, gemm_launch_count(M->gemm_kind, bf, io.split_k, &e), NV_K_GEMM,
+          N * K * es + R * K * es + out_bytes,
           2 * R * N * K, [&] {
             gst = gemm_run(M->gemm_plans, M->gemm_kind, bf, X, (int)ldx, W, (int)N, (int)K, io.rs.nrows,
                            io.rs.max_rows, io.Y, io.split_k, &e, io.tile_counters, io.epi_grid, pf,
@@ -325,9 +329,41 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
           [&] { launch_rmsnorm_rows(bf, io.rs, Lw.mlp_norm, io.act, M->d, M->cfg.rms_eps, st); });
   }
   NV_TRY(gemm(EPI_SWIGLU, io.act, d, Lw.w_gu, 2 * F, d, R * F * es, Lw.w_d, d * F * es));
-  NV_TRY(gemm(EPI_RESID, io.u, F, Lw.w_d, d, F, R * d * 8, io.prefetch_next && nextL ? nextL->w_qkv : nullptr,
-              3 * HQ * d * es));
+  const void* pf_next = io.prefetch_next && nextL ? nextL->w_qkv : nullptr;
+  if (next_norm && M->gemm_kind == GEMM_TC && io.split_k) {
+    // down projection slices summed into h by the norm kernel, which also
+    // writes the next layer's normed rows
+    int sg = 0;
+    timed(prof, launches, 1, NV_K_GEMM, d * F * es + R * F * es + R * d * 4, 2 * R * d * F, [&] {
+      gst = gemm_run(M->gemm_plans, M->gemm_kind, bf, io.u, (int)F, Lw.w_d, (int)d, (int)F, io.rs.nrows,
+                     io.rs.max_rows, io.Y, true, nullptr, io.tile_counters, io.epi_grid, pf_next,
+                     (size_t)(3 * HQ * d * es), st, &sg);
+    });
+    NV_TRY(gst);
+    timed(prof, launches, 1, NV_K_NORM, R * d * (8 + es), 0, [&] {
+      launch_resid_norm(bf, io.rs, io.Y, sg, M->d, M->F, tc_split_stride_elems(M->d), next_norm, io.act, M->d,
+                        M->cfg.rms_eps, st);
+    });
+    return NV_OK;
+  }
+  NV_TRY(gemm(EPI_RESID, io.u, F, Lw.w_d, d, F, R * d * 8, pf_next, 3 * HQ * d * es));
+  if (next_norm)
+    timed(prof, launches, 1, NV_K_NORM, R * d * (4 + es), 0,
+          [&] { launch_rmsnorm_rows(bf, io.rs, next_norm, io.act, M->d, M->cfg.rms_eps, st); });
   return NV_OK;
+}
+
+// Layers between two exits run the same rows (exits happen only after a
+// block's last layer, and a block's layers keep equal cache lengths), so a
+// block is planned once, at its first layer.
+int block_layers(const nv_model* M, int layer) {
+  int n = 1;
+  while (layer + n - 1 < M->L - 1 && M->exit_at[layer + n - 1] < 0) ++n;
+  return n;
+}
+// the next layer's attention-norm gain when it runs the same rows as `layer`
+const void* next_norm_in_block(const nv_model* M, int layer) {
+  return (layer + 1 < M->L && M->exit_at[layer] < 0) ? M->layers[layer + 1].attn_norm : nullptr;
 }
 
 LayerIO state_io(nv_state* s) {
@@ -376,6 +412,7 @@ PlanArgs state_plan(nv_state* s, int layer, int mode) {
   p.max_rows = s->max_rows;
   p.status = s->status;
   p.counters = s->counters;
+  p.nlayers = 1;
   p.weight_bytes = M->layer_weight_bytes;
   p.kv_pos_bytes = (long long)2 * M->HQ * (long long)M->esz;
   p.h = s->hbuf;
@@ -414,15 +451,18 @@ nv_status record_layers(nv_state* s, cudaStream_t st, Prof* prof, long long* lau
   const long long es = (long long)M->esz;
   LayerIO io = state_io(s);
   for (int layer = l0; layer < l1; ++layer) {
-    PlanArgs p = state_plan(s, layer, 0);
-    timed(prof, launches, 1, NV_K_PLAN_NORM, 0, 0, [&] {
-      launch_plan_norm(bf, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
-    });
-    if (prof) {
-      NV_TRY(prof_read_plan(s, prof, st));
-      prof->recs.back().bytes = (long long)prof->R * M->d * (4 + es);
+    if (layer == l0 || M->exit_at[layer - 1] >= 0) {
+      PlanArgs p = state_plan(s, layer, 0);
+      p.nlayers = block_layers(M, layer);
+      timed(prof, launches, 1, NV_K_PLAN_NORM, 0, 0, [&] {
+        launch_plan_norm(bf, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
+      });
+      if (prof) {
+        NV_TRY(prof_read_plan(s, prof, st));
+        prof->recs.back().bytes = (long long)prof->R * M->d * (4 + es);
+      }
     }
-    NV_TRY(layer_body(M, layer, io, st, prof, launches));
+    NV_TRY(layer_body(M, layer, io, st, prof, launches, next_norm_in_block(M, layer)));
     const int k = M->exit_at[layer];
     if (k < 0) continue;
     JuncArgs j{};
@@ -1263,6 +1303,7 @@ nv_status nv_decode_step_profiled(nv_state* s, uint64_t seed, int32_t* tokens_ou
     nv_kernel_stat& k = stats[r.kind];
     k.ms += ms;
     k.launches += 1;
+    k.kernels += r.kernels;
     k.bytes += r.bytes;
     k.flops += r.flops;
   }
@@ -1280,10 +1321,13 @@ nv_status nv_flush_deferred(nv_state* s, void* stream) {
   LayerIO io = state_io(s);
   long long launches = 0;
   for (int layer = M->cfg.exit_layers[0]; layer < M->L; ++layer) {
-    PlanArgs p = state_plan(s, layer, 1);
-    launch_plan_norm(M->bf16, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
-    ++launches;
-    NV_TRY(layer_body(M, layer, io, st, nullptr, &launches));
+    if (layer == M->cfg.exit_layers[0] || M->exit_at[layer - 1] >= 0) {
+      PlanArgs p = state_plan(s, layer, 1);
+      p.nlayers = block_layers(M, layer);
+      launch_plan_norm(M->bf16, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
+      ++launches;
+    }
+    NV_TRY(layer_body(M, layer, io, st, nullptr, &launches, next_norm_in_block(M, layer)));
   }
   s->launches_total += launches;
   NV_CUDA_TRY(cudaGetLastError());
@@ -1560,6 +1604,7 @@ nv_status nv_score_mixture_profiled(nv_model* M, const int32_t* tokens, int B, i
     nv_kernel_stat& k = stats[r.kind];
     k.ms += ms;
     k.launches += 1;
+    k.kernels += r.kernels;
     k.bytes += r.bytes;
     k.flops += r.flops;
   }

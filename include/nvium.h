@@ -225,16 +225,19 @@ nv_status nv_philox4x32_10_noalloc(uint64_t seed, const uint32_t *ctr, int n,
 
 /* Per-kernel timing of one decode step (a measurement hook, not a second
  * code path): the step's kernels are launched directly on `stream`, each
- * bracketed by CUDA events, instead of as one graph replay; the step's
+ * call bracketed by CUDA events, instead of as one graph replay; the step's
  * results are identical.  stats[kind] accumulates, for NV_K_* kinds, the
- * summed event time, the launches, and the algorithmic bytes (the bytes the
- * kernel must move: weights once, K/V of the attended positions once,
- * activations in and out) and flops of those launches.  Synchronous. */
+ * summed event time, the calls (`launches`: one GEMM with its split-K sum
+ * epilogue is one call), the kernels those calls launched (`kernels`), and
+ * the algorithmic bytes (the bytes the kernel must move: weights once, K/V
+ * of the attended positions once, activations in and out) and flops of those
+ * calls.  Synchronous. */
 typedef struct nv_kernel_stat {
   double ms;
   int64_t launches;
   int64_t bytes;
   int64_t flops;
+  int64_t kernels;
 } nv_kernel_stat;
 enum {
   NV_K_PLAN_NORM = 0, /* work-list planner + attention RMSNorm    */
