@@ -214,7 +214,6 @@ def run_ours(args):
     weights = W.make_weights(cfg, seed=0)
     max_seq = int(lens.max()) + steps + 64
     model = nv.Model(cfg, weights, max_batch=B, max_seq=max_seq, max_pending=256)
-    del weights
     st = nv.State(model, B)
     tok_host = torch.from_numpy(np.concatenate(prompts).astype(np.int32)).pin_memory()
     stream = torch.cuda.current_stream(dev)
@@ -279,6 +278,53 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e2.elapsed_time(e3), dev)
     e2e_value = tokens_per_step * world * args.steps / (e2e_ms / 1e3)
 
+    # prefill and the final flush on their own (decode tokens/s excludes the
+    # prefill; the flush is owed work and sits inside every timed pass)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ea.record(stream)
+    st.prefill(tok_host, lens)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    prefill_ms = ea.elapsed_time(eb)
+    for s in range(steps):
+        st.decode_step(xseed + s, tok_d, ex_d)
+    ea.record(stream)
+    st.flush()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    flush_ms = ea.elapsed_time(eb)
+
+    # the same kernels forced to full depth (every token leaves at the last
+    # exit): the dense-decode comparison of the same workload
+    fmodel = nv.Model(cfg, weights, max_batch=B, max_seq=max_seq, max_pending=256,
+                      router_mode=nv.NV_ROUTER_FORCE_LAST)
+    del weights
+    fst = nv.State(fmodel, B)
+    fst.prefill(tok_host, lens)
+
+    def full_pass(seed):
+        fst.rewind()
+        for s in range(steps):
+            fst.decode_step(seed + s, tok_d, ex_d)
+        fst.flush()
+
+    for i in range(args.warmup):
+        full_pass(xseed + 100000 * (i + 1))
+    torch.cuda.synchronize()
+    barrier()
+    ea.record(stream)
+    for i in range(args.steps):
+        full_pass(xseed)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    full_ms = max_over_ranks(ea.elapsed_time(eb), dev) / args.steps
+    fst.sync_status()
+    fst.close()
+    fmodel.close()
+    full_value = tokens_per_step * world / (full_ms / 1e3)
+
     # per-kernel times: one profiled pass (each launch bracketed by events)
     stats = (nv.KernelStat * len(nv.KERNEL_KINDS))()
     st.rewind()
@@ -317,7 +363,12 @@ def run_ours(args):
                    "d2h_bytes_per_step": int(steps * B * 8)},
            "gpu_launches": launches,
            "roofline": roofline,
-           "realised_exit_mass": exit_mass}
+           "realised_exit_mass": exit_mass,
+           "full_depth": {"value": round(full_value, 1), "unit": "tokens/s", "ms_per_step": round(full_ms, 3),
+                          "speedup": round(value / full_value, 3),
+                          "what": "same workload and kernels, router forced to the last exit"},
+           "prefill_ms": round(prefill_ms, 3),
+           "flush_ms": round(flush_ms, 3)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, weights_seed=0, lens=lens, prompts=prompts, xseed=xseed)
     out["clocks"] = clk.summary()
