@@ -96,6 +96,7 @@ _SIGS = [
     ("nv_philox4x32_10", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
     ("nv_decode_step_profiled", _I, [_P, ctypes.c_uint64, _P, _P, _P, _P]),
     ("nv_philox4x32_10_noalloc", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
+    ("nv_selftest_bounded_wait", _I, [_I, _P, _P]),
     ("nv_score_mixture_profiled", _I, [_P, _P, _I, _I, _P, _P, _P, _P]),
     ("nv_last_error", ctypes.c_char_p, []),
 ]
@@ -310,6 +311,14 @@ def philox4x32_10(seed: int, counters: np.ndarray) -> np.ndarray:
     out = np.zeros_like(ctr)
     _check(lib().nv_philox4x32_10(ctypes.c_uint64(seed), _ptr(ctr), ctr.shape[0], _ptr(out), None))
     return out
+
+
+def selftest_bounded_wait(limit_us: int) -> bool:
+    """Run the bounded-wait self-test (a wait that nothing completes, given
+    up after limit_us); True when the wait gave up as it should."""
+    out = np.zeros(1, np.int32)
+    _check(lib().nv_selftest_bounded_wait(int(limit_us), _ptr(out), None))
+    return bool(out[0])
 
 
 def philox4x32_10_noalloc(seed: int, counters: np.ndarray) -> np.ndarray:

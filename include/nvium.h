@@ -223,6 +223,17 @@ nv_status nv_philox4x32_10(uint64_t seed, const uint32_t *ctr, int n,
 nv_status nv_philox4x32_10_noalloc(uint64_t seed, const uint32_t *ctr, int n,
                                    uint32_t *out, void *stream);
 
+/* Self-test of the bounded-wait rule that every wait in the library's
+ * kernels follows (a wait on an mbarrier or flag gives up after a time
+ * limit, records a timeout in the device status word and returns, leaving
+ * the CUDA context usable).  One thread waits on a shared-memory mbarrier
+ * that nothing completes, for at most limit_us microseconds (1 ..
+ * 1000000; else NV_ERR_INVALID_ARG), and *expired_out is set to 1 when the
+ * wait gave up (the expected outcome), 0 otherwise.  No copy is in flight
+ * while it waits.  Synchronous on `stream`.  The paper has no counterpart:
+ * it is failure-detection test infrastructure. */
+nv_status nv_selftest_bounded_wait(int limit_us, int *expired_out, void *stream);
+
 /* Per-kernel timing of one decode step (a measurement hook, not a second
  * code path): the step's kernels are launched directly on `stream`, each
  * call bracketed by CUDA events, instead of as one graph replay; the step's

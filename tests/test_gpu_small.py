@@ -171,3 +171,13 @@ def test_mma_and_simt_scoring_attention_agree(weights):
         m.close()
     assert np.all(np.isfinite(out["mma"]))
     np.testing.assert_allclose(out["mma"], out["simt"], atol=tolerance(CFG), rtol=0)
+
+
+def test_decode_parity_bf16_degenerate_and_ragged_prompts(weights):
+    """A one-token prompt (no prefill rows), one ending a 64-row query tile
+    plus one row, and one spanning several key tiles, through the MMA
+    attention kernels."""
+    wl = W.WORKLOADS["S"]
+    prompts = [p[:n] for p, n in zip(W.make_prompts(wl), (1, 65, 130))]
+    chk, state, dec, _ = run_decode_parity(nv, CFG, weights, prompts, 12)
+    assert chk.steps == 12

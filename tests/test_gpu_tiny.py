@@ -177,3 +177,59 @@ def test_conditional_and_flat_step_graphs_agree(cfg_name):
         np.testing.assert_array_equal(a[1], b[1])
     # the conditional graph launches no more kernels than the flat one
     assert outs["1"][2][nv.CTR["launches"]] <= outs["0"][2][nv.CTR["launches"]]
+
+
+def test_decode_parity_batch_wider_than_one_planner_block(weights):
+    """300 sequences: the planner's 256 threads each take two sequences; the
+    attention and junction grids span several waves."""
+    rng = np.random.default_rng(5)
+    lens = rng.integers(1, 13, size=300)
+    prompts = [W.make_prompts(W.WORKLOADS["T"], seed=10 + i)[0][:n] for i, n in enumerate(lens)]
+    chk, state, dec, _ = run_decode_parity(nv, CFG, weights, prompts, 4, max_seq=32)
+    assert chk.steps == 4 and chk.exit_ties == 0 and chk.token_ties == 0
+
+
+def test_host_argument_and_capacity_errors(weights):
+    """Argument and state errors come back as statuses, and a sequence that
+    reaches max_seq stops with NV_ERR_CAPACITY; the state stays usable."""
+    prompt = W.make_prompts(W.WORKLOADS["T"])[0][:10]
+    model = nv.Model(CFG, weights, max_batch=2, max_seq=16)
+    st = nv.State(model, 1)
+    tok, ex = np.zeros(1, np.int32), np.zeros(1, np.int32)
+    with pytest.raises(nv.NviumError) as e:
+        st.decode_step(1, tok, ex)
+    assert e.value.status == nv.NV_ERR_STATE
+    with pytest.raises(nv.NviumError) as e:
+        st.prefill(prompt, [0])
+    assert e.value.status == nv.NV_ERR_INVALID_ARG
+    bad = prompt.copy()
+    bad[3] = CFG.vocab
+    with pytest.raises(nv.NviumError) as e:
+        st.prefill(bad, [10])
+    assert e.value.status == nv.NV_ERR_INVALID_ARG
+    st.prefill(prompt, [10])
+    n = 0
+    with pytest.raises(nv.NviumError) as e:
+        for s in range(16):
+            st.decode_step(5 + s, tok, ex)
+            n += 1
+    assert e.value.status == nv.NV_ERR_CAPACITY
+    # steps at positions 9 .. 14 sample tokens for 10 .. 15; the next would
+    # sample position 16 = max_seq
+    assert n == 16 - 10
+    st.sync_status()
+    st.rewind()
+    st.decode_step(5, tok, ex)
+    st.sync_status()
+    st.close()
+    model.close()
+
+
+def test_bounded_wait_gives_up_and_leaves_the_context_usable():
+    """Failure detection without a GPU fault: a wait that nothing completes
+    gives up after its limit and reports it; the next launches still work."""
+    assert nv.selftest_bounded_wait(20000)
+    ctr = np.arange(64, dtype=np.uint32).reshape(16, 4)
+    out = nv.philox4x32_10(7, ctr)
+    ref = O.philox4x32_10([ctr[:, i] for i in range(4)], (7, 0))
+    np.testing.assert_array_equal(out, np.stack([r.astype(np.uint32) for r in ref], 1))
