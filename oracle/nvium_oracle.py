@@ -226,6 +226,15 @@ def mixture_logprob(log_p: np.ndarray, log_pi: np.ndarray) -> np.ndarray:
     return logsumexp(log_p + log_pi, axis=-1)
 
 
+def expected_depth(log_p: np.ndarray, exit_layers: Sequence[int], n_layers: int) -> np.ndarray:
+    """Expected normalised layer depth of a token (section 2 "Training": the
+    compute penalty L_compute is the expected normalised depth): a token that
+    exits at node k has run exit_layers[k] of the n_layers layers, so
+    E[depth] = sum_k p_k * exit_layers[k] / n_layers."""
+    frac = np.asarray(exit_layers, dtype=np.float64) / float(n_layers)
+    return np.exp(np.asarray(log_p, dtype=np.float64)) @ frac
+
+
 # --------------------------------------------------------------------------
 # backbone (LLaMA-2, section 4) on rows of one sequence
 # --------------------------------------------------------------------------
@@ -377,10 +386,19 @@ def score_mixture(model: OracleModel, tokens: np.ndarray):
     with log p_k from the routers at position t and
     log pi_k(v) = logit_k[v] - LSE_v logit_k.
     """
+    logp, nll, _, _ = score_mixture_with_depth(model, tokens)
+    return logp, nll
+
+
+def score_mixture_with_depth(model: OracleModel, tokens: np.ndarray):
+    """score_mixture plus the compute-penalty forward: (logp [B, S-1], mean
+    NLL, depth [B, S-1], mean depth), depth[b, t] = expected normalised layer
+    depth of position t (expected_depth of its exit probabilities)."""
     cfg = model.cfg
     tokens = np.asarray(tokens)
     B, S = tokens.shape
     out = np.empty((B, S - 1))
+    depth = np.empty((B, S - 1))
     for b in range(B):
         _, states, _ = model.forward_sequence(tokens[b, : S - 1])
         tgt = tokens[b, 1:].astype(np.int64)
@@ -392,8 +410,10 @@ def score_mixture(model: OracleModel, tokens: np.ndarray):
                 z[:, k] = model.router_logit(k, nk)
             lg = model.head_logits(k, nk)
             logpi[:, k] = lg[np.arange(S - 1), tgt] - logsumexp(lg, axis=-1)
-        out[b] = mixture_logprob(log_exit_probs(z, model.mode), logpi)
-    return out, float(-out.mean())
+        lp = log_exit_probs(z, model.mode)
+        out[b] = mixture_logprob(lp, logpi)
+        depth[b] = expected_depth(lp, cfg.exit_layers, cfg.n_layers)
+    return out, float(-out.mean()), depth, float(depth.mean())
 
 
 def dense_logprobs(model: OracleModel, tokens: Sequence[int]) -> np.ndarray:

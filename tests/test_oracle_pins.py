@@ -357,3 +357,45 @@ def test_decoder_step_uses_the_vectorised_sampler():
 
 def test_gumbel_argmax_ties_to_lowest_id():
     assert int(O.gumbel_argmax(np.array([1.0, 3.0, 3.0, 2.0]), np.zeros(4))) == 1
+
+
+# ---------------------------------------------------------------------------
+# compute-penalty forward: expected normalised layer depth
+# ---------------------------------------------------------------------------
+def test_expected_depth_closed_forms():
+    """Zero intermediate mass: every token runs all L layers (depth 1). A
+    router that always stops at the first node: depth l_1 / L."""
+    z = np.random.default_rng(3).normal(size=(50, 3))
+    exits, L = (3, 6, 9, 12), 12
+    d_last = O.expected_depth(O.log_exit_probs(z, O.ROUTER_FORCE_LAST), exits, L)
+    np.testing.assert_array_equal(d_last, np.ones(50))
+    d_first = O.expected_depth(O.log_exit_probs(np.full((4, 3), 60.0)), exits, L)
+    np.testing.assert_allclose(d_first, 3 / 12, rtol=0, atol=1e-12)
+    d_never = O.expected_depth(O.log_exit_probs(np.full((4, 3), -60.0)), exits, L)
+    np.testing.assert_allclose(d_never, 1.0, rtol=0, atol=1e-12)
+
+
+def test_expected_depth_matches_sampled_exits():
+    """E[depth] equals the mean depth of exits drawn by the sequential
+    stop/continue sampler (itself pinned to p_k above): 2e5 draws, 5 sigma."""
+    w = np.array([0.35, 0.4, 0.55])
+    z = np.log(w / (1 - w))
+    exits, L = (2, 5, 7, 11), 11
+    want = float(O.expected_depth(O.log_exit_probs(z[None, :]), exits, L)[0])
+    seeds = np.arange(200000, dtype=np.uint64)
+    u = np.stack([O.exit_uniform(seeds, 0, 3, k) for k in (1, 2, 3)], -1)
+    depth = np.asarray(exits, dtype=np.float64)[O.sample_exit(u, w) - 1] / L
+    assert abs(depth.mean() - want) < 5 * depth.std() / np.sqrt(len(depth))
+
+
+def test_scoring_depth_uses_the_scoring_exit_probabilities():
+    """score_mixture_with_depth returns score_mixture's values plus the depth
+    of the same log p_k (its definition on the tiny model)."""
+    model, _ = tiny_model()
+    toks = np.stack([W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:12] for s in (1, 2)])
+    lp, nll = O.score_mixture(model, toks)
+    lp2, nll2, depth, mean_depth = O.score_mixture_with_depth(model, toks)
+    np.testing.assert_array_equal(lp, lp2)
+    assert nll == nll2
+    assert depth.shape == lp.shape and abs(mean_depth - depth.mean()) < 1e-15
+    assert np.all(depth >= model.cfg.exit_layers[0] / model.cfg.n_layers - 1e-12) and np.all(depth <= 1 + 1e-12)
