@@ -267,6 +267,10 @@ class OracleModel:
             if k < cfg.n_exits - 1:
                 e["router_w"] = f(E["router_w"])
                 e["router_b"] = float(E["router_b"])
+                if getattr(cfg, "router_hidden", 0):
+                    e["router_w1"] = f(E["router_w1"])
+                    e["router_b1"] = np.asarray(E["router_b1"], dtype=np.float32)
+                    e["router_w2"] = np.asarray(E["router_w2"], dtype=np.float32)
             self.exits.append(e)
         self.exit_at = {l: k for k, l in enumerate(cfg.exit_layers)}  # layer -> exit index (0-based)
 
@@ -338,8 +342,13 @@ class OracleModel:
         return self.rnd(rmsnorm(h, widen(self.exits[k]["norm"]), self.cfg.rms_eps))
 
     def router_logit(self, k: int, nk: np.ndarray) -> np.ndarray:
-        """z_k = r_k . n_k + b_k (k < N_V - 1, 0-based)."""
+        """z_k = r_k . n_k + b_k (k < N_V - 1, 0-based), or, with a router MLP
+        (section 2 "Architektur": a router MLP maps the node's hidden state to
+        w_k), z_k = v_k . silu(U_k n_k + c_k) + b_k, silu(x) = x sigmoid(x)."""
         e = self.exits[k]
+        if "router_w1" in e:
+            a = np.asarray(nk, dtype=np.float64) @ widen(e["router_w1"]).T + widen(e["router_b1"])
+            return silu(a) @ widen(e["router_w2"]) + e["router_b"]
         return nk @ widen(e["router_w"]) + e["router_b"]
 
     def router_prob(self, k: int, nk: np.ndarray) -> np.ndarray:

@@ -399,3 +399,48 @@ def test_scoring_depth_uses_the_scoring_exit_probabilities():
     assert nll == nll2
     assert depth.shape == lp.shape and abs(mean_depth - depth.mean()) < 1e-15
     assert np.all(depth >= model.cfg.exit_layers[0] / model.cfg.n_layers - 1e-12) and np.all(depth <= 1 + 1e-12)
+
+
+# ---------------------------------------------------------------------------
+# router MLP (section 2 "Architektur": a router MLP maps h at node k to w_k)
+# ---------------------------------------------------------------------------
+def _mlp_router_model(U_of, c_of, v_of, mode=O.ROUTER_NORMAL):
+    import dataclasses
+    model, w = tiny_model(mode)
+    r = U_of(w["exits"][0]).shape[0]
+    cfg = dataclasses.replace(W.TINY, router_hidden=r)
+    w2 = {**w, "exits": [dict(e) for e in w["exits"]]}
+    for k in range(cfg.n_exits - 1):
+        e = w2["exits"][k]
+        e["router_w1"], e["router_b1"], e["router_w2"] = U_of(e), c_of(e), v_of(e)
+    return O.OracleModel(cfg, w2, mode), model
+
+
+def test_router_mlp_reduces_to_the_scalar_router():
+    """silu(x) - silu(-x) = x, so hidden units U = [r; -r], c = 0, v = [1, -1]
+    give z = r . n + b: mixture scoring equals the (pinned) scalar router's."""
+    mlp, scalar = _mlp_router_model(lambda e: np.stack([e["router_w"], -e["router_w"]]),
+                                    lambda e: np.zeros(2, np.float32), lambda e: np.array([1.0, -1.0], np.float32))
+    toks = np.stack([W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:16] for s in (1, 2)])
+    a, _ = O.score_mixture(mlp, toks)
+    b, _ = O.score_mixture(scalar, toks)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_router_mlp_hidden_unit_is_torch_silu():
+    """One hidden unit: z = silu(r . n + c) + b, against torch's SiLU; a second
+    unit with output weight 0 changes nothing."""
+    import torch
+    c0 = np.float32(0.37)
+    mlp, scalar = _mlp_router_model(lambda e: e["router_w"][None, :], lambda e: np.array([c0], np.float32),
+                                    lambda e: np.array([1.0], np.float32))
+    rng = np.random.default_rng(2)
+    n = rng.normal(size=(32, W.TINY.d_model))
+    for k in range(W.TINY.n_exits - 1):
+        pre = n @ O.widen(scalar.exits[k]["router_w"]) + float(c0)
+        want = torch.nn.functional.silu(torch.from_numpy(pre)).numpy() + scalar.exits[k]["router_b"]
+        np.testing.assert_allclose(mlp.router_logit(k, n), want, rtol=0, atol=1e-13)
+    wide, _ = _mlp_router_model(lambda e: np.stack([e["router_w"], e["router_w"] * 3]),
+                                lambda e: np.array([c0, 1.0], np.float32), lambda e: np.array([1.0, 0.0], np.float32))
+    for k in range(W.TINY.n_exits - 1):
+        np.testing.assert_allclose(wide.router_logit(k, n), mlp.router_logit(k, n), rtol=0, atol=1e-13)

@@ -53,6 +53,8 @@ class ModelConfig:
     dtype: int  # F32 or BF16
     rms_eps: float = 1e-5
     rope_theta: float = 10000.0
+    # hidden width of the router MLP of every exit but the last; 0: scalar router
+    router_hidden: int = 0
 
     @property
     def n_exits(self) -> int:
@@ -191,7 +193,9 @@ def make_weights(cfg: ModelConfig, seed: int = 0, random_gains: bool = False,
     Returns {"dtype", "tok_emb", "layers": [dict], "exits": [dict]}; tensors
     are float32 (F32 configs) or bf16 bits as uint16 (BF16 configs).  Each
     exit dict has "norm", "head", and for k < N_V "router_w" and the float
-    "router_b".
+    "router_b"; with cfg.router_hidden = r > 0 also the router MLP's
+    "router_w1" [r, d] (model dtype), "router_b1" [r] and "router_w2" [r]
+    (float32).
     """
     specs = _tensor_specs(cfg)
 
@@ -232,6 +236,17 @@ def make_weights(cfg: ModelConfig, seed: int = 0, random_gains: bool = False,
                                                   [1.0 / cfg.n_exits] * cfg.n_exits)
     for k in range(cfg.n_exits - 1):
         w["exits"][k]["router_b"] = float(np.float32(router_bias[k]))
+    if cfg.router_hidden:
+        # router MLP z = v . silu(U n + c) + b: U ~ N(0, 1/d) (model dtype),
+        # c ~ N(0, 0.1^2), v ~ N(0, 1/r) (float32); streams after the manifest's
+        r, d = cfg.router_hidden, cfg.d_model
+        for k in range(cfg.n_exits - 1):
+            rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(len(specs) + 1 + k,))))
+            U = rng.standard_normal(size=(r, d), dtype=np.float32) * np.float32(1.0 / np.sqrt(d))
+            w["exits"][k]["router_w1"] = f32_to_bf16_bits(U) if cfg.dtype == BF16 else U
+            w["exits"][k]["router_b1"] = (rng.standard_normal(size=r, dtype=np.float32) * np.float32(0.1))
+            w["exits"][k]["router_w2"] = (rng.standard_normal(size=r, dtype=np.float32) *
+                                          np.float32(1.0 / np.sqrt(r)))
     return w
 
 
