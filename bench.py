@@ -441,6 +441,13 @@ def run_scoring(args):
     e3.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e2.elapsed_time(e3), dev) / args.steps
+    # the compute-penalty forward on the same batch (untimed): mean expected
+    # normalised layer depth
+    depth_d = torch.zeros_like(logp_d)
+    mdepth_d = torch.zeros(1, dtype=torch.float32, device=dev)
+    model.score_mixture_ex(tok_d, logp_d, nll_d, depth_d, mdepth_d)
+    torch.cuda.synchronize()
+    mean_depth = float(mdepth_d.item())
     stats = model.score_mixture_profiled(tok_d, logp_d, nll_d)
     kern = {k: dict(ms=stats[i].ms, launches=int(stats[i].launches), kernels=int(stats[i].kernels),
                     flops=int(stats[i].flops))
@@ -464,7 +471,8 @@ def run_scoring(args):
                         "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
                         "peak_source": src, "kernel_share": {k: round(v["ms"] / total_k, 4) for k, v in kern.items()},
                         "gemm_tflop_per_step": round(gemm_flops / 1e12, 2)},
-           "mean_nll": float(nll_d.item())}
+           "mean_nll": float(nll_d.item()),
+           "mean_expected_depth": round(mean_depth, 5)}
     out["clocks"] = clk.summary()
     if rank == 0:
         print(json.dumps(out))

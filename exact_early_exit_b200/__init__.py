@@ -57,7 +57,7 @@ class Config(ctypes.Structure):
                 ("n_exits", ctypes.c_int), ("exit_layers", ctypes.c_int * NV_MAX_EXITS), ("dtype", ctypes.c_int),
                 ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("max_batch", ctypes.c_int),
                 ("max_seq", ctypes.c_int), ("page_size", ctypes.c_int), ("max_pending", ctypes.c_int),
-                ("router_mode", ctypes.c_int)]
+                ("router_mode", ctypes.c_int), ("router_hidden", ctypes.c_int)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -66,7 +66,8 @@ class LayerWeights(ctypes.Structure):
 
 class ExitWeights(ctypes.Structure):
     _fields_ = [("norm", ctypes.c_void_p), ("head", ctypes.c_void_p), ("router_w", ctypes.c_void_p),
-                ("router_b", ctypes.c_float)]
+                ("router_b", ctypes.c_float), ("router_w1", ctypes.c_void_p), ("router_b1", ctypes.c_void_p),
+                ("router_w2", ctypes.c_void_p)]
 
 
 class Weights(ctypes.Structure):
@@ -98,6 +99,7 @@ _SIGS = [
     ("nv_philox4x32_10_noalloc", _I, [ctypes.c_uint64, _P, _I, _P, _P]),
     ("nv_selftest_bounded_wait", _I, [_I, _P, _P]),
     ("nv_score_mixture_profiled", _I, [_P, _P, _I, _I, _P, _P, _P, _P]),
+    ("nv_score_mixture_ex", _I, [_P, _P, _I, _I, _P, _P, _P, _P, _P]),
     ("nv_last_error", ctypes.c_char_p, []),
 ]
 
@@ -171,6 +173,7 @@ def make_config(model_cfg, max_batch: int, max_seq: int, page_size: int = 64, ma
     c.page_size = page_size
     c.max_pending = max_pending
     c.router_mode = router_mode
+    c.router_hidden = int(getattr(model_cfg, "router_hidden", 0))
     return c
 
 
@@ -206,6 +209,9 @@ class Model:
             ew[k].head = p(E["head"])
             ew[k].router_w = p(E["router_w"]) if "router_w" in E else None
             ew[k].router_b = float(E.get("router_b", 0.0))
+            for f in ("router_w1", "router_b1", "router_w2"):
+                if f in E:
+                    setattr(ew[k], f, p(E[f]))
         w = Weights(p(weights["tok_emb"]), lw, ew)
         h = ctypes.c_void_p()
         _check(lib().nv_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(h)))
@@ -217,6 +223,14 @@ class Model:
         B, S = tokens.shape
         _check(lib().nv_score_mixture(self.handle, _ptr(tokens), B, S, _ptr(logp_out), _ptr(mean_nll_out),
                                       _stream(stream)))
+
+    def score_mixture_ex(self, tokens, logp_out, mean_nll_out=None, depth_out=None, mean_depth_out=None,
+                         stream=None):
+        """score_mixture plus the expected normalised layer depth of every
+        position (depth_out [B, S-1]) and its mean (mean_depth_out [1])."""
+        B, S = tokens.shape
+        _check(lib().nv_score_mixture_ex(self.handle, _ptr(tokens), B, S, _ptr(logp_out), _ptr(mean_nll_out),
+                                         _ptr(depth_out), _ptr(mean_depth_out), _stream(stream)))
 
     def score_mixture_profiled(self, tokens, logp_out, mean_nll_out=None, stats=None, stream=None):
         """score_mixture with per-kernel CUDA-event timing (KernelStat array)."""

@@ -111,6 +111,9 @@ struct ExitDev {
   const void* head;      // [V, d]
   const void* router_w;  // [d] (unused for the last exit)
   float router_b;
+  const void* router_w1;    // router MLP [r, d] (model dtype), or null
+  const float* router_b1;   // [r]
+  const float* router_w2;   // [r]
 };
 
 // Rows processed together at one layer.  Rows of a sequence are contiguous and

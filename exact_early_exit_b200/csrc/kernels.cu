@@ -1003,11 +1003,31 @@ void launch_step_end(const StepArgs& a, cudaStream_t st) {
 
 // ---------------------------------------------------------------------------
 // Exit junction k (section 2 "Architektur": router w_k, stop/continue).
-// n_k = RMSNorm_k(h) (rounded to the model dtype), z = r_k . n_k + b_k,
+// n_k = RMSNorm_k(h) (rounded to the model dtype), z = r_k . n_k + b_k or,
+// with a router MLP of width r, z = v . silu(U n_k + c) + b_k;
 // w_k = sigmoid(z) (0 when routing is forced to the last exit), and the token
 // stops here iff u_k < w_k; the last exit always stops.  u_k is the Philox
 // uniform of counter (b, t, 0, k/4), lane k%4 (k 0-based).
 // ---------------------------------------------------------------------------
+// Router MLP of one row, by one warp over the hidden units j = j0, j0 + dj,
+// ...: returns this warp's share of sum_j v_j silu(U_j . n + c_j) (in every
+// lane); n is the row's exit-normalised state in the model dtype.
+template <typename T>
+__device__ __forceinline__ float router_mlp_part(const T* __restrict__ n, const T* __restrict__ U,
+                                                 const float* __restrict__ c, const float* __restrict__ v, int d,
+                                                 int r, int j0, int dj) {
+  const int lane = threadIdx.x & 31;
+  float z = 0.f;
+  for (int j = j0; j < r; j += dj) {
+    const T* u = U + (size_t)j * d;
+    float a = 0.f;
+    for (int i = lane; i < d; i += 32) a = fmaf(ld(n + i), ld(u + i), a);
+    a = warp_sum(a) + c[j];
+    z = fmaf(v[j], a / (1.0f + expf(-a)), z);
+  }
+  return z;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_junction(JuncArgs a) {
   pdl_wait();
@@ -1029,6 +1049,13 @@ __global__ void __launch_bounds__(256) k_junction(JuncArgs a) {
     const float n = rnd<T>(h[i] * inv * ld(g + i));
     out[i] = cvt<T>(n);
     if (!last) z = fmaf(n, ld(rw + i), z);
+  }
+  if (!last && a.router_hidden > 0) {
+    // every thread's n_k is in exit_act: the eight warps split the hidden units
+    __syncthreads();
+    const float zp = router_mlp_part<T>(out, (const T*)a.router_w1, a.router_b1, a.router_w2, a.d, a.router_hidden,
+                                        threadIdx.x >> 5, 8);
+    z = (threadIdx.x & 31) == 0 ? zp : 0.f;
   }
   z = block_sum<256>(z);
   if (threadIdx.x == 0) {
@@ -1264,13 +1291,15 @@ void launch_head_reduce(const HeadArgs& a, cudaStream_t st) {
 // Scoring (section 2: the mixture and its cross-entropy)
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void k_exit_rows(RowSet rs, const T* __restrict__ g, const T* __restrict__ rw, float rb, int k,
-                            int n_exits, T* __restrict__ act, float* __restrict__ z, int d, float eps) {
+__global__ void k_exit_rows(RowSet rs, ExitDev e, int rh, int k, int n_exits, T* __restrict__ act,
+                            float* __restrict__ z, int d, float eps) {
   pdl_wait();
   pdl_launch();
   const int R = *rs.nrows;
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   const bool last = k == n_exits - 1;
+  const T* g = (const T*)e.norm;
+  const T* rw = (const T*)e.router_w;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb) {
     const float* h = rs.h + (size_t)rs.row_hrow[r] * d;
     float ss = 0.f;
@@ -1281,21 +1310,25 @@ __global__ void k_exit_rows(RowSet rs, const T* __restrict__ g, const T* __restr
     for (int i = lane; i < d; i += 32) {
       const float n = rnd<T>(h[i] * inv * ld(g + i));
       act[(size_t)r * d + i] = cvt<T>(n);
-      if (!last) zz = fmaf(n, ld(rw + i), zz);
+      if (!last && rh == 0) zz = fmaf(n, ld(rw + i), zz);
     }
-    zz = warp_sum(zz);
-    if (!last && lane == 0) z[(size_t)r * (n_exits - 1) + k] = zz + rb;
+    if (!last && rh > 0) {
+      __syncwarp();
+      zz = router_mlp_part<T>(act + (size_t)r * d, (const T*)e.router_w1, e.router_b1, e.router_w2, d, rh, 0, 1);
+    } else {
+      zz = warp_sum(zz);
+    }
+    if (!last && lane == 0) z[(size_t)r * (n_exits - 1) + k] = zz + e.router_b;
   }
 }
-void launch_exit_rows(bool bf16, RowSet rs, const void* norm, const void* router_w, float router_b, int k,
-                      int n_exits, void* act, float* z, int d, float eps, cudaStream_t st) {
+void launch_exit_rows(bool bf16, RowSet rs, const ExitDev& e, int router_hidden, int k, int n_exits, void* act,
+                      float* z, int d, float eps, cudaStream_t st) {
   int grid = (rs.max_rows + 7) / 8;
   if (grid > 2048) grid = 2048;
   if (bf16)
-    launch_k(k_exit_rows<__nv_bfloat16>, grid, 256, 0, st, rs, (const __nv_bfloat16*)norm, (const __nv_bfloat16*)router_w,
-                                                     router_b, k, n_exits, (__nv_bfloat16*)act, z, d, eps);
-  else launch_k(k_exit_rows<float>, grid, 256, 0, st, rs, (const float*)norm, (const float*)router_w, router_b, k, n_exits,
-                                                (float*)act, z, d, eps);
+    launch_k(k_exit_rows<__nv_bfloat16>, grid, 256, 0, st, rs, e, router_hidden, k, n_exits, (__nv_bfloat16*)act, z,
+             d, eps);
+  else launch_k(k_exit_rows<float>, grid, 256, 0, st, rs, e, router_hidden, k, n_exits, (float*)act, z, d, eps);
 }
 
 // log pi_k(target) = logit[target] - LSE(logits), one warp per row.
@@ -1330,14 +1363,17 @@ __device__ __forceinline__ float log_sigmoid(float z) {
 }
 
 // log pi_mix = LSE_k(log p_k + log pi_k), log p_k = log sigma(z_k) + sum_{j<k} log sigma(-z_j).
+// log pi_mix = LSE_k(log p_k + log pi_k) per row; with `depth`, also the
+// expected normalised layer depth sum_k p_k * exit_frac[k] (section 2
+// "Training": the compute penalty is the expected normalised depth).
 __global__ void k_mixture(const float* __restrict__ z, const float* __restrict__ logpi, int R, int n_exits, int mode,
-                          float* __restrict__ logp) {
+                          float* __restrict__ logp, float* __restrict__ depth, ExitFrac ef) {
   pdl_wait();
   pdl_launch();
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= R) return;
   float terms[NV_MAX_EXITS];
-  float acc = 0.f, M = -CUDART_INF_F;
+  float acc = 0.f, M = -CUDART_INF_F, dep = 0.f;
   for (int k = 0; k < n_exits; ++k) {
     float lp;
     if (mode == NV_ROUTER_FORCE_LAST) {
@@ -1349,27 +1385,30 @@ __global__ void k_mixture(const float* __restrict__ z, const float* __restrict__
     } else {
       lp = acc;
     }
+    if (lp != -CUDART_INF_F) dep += expf(lp) * ef.f[k];
     terms[k] = lp + logpi[(size_t)r * n_exits + k];
     M = fmaxf(M, terms[k]);
   }
   float s = 0.f;
   for (int k = 0; k < n_exits; ++k) s += (terms[k] == -CUDART_INF_F) ? 0.f : expf(terms[k] - M);
   logp[r] = M + logf(s);
+  if (depth) depth[r] = dep;
 }
 
-__global__ void k_mean_nll(const float* __restrict__ logp, int R, float* __restrict__ out) {
+// *out = scale * mean(x[0..R)), accumulated in double in a fixed order
+__global__ void k_mean(const float* __restrict__ x, int R, float scale, float* __restrict__ out) {
   pdl_wait();
   pdl_launch();
   __shared__ double s[256];
   double a = 0.0;
-  for (int r = threadIdx.x; r < R; r += 256) a += (double)logp[r];
+  for (int r = threadIdx.x; r < R; r += 256) a += (double)x[r];
   s[threadIdx.x] = a;
   __syncthreads();
   for (int o = 128; o; o >>= 1) {
     if (threadIdx.x < o) s[threadIdx.x] += s[threadIdx.x + o];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *out = (float)(-s[0] / (double)R);
+  if (threadIdx.x == 0) *out = (float)((double)scale * s[0] / (double)R);
 }
 
 __global__ void k_philox(unsigned long long seed, const uint4* ctr, int n, uint4* out) {
@@ -1419,10 +1458,19 @@ cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes) {
   return e;
 }
 
-void launch_mixture(const float* z, const float* logpi, int R, int n_exits, int mode, float* logp, float* mean_nll,
-                    cudaStream_t st) {
-  launch_k(k_mixture, (R + 255) / 256, 256, 0, st, z, logpi, R, n_exits, mode, logp);
-  if (mean_nll) launch_k(k_mean_nll, 1, 256, 0, st, logp, R, mean_nll);
+int launch_mixture(const float* z, const float* logpi, int R, int n_exits, int mode, float* logp, float* mean_nll,
+                   float* depth, float* mean_depth, const ExitFrac& ef, cudaStream_t st) {
+  int n = 1;
+  launch_k(k_mixture, (R + 255) / 256, 256, 0, st, z, logpi, R, n_exits, mode, logp, depth, ef);
+  if (mean_nll) {
+    launch_k(k_mean, 1, 256, 0, st, (const float*)logp, R, -1.0f, mean_nll);
+    ++n;
+  }
+  if (depth && mean_depth) {
+    launch_k(k_mean, 1, 256, 0, st, (const float*)depth, R, 1.0f, mean_depth);
+    ++n;
+  }
+  return n;
 }
 
 }  // namespace nv

@@ -147,6 +147,10 @@ struct JuncArgs {
   const void* norm;
   const void* router_w;
   float router_b;
+  int router_hidden;     // router MLP width (0: scalar router)
+  const void* router_w1; // [r][d] model dtype
+  const float* router_b1;
+  const float* router_w2;
   void* exit_act;        // [B][d]
   const unsigned long long* seed;
   long long* counters;
@@ -174,8 +178,10 @@ void launch_head_sample(bool bf16, const HeadArgs& a, cudaStream_t st);
 void launch_head_reduce(const HeadArgs& a, cudaStream_t st);
 
 // scoring
-void launch_exit_rows(bool bf16, RowSet rs, const void* norm, const void* router_w, float router_b, int k,
-                      int n_exits, void* act, float* z, int d, float eps, cudaStream_t st);
+// Scoring rows at exit k: act = RMSNorm_k(h) (model dtype) and the router
+// logit z[r][k] (scalar router, or the router MLP when router_hidden > 0).
+void launch_exit_rows(bool bf16, RowSet rs, const ExitDev& e, int router_hidden, int k, int n_exits, void* act,
+                      float* z, int d, float eps, cudaStream_t st);
 void launch_lse_target(const float* Y, int r_begin, int n, int V, const int* target, float* logpi, int k,
                        int n_exits, cudaStream_t st);
 // Sets conditional `h` to (any active[b] or force[b]); when set, adds
@@ -187,7 +193,13 @@ void launch_philox(unsigned long long seed, const void* ctr, int n, void* out, c
 // Opt-in shared memory for the head sampler and the planner.
 cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes);
 
-void launch_mixture(const float* z, const float* logpi, int R, int n_exits, int mode, float* logp,
-                    float* mean_nll, cudaStream_t st);
+// Normalised depth of each exit: exit_layers[k] / n_layers.
+struct ExitFrac {
+  float f[NV_MAX_EXITS];
+};
+// log pi_mix per row, optional mean NLL, optional expected normalised depth
+// per row and its mean; returns the number of kernels launched.
+int launch_mixture(const float* z, const float* logpi, int R, int n_exits, int mode, float* logp, float* mean_nll,
+                   float* depth, float* mean_depth, const ExitFrac& ef, cudaStream_t st);
 
 }  // namespace nv

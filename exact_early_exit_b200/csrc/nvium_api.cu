@@ -90,7 +90,8 @@ struct nv_model {
   int gemm_kind = GEMM_SIMT;
   GemmPlanCache* gemm_plans = nullptr;
   // scoring scratch
-  Buf sc_h, sc_act, sc_u, sc_ctr, sc_q, sc_o, sc_Y, sc_kv, sc_part, sc_z, sc_logpi, sc_logp, sc_i32, sc_nll;
+  Buf sc_h, sc_act, sc_u, sc_ctr, sc_q, sc_o, sc_Y, sc_kv, sc_part, sc_z, sc_logpi, sc_logp, sc_i32, sc_nll,
+      sc_depth, sc_mdepth;
 };
 
 struct nv_state {
@@ -486,6 +487,10 @@ nv_status record_layers(nv_state* s, cudaStream_t st, Prof* prof, long long* lau
     j.norm = M->exits[k].norm;
     j.router_w = M->exits[k].router_w;
     j.router_b = M->exits[k].router_b;
+    j.router_hidden = M->cfg.router_hidden;
+    j.router_w1 = M->exits[k].router_w1;
+    j.router_b1 = M->exits[k].router_b1;
+    j.router_w2 = M->exits[k].router_w2;
     j.exit_act = s->exit_act;
     j.seed = s->seed_dev;
     j.counters = s->counters;
@@ -734,6 +739,7 @@ nv_status validate_config(const nv_config* c) {
   if (c->page_size < ATTN_KT || c->page_size % ATTN_KT) return bad("page_size must be a multiple of 64");
   if (c->max_pending < 2) return bad("max_pending must be >= 2");
   if (c->router_mode != NV_ROUTER_NORMAL && c->router_mode != NV_ROUTER_FORCE_LAST) return bad("router_mode");
+  if (c->router_hidden < 0 || c->router_hidden > 1024) return bad("router_hidden must be in [0, 1024]");
   if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return bad("rms_eps / rope_theta");
   return NV_OK;
 }
@@ -782,8 +788,11 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
       return NV_ERR_INVALID_ARG;
     }
   }
+  const int RH = cfg->router_hidden;
   for (int k = 0; k < M->NE; ++k) {
-    if (!w->exits[k].norm || !w->exits[k].head || (k < M->NE - 1 && !w->exits[k].router_w)) {
+    const nv_exit_weights& ew = w->exits[k];
+    const bool router_ok = k == M->NE - 1 || (RH ? (ew.router_w1 && ew.router_b1 && ew.router_w2) : ew.router_w != nullptr);
+    if (!ew.norm || !ew.head || !router_ok) {
       set_error("weights: null exit tensor");
       delete M;
       return NV_ERR_INVALID_ARG;
@@ -808,7 +817,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
     o_l[i * 6 + 5] = take(d * F * esz);
   }
   // heads: identical pointers share one packed copy
-  std::vector<size_t> o_e(M->NE * 3);
+  std::vector<size_t> o_e(M->NE * 3), o_r(M->NE * 3, 0);
   for (int k = 0; k < M->NE; ++k) {
     o_e[k * 3 + 0] = take(d * esz);
     int same = -1;
@@ -816,6 +825,11 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
       if (w->exits[j].head == w->exits[k].head) same = j;
     o_e[k * 3 + 1] = same >= 0 ? o_e[same * 3 + 1] : take(V * d * esz);
     o_e[k * 3 + 2] = take(d * esz);
+    if (RH && k < M->NE - 1) {  // router MLP: U [r, d], c [r], v [r]
+      o_r[k * 3 + 0] = take((size_t)RH * d * esz);
+      o_r[k * 3 + 1] = take((size_t)RH * 4);
+      o_r[k * 3 + 2] = take((size_t)RH * 4);
+    }
   }
   const size_t o_rope = take((size_t)cfg->max_seq * (M->hd / 2) * sizeof(float2));
   nv_status st = dalloc_bytes(&M->pool, off);
@@ -866,8 +880,17 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
     const nv_exit_weights& ew = w->exits[k];
     NV_CP(o_e[k * 3 + 0], ew.norm, d * esz);
     NV_CP(o_e[k * 3 + 1], ew.head, V * d * esz);
-    if (k < M->NE - 1) NV_CP(o_e[k * 3 + 2], ew.router_w, d * esz);
-    M->exits[k] = ExitDev{P + o_e[k * 3 + 0], P + o_e[k * 3 + 1], P + o_e[k * 3 + 2], ew.router_b};
+    if (k < M->NE - 1 && ew.router_w) NV_CP(o_e[k * 3 + 2], ew.router_w, d * esz);
+    M->exits[k] = ExitDev{P + o_e[k * 3 + 0], P + o_e[k * 3 + 1], P + o_e[k * 3 + 2], ew.router_b,
+                          nullptr, nullptr, nullptr};
+    if (RH && k < M->NE - 1) {
+      NV_CP(o_r[k * 3 + 0], ew.router_w1, (size_t)RH * d * esz);
+      NV_CP(o_r[k * 3 + 1], ew.router_b1, (size_t)RH * 4);
+      NV_CP(o_r[k * 3 + 2], ew.router_w2, (size_t)RH * 4);
+      M->exits[k].router_w1 = P + o_r[k * 3 + 0];
+      M->exits[k].router_b1 = (const float*)(P + o_r[k * 3 + 1]);
+      M->exits[k].router_w2 = (const float*)(P + o_r[k * 3 + 2]);
+    }
   }
 #undef NV_CP
   M->rope = (float2*)(P + o_rope);
@@ -907,7 +930,7 @@ nv_status nv_destroy(nv_model* M) {
   if (M->pool) cudaFree(M->pool);
   gemm_plans_destroy(M->gemm_plans);
   for (Buf* b : {&M->sc_h, &M->sc_act, &M->sc_u, &M->sc_ctr, &M->sc_q, &M->sc_o, &M->sc_Y, &M->sc_kv, &M->sc_part, &M->sc_z,
-                 &M->sc_logpi, &M->sc_logp, &M->sc_i32, &M->sc_nll})
+                 &M->sc_logpi, &M->sc_logp, &M->sc_i32, &M->sc_nll, &M->sc_depth, &M->sc_mdepth})
     b->release();
   delete M;
   return NV_OK;
@@ -1433,7 +1456,7 @@ nv_status nv_sync_status(nv_state* s) {
 
 namespace {
 nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll, cudaStream_t st,
-                     Prof* prof) {
+                     Prof* prof, float* depth = nullptr, float* mean_depth = nullptr) {
   if (!M || !tokens || !logp) {
     set_error("null argument");
     return NV_ERR_INVALID_ARG;
@@ -1477,6 +1500,10 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
   NV_TRY(M->sc_logpi.need((size_t)R * NE * 4));
   NV_TRY(M->sc_logp.need((size_t)R * 4));
   NV_TRY(M->sc_nll.need(4));
+  if (depth || mean_depth) {
+    NV_TRY(M->sc_depth.need((size_t)R * 4));
+    NV_TRY(M->sc_mdepth.need(4));
+  }
   const int nchunks = (R + head_chunk - 1) / head_chunk;
   NV_TRY(M->sc_i32.need(((size_t)R * 5 + B + 2 + (size_t)B * pps + nchunks) * 4));
   int* d_b = M->sc_i32.as<int>();
@@ -1558,7 +1585,7 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
     const int k = M->exit_at[layer];
     if (k < 0) continue;
     timed(prof, nullptr, 1, NV_K_JUNCTION, (long long)R * M->d * (4 + es), 0, [&] {
-      launch_exit_rows(M->bf16, io.rs, M->exits[k].norm, M->exits[k].router_w, M->exits[k].router_b, k, NE, io.act,
+      launch_exit_rows(M->bf16, io.rs, M->exits[k], M->cfg.router_hidden, k, NE, io.act,
                        M->sc_z.as<float>(), M->d, M->cfg.rms_eps, st);
     });
     for (int c = 0; c < nchunks; ++c) {
@@ -1575,12 +1602,19 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
       NV_TRY(hst);
     }
   }
-  timed(prof, nullptr, 2, NV_K_STEP, 0, 0, [&] {
+  ExitFrac ef{};
+  for (int k = 0; k < NE; ++k) ef.f[k] = (float)M->cfg.exit_layers[k] / (float)M->L;
+  const bool want_depth = depth || mean_depth;
+  const int mix_kernels = 1 + 1 + (want_depth ? 1 : 0);
+  timed(prof, nullptr, mix_kernels, NV_K_STEP, 0, 0, [&] {
     launch_mixture(M->sc_z.as<float>(), M->sc_logpi.as<float>(), R, NE, M->cfg.router_mode, M->sc_logp.as<float>(),
-                   M->sc_nll.as<float>(), st);
+                   M->sc_nll.as<float>(), want_depth ? M->sc_depth.as<float>() : nullptr,
+                   want_depth ? M->sc_mdepth.as<float>() : nullptr, ef, st);
   });
   NV_CUDA_TRY(cudaMemcpyAsync(logp, M->sc_logp.p, (size_t)R * 4, cudaMemcpyDefault, st));
   if (mean_nll) NV_CUDA_TRY(cudaMemcpyAsync(mean_nll, M->sc_nll.p, 4, cudaMemcpyDefault, st));
+  if (depth) NV_CUDA_TRY(cudaMemcpyAsync(depth, M->sc_depth.p, (size_t)R * 4, cudaMemcpyDefault, st));
+  if (mean_depth) NV_CUDA_TRY(cudaMemcpyAsync(mean_depth, M->sc_mdepth.p, 4, cudaMemcpyDefault, st));
   NV_CUDA_TRY(cudaGetLastError());
   return NV_OK;
 }
@@ -1591,6 +1625,11 @@ extern "C" {
 nv_status nv_score_mixture(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll,
                            void* stream) {
   return score_impl(M, tokens, B, S, logp, mean_nll, (cudaStream_t)stream, nullptr);
+}
+
+nv_status nv_score_mixture_ex(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll,
+                              float* depth, float* mean_depth, void* stream) {
+  return score_impl(M, tokens, B, S, logp, mean_nll, (cudaStream_t)stream, nullptr, depth, mean_depth);
 }
 
 nv_status nv_score_mixture_profiled(nv_model* M, const int32_t* tokens, int B, int S, float* logp, float* mean_nll,

@@ -86,6 +86,11 @@ typedef struct nv_config {
   float rope_theta; /* RoPE base, 10000 for LLaMA-2               */
   int max_batch, max_seq, page_size, max_pending;
   int router_mode;
+  /* 0: scalar router (router_w, router_b).  r in [1, 1024]: a router MLP of
+   * hidden width r on the exit-normalised state (section 2 "Architektur":
+   * "a router MLP"), z = router_w2 . silu(router_w1 n_k + router_b1) +
+   * router_b; router_w is then unused. */
+  int router_hidden;
 } nv_config;
 
 /* One backbone layer.  Row-major, PyTorch "out x in" convention (y = x W^T).
@@ -98,12 +103,18 @@ typedef struct nv_layer_weights {
 } nv_layer_weights;
 
 /* One exit: its RMSNorm gain [d_model], its linear head [vocab, d_model], and
- * for k < N_V its scalar sigmoid router w_k = sigma(router_w . n_k + router_b)
- * on the exit-normalised state n_k (router_w [d_model]; ignored for the last
- * exit).  Giving every exit the same `head` pointer shares one head. */
+ * for k < N_V its sigmoid router w_k = sigma(z) on the exit-normalised state
+ * n_k: z = router_w . n_k + router_b (router_w [d_model]), or with
+ * router_hidden = r > 0 the router MLP z = router_w2 . silu(router_w1 n_k +
+ * router_b1) + router_b (router_w1 [r, d_model] in the model dtype,
+ * router_b1 and router_w2 [r] float; silu(x) = x sigmoid(x)).  Router fields
+ * are ignored for the last exit.  Giving every exit the same `head` pointer
+ * shares one head. */
 typedef struct nv_exit_weights {
   const void *norm, *head, *router_w;
   float router_b;
+  const void *router_w1;
+  const float *router_b1, *router_w2;
 } nv_exit_weights;
 
 typedef struct nv_weights {
@@ -129,6 +140,16 @@ nv_status nv_destroy(nv_model *m);
  * Synchronous with respect to `stream` when an output is host memory. */
 nv_status nv_score_mixture(nv_model *m, const int32_t *tokens, int B, int S,
                            float *logp, float *mean_nll, void *stream);
+
+/* nv_score_mixture plus the forward of the compute penalty (section 2
+ * "Training": L_compute is the expected normalised layer depth).  depth
+ * [B, S-1] float (host or device, may be NULL): depth[b][t] = sum_k p_k *
+ * exit_layers[k] / n_layers with the exit probabilities p_k of position t
+ * (those used by logp[b][t]); mean_depth (host or device, may be NULL) =
+ * mean(depth).  Other arguments, results and errors as nv_score_mixture. */
+nv_status nv_score_mixture_ex(nv_model *m, const int32_t *tokens, int B, int S,
+                              float *logp, float *mean_nll, float *depth,
+                              float *mean_depth, void *stream);
 
 /* A decode state for B sequences (B <= max_batch): paged KV cache with its own
  * length per (sequence, layer), deferred-row store, work lists, CUDA graph. */

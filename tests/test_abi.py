@@ -46,7 +46,7 @@ def _cfg(**kw):
 
 @pytest.mark.parametrize("field,value", [
     ("n_layers", 0), ("head_dim", 48), ("dtype", 7), ("page_size", 48), ("max_pending", 1),
-    ("max_batch", 0), ("router_mode", 5), ("n_exits", 0),
+    ("max_batch", 0), ("router_mode", 5), ("n_exits", 0), ("router_hidden", -1), ("router_hidden", 4096),
 ])
 def test_create_rejects_bad_config_on_host(field, value):
     c = _cfg(**{field: value})

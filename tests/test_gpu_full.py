@@ -45,13 +45,18 @@ def test_scoring_16x2048_prefix_matches_oracle(weights, oracle_model):
     model = nv.Model(CFG, weights, max_batch=1, max_seq=2048)
     logp = np.zeros((16, 2047), np.float32)
     nll = np.zeros(1, np.float32)
-    model.score_mixture(toks, logp, nll)
+    depth = np.zeros((16, 2047), np.float32)
+    mean_depth = np.zeros(1, np.float32)
+    model.score_mixture_ex(toks, logp, nll, depth, mean_depth)
     model.close()
     assert np.all(np.isfinite(logp)) and np.all(logp < 0)
     assert abs(float(nll[0]) + float(logp.astype(np.float64).mean())) < 1e-3
+    assert np.all(depth >= 12 / 48 - 1e-6) and np.all(depth <= 1 + 1e-6)
+    assert abs(float(mean_depth[0]) - float(depth.astype(np.float64).mean())) < 1e-5
     T = 40
-    ref, _ = O.score_mixture(oracle_model, toks[5:6, : T + 1])
+    ref, _, ref_depth, _ = O.score_mixture_with_depth(oracle_model, toks[5:6, : T + 1])
     np.testing.assert_allclose(logp[5, :T], ref[0], atol=tolerance(CFG), rtol=0)
+    np.testing.assert_allclose(depth[5, :T], ref_depth[0], atol=tolerance(CFG), rtol=0)
 
 
 def test_decode_b64_sampled_sequence_matches_oracle(weights, oracle_model):

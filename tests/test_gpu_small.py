@@ -26,10 +26,14 @@ def test_scoring_matches_oracle(weights):
     model = nv.Model(CFG, weights, max_batch=1, max_seq=128)
     logp = np.zeros((2, 95), np.float32)
     nll = np.zeros(1, np.float32)
-    model.score_mixture(toks, logp, nll)
-    ref, ref_nll = O.score_mixture(O.OracleModel(CFG, weights), toks)
+    depth = np.zeros((2, 95), np.float32)
+    mean_depth = np.zeros(1, np.float32)
+    model.score_mixture_ex(toks, logp, nll, depth, mean_depth)
+    ref, ref_nll, ref_depth, ref_mean_depth = O.score_mixture_with_depth(O.OracleModel(CFG, weights), toks)
     np.testing.assert_allclose(logp, ref, atol=2e-2, rtol=0)
     assert abs(nll[0] - ref_nll) <= 2e-2
+    np.testing.assert_allclose(depth, ref_depth, atol=2e-2, rtol=0)
+    assert abs(mean_depth[0] - ref_mean_depth) <= 2e-2
 
 
 def test_decode_parity_b4(weights):
@@ -180,4 +184,22 @@ def test_decode_parity_bf16_degenerate_and_ragged_prompts(weights):
     wl = W.WORKLOADS["S"]
     prompts = [p[:n] for p, n in zip(W.make_prompts(wl), (1, 65, 130))]
     chk, state, dec, _ = run_decode_parity(nv, CFG, weights, prompts, 12)
+    assert chk.steps == 12
+
+
+def test_router_mlp_bf16_scoring_and_decode_match_oracle():
+    """Router MLP of width 64 on the bf16 model: scoring and decode parity."""
+    import dataclasses
+    cfg = dataclasses.replace(CFG, router_hidden=64)
+    w = W.make_weights(cfg, seed=0)
+    wl = W.WORKLOADS["S"]
+    toks = np.stack([W.make_prompts(wl, seed=s)[0][:80] for s in (1, 2)]).astype(np.int32)
+    model = nv.Model(cfg, w, max_batch=1, max_seq=128)
+    logp = np.zeros((2, 79), np.float32)
+    model.score_mixture(toks, logp)
+    ref, _ = O.score_mixture(O.OracleModel(cfg, w), toks)
+    np.testing.assert_allclose(logp, ref, atol=tolerance(cfg), rtol=0)
+    model.close()
+    prompts = [p[:n] for p, n in zip(W.make_prompts(wl), (40, 9, 70))]
+    chk, *_ = run_decode_parity(nv, cfg, w, prompts, 12)
     assert chk.steps == 12

@@ -37,10 +37,18 @@ def test_scoring_matches_oracle(weights, mode):
     model = nv.Model(CFG, weights, max_batch=1, max_seq=64, router_mode=mode)
     logp = np.zeros((3, 31), np.float32)
     nll = np.zeros(1, np.float32)
-    model.score_mixture(toks, logp, nll)
-    ref, ref_nll = O.score_mixture(O.OracleModel(CFG, weights, mode), toks)
+    depth = np.zeros((3, 31), np.float32)
+    mean_depth = np.zeros(1, np.float32)
+    model.score_mixture_ex(toks, logp, nll, depth, mean_depth)
+    ref, ref_nll, ref_depth, ref_mean_depth = O.score_mixture_with_depth(O.OracleModel(CFG, weights, mode), toks)
     np.testing.assert_allclose(logp, ref, atol=1e-4, rtol=0)
     assert abs(nll[0] - ref_nll) <= 1e-4
+    # the compute-penalty forward: expected normalised depth per position
+    np.testing.assert_allclose(depth, ref_depth, atol=1e-4, rtol=0)
+    assert abs(mean_depth[0] - ref_mean_depth) <= 1e-4
+    logp2 = np.zeros((3, 31), np.float32)
+    model.score_mixture(toks, logp2)
+    np.testing.assert_array_equal(logp2, logp)
     if mode == O.ROUTER_FORCE_LAST:
         dense = O.dense_logprobs(O.OracleModel(CFG, weights, mode), toks[0, :-1])
         np.testing.assert_allclose(logp[0], dense[np.arange(31), toks[0, 1:]], atol=1e-4, rtol=0)
@@ -233,3 +241,25 @@ def test_bounded_wait_gives_up_and_leaves_the_context_usable():
     out = nv.philox4x32_10(7, ctr)
     ref = O.philox4x32_10([ctr[:, i] for i in range(4)], (7, 0))
     np.testing.assert_array_equal(out, np.stack([r.astype(np.uint32) for r in ref], 1))
+
+
+def test_router_mlp_scoring_and_decode_match_oracle():
+    """Router MLP (width 8) instead of the scalar router: mixture scoring and
+    teacher-forced decode against the oracle, fp32 tolerance."""
+    import dataclasses
+    cfg = dataclasses.replace(CFG, router_hidden=8)
+    w = W.make_weights(cfg, seed=0)
+    toks = np.stack([W.make_prompts(W.WORKLOADS["T"], seed=s)[0] for s in (1, 2)]).astype(np.int32)
+    model = nv.Model(cfg, w, max_batch=1, max_seq=64)
+    logp = np.zeros((2, 31), np.float32)
+    depth = np.zeros((2, 31), np.float32)
+    model.score_mixture_ex(toks, logp, None, depth)
+    ref, _, ref_depth, _ = O.score_mixture_with_depth(O.OracleModel(cfg, w), toks)
+    np.testing.assert_allclose(logp, ref, atol=1e-4, rtol=0)
+    np.testing.assert_allclose(depth, ref_depth, atol=1e-4, rtol=0)
+    model.close()
+    prompts = [W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:n] for s, n in ((1, 7), (2, 20), (3, 1))]
+    chk, state, dec, _ = run_decode_parity(nv, cfg, w, prompts, 16)
+    assert chk.steps == 16 and chk.exit_ties == 0 and chk.token_ties == 0
+    c = state.counters()
+    assert c[nv.CTR["exit0"]:nv.CTR["exit0"] + 4].sum() == 48
