@@ -271,7 +271,11 @@ class OracleModel:
                     e["router_w1"] = f(E["router_w1"])
                     e["router_b1"] = np.asarray(E["router_b1"], dtype=np.float32)
                     e["router_w2"] = np.asarray(E["router_w2"], dtype=np.float32)
+                if getattr(cfg, "adapter_hidden", 0):
+                    e["adapter_w1"] = f(E["adapter_w1"])
+                    e["adapter_w2"] = f(E["adapter_w2"])
             self.exits.append(e)
+        self.adapters = bool(getattr(cfg, "adapter_hidden", 0))
         self.exit_at = {l: k for k, l in enumerate(cfg.exit_layers)}  # layer -> exit index (0-based)
 
     # rounding point of the bf16 numerics contract
@@ -357,15 +361,35 @@ class OracleModel:
         z = self.router_logit(k, nk)
         return 1.0 / (1.0 + np.exp(-z))
 
-    def head_logits(self, k: int, nk: np.ndarray) -> np.ndarray:
-        return self.mm(np.atleast_2d(nk), self.exits[k]["head"])
+    def head_input(self, k: int, h: np.ndarray) -> np.ndarray:
+        """What exit k's head reads.  Per-exit heads: the exit state n_k.
+        Shared head (section 2 "Architektur": all exits share the final LM
+        head, light adapter MLPs map the intermediate states to the geometry
+        the head expects): for k < N_V - 1, m = h + W2 silu(W1 n_k) and the
+        head reads the final norm of m (the last exit's norm); the last exit
+        reads its own state."""
+        if not self.adapters or k == self.cfg.n_exits - 1:
+            return self.exit_state(k, h)
+        e = self.exits[k]
+        nk = self.exit_state(k, h)
+        hid = self.rnd(silu(self.mm(np.atleast_2d(nk), e["adapter_w1"])))
+        m = np.atleast_2d(h) + self.mm(hid, e["adapter_w2"])
+        last = self.cfg.n_exits - 1
+        return self.rnd(rmsnorm(m, widen(self.exits[last]["norm"]), self.cfg.rms_eps)).reshape(np.shape(h))
+
+    def head_logits(self, k: int, x: np.ndarray) -> np.ndarray:
+        """Logits of exit k from its head input x (head_input): exit k's own
+        head, or with adapters the one shared head (the last exit's)."""
+        head = self.exits[-1]["head"] if self.adapters else self.exits[k]["head"]
+        return self.mm(np.atleast_2d(x), head)
 
     # ---- full forward over whole sequences ------------------------------
     def forward_sequence(self, tokens: Sequence[int], cache: Optional[SeqCache] = None,
-                         collect_exits: bool = True):
+                         collect_exits: bool = True, with_heads: bool = False):
         """Standard full-depth forward over positions 0..n-1 of one sequence.
 
-        Returns (h_final [n, d], exit states {k: n_k [n, d]}, cache).
+        Returns (h_final [n, d], exit states {k: n_k [n, d]}, cache), and with
+        with_heads also {k: head input [n, d]} (head_input of each exit).
         """
         cfg = self.cfg
         n = len(tokens)
@@ -373,13 +397,17 @@ class OracleModel:
             cache = SeqCache(cfg.n_layers, n, cfg.n_heads, cfg.head_dim)
         h = self.embed(tokens)
         pos = np.arange(n)
-        states = {}
+        states, heads = {}, {}
         for m in range(cfg.n_layers):
             h = self.layer_rows(m, h, pos, cache)
             cache.lens[m] = n
             if collect_exits and (m + 1) in self.exit_at:
                 k = self.exit_at[m + 1]
                 states[k] = self.exit_state(k, h)
+                if with_heads:
+                    heads[k] = self.head_input(k, h)
+        if with_heads:
+            return h, states, cache, heads
         return h, states, cache
 
 
@@ -409,7 +437,7 @@ def score_mixture_with_depth(model: OracleModel, tokens: np.ndarray):
     out = np.empty((B, S - 1))
     depth = np.empty((B, S - 1))
     for b in range(B):
-        _, states, _ = model.forward_sequence(tokens[b, : S - 1])
+        _, states, _, heads = model.forward_sequence(tokens[b, : S - 1], with_heads=True)
         tgt = tokens[b, 1:].astype(np.int64)
         z = np.zeros((S - 1, cfg.n_exits - 1))
         logpi = np.empty((S - 1, cfg.n_exits))
@@ -417,7 +445,7 @@ def score_mixture_with_depth(model: OracleModel, tokens: np.ndarray):
             nk = states[k]
             if k < cfg.n_exits - 1:
                 z[:, k] = model.router_logit(k, nk)
-            lg = model.head_logits(k, nk)
+            lg = model.head_logits(k, heads[k])
             logpi[:, k] = lg[np.arange(S - 1), tgt] - logsumexp(lg, axis=-1)
         lp = log_exit_probs(z, model.mode)
         out[b] = mixture_logprob(lp, logpi)
@@ -563,7 +591,8 @@ class OracleDecoder:
                 fe = None if forced_exits is None else int(forced_exits[b])
                 if (own_stop if fe is None else fe == k0 + 1):
                     active[b] = False
-                    lg = model.head_logits(k0, nk)[0]
+                    hin = model.head_input(k0, self.pending[b][t]) if model.adapters else nk
+                    lg = model.head_logits(k0, hin)[0]
                     sc = lg + gumbel_noise(seed, self.ids[b], t, cfg.vocab)
                     rec.scores = sc
                     rec.oracle_token = int(np.argmax(sc))
@@ -619,6 +648,7 @@ def step_distribution(model: OracleModel, junction_states: List[np.ndarray]):
     token: returns (p [N_V], pi [N_V, V]) with p the stick-breaking exit
     probabilities and pi_k = softmax(head_k n_k)."""
     cfg = model.cfg
+    assert not model.adapters, "exit states are the head inputs only without adapters"
     w = np.array([np.asarray(model.router_prob(k, junction_states[k])).item() for k in range(cfg.n_exits - 1)])
     p = exit_probs(w)
     pi = np.empty((cfg.n_exits, cfg.vocab))

@@ -444,3 +444,57 @@ def test_router_mlp_hidden_unit_is_torch_silu():
                                 lambda e: np.array([c0, 1.0], np.float32), lambda e: np.array([1.0, 0.0], np.float32))
     for k in range(W.TINY.n_exits - 1):
         np.testing.assert_allclose(wide.router_logit(k, n), mlp.router_logit(k, n), rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# shared head + exit adapters (section 2 "Architektur": all exits share the
+# final LM head; light adapter MLPs map intermediate states to its geometry)
+# ---------------------------------------------------------------------------
+def _adapter_model(W1_of, W2_of, same_norms=False, mode=O.ROUTER_NORMAL):
+    import dataclasses
+    _, w = tiny_model(mode)
+    a = W1_of(w["exits"][0]).shape[0]
+    cfg = dataclasses.replace(W.TINY, adapter_hidden=a)
+    w2 = {**w, "exits": [dict(e) for e in w["exits"]]}
+    last = w2["exits"][-1]
+    for k in range(cfg.n_exits - 1):
+        e = w2["exits"][k]
+        e["adapter_w1"], e["adapter_w2"] = W1_of(e), W2_of(e)
+        if same_norms:
+            e["norm"] = last["norm"]
+    return O.OracleModel(cfg, w2, mode), w2
+
+
+def test_adapters_with_zero_output_are_the_shared_head_model():
+    """W2 = 0 and every exit norm equal to the final norm: the adapter model is
+    the per-exit-head model whose heads are all the final LM head (pinned
+    through the independent LLaMA above)."""
+    d = W.TINY.d_model
+    rng = np.random.default_rng(4)
+    ad, w2 = _adapter_model(lambda e: rng.normal(size=(32, d)).astype(np.float32),
+                            lambda e: np.zeros((d, 32), np.float32), same_norms=True)
+    per = {**w2, "exits": [dict(e, head=w2["exits"][-1]["head"]) for e in w2["exits"]]}
+    ref = O.OracleModel(W.TINY, per)
+    toks = np.stack([W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:16] for s in (1, 2)])
+    np.testing.assert_allclose(O.score_mixture(ad, toks)[0], O.score_mixture(ref, toks)[0], rtol=0, atol=1e-12)
+
+
+def test_adapter_head_input_against_torch():
+    """One exit's head input, m = h + W2 silu(W1 n_k) then the final RMSNorm,
+    against torch's silu and rms_norm in float64 (fp32 model: no rounding)."""
+    import torch
+    import torch.nn.functional as F
+    d = W.TINY.d_model
+    rng = np.random.default_rng(6)
+    ad, w2 = _adapter_model(lambda e: (rng.normal(size=(16, d)) / np.sqrt(d)).astype(np.float32),
+                            lambda e: (rng.normal(size=(d, 16)) * 0.3).astype(np.float32))
+    h = rng.normal(size=(8, d))
+    for k in range(W.TINY.n_exits - 1):
+        e = w2["exits"][k]
+        n = F.rms_norm(torch.from_numpy(h), (d,), torch.from_numpy(e["norm"].astype(np.float64)), 1e-5)
+        m = torch.from_numpy(h) + F.silu(n @ torch.from_numpy(e["adapter_w1"].astype(np.float64)).T) @ \
+            torch.from_numpy(e["adapter_w2"].astype(np.float64)).T
+        want = F.rms_norm(m, (d,), torch.from_numpy(w2["exits"][-1]["norm"].astype(np.float64)), 1e-5).numpy()
+        np.testing.assert_allclose(ad.head_input(k, h), want, rtol=0, atol=1e-12)
+    # the last exit reads its own state, adapters or not
+    np.testing.assert_array_equal(ad.head_input(3, h), ad.exit_state(3, h))

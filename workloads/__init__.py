@@ -55,6 +55,9 @@ class ModelConfig:
     rope_theta: float = 10000.0
     # hidden width of the router MLP of every exit but the last; 0: scalar router
     router_hidden: int = 0
+    # hidden width of the exit adapters in front of one shared LM head (the
+    # last exit's head and norm); 0: every exit has its own head
+    adapter_hidden: int = 0
 
     @property
     def n_exits(self) -> int:
@@ -195,7 +198,9 @@ def make_weights(cfg: ModelConfig, seed: int = 0, random_gains: bool = False,
     exit dict has "norm", "head", and for k < N_V "router_w" and the float
     "router_b"; with cfg.router_hidden = r > 0 also the router MLP's
     "router_w1" [r, d] (model dtype), "router_b1" [r] and "router_w2" [r]
-    (float32).
+    (float32); with cfg.adapter_hidden = a > 0 also the exit adapter's
+    "adapter_w1" [a, d] and "adapter_w2" [d, a] (model dtype), and the exits
+    then share the last exit's head and norm.
     """
     specs = _tensor_specs(cfg)
 
@@ -247,6 +252,16 @@ def make_weights(cfg: ModelConfig, seed: int = 0, random_gains: bool = False,
             w["exits"][k]["router_b1"] = (rng.standard_normal(size=r, dtype=np.float32) * np.float32(0.1))
             w["exits"][k]["router_w2"] = (rng.standard_normal(size=r, dtype=np.float32) *
                                           np.float32(1.0 / np.sqrt(r)))
+    if cfg.adapter_hidden:
+        # exit adapters m = h + W2 silu(W1 n_k): W1 ~ N(0, 1/d), W2 ~ N(0, 0.02^2)
+        # (model dtype); streams after the router MLP's
+        a, d = cfg.adapter_hidden, cfg.d_model
+        for k in range(cfg.n_exits - 1):
+            rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(len(specs) + 101 + k,))))
+            W1 = rng.standard_normal(size=(a, d), dtype=np.float32) * np.float32(1.0 / np.sqrt(d))
+            W2 = rng.standard_normal(size=(d, a), dtype=np.float32) * np.float32(0.02)
+            w["exits"][k]["adapter_w1"] = f32_to_bf16_bits(W1) if cfg.dtype == BF16 else W1
+            w["exits"][k]["adapter_w2"] = f32_to_bf16_bits(W2) if cfg.dtype == BF16 else W2
     return w
 
 
