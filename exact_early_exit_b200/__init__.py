@@ -57,7 +57,7 @@ class Config(ctypes.Structure):
                 ("n_exits", ctypes.c_int), ("exit_layers", ctypes.c_int * NV_MAX_EXITS), ("dtype", ctypes.c_int),
                 ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("max_batch", ctypes.c_int),
                 ("max_seq", ctypes.c_int), ("page_size", ctypes.c_int), ("max_pending", ctypes.c_int),
-                ("router_mode", ctypes.c_int), ("router_hidden", ctypes.c_int)]
+                ("router_mode", ctypes.c_int), ("router_hidden", ctypes.c_int), ("adapter_hidden", ctypes.c_int)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -67,7 +67,7 @@ class LayerWeights(ctypes.Structure):
 class ExitWeights(ctypes.Structure):
     _fields_ = [("norm", ctypes.c_void_p), ("head", ctypes.c_void_p), ("router_w", ctypes.c_void_p),
                 ("router_b", ctypes.c_float), ("router_w1", ctypes.c_void_p), ("router_b1", ctypes.c_void_p),
-                ("router_w2", ctypes.c_void_p)]
+                ("router_w2", ctypes.c_void_p), ("adapter_w1", ctypes.c_void_p), ("adapter_w2", ctypes.c_void_p)]
 
 
 class Weights(ctypes.Structure):
@@ -174,6 +174,7 @@ def make_config(model_cfg, max_batch: int, max_seq: int, page_size: int = 64, ma
     c.max_pending = max_pending
     c.router_mode = router_mode
     c.router_hidden = int(getattr(model_cfg, "router_hidden", 0))
+    c.adapter_hidden = int(getattr(model_cfg, "adapter_hidden", 0))
     return c
 
 
@@ -206,10 +207,10 @@ class Model:
         ew = (ExitWeights * n_exits)()
         for k, E in enumerate(weights["exits"]):
             ew[k].norm = p(E["norm"])
-            ew[k].head = p(E["head"])
+            ew[k].head = p(E["head"]) if "head" in E else None
             ew[k].router_w = p(E["router_w"]) if "router_w" in E else None
             ew[k].router_b = float(E.get("router_b", 0.0))
-            for f in ("router_w1", "router_b1", "router_w2"):
+            for f in ("router_w1", "router_b1", "router_w2", "adapter_w1", "adapter_w2"):
                 if f in E:
                     setattr(ew[k], f, p(E[f]))
         w = Weights(p(weights["tok_emb"]), lw, ew)

@@ -114,6 +114,8 @@ struct ExitDev {
   const void* router_w1;    // router MLP [r, d] (model dtype), or null
   const float* router_b1;   // [r]
   const float* router_w2;   // [r]
+  const void* adapter_w1;   // exit adapter [a, d] (model dtype), or null
+  const void* adapter_w2;   // [d, a]
 };
 
 // Rows processed together at one layer.  Rows of a sequence are contiguous and

@@ -1086,6 +1086,106 @@ void launch_junction(bool bf16, const JuncArgs& a, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
+// Exit adapter (section 2 "Architektur": all exits share the final LM head,
+// light adapter MLPs map the intermediate states to its geometry).  One CTA
+// per sequence that stopped here: hidden = silu(W1 n_k) (rounded to the model
+// dtype: it multiplies W2), m = h + W2 hidden (fp32), head input = final
+// RMSNorm of m.  Shared memory: hidden [a] and m [d].
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) k_exit_adapter(AdapterArgs p) {
+  pdl_wait();
+  pdl_launch();
+  const int b = blockIdx.x;
+  if (!p.stop[b]) return;
+  extern __shared__ float s_ad[];
+  float* s_hid = s_ad;
+  float* s_m = s_ad + p.a;
+  T* x = (T*)p.exit_act + (size_t)b * p.d;
+  const float* h = p.hbuf + ((size_t)b * p.cap + p.t[b] % p.cap) * p.d;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int j = w; j < p.a; j += 8) {
+    const T* u = (const T*)p.w1 + (size_t)j * p.d;
+    float acc = 0.f;
+    for (int i = lane; i < p.d; i += 32) acc = fmaf(ld(x + i), ld(u + i), acc);
+    acc = warp_sum(acc);
+    if (lane == 0) s_hid[j] = rnd<T>(acc / (1.0f + expf(-acc)));
+  }
+  __syncthreads();
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < p.d; i += 256) {
+    const T* v = (const T*)p.w2 + (size_t)i * p.a;
+    float o = 0.f;
+    for (int j = 0; j < p.a; ++j) o = fmaf(ld(v + j), s_hid[j], o);
+    const float m = h[i] + o;
+    s_m[i] = m;
+    ss = fmaf(m, m, ss);
+  }
+  ss = block_sum<256>(ss);
+  const float inv = 1.0f / sqrtf(ss / (float)p.d + p.eps);
+  const T* g = (const T*)p.final_norm;
+  for (int i = threadIdx.x; i < p.d; i += 256) x[i] = cvt<T>(rnd<T>(s_m[i] * inv * ld(g + i)));
+}
+void launch_exit_adapter(bool bf16, const AdapterArgs& a, cudaStream_t st) {
+  const size_t sm = (size_t)(a.a + a.d) * sizeof(float);
+  if (bf16) launch_k(k_exit_adapter<__nv_bfloat16>, a.B, 256, sm, st, a);
+  else launch_k(k_exit_adapter<float>, a.B, 256, sm, st, a);
+}
+cudaError_t exit_adapter_prepare(bool bf16, int d, int a) {
+  const size_t sm = (size_t)(a + d) * sizeof(float);
+  if (sm <= 48 * 1024) return cudaSuccess;
+  return bf16 ? cudaFuncSetAttribute(k_exit_adapter<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)
+              : cudaFuncSetAttribute(k_exit_adapter<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+}
+
+template <typename T>
+__global__ void k_silu_rows(const int* __restrict__ nrows, const float* __restrict__ Y, int a, T* __restrict__ u) {
+  pdl_wait();
+  pdl_launch();
+  const size_t n = (size_t)(*nrows) * a;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float y = Y[i];
+    u[i] = cvt<T>(rnd<T>(y / (1.0f + expf(-y))));
+  }
+}
+void launch_silu_rows(bool bf16, const int* nrows, const float* Y, int a, void* u, int max_rows, cudaStream_t st) {
+  long long g = ((long long)max_rows * a + 255) / 256;
+  const int grid = (int)(g < 4096 ? (g < 1 ? 1 : g) : 4096);
+  if (bf16) launch_k(k_silu_rows<__nv_bfloat16>, grid, 256, 0, st, nrows, Y, a, (__nv_bfloat16*)u);
+  else launch_k(k_silu_rows<float>, grid, 256, 0, st, nrows, Y, a, (float*)u);
+}
+
+template <typename T>
+__global__ void k_adapter_norm_rows(RowSet rs, const float* __restrict__ Y, const T* __restrict__ g,
+                                    T* __restrict__ act, int d, float eps) {
+  pdl_wait();
+  pdl_launch();
+  const int R = *rs.nrows;
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb) {
+    const float* h = rs.h + (size_t)rs.row_hrow[r] * d;
+    const float* y = Y + (size_t)r * d;
+    float ss = 0.f;
+    for (int i = lane; i < d; i += 32) {
+      const float m = h[i] + y[i];
+      ss = fmaf(m, m, ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    for (int i = lane; i < d; i += 32) act[(size_t)r * d + i] = cvt<T>(rnd<T>((h[i] + y[i]) * inv * ld(g + i)));
+  }
+}
+void launch_adapter_norm_rows(bool bf16, RowSet rs, const float* Y, const void* final_norm, void* act, int d,
+                              float eps, cudaStream_t st) {
+  int grid = (rs.max_rows + 7) / 8;
+  if (grid > 2048) grid = 2048;
+  if (bf16)
+    launch_k(k_adapter_norm_rows<__nv_bfloat16>, grid, 256, 0, st, rs, Y, (const __nv_bfloat16*)final_norm,
+             (__nv_bfloat16*)act, d, eps);
+  else launch_k(k_adapter_norm_rows<float>, grid, 256, 0, st, rs, Y, (const float*)final_norm, (float*)act, d, eps);
+}
+
+// ---------------------------------------------------------------------------
 // Fused exit-head sampler (exact sampling, section 3; Gumbel-max reading).
 // For the rows that stopped at exit k: logit_v = W_k[v] . n_k with 16-byte
 // coalesced loads of each head row, score_v = logit_v + Gumbel(U_v) with U_v

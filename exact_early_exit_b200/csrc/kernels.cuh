@@ -159,6 +159,29 @@ struct JuncArgs {
 };
 void launch_junction(bool bf16, const JuncArgs& a, cudaStream_t st);
 
+// Exit adapter in front of the shared head (decode): for every sequence that
+// stopped at this exit, exit_act[b] (n_k on entry) becomes the final
+// RMSNorm of m = h + W2 silu(W1 n_k).
+struct AdapterArgs {
+  int B, cap, d, a;
+  float eps;
+  const int* t;
+  const int* stop;        // [B] flags of this exit
+  const float* hbuf;
+  const void* w1;         // [a][d]
+  const void* w2;         // [d][a]
+  const void* final_norm; // [d] (the last exit's norm)
+  void* exit_act;         // [B][d]
+};
+void launch_exit_adapter(bool bf16, const AdapterArgs& a, cudaStream_t st);
+cudaError_t exit_adapter_prepare(bool bf16, int d, int a);
+// Scoring side of the same adapter, after the two GEMMs of W1 and W2:
+// u = silu(Y) (model dtype) over the [rows][a] hidden, and act = final
+// RMSNorm of h + Y over the [rows][d] output.
+void launch_silu_rows(bool bf16, const int* nrows, const float* Y, int a, void* u, int max_rows, cudaStream_t st);
+void launch_adapter_norm_rows(bool bf16, RowSet rs, const float* Y, const void* final_norm, void* act, int d,
+                              float eps, cudaStream_t st);
+
 struct HeadArgs {
   int B, d, V, k;
   const int* t;

@@ -498,6 +498,24 @@ nv_status record_layers(nv_state* s, cudaStream_t st, Prof* prof, long long* lau
     j.head_bytes = (long long)M->V * M->d * es;
     timed(prof, launches, 1, NV_K_JUNCTION, (long long)s->B * M->d * (4 + es), 0,
           [&] { launch_junction(bf, j, st); });
+    if (M->cfg.adapter_hidden && k < M->NE - 1) {
+      // the shared head reads the adapter's output, not n_k
+      AdapterArgs ad{};
+      ad.B = s->B;
+      ad.cap = s->cap;
+      ad.d = M->d;
+      ad.a = M->cfg.adapter_hidden;
+      ad.eps = M->cfg.rms_eps;
+      ad.t = s->t;
+      ad.stop = j.stop;
+      ad.hbuf = s->hbuf;
+      ad.w1 = M->exits[k].adapter_w1;
+      ad.w2 = M->exits[k].adapter_w2;
+      ad.final_norm = M->exits[M->NE - 1].norm;
+      ad.exit_act = s->exit_act;
+      timed(prof, launches, 1, NV_K_JUNCTION, 2LL * ad.a * M->d * es, 4LL * s->B * ad.a * M->d,
+            [&] { launch_exit_adapter(bf, ad, st); });
+    }
     HeadArgs h{};
     h.B = s->B;
     h.d = M->d;
@@ -740,6 +758,8 @@ nv_status validate_config(const nv_config* c) {
   if (c->max_pending < 2) return bad("max_pending must be >= 2");
   if (c->router_mode != NV_ROUTER_NORMAL && c->router_mode != NV_ROUTER_FORCE_LAST) return bad("router_mode");
   if (c->router_hidden < 0 || c->router_hidden > 1024) return bad("router_hidden must be in [0, 1024]");
+  if (c->adapter_hidden < 0 || c->adapter_hidden > 4096) return bad("adapter_hidden must be in [0, 4096]");
+  if (c->adapter_hidden && c->dtype == NV_BF16 && c->adapter_hidden % 128) return bad("bf16 adapter_hidden % 128");
   if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return bad("rms_eps / rope_theta");
   return NV_OK;
 }
@@ -788,11 +808,13 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
       return NV_ERR_INVALID_ARG;
     }
   }
-  const int RH = cfg->router_hidden;
+  const int RH = cfg->router_hidden, AH = cfg->adapter_hidden;
   for (int k = 0; k < M->NE; ++k) {
     const nv_exit_weights& ew = w->exits[k];
-    const bool router_ok = k == M->NE - 1 || (RH ? (ew.router_w1 && ew.router_b1 && ew.router_w2) : ew.router_w != nullptr);
-    if (!ew.norm || !ew.head || !router_ok) {
+    const bool last = k == M->NE - 1;
+    const bool router_ok = last || (RH ? (ew.router_w1 && ew.router_b1 && ew.router_w2) : ew.router_w != nullptr);
+    const bool head_ok = AH ? (last ? ew.head != nullptr : (ew.adapter_w1 && ew.adapter_w2)) : ew.head != nullptr;
+    if (!ew.norm || !head_ok || !router_ok) {
       set_error("weights: null exit tensor");
       delete M;
       return NV_ERR_INVALID_ARG;
@@ -817,13 +839,19 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
     o_l[i * 6 + 5] = take(d * F * esz);
   }
   // heads: identical pointers share one packed copy
-  std::vector<size_t> o_e(M->NE * 3), o_r(M->NE * 3, 0);
+  std::vector<size_t> o_e(M->NE * 3), o_r(M->NE * 3, 0), o_a(M->NE * 2, 0);
+  // with adapters every exit reads the last exit's head: pack it first
+  const size_t o_shared = AH ? take(V * d * esz) : 0;
   for (int k = 0; k < M->NE; ++k) {
     o_e[k * 3 + 0] = take(d * esz);
     int same = -1;
     for (int j = 0; j < k; ++j)
       if (w->exits[j].head == w->exits[k].head) same = j;
-    o_e[k * 3 + 1] = same >= 0 ? o_e[same * 3 + 1] : take(V * d * esz);
+    o_e[k * 3 + 1] = AH ? o_shared : (same >= 0 ? o_e[same * 3 + 1] : take(V * d * esz));
+    if (AH && k < M->NE - 1) {  // adapter W1 [a, d], W2 [d, a]
+      o_a[k * 2 + 0] = take((size_t)AH * d * esz);
+      o_a[k * 2 + 1] = take((size_t)AH * d * esz);
+    }
     o_e[k * 3 + 2] = take(d * esz);
     if (RH && k < M->NE - 1) {  // router MLP: U [r, d], c [r], v [r]
       o_r[k * 3 + 0] = take((size_t)RH * d * esz);
@@ -879,10 +907,16 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
   for (int k = 0; k < M->NE; ++k) {
     const nv_exit_weights& ew = w->exits[k];
     NV_CP(o_e[k * 3 + 0], ew.norm, d * esz);
-    NV_CP(o_e[k * 3 + 1], ew.head, V * d * esz);
+    if (!AH || k == M->NE - 1) NV_CP(o_e[k * 3 + 1], ew.head, V * d * esz);
     if (k < M->NE - 1 && ew.router_w) NV_CP(o_e[k * 3 + 2], ew.router_w, d * esz);
     M->exits[k] = ExitDev{P + o_e[k * 3 + 0], P + o_e[k * 3 + 1], P + o_e[k * 3 + 2], ew.router_b,
-                          nullptr, nullptr, nullptr};
+                          nullptr, nullptr, nullptr, nullptr, nullptr};
+    if (AH && k < M->NE - 1) {
+      NV_CP(o_a[k * 2 + 0], ew.adapter_w1, (size_t)AH * d * esz);
+      NV_CP(o_a[k * 2 + 1], ew.adapter_w2, (size_t)AH * d * esz);
+      M->exits[k].adapter_w1 = P + o_a[k * 2 + 0];
+      M->exits[k].adapter_w2 = P + o_a[k * 2 + 1];
+    }
     if (RH && k < M->NE - 1) {
       NV_CP(o_r[k * 3 + 0], ew.router_w1, (size_t)RH * d * esz);
       NV_CP(o_r[k * 3 + 1], ew.router_b1, (size_t)RH * 4);
@@ -908,6 +942,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
     const size_t head_sm = (((size_t)cfg->max_batch * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * d * esz;
     cudaError_t e2 = kernels_set_smem_limits(head_sm, (size_t)(cfg->max_batch + 1) * 4);
     if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_mma_prepare();
+    if (e2 == cudaSuccess && cfg->adapter_hidden) e2 = exit_adapter_prepare(M->bf16, M->d, cfg->adapter_hidden);
     if (e2 != cudaSuccess) {
       set_error(std::string("shared memory limits: ") + cudaGetErrorString(e2));
       nv_destroy(M);
@@ -1483,11 +1518,13 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
   const int pps = (S + ps - 1) / ps;
   const size_t wide = M->d > M->F ? M->d : M->F;
   const int head_chunk = std::min(R, 4096);
-  const size_t y_layers = gemm_workspace_elems(M->gemm_kind, R, 3 * M->HQ > 2 * M->F ? 3 * M->HQ : 2 * M->F);
+  const int AH = M->cfg.adapter_hidden;
+  const size_t y_layers = gemm_workspace_elems(
+      M->gemm_kind, R, std::max<size_t>(3 * M->HQ > 2 * M->F ? 3 * M->HQ : 2 * M->F, (size_t)AH));
   const size_t y_head = gemm_workspace_elems(M->gemm_kind, head_chunk, M->V);
   NV_TRY(M->sc_h.need((size_t)R * M->d * 4));
   NV_TRY(M->sc_act.need((size_t)R * wide * M->esz));
-  NV_TRY(M->sc_u.need((size_t)R * M->F * M->esz));
+  NV_TRY(M->sc_u.need((size_t)R * std::max<size_t>(M->F, (size_t)AH) * M->esz));
   if (!M->sc_ctr.p) {
     NV_TRY(M->sc_ctr.need((size_t)kTileCounters * 4));
     NV_CUDA_TRY(cudaMemset(M->sc_ctr.p, 0, (size_t)kTileCounters * 4));
@@ -1588,6 +1625,26 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
       launch_exit_rows(M->bf16, io.rs, M->exits[k], M->cfg.router_hidden, k, NE, io.act,
                        M->sc_z.as<float>(), M->d, M->cfg.rms_eps, st);
     });
+    if (AH && k < NE - 1) {
+      // exit adapter before the shared head: hidden = silu(n_k W1^T), then
+      // act = final RMSNorm of h + hidden W2^T
+      nv_status ast = NV_OK;
+      timed(prof, nullptr, gemm_launch_count(M->gemm_kind, M->bf16, false, nullptr) * 2 + 2, NV_K_HEAD,
+            2LL * AH * M->d * es, 4LL * R * AH * M->d, [&] {
+              ast = gemm_run(M->gemm_plans, M->gemm_kind, M->bf16, io.act, M->d, M->exits[k].adapter_w1, AH, M->d,
+                             io.rs.nrows, io.rs.max_rows, io.Y, false, nullptr, io.tile_counters, io.epi_grid,
+                             nullptr, 0, st);
+              if (ast != NV_OK) return;
+              launch_silu_rows(M->bf16, io.rs.nrows, io.Y, AH, io.u, io.rs.max_rows, st);
+              ast = gemm_run(M->gemm_plans, M->gemm_kind, M->bf16, io.u, AH, M->exits[k].adapter_w2, M->d, AH,
+                             io.rs.nrows, io.rs.max_rows, io.Y, false, nullptr, io.tile_counters, io.epi_grid,
+                             nullptr, 0, st);
+              if (ast != NV_OK) return;
+              launch_adapter_norm_rows(M->bf16, io.rs, io.Y, M->exits[NE - 1].norm, io.act, M->d, M->cfg.rms_eps,
+                                       st);
+            });
+      NV_TRY(ast);
+    }
     for (int c = 0; c < nchunks; ++c) {
       const int r0 = c * head_chunk;
       const long long rc = std::min(head_chunk, R - r0);

@@ -91,6 +91,12 @@ typedef struct nv_config {
    * "a router MLP"), z = router_w2 . silu(router_w1 n_k + router_b1) +
    * router_b; router_w is then unused. */
   int router_hidden;
+  /* 0: every exit has its own norm and head.  a > 0: the exits share one LM
+   * head, the last exit's (section 2 "Architektur": a shared head with light
+   * adapter MLPs): exit k < N_V's head reads the final RMSNorm (the last
+   * exit's norm) of m = h + adapter_w2 silu(adapter_w1 n_k), n_k still
+   * feeding the router.  a in [1, 4096]; bf16 models need a % 128 == 0. */
+  int adapter_hidden;
 } nv_config;
 
 /* One backbone layer.  Row-major, PyTorch "out x in" convention (y = x W^T).
@@ -115,6 +121,10 @@ typedef struct nv_exit_weights {
   float router_b;
   const void *router_w1;
   const float *router_b1, *router_w2;
+  /* adapter_hidden = a > 0, exits before the last: adapter_w1 [a, d_model],
+   * adapter_w2 [d_model, a] (model dtype); `head` is then read from the last
+   * exit only. */
+  const void *adapter_w1, *adapter_w2;
 } nv_exit_weights;
 
 typedef struct nv_weights {

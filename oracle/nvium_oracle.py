@@ -263,7 +263,9 @@ class OracleModel:
         self.layers = [{k: f(v) for k, v in L.items()} for L in weights["layers"]]
         self.exits = []
         for k, E in enumerate(weights["exits"]):
-            e = {"norm": f(E["norm"]), "head": f(E["head"])}
+            e = {"norm": f(E["norm"])}
+            if "head" in E:  # with adapters only the last exit's head is read
+                e["head"] = f(E["head"])
             if k < cfg.n_exits - 1:
                 e["router_w"] = f(E["router_w"])
                 e["router_b"] = float(E["router_b"])

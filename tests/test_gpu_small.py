@@ -203,3 +203,26 @@ def test_router_mlp_bf16_scoring_and_decode_match_oracle():
     prompts = [p[:n] for p, n in zip(W.make_prompts(wl), (40, 9, 70))]
     chk, *_ = run_decode_parity(nv, cfg, w, prompts, 12)
     assert chk.steps == 12
+
+
+@pytest.mark.parametrize("batch", [3, 16])
+def test_shared_head_with_adapters_bf16_matches_oracle(batch):
+    """Shared head behind adapters of width 128 on the bf16 model: scoring
+    (tcgen05 GEMMs for the adapters) and decode, with the SIMT head (B=3) and
+    the tensor-core head (B=16)."""
+    import dataclasses
+    cfg = dataclasses.replace(CFG, adapter_hidden=128)
+    w = W.make_weights(cfg, seed=0)
+    wl = W.WORKLOADS["S"]
+    if batch == 3:
+        toks = np.stack([W.make_prompts(wl, seed=s)[0][:80] for s in (1, 2)]).astype(np.int32)
+        model = nv.Model(cfg, w, max_batch=1, max_seq=128)
+        logp = np.zeros((2, 79), np.float32)
+        model.score_mixture(toks, logp)
+        ref, _ = O.score_mixture(O.OracleModel(cfg, w), toks)
+        np.testing.assert_allclose(logp, ref, atol=tolerance(cfg), rtol=0)
+        model.close()
+    prompts = [p[:n] for p, n in zip(W.make_prompts(wl, seed=4, lengths=[70] * batch),
+                                     np.random.default_rng(1).integers(1, 70, size=batch))]
+    chk, *_ = run_decode_parity(nv, cfg, w, prompts, 8, check_kv=batch == 3)
+    assert chk.steps == 8

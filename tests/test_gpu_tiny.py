@@ -263,3 +263,23 @@ def test_router_mlp_scoring_and_decode_match_oracle():
     assert chk.steps == 16 and chk.exit_ties == 0 and chk.token_ties == 0
     c = state.counters()
     assert c[nv.CTR["exit0"]:nv.CTR["exit0"] + 4].sum() == 48
+
+
+def test_shared_head_with_adapters_matches_oracle():
+    """Exits share the last exit's head behind adapters of width 32: scoring
+    and teacher-forced decode against the oracle (fp32)."""
+    import dataclasses
+    cfg = dataclasses.replace(CFG, adapter_hidden=32)
+    w = W.make_weights(cfg, seed=0)
+    for k in range(cfg.n_exits - 1):
+        del w["exits"][k]["head"]  # only the last exit's head is read
+    toks = np.stack([W.make_prompts(W.WORKLOADS["T"], seed=s)[0] for s in (1, 2)]).astype(np.int32)
+    model = nv.Model(cfg, w, max_batch=1, max_seq=64)
+    logp = np.zeros((2, 31), np.float32)
+    model.score_mixture(toks, logp)
+    ref, _ = O.score_mixture(O.OracleModel(cfg, w), toks)
+    np.testing.assert_allclose(logp, ref, atol=1e-4, rtol=0)
+    model.close()
+    prompts = [W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:n] for s, n in ((1, 9), (2, 1), (3, 30))]
+    chk, *_ = run_decode_parity(nv, cfg, w, prompts, 16)
+    assert chk.steps == 16 and chk.exit_ties == 0 and chk.token_ties == 0
