@@ -9,8 +9,10 @@
 // still issues full 128-row MMAs and streams each weight tile once.
 //
 // Persistent, warp-specialised CTAs (one per SM):
-//   warp 4, one lane: TMA producer, 4-stage ring of (W tile 128x64, X tile
-//                     <=256x64), 128-byte swizzle, mbarrier complete_tx;
+//   warp 4, one lane: TMA producer, ring of (W tile 128x64, X tile
+//                     <=256x64) stages, 128-byte swizzle, mbarrier
+//                     complete_tx; the stage count follows the row tile (4
+//                     stages at 256 rows, up to 12 for a handful of rows);
 //   warp 5, one lane: issues tcgen05.mma (kind::f16, M=128, N=32..256,
 //                     K=16) into one of two TMEM accumulators, commits to the
 //                     stage's "empty" barrier and to "accumulator full";
@@ -20,8 +22,11 @@
 // range is split (tc_split_count); the partial slices are summed in a fixed
 // order by the epilogue kernel that follows.  Without a split, the layer
 // epilogue (RoPE + KV write, residual, SwiGLU) runs in the epilogue warps
-// from a staged tile.  Every mbarrier wait is bounded: on expiry
-// the CTA flags DEV_ERR_TIMEOUT, stops issuing work, frees its TMEM and exits.
+// from a staged tile (or, for the exit heads, the Gumbel-max sampler and
+// log-sum-exp of each 128-token tile).  Before griddepcontrol.wait a CTA pulls
+// its own first weight tiles and the next GEMM's weights into L2.  Every
+// mbarrier wait is bounded: on expiry the CTA flags DEV_ERR_TIMEOUT, stops
+// issuing work, frees its TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

@@ -540,7 +540,9 @@ void launch_epilogue(bool bf16, const EpiArgs& a, int grid, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
-// Paged attention with per-(sequence, layer) cache lengths.
+// Paged attention with per-(sequence, layer) cache lengths, SIMT (the fp32
+// model's prefill and scoring attention, and the NVIUM_ATTN=simt comparison
+// path; bf16 models with head_dim 64 use k_attn_fa_mma).
 //
 // CTA (b, head, z): z = row group * kv_splits + split.  The row group is up to
 // 32 consecutive rows of sequence b (ascending positions p); row p attends
@@ -689,7 +691,8 @@ __global__ void k_attn_combine(AttnArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Decode attention: CTA (b, head, chunk) handles keys [chunk*128, chunk*128 +
+// Decode attention, SIMT (the fp32 model's and the comparison path; bf16
+// models with head_dim 64 use k_attn_dec_mma): CTA (b, head, chunk) handles keys [chunk*128, chunk*128 +
 // 128) of sequence b at this layer for every row of b whose position reaches
 // the chunk.  One thread issues TMA bulk copies of the chunk's K and V pages
 // (each page of one head is contiguous), completing on an mbarrier, so the
