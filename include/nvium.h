@@ -186,9 +186,10 @@ nv_status nv_rewind(nv_state *s, void *stream);
  * argmax_v(logit_k[v] + Gumbel(U_v)), U_v from counter (b, t, 1, v/4), lane
  * v%4, ties to the lowest id.  Layers above the exit are deferred; at each
  * layer the deferred rows of a sequence whose new token reaches that layer
- * run in the same packed pass.  Outputs (host or device, [B]): tokens_out =
- * sampled ids, exits_out = exit used (1..N_V), logp_out (may be NULL) =
- * log pi_exit(token). */
+ * run in the same packed pass.  With adapter_hidden > 0 the logits come
+ * from the shared head applied to the exit's adapter output.  Outputs (host
+ * or device, [B]): tokens_out = sampled ids, exits_out = exit used (1..N_V),
+ * logp_out (may be NULL) = log pi_exit(token). */
 nv_status nv_decode_step(nv_state *s, uint64_t philox_seed, int32_t *tokens_out,
                          int32_t *exits_out, float *logp_out, void *stream);
 
