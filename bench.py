@@ -36,6 +36,7 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "decode tokens/s, 1.5B 4-exit model, B=1/B=64 on 1 B200; % of HBM roofline"
+SCORE_METRIC = "mixture scoring tokens/s, 1.5B 4-exit model, 16 x 2048; GEMMs as % of bf16 tensor peak"
 FALLBACK_HBM_GBS = 6650.0
 PHILOX_SEED = 1234
 
@@ -457,7 +458,7 @@ def run_scoring(args):
     gemm_flops = kern["gemm"]["flops"] + kern["head"]["flops"]
     achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
     peak, src = measured_tensor_peak()
-    out = {"metric": "mixture scoring tokens/s, 1.5B 4-exit model, 16 x 2048; GEMMs as % of bf16 tensor peak",
+    out = {"metric": SCORE_METRIC,
            "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -516,11 +517,40 @@ def cpu_baseline(wl, weights_seed, lens, prompts, xseed, prefix=128, n_steps=2):
                       f"{n_steps} decode steps timed (1 token each), float64 numpy"}
 
 
+def run_reference_scoring(args, wl, world):
+    """The oracle's mixture scoring on a bounded sample of the scoring
+    workload: one sequence's first 65 tokens (64 scored positions) per step."""
+    from oracle import nvium_oracle as O
+    pseed, _, _ = rank_seeds(0)
+    toks = np.stack(W.make_prompts(wl, seed=pseed)).astype(np.int32)[:1, :65]
+    om = O.OracleModel(wl.model, W.make_weights(wl.model, seed=0))
+    for _ in range(args.warmup):
+        O.score_mixture(om, toks[:, :9])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.score_mixture(om, toks)
+    dt = time.perf_counter() - t0
+    value = args.steps * (toks.shape[1] - 1) / dt
+    sample = "sequence 0, first 65 tokens (64 scored positions) per step, float64 numpy oracle"
+    out = {"metric": SCORE_METRIC, "impl": "reference", "value": round(value, 4), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(dt / args.steps * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": wl.name, "model": wl.model.name, "global_batch": wl.batch, "seq_len": wl.prompt_len},
+           "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
 def run_reference(args):
     rank, world, _ = rank_env()
     if rank != 0:
         return
     wl = W.WORKLOADS[args.workload]
+    if args.workload == "XS":
+        run_reference_scoring(args, wl, world)
+        return
     pseed, lseed, xseed = rank_seeds(0)
     lens = W.make_prompt_lengths(wl, seed=lseed)
     prompts = W.make_prompts(wl, seed=pseed, lengths=lens)

@@ -5,6 +5,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 import bench
@@ -56,3 +57,30 @@ def test_bench_rejects_short_warmup():
     import pytest
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "1"])
+
+
+def _reference_line(workload):
+    import contextlib
+    import io
+    import json
+    import bench
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", workload, "--steps", "1", "--warmup", "3"])
+    lines = [l for l in buf.getvalue().splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    return json.loads(lines[0])
+
+
+@pytest.mark.parametrize("workload,metric", [("T", "METRIC"), ("XS", "SCORE_METRIC")])
+def test_reference_arm_prints_the_contract_line(workload, metric):
+    """The reference arm (the oracle on the host cores) prints one JSON line
+    with the base contract's keys, its cpu_baseline and an e2e of zero bytes."""
+    d = _reference_line(workload)
+    assert d["impl"] == "reference" and d["metric"] == getattr(bench, metric)
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    for k in ("n_gpus", "steps", "warmup", "ms_per_step", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert k in d
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
