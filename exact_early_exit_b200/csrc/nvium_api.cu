@@ -930,7 +930,13 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
   M->rope = (float2*)(P + o_rope);
   launch_rope_table(M->rope, cfg->max_seq, M->hd, (double)cfg->rope_theta, 0);
   M->layer_weight_bytes = (long long)(4 * HQ * d + 3 * F * d) * (long long)esz;
-  M->gemm_kind = M->bf16 ? gemm_default_kind() : GEMM_SIMT;
+  // the tcgen05 engine tiles N by 128 and K by 64: every packed weight of the
+  // model must fit (QKV, O, gate/up, down, the heads, the adapters), and the
+  // fused QKV epilogue wants whole 128-feature tiles of q, k and v; other
+  // bf16 shapes run on the SIMT engine
+  const bool tc_shapes = d % 128 == 0 && HQ % 128 == 0 && (2 * F) % 128 == 0 && F % 64 == 0 &&
+                         V % 128 == 0 && cfg->adapter_hidden % 128 == 0;
+  M->gemm_kind = (M->bf16 && tc_shapes) ? gemm_default_kind() : GEMM_SIMT;
   M->gemm_plans = gemm_plans_create();
   // kernels that need more than 48 KB of dynamic shared memory
   nv_status gs = gemm_prepare(M->gemm_kind, M->bf16);
