@@ -512,9 +512,20 @@ def cpu_baseline(wl, weights_seed, lens, prompts, xseed, prefix=128, n_steps=2):
     for s in range(n_steps):
         dec.step(xseed + s)
     dt = time.perf_counter() - t0
-    return {"value": round(n_steps / dt, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"sequence {b}, first {min(prefix, len(prompts[b]))} prompt tokens prefilled untimed, "
-                      f"{n_steps} decode steps timed (1 token each), float64 numpy"}
+    out = {"value": round(n_steps / dt, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"sequence {b}, first {min(prefix, len(prompts[b]))} prompt tokens prefilled untimed, "
+                     f"{n_steps} decode steps timed (1 token each), float64 numpy"}
+    # the same sample on one host thread (the oracle's matrix products are the
+    # only multi-threaded part)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            dec.step(xseed + n_steps)
+            out["value_1_thread"] = round(1.0 / (time.perf_counter() - t0), 4)
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference_scoring(args, wl, world):

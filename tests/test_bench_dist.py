@@ -84,3 +84,14 @@ def test_reference_arm_prints_the_contract_line(workload, metric):
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_cpu_baseline_reports_all_threads_and_one_thread():
+    """The CPU baseline times the oracle on a bounded sample with the host's
+    BLAS threads and again on one thread."""
+    wl = W.WORKLOADS["T"]
+    lens = W.make_prompt_lengths(wl)
+    prompts = W.make_prompts(wl, lengths=lens)
+    cb = bench.cpu_baseline(wl, weights_seed=0, lens=lens, prompts=prompts, xseed=7, prefix=16, n_steps=2)
+    assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["cores"] >= 1
+    assert cb["value"] > 0 and cb["value_1_thread"] > 0 and "sample" in cb
