@@ -478,6 +478,9 @@ def run_scoring(args):
     if rank == 0:
         print(json.dumps(out))
     model.close()
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------------------
