@@ -498,3 +498,27 @@ def test_adapter_head_input_against_torch():
         np.testing.assert_allclose(ad.head_input(k, h), want, rtol=0, atol=1e-12)
     # the last exit reads its own state, adapters or not
     np.testing.assert_array_equal(ad.head_input(3, h), ad.exit_state(3, h))
+
+
+@pytest.mark.parametrize("pattern", ["random", "all1", "last"])
+def test_layers_of_an_exit_block_keep_equal_cache_lengths(pattern):
+    """Exits happen only after a block's last layer, so at every step the
+    layers between two exits have equal cache lengths and hence run the same
+    rows: the GPU plans each block once.  Checked on a 6-layer model with
+    blocks of two layers, under forced exit patterns, and after the flush."""
+    cfg = W.ModelConfig("blocks-of-two", 6, 64, 2, 32, 172, 256, (2, 4, 6), W.F32)
+    model = O.OracleModel(cfg, W.make_weights(cfg, seed=1))
+    prompts = [W.make_prompts(W.WORKLOADS["T"], seed=s)[0][:n] for s, n in ((1, 5), (2, 11), (3, 1))]
+    dec = O.OracleDecoder(model, prompts, 24)
+    rng = np.random.default_rng(9)
+    blocks = [(0, 2), (2, 4), (4, 6)]
+    for s in range(24):
+        ex = {"random": list(rng.integers(1, 4, size=3)), "all1": [1, 1, 1], "last": [3, 3, 3]}[pattern]
+        dec.step(77 + s, forced_exits=ex)
+        for b in range(3):
+            lens = dec.caches[b].lens
+            for l0, l1 in blocks:
+                assert len(set(lens[l0:l1])) == 1, (s, b, lens)
+    dec.flush()
+    for b in range(3):
+        assert len(set(dec.caches[b].lens)) == 1
