@@ -353,7 +353,7 @@ def run_ours(args):
            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == W.BF16 else "f32",
            "data": "synthetic",
-           "config": {"workload": wl.name, "model": cfg.name, "global_batch": B * world,
+           "config": {"workload": wl.name, "global_batch": B * world,
                       "prompt_len": (f"U[{wl.prompt_len_lo},{wl.prompt_len}]" if wl.prompt_len_lo != wl.prompt_len
                                      else wl.prompt_len),
                       "decode_steps": steps, "parallelism": f"dp{world}" if world > 1 else "single",
@@ -462,7 +462,7 @@ def run_scoring(args):
            "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": wl.name, "model": cfg.name, "global_batch": B * world, "seq_len": S,
+           "config": {"workload": wl.name, "global_batch": B * world, "seq_len": S,
                       "parallelism": f"dp{world}" if world > 1 else "single",
                       "l2": "inputs larger than L2 (weights and activations streamed each step)"},
            "e2e": {"value": round(tokens * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
@@ -550,7 +550,7 @@ def run_reference_scoring(args, wl, world):
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(dt / args.steps * 1e3, 1), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": wl.name, "model": wl.model.name, "global_batch": wl.batch, "seq_len": wl.prompt_len},
+           "config": {"workload": wl.name, "global_batch": wl.batch, "seq_len": wl.prompt_len},
            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -583,7 +583,7 @@ def run_reference(args):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "f64", "data": "synthetic",
-           "config": {"workload": wl.name, "model": wl.model.name, "global_batch": wl.batch,
+           "config": {"workload": wl.name, "global_batch": wl.batch,
                       "decode_steps": wl.steps},
            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                             "sample": sample},

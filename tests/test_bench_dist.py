@@ -81,6 +81,8 @@ def test_reference_arm_prints_the_contract_line(workload, metric):
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     for k in ("n_gpus", "steps", "warmup", "ms_per_step", "scaling", "vs_baseline", "dtype", "data", "config"):
         assert k in d
+    # the config names the workload, without model keys
+    assert d["config"]["workload"] and "model" not in d["config"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
