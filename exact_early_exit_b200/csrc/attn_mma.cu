@@ -32,14 +32,12 @@
 namespace nv {
 namespace {
 
-constexpr int CK = ATTN_DEC_CK;  // keys per CTA
 constexpr int HD = 64;           // head dim (128-byte rows)
 constexpr int RG = 16;           // rows per MMA pass
 constexpr int QLD = HD + 8;      // padded Q row: 144 bytes, conflict-free ldmatrix
 constexpr int OLD = HD + 2;      // per-warp partial row: HD sums, max, weight sum
 constexpr int BOX = 64;          // positions per TMA box (a page holds 64 or 128)
 constexpr int BOX_BYTES = BOX * HD * 2;
-
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(const_cast<void*>(p));

@@ -96,9 +96,11 @@ struct AttnArgs {
   int* dec_ctr;               // [B][H] split arrival counters (zero between launches)
 };
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
-// Decode / flush attention: 128-key chunks (grid z = kv_splits = chunks of
-// max_seq), TMA bulk loads of K/V pages, partials merged per row.  Needs
-// head_dim * element size == 128 bytes and page_size == 64.
+// Decode / flush attention.  bf16 with head_dim 64 and a KV tensor map: the
+// warp-MMA kernel below (a.dec_splits key-range splits).  Otherwise the SIMT
+// kernel: 128-key chunks (grid z = kv_splits = chunks of max_seq), TMA bulk
+// loads of K/V pages, partials merged per row by a combine kernel.  Both
+// need head_dim * element size == 128 bytes and page_size a multiple of 64.
 constexpr int ATTN_DEC_CK = 128;
 void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st);
 // kernels launch_attention_decode runs for these arguments (1 or 2)
