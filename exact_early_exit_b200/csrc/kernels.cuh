@@ -100,7 +100,7 @@ void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
 // warp-MMA kernel below (a.dec_splits key-range splits).  Otherwise the SIMT
 // kernel: 128-key chunks (grid z = kv_splits = chunks of max_seq), TMA bulk
 // loads of K/V pages, partials merged per row by a combine kernel.  Both
-// need head_dim * element size == 128 bytes and page_size a multiple of 64.
+// need head_dim * element size == 128 bytes and page_size 64 or 128.
 constexpr int ATTN_DEC_CK = 128;
 void launch_attention_decode(bool bf16, const AttnArgs& a, cudaStream_t st);
 // kernels launch_attention_decode runs for these arguments (1 or 2)
