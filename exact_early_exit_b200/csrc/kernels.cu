@@ -295,8 +295,10 @@ void launch_resid_norm(bool bf16, RowSet rs, const float* Y, int split_grid, int
 // reading): when b's new token is still active at m, its deferred positions
 // [len[b][m], t_b) followed by the new position t_b; when the sequence must
 // complete early (its deferred store is full) the deferred positions alone;
-// in flush mode every deferred position [len[b][m], t_b).  Every CTA computes
-// the same prefix sums in shared memory; CTA 0 publishes the list.
+// in flush mode every deferred position [len[b][m], t_b).  The layers between
+// two exits keep equal cache lengths, so a plan made at a block's first layer
+// serves the whole block (counters count it for a.nlayers layers).  Every CTA
+// computes the same prefix sums in shared memory; CTA 0 publishes the list.
 // ---------------------------------------------------------------------------
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT) k_plan_norm(PlanArgs a, const T* __restrict__ gain, T* __restrict__ act,
@@ -692,9 +694,9 @@ __global__ void k_attn_combine(AttnArgs a) {
 
 // ---------------------------------------------------------------------------
 // Decode attention, SIMT (the fp32 model's and the comparison path; bf16
-// models with head_dim 64 use k_attn_dec_mma): CTA (b, head, chunk) handles keys [chunk*128, chunk*128 +
-// 128) of sequence b at this layer for every row of b whose position reaches
-// the chunk.  One thread issues TMA bulk copies of the chunk's K and V pages
+// models with head_dim 64 use k_attn_dec_mma): CTA (b, head, chunk) handles
+// keys [chunk*128, chunk*128 + 128) of sequence b at this layer for every row
+// of b whose position reaches the chunk.  One thread issues TMA bulk copies of the chunk's K and V pages
 // (each page of one head is contiguous), completing on an mbarrier, so the
 // whole 2 x 16 KB chunk is in flight at once.  Scores: one lane per key,
 // 16-byte reads of the key row in a per-lane rotated order (conflict-free);
