@@ -522,3 +522,20 @@ def test_layers_of_an_exit_block_keep_equal_cache_lengths(pattern):
     dec.flush()
     for b in range(3):
         assert len(set(dec.caches[b].lens)) == 1
+
+
+def test_router_bias_calibration_hits_the_target_stop_rates():
+    """The calibrated biases make E[sigmoid(b_k + eps)], eps ~ N(0, 0.02^2 d),
+    the conditional stop rate of each junction (target exit mass
+    0.4/0.25/0.2/0.15): checked by Monte Carlo, not by the quadrature used to
+    solve for them, and the implied exit masses multiply back to the target."""
+    d = 1536
+    b = W.calibrate_router_biases(d)
+    eps = np.random.default_rng(0).normal(0.0, 0.02 * np.sqrt(d), size=2_000_000)
+    c = [float(np.mean(1.0 / (1.0 + np.exp(-(bk + eps))))) for bk in b]
+    mass, left = [], 1.0
+    for ck in c:
+        mass.append(left * ck)
+        left *= 1.0 - ck
+    mass.append(left)
+    np.testing.assert_allclose(mass, W.TARGET_EXIT_MASS, rtol=0, atol=2e-3)
