@@ -277,6 +277,48 @@ def test_deferred_kv_equals_full_depth(pattern):
             np.testing.assert_allclose(dec.caches[b].V[m][:t], full.V[m][:t], rtol=1e-10, atol=1e-13)
 
 
+@pytest.mark.parametrize("pattern", ["routed", "all1"])
+def test_early_completion_changes_nothing(pattern):
+    """Reading r7: completing a sequence's deferred rows before the lazy rule
+    would run them (what the GPU does when a sequence's deferred store is
+    full) changes no value.  A decoder that flushes part-way takes the same
+    exits and tokens with the same log-probabilities and junction draws as
+    the lazy one, and both end with the same caches."""
+    cfg = W.TINY
+    model, _ = tiny_model()
+    prompts = [W.make_prompts(W.WORKLOADS["T"])[0][:9], W.make_prompts(W.WORKLOADS["T"], seed=7)[0][:14]]
+    steps = 16
+    lazy = O.OracleDecoder(model, prompts, steps)
+    eager = O.OracleDecoder(model, prompts, steps)
+    completed = 0
+    for s in range(steps):
+        ex = [1, 1] if pattern == "all1" else None
+        if s in (4, 9):
+            completed += sum(eager.deferred_rows(b) for b in range(2))
+            eager.flush()
+        ra = lazy.step(1234, forced_exits=ex)
+        rb = eager.step(1234, forced_exits=ex)
+        for a, b in zip(ra, rb):
+            assert (a.exit, a.token) == (b.exit, b.token)
+            np.testing.assert_allclose(b.logp, a.logp, rtol=1e-10, atol=1e-12)
+            assert len(a.junctions) == len(b.junctions)
+            for (ka, ua, wa), (kb, ub, wb) in zip(a.junctions, b.junctions):
+                assert (ka, ua) == (kb, ub)
+                np.testing.assert_allclose(wb, wa, rtol=1e-10)
+    assert completed > 0, "nothing was deferred when the early completion ran"
+    lazy.flush()
+    eager.flush()
+    for b in range(2):
+        t = lazy.t[b]
+        assert eager.t[b] == t and lazy.caches[b].lens == eager.caches[b].lens == [t] * cfg.n_layers
+        # both against an undeferred full-depth forward of the same tokens
+        _, _, full = model.forward_sequence(lazy.tokens[b][:t])
+        for m in range(cfg.n_layers):
+            for dec in (lazy, eager):
+                np.testing.assert_allclose(dec.caches[b].K[m][:t], full.K[m][:t], rtol=1e-10, atol=1e-13)
+                np.testing.assert_allclose(dec.caches[b].V[m][:t], full.V[m][:t], rtol=1e-10, atol=1e-13)
+
+
 def test_decode_step_law_matches_full_depth_states():
     """The h a new token reaches each junction with, under deferral, is the
     full-depth forward's h: the step's (u, w) and scores use it."""
