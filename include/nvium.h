@@ -308,6 +308,10 @@ nv_status nv_score_mixture_profiled(nv_model *m, const int32_t *tokens, int B,
 /* Synchronise the state's work and return any device-detected error. */
 nv_status nv_sync_status(nv_state *s);
 
+/* The calling thread's most recent error message (thread-local): every failing
+ * call records one, except a null-handle rejection, which only returns
+ * NV_ERR_INVALID_ARG.  The pointer stays valid until that thread records the
+ * next message; never NULL. */
 const char *nv_last_error(void);
 
 #ifdef __cplusplus

@@ -77,3 +77,27 @@ def test_null_handles_are_rejected():
     assert L.nv_decode_step(None, 1, None, None, None, None) == nv.NV_ERR_INVALID_ARG
     assert L.nv_score_mixture(None, None, 1, 2, None, None, None) == nv.NV_ERR_INVALID_ARG
     assert L.nv_philox4x32_10(1, None, 4, None, None) == nv.NV_ERR_INVALID_ARG
+
+
+def test_last_error_is_per_thread():
+    """nv_last_error is thread-local: another thread's failing call does not
+    replace this thread's message."""
+    import threading
+    L = nv.lib()
+    h = ctypes.c_void_p()
+    assert L.nv_create(ctypes.byref(_cfg(n_layers=0)), ctypes.byref(nv.Weights()), ctypes.byref(h)) == \
+        nv.NV_ERR_INVALID_ARG
+    mine = L.nv_last_error()
+    other = []
+
+    def fail_elsewhere():
+        c = _cfg()
+        c.exit_layers[1] = 1
+        L.nv_create(ctypes.byref(c), ctypes.byref(nv.Weights()), ctypes.byref(ctypes.c_void_p()))
+        other.append(L.nv_last_error())
+
+    t = threading.Thread(target=fail_elsewhere)
+    t.start()
+    t.join()
+    assert other and other[0] != mine
+    assert L.nv_last_error() == mine
