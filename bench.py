@@ -197,22 +197,22 @@ def workload_for(args):
 # ---------------------------------------------------------------------------
 # the CUDA arm
 # ---------------------------------------------------------------------------
-def run_ours(args):
+def measure_decode(args, wl, n_steps, n_warmup, dev, rank, world, weights=None, want_cpu=False):
+    """Decode passes of workload `wl` (the bench step: rewind + decode_steps
+    decode steps + flush), e2e through the C ABI from host buffers, the same
+    kernels forced to full depth, and the per-kernel profiled pass; returns
+    the measurement dict (the JSON line's keys)."""
     import torch
 
     import exact_early_exit_b200 as nv
 
-    rank, world = dist_init("nccl")
-    _, _, local = rank_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    wl = workload_for(args)
     cfg = wl.model
     pseed, lseed, xseed = rank_seeds(rank)
     lens = W.make_prompt_lengths(wl, seed=lseed)
     prompts = W.make_prompts(wl, seed=pseed, lengths=lens)
     B, steps = wl.batch, wl.steps
-    weights = W.make_weights(cfg, seed=0)
+    if weights is None:
+        weights = W.make_weights(cfg, seed=0)
     max_seq = int(lens.max()) + steps + 64
     model = nv.Model(cfg, weights, max_batch=B, max_seq=max_seq, max_pending=256)
     st = nv.State(model, B)
@@ -229,17 +229,17 @@ def run_ours(args):
             st.decode_step(seed + s, tok_d, ex_d)
         st.flush()
 
-    for i in range(args.warmup):
+    for i in range(n_warmup):
         gen_pass(xseed + 100000 * (i + 1))
     torch.cuda.synchronize()
     st.sync_status()
     st.reset_counters()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
-        for i in range(args.steps):
+        for i in range(n_steps):
             gen_pass(xseed)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -248,15 +248,15 @@ def run_ours(args):
     st.sync_status()
     ctr = st.counters()
     ms_max = max_over_ranks(ms_total, dev)
-    ms_per_step = ms_max / args.steps
+    ms_per_step = ms_max / n_steps
     tokens_per_step = B * steps
-    value = tokens_per_step * world * args.steps / (ms_max / 1e3)
+    value = tokens_per_step * world * n_steps / (ms_max / 1e3)
     launches = int(ctr[nv.CTR["launches"]])
 
     # algorithmic bytes of one pass (weights per layer run, K/V attended and
     # written, exit heads), from the device counters of the timed passes
     pass_bytes = float(ctr[nv.CTR["weight_bytes"]] + ctr[nv.CTR["kv_read_bytes"]] +
-                       ctr[nv.CTR["kv_write_bytes"]] + ctr[nv.CTR["head_bytes"]]) / args.steps
+                       ctr[nv.CTR["kv_write_bytes"]] + ctr[nv.CTR["head_bytes"]]) / n_steps
     exits = ctr[nv.CTR["exit0"]:nv.CTR["exit0"] + cfg.n_exits].astype(float)
     exit_mass = (exits / max(exits.sum(), 1)).round(4).tolist()
 
@@ -268,7 +268,7 @@ def run_ours(args):
     e2 = torch.cuda.Event(enable_timing=True)
     e3 = torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    for i in range(args.steps):
+    for i in range(n_steps):
         st.prefill(tok_host, lens)
         for s in range(steps):
             st.decode_step(xseed + s, tok_h, ex_h)
@@ -277,7 +277,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e2.elapsed_time(e3), dev)
-    e2e_value = tokens_per_step * world * args.steps / (e2e_ms / 1e3)
+    e2e_value = tokens_per_step * world * n_steps / (e2e_ms / 1e3)
 
     # prefill and the final flush on their own (decode tokens/s excludes the
     # prefill; the flush is owed work and sits inside every timed pass)
@@ -300,7 +300,6 @@ def run_ours(args):
     # exit): the dense-decode comparison of the same workload
     fmodel = nv.Model(cfg, weights, max_batch=B, max_seq=max_seq, max_pending=256,
                       router_mode=nv.NV_ROUTER_FORCE_LAST)
-    del weights
     fst = nv.State(fmodel, B)
     fst.prefill(tok_host, lens)
 
@@ -310,17 +309,17 @@ def run_ours(args):
             fst.decode_step(seed + s, tok_d, ex_d)
         fst.flush()
 
-    for i in range(args.warmup):
+    for i in range(n_warmup):
         full_pass(xseed + 100000 * (i + 1))
     torch.cuda.synchronize()
     barrier()
     ea.record(stream)
-    for i in range(args.steps):
+    for i in range(n_steps):
         full_pass(xseed)
     eb.record(stream)
     torch.cuda.synchronize()
     barrier()
-    full_ms = max_over_ranks(ea.elapsed_time(eb), dev) / args.steps
+    full_ms = max_over_ranks(ea.elapsed_time(eb), dev) / n_steps
     fst.sync_status()
     fst.close()
     fmodel.close()
@@ -349,8 +348,8 @@ def run_ours(args):
                 "step_algorithmic_GBps": round(pass_bytes / (ms_per_step / 1e3) / 1e9, 1),
                 "step_frac": round(pass_bytes / (ms_per_step / 1e3) / 1e9 / peak, 4)}
 
-    out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": n_steps,
+           "warmup": n_warmup, "ms_per_step": round(ms_per_step, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == W.BF16 else "f32",
            "data": "synthetic",
            "config": {"workload": wl.name, "global_batch": B * world,
@@ -370,13 +369,50 @@ def run_ours(args):
                           "what": "same workload and kernels, router forced to the last exit"},
            "prefill_ms": round(prefill_ms, 3),
            "flush_ms": round(flush_ms, 3)}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, weights_seed=0, lens=lens, prompts=prompts, xseed=xseed)
+    if want_cpu:
+        out["cpu_baseline"] = cpu_baseline(wl, lens=lens, prompts=prompts, xseed=xseed)
     out["clocks"] = clk.summary()
-    if rank == 0:
-        print(json.dumps(out))
     st.close()
     model.close()
+    return out
+
+
+SUB_KEYS = ("value", "unit", "steps", "warmup", "ms_per_step", "config", "e2e", "gpu_launches", "roofline",
+            "realised_exit_mass", "full_depth", "prefill_ms", "flush_ms", "mean_nll", "mean_expected_depth",
+            "clocks")
+
+
+def sub_line(d: dict, metric: str) -> dict:
+    """A second workload's measurement nested inside the headline line."""
+    out = {"metric": metric}
+    out.update({k: d[k] for k in SUB_KEYS if k in d})
+    return out
+
+
+def run_ours(args):
+    """The decode workload's JSON line; with the default workload (B=64) on
+    one GPU it also carries the B=1 decode (`b1`) and the 16 x 2048 scoring
+    (`scoring`) measurements, each with its own roofline and e2e."""
+    import torch
+
+    rank, world = dist_init("nccl")
+    _, _, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = workload_for(args)
+    weights = W.make_weights(wl.model, seed=0)
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    out = measure_decode(args, wl, args.steps, args.warmup, dev, rank, world, weights=weights, want_cpu=want_cpu)
+    if args.workload == "X64" and not args.layers and not args.decode_steps and not args.headline_only:
+        # the other two configurations of the metric, with fewer timed passes
+        sub_steps = max(3, min(args.steps, 5))
+        b1 = measure_decode(args, W.WORKLOADS["X1"], sub_steps, 3, dev, rank, world, weights=weights)
+        out["b1"] = sub_line(b1, METRIC)
+        del weights
+        sc = measure_scoring(W.WORKLOADS["XS"], sub_steps, 3, dev, rank, world)
+        out["scoring"] = sub_line(sc, SCORE_METRIC)
+    if rank == 0:
+        print(json.dumps(out))
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()
@@ -391,18 +427,14 @@ def measured_tensor_peak():
         return 1400.0, "fallback sustained"
 
 
-def run_scoring(args):
+def measure_scoring(wl, n_steps, n_warmup, dev, rank, world):
     """Mixture scoring of 16 x 2048 tokens (log pi_mix at every position and
-    the mean NLL): one nv_score_mixture call per step."""
+    the mean NLL): one nv_score_mixture call per step; returns the
+    measurement dict."""
     import torch
 
     import exact_early_exit_b200 as nv
 
-    rank, world = dist_init("nccl")
-    _, _, local = rank_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    wl = workload_for(args)
     cfg = wl.model
     pseed, _, _ = rank_seeds(rank)
     toks = np.stack(W.make_prompts(wl, seed=pseed)).astype(np.int32)
@@ -414,20 +446,20 @@ def run_scoring(args):
     logp_d = torch.zeros((B, S - 1), dtype=torch.float32, device=dev)
     nll_d = torch.zeros(1, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    for _ in range(args.warmup):
+    for _ in range(n_warmup):
         model.score_mixture(tok_d, logp_d, nll_d)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(n_steps):
             model.score_mixture(tok_d, logp_d, nll_d)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    ms = max_over_ranks(e0.elapsed_time(e1), dev) / n_steps
     tokens = B * (S - 1)
     value = tokens * world / (ms / 1e3)
     # e2e: host tokens in, host log-probs out
@@ -437,11 +469,11 @@ def run_scoring(args):
     torch.cuda.synchronize()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    for _ in range(args.steps):
+    for _ in range(n_steps):
         model.score_mixture(tok_h, logp_h, nll_h)
     e3.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e2.elapsed_time(e3), dev) / args.steps
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3), dev) / n_steps
     # the compute-penalty forward on the same batch (untimed): mean expected
     # normalised layer depth
     depth_d = torch.zeros_like(logp_d)
@@ -459,15 +491,15 @@ def run_scoring(args):
     achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
     peak, src = measured_tensor_peak()
     out = {"metric": SCORE_METRIC,
-           "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+           "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": n_steps,
+           "warmup": n_warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
            "config": {"workload": wl.name, "global_batch": B * world, "seq_len": S,
                       "parallelism": f"dp{world}" if world > 1 else "single",
                       "l2": "inputs larger than L2 (weights and activations streamed each step)"},
            "e2e": {"value": round(tokens * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                    "h2d_bytes_per_step": int(toks.nbytes), "d2h_bytes_per_step": int(B * (S - 1) * 4 + 4)},
-           "gpu_launches": sum(v["kernels"] for v in kern.values()) * args.steps,
+           "gpu_launches": sum(v["kernels"] for v in kern.values()) * n_steps,
            "roofline": {"bound": "tensor", "kernel": "gemm (layers + exit heads)", "achieved": round(achieved, 1),
                         "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
                         "peak_source": src, "kernel_share": {k: round(v["ms"] / total_k, 4) for k, v in kern.items()},
@@ -475,9 +507,20 @@ def run_scoring(args):
            "mean_nll": float(nll_d.item()),
            "mean_expected_depth": round(mean_depth, 5)}
     out["clocks"] = clk.summary()
+    model.close()
+    return out
+
+
+def run_scoring(args):
+    import torch
+
+    rank, world = dist_init("nccl")
+    _, _, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    out = measure_scoring(workload_for(args), args.steps, args.warmup, dev, rank, world)
     if rank == 0:
         print(json.dumps(out))
-    model.close()
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()
@@ -495,29 +538,32 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_setup(wl, lens, prompts, prefix):
+def oracle_setup(wl, lens, prompts, max_new=64):
+    """The oracle decoder on one sequence of the workload: the batch's
+    shortest prompt (all of it), prefilled at full depth (untimed)."""
     from oracle import nvium_oracle as O
     weights = W.make_weights(wl.model, seed=0)
     om = O.OracleModel(wl.model, weights)
     b = int(np.argmin(lens))
-    p = prompts[b][:prefix]
-    dec = O.OracleDecoder(om, [p], 64)
+    dec = O.OracleDecoder(om, [prompts[b]], max_new)
     dec.ids = [b]
     return dec, b
 
 
-def cpu_baseline(wl, weights_seed, lens, prompts, xseed, prefix=128, n_steps=2):
-    """The oracle on a bounded sample: one sequence (the batch's shortest
-    prompt, first `prefix` tokens prefilled untimed), `n_steps` decode steps
-    timed; tokens/s of that sample."""
-    dec, b = oracle_setup(wl, lens, prompts, prefix)
+def cpu_baseline(wl, lens, prompts, xseed, n_steps=16):
+    """The oracle on a bounded sample of the workload: one of its sequences
+    (the shortest prompt, prefilled in full, untimed), the first `n_steps`
+    decode steps of that sequence timed with the workload's Philox seeds;
+    tokens/s of that sample (the oracle's per-token rate, extrapolated to the
+    workload)."""
+    dec, b = oracle_setup(wl, lens, prompts)
     t0 = time.perf_counter()
     for s in range(n_steps):
         dec.step(xseed + s)
     dt = time.perf_counter() - t0
     out = {"value": round(n_steps / dt, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-           "sample": f"sequence {b}, first {min(prefix, len(prompts[b]))} prompt tokens prefilled untimed, "
-                     f"{n_steps} decode steps timed (1 token each), float64 numpy"}
+           "sample": f"sequence {b} of the workload ({len(prompts[b])}-token prompt prefilled untimed), its first "
+                     f"{n_steps} decode steps timed (1 token each), float64 numpy; tokens/s extrapolated per token"}
     # the same sample on one host thread (the oracle's matrix products are the
     # only multi-threaded part)
     try:
@@ -568,17 +614,18 @@ def run_reference(args):
     pseed, lseed, xseed = rank_seeds(0)
     lens = W.make_prompt_lengths(wl, seed=lseed)
     prompts = W.make_prompts(wl, seed=pseed, lengths=lens)
-    dec, b = oracle_setup(wl, lens, prompts, 128)
+    dec, b = oracle_setup(wl, lens, prompts, max_new=args.warmup + args.steps + 1)
+    # warm-up steps are the sequence's first decode steps; the timed steps follow them
     for i in range(args.warmup):
-        dec.step(xseed + 1000 + i)
+        dec.step(xseed + i)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        dec.step(xseed + i)
+        dec.step(xseed + args.warmup + i)
     dt = time.perf_counter() - t0
     value = args.steps / dt
     cores = blas_threads()
-    sample = (f"sequence {b}, first 128 prompt tokens prefilled untimed; each step = 1 decode step of that "
-              f"sequence (1 token), float64 numpy oracle")
+    sample = (f"sequence {b} of the workload ({len(prompts[b])}-token prompt prefilled untimed); each step = 1 "
+              f"decode step of that sequence (1 token), float64 numpy oracle; tokens/s extrapolated per token")
     out = {"metric": METRIC, "impl": "reference", "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -599,6 +646,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["X64", "X1", "XS", "S", "T"], default="X64")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="default workload: skip the nested B=1 and scoring measurements")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: the workload's model with this many layers (exits spread evenly)")
     ap.add_argument("--decode-steps", type=int, default=0, help="profiling only: decode steps per pass")

@@ -91,6 +91,7 @@ _SIGS = [
     ("nv_decode_step", _I, [_P, ctypes.c_uint64, _P, _P, _P, _P]),
     ("nv_flush_deferred", _I, [_P, _P]),
     ("nv_read_kv", _I, [_P, _I, _I, _P, _P, ctypes.POINTER(_I), _P]),
+    ("nv_read_router_probs", _I, [_P, _P, _P]),
     ("nv_read_counters", _I, [_P, _P, _I]),
     ("nv_reset_counters", _I, [_P]),
     ("nv_sync_status", _I, [_P]),
@@ -296,6 +297,16 @@ class State:
         n = ctypes.c_int()
         _check(lib().nv_read_kv(self.handle, b, layer, _ptr(K), _ptr(V), ctypes.byref(n), _stream(None)))
         return K[: n.value], V[: n.value], n.value
+
+    def router_probs(self) -> np.ndarray:
+        """[n_exits - 1, B] float32: the w_k each sequence's token was compared
+        against at junction k in the last decode step (NaN where the token
+        stopped earlier)."""
+        c = self.model.cfg
+        out = np.zeros((c.n_exits - 1, self.B), dtype=np.float32)
+        if out.size:
+            _check(lib().nv_read_router_probs(self.handle, _ptr(out), _stream(None)))
+        return out
 
     def counters(self) -> np.ndarray:
         out = np.zeros(NV_CTR_COUNT, dtype=np.int64)

@@ -975,7 +975,10 @@ __global__ void k_step_begin(StepArgs a) {
     const int f = (pending + 1 >= a.cap) ? 1 : 0;
     a.force[b] = f;
     if (f && a.counters) atomicAdd((unsigned long long*)&a.counters[NV_CTR_FORCED], 1ull);
-    for (int k = 0; k < a.n_exits; ++k) a.stop[k * a.B + b] = 0;
+    for (int k = 0; k < a.n_exits; ++k) {
+      a.stop[k * a.B + b] = 0;
+      a.router_p[k * a.B + b] = CUDART_NAN_F;
+    }
     if (b == 0) {
       *a.seed_dev = a.seed;
       for (int k = 0; k < a.n_exits; ++k) a.nstop[k] = 0;
@@ -1067,6 +1070,7 @@ __global__ void __launch_bounds__(256) k_junction(JuncArgs a) {
     bool stop = true;
     if (!last) {
       const float w = (a.router_mode == NV_ROUTER_FORCE_LAST) ? 0.f : 1.0f / (1.0f + expf(-(z + a.router_b)));
+      a.router_p[b] = w;
       const unsigned long long seed = *a.seed;
       const uint4 r = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)tb, STREAM_EXIT, (uint32_t)(a.k / 4)),
                                     (uint32_t)seed, (uint32_t)(seed >> 32));

@@ -124,6 +124,7 @@ struct StepArgs {
   int* force;
   int* stop;             // [n_exits][B]
   int* nstop;            // [n_exits]
+  float* router_p;       // [n_exits][B] w_k of this step (NaN: junction not reached)
   const int* lens;
   float* hbuf;
   const void* emb;
@@ -145,6 +146,7 @@ struct JuncArgs {
   int* active;
   int* exit_id;
   int* stop;             // [B] flags of this exit
+  float* router_p;       // [B] w_k of this exit's junction, per sequence
   const float* hbuf;
   const void* norm;
   const void* router_w;

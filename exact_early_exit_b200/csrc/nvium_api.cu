@@ -115,6 +115,8 @@ struct nv_state {
   bool tc_head = false;  // exit heads on tensor cores (bf16, B >= 16)
   int *prompt_len = nullptr, *prompt_last = nullptr;
   float* logp = nullptr;
+  float* router_p = nullptr;  // [NV_MAX_EXITS][B] router probabilities of the last step
+  bool stepped = false;       // a decode step has run since nv_prefill
   float* hbuf = nullptr;
   // work list and activations
   int *row_b = nullptr, *row_pos = nullptr, *row_hrow = nullptr, *seq_start = nullptr, *nrows = nullptr;
@@ -483,6 +485,7 @@ nv_status record_layers(nv_state* s, cudaStream_t st, Prof* prof, long long* lau
     j.active = s->active;
     j.exit_id = s->exit_id;
     j.stop = s->stop + (size_t)k * s->B;
+    j.router_p = s->router_p + (size_t)k * s->B;
     j.hbuf = s->hbuf;
     j.norm = M->exits[k].norm;
     j.router_w = M->exits[k].router_w;
@@ -1030,6 +1033,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   A((void**)&s->d_B, 4);
   A((void**)&s->d_block_launches, NV_MAX_EXITS * 4);
   A((void**)&s->logp, (size_t)B * 4);
+  A((void**)&s->router_p, (size_t)NV_MAX_EXITS * B * 4);
   A((void**)&s->hbuf, (size_t)B * s->cap * d * 4);
   for (int** p : {&s->row_b, &s->row_pos, &s->row_hrow}) A((void**)p, (size_t)s->max_rows * 4);
   A((void**)&s->seq_start, (size_t)(B + 1) * 4);
@@ -1235,6 +1239,7 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
   s->h_prompt_len.assign(lens, lens + B);
   s->h_t = t0;
   s->prefilled = true;
+  s->stepped = false;
   return check_status(s);
 }
 
@@ -1257,6 +1262,7 @@ nv_status nv_rewind(nv_state* s, void* stream) {
   NV_CUDA_TRY(cudaMemcpyAsync(s->lens, ln.data(), ln.size() * 4, cudaMemcpyHostToDevice, st));
   NV_CUDA_TRY(cudaStreamSynchronize(st));
   s->h_t = t0;
+  s->stepped = false;
   return NV_OK;
 }
 
@@ -1297,6 +1303,7 @@ nv_status decode_step_impl(nv_state* s, uint64_t seed, int32_t* tokens_out, int3
   sa.force = s->force;
   sa.stop = s->stop;
   sa.nstop = s->nstop;
+  sa.router_p = s->router_p;
   sa.lens = s->lens;
   sa.hbuf = s->hbuf;
   sa.emb = M->tok_emb;
@@ -1345,6 +1352,7 @@ nv_status decode_step_impl(nv_state* s, uint64_t seed, int32_t* tokens_out, int3
   NV_CUDA_TRY(cudaMemcpyAsync(exits_out, s->out_exit, s->B * 4, cudaMemcpyDefault, st));
   if (logp_out) NV_CUDA_TRY(cudaMemcpyAsync(logp_out, s->logp, s->B * 4, cudaMemcpyDefault, st));
   for (int b = 0; b < s->B; ++b) s->h_t[b] += 1;
+  s->stepped = true;
   return NV_OK;
 }
 }  // namespace
@@ -1437,6 +1445,23 @@ nv_status nv_read_kv(nv_state* s, int b, int layer, void* k_out, void* v_out, in
         NV_CUDA_TRY(cudaMemcpy2DAsync(dst, (size_t)M->H * row, src, row, row, n, cudaMemcpyDefault, st));
       }
   }
+  NV_CUDA_TRY(cudaStreamSynchronize(st));
+  return NV_OK;
+}
+
+nv_status nv_read_router_probs(nv_state* s, float* w_out, void* stream) {
+  if (!s || !w_out) {
+    set_error("null argument");
+    return NV_ERR_INVALID_ARG;
+  }
+  if (!s->stepped) {
+    set_error("nv_read_router_probs before the first decode step");
+    return NV_ERR_STATE;
+  }
+  const int n = (s->m->NE - 1) * s->B;
+  if (n == 0) return NV_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  NV_CUDA_TRY(cudaMemcpyAsync(w_out, s->router_p, (size_t)n * 4, cudaMemcpyDeviceToHost, st));
   NV_CUDA_TRY(cudaStreamSynchronize(st));
   return NV_OK;
 }

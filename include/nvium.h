@@ -204,6 +204,16 @@ nv_status nv_flush_deferred(nv_state *s, void *stream);
 nv_status nv_read_kv(nv_state *s, int b, int layer, void *k_out, void *v_out,
                      int *len_out, void *stream);
 
+/* Test hook: the router probabilities of the last decode step (section 2
+ * "Architektur": w_k of exit k's router).  w_out (host, (n_exits-1) x B
+ * float, exit-major): w_out[(k-1)*B + b] = the w_k that sequence b's token
+ * compared its uniform u_k against at junction k, as the kernel computed it
+ * (0 under NV_ROUTER_FORCE_LAST), or NaN when that token stopped before
+ * junction k.  Lets a caller check every stop decision against the device's
+ * own w_k (stop iff u_k < w_k) and measure |w_k - w_k(reference)|.
+ * Returns NV_ERR_STATE before the first decode step.  Synchronous. */
+nv_status nv_read_router_probs(nv_state *s, float *w_out, void *stream);
+
 /* Per-state counters, int64, accumulated since nv_state_create or the last
  * nv_reset_counters (synchronous).  Indices: see NV_CTR_*. */
 enum {
@@ -247,7 +257,10 @@ nv_status nv_philox4x32_10(uint64_t seed, const uint32_t *ctr, int n,
  * ctr, out: n x 4 uint32 (host or device); 1 <= n <= NV_PHILOX_NOALLOC_MAX,
  * larger n returns NV_ERR_INVALID_ARG with a message.  The first call on a
  * device looks up the array's device address once, with that device
- * current; make that first call before any stream capture.  All calls share
+ * current, and keeps it for the life of the process; make that first call
+ * before any stream capture.  A cudaDeviceReset (or any reset of the primary
+ * context) unloads the array, so the kept address is no longer valid: do
+ * not call this entry point on that device again after such a reset.  All calls share
  * the array and it keeps the last call's contents, so calls that overlap on
  * the GPU (other streams, other host threads) race; serialise them.
  * Synchronous. */

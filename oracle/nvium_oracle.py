@@ -167,6 +167,42 @@ def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
+def attention_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, p: int, scale: float) -> np.ndarray:
+    """Causal softmax attention of one row at position p (LLaMA-2): q [H, hd]
+    against the cached keys and values of positions 0..p (K, V [>= p+1, H, hd]);
+    o_h = sum_j softmax_j(q_h . k_jh * scale) v_jh.  Returns [H, hd]."""
+    Kc, Vc = K[: p + 1], V[: p + 1]
+    s = np.einsum("hd,jhd->hj", q, Kc) * scale
+    s = s - s.max(axis=1, keepdims=True)
+    e = np.exp(s)
+    a = e / e.sum(axis=1, keepdims=True)
+    return np.einsum("hj,jhd->hd", a, Vc)
+
+
+def causal_attention_rows(q: np.ndarray, K: np.ndarray, V: np.ndarray, pos: np.ndarray, scale: float,
+                          rows_per_block: int = 256) -> np.ndarray:
+    """attention_row for many rows of one sequence at once: q [n, H, hd],
+    positions pos [n]; row i attends to positions 0..pos[i].  The same
+    definition, evaluated as one score matrix per block of rows with the keys
+    beyond each row's position masked out (they get weight exactly 0).
+    Returns [n, H, hd]."""
+    pos = np.asarray(pos, dtype=np.int64)
+    n = q.shape[0]
+    out = np.empty_like(q)
+    for r0 in range(0, n, rows_per_block):
+        r1 = min(n, r0 + rows_per_block)
+        P = int(pos[r0:r1].max()) + 1
+        qh = q[r0:r1].transpose(1, 0, 2)                       # [H, m, hd]
+        s = np.matmul(qh, K[:P].transpose(1, 2, 0)) * scale     # [H, m, P]
+        beyond = np.arange(P)[None, :] > pos[r0:r1, None]       # [m, P]
+        s = np.where(beyond[None], -np.inf, s)
+        s = s - s.max(axis=2, keepdims=True)
+        e = np.exp(s)
+        a = e / e.sum(axis=2, keepdims=True)
+        out[r0:r1] = np.matmul(a, V[:P].transpose(1, 0, 2)).transpose(1, 0, 2)
+    return out
+
+
 def log_sigmoid(z):
     """log sigma(z) = -softplus(-z), computed stably."""
     z = np.asarray(z, dtype=np.float64)
@@ -279,6 +315,9 @@ class OracleModel:
             self.exits.append(e)
         self.adapters = bool(getattr(cfg, "adapter_hidden", 0))
         self.exit_at = {l: k for k, l in enumerate(cfg.exit_layers)}  # layer -> exit index (0-based)
+        # rows of one sequence attend through one masked product per block of
+        # rows (causal_attention_rows); False: one row at a time (attention_row)
+        self.block_attention = True
 
     # rounding point of the bf16 numerics contract
     def rnd(self, x):
@@ -325,16 +364,14 @@ class OracleModel:
         for i in range(n):
             caches[i].K[m][pos[i]] = k[i]
             caches[i].V[m][pos[i]] = v[i]
-        o = np.empty((n, H, hd))
         scale = 1.0 / math.sqrt(hd)
-        for i in range(n):
-            p = int(pos[i])
-            Kc, Vc = caches[i].K[m][: p + 1], caches[i].V[m][: p + 1]          # [p+1, H, hd]
-            s = np.einsum("hd,jhd->hj", q[i], Kc) * scale
-            s = s - s.max(axis=1, keepdims=True)
-            e = np.exp(s)
-            a = e / e.sum(axis=1, keepdims=True)
-            o[i] = np.einsum("hj,jhd->hd", a, Vc)
+        one_seq = n > 1 and all(c is caches[0] for c in caches)
+        if one_seq and self.block_attention:
+            o = causal_attention_rows(q, caches[0].K[m], caches[0].V[m], pos, scale)
+        else:
+            o = np.empty((n, H, hd))
+            for i in range(n):
+                o[i] = attention_row(q[i], caches[i].K[m], caches[i].V[m], int(pos[i]), scale)
         o = self.rnd(o.reshape(n, H * hd))
         h = h + self.mm(o, L["wo"])
         # MLP sub-block (SwiGLU)

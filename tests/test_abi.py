@@ -101,3 +101,16 @@ def test_last_error_is_per_thread():
     t.join()
     assert other and other[0] != mine
     assert L.nv_last_error() == mine
+
+
+def test_binding_constants_match_the_header():
+    """Limits the binding repeats from include/nvium.h have the header's values."""
+    text = open(HEADER).read()
+    for name in ("NV_PHILOX_NOALLOC_MAX", "NV_MAX_EXITS"):
+        m = re.search(r"#define\s+" + name + r"\s+(\d+)", text)
+        assert m, name
+        assert int(m.group(1)) == getattr(nv, name), name
+
+
+def test_router_probs_rejects_null_state():
+    assert nv.lib().nv_read_router_probs(None, None, None) == nv.NV_ERR_INVALID_ARG

@@ -94,6 +94,16 @@ def test_cpu_baseline_reports_all_threads_and_one_thread():
     wl = W.WORKLOADS["T"]
     lens = W.make_prompt_lengths(wl)
     prompts = W.make_prompts(wl, lengths=lens)
-    cb = bench.cpu_baseline(wl, weights_seed=0, lens=lens, prompts=prompts, xseed=7, prefix=16, n_steps=2)
+    cb = bench.cpu_baseline(wl, lens=lens, prompts=prompts, xseed=7, n_steps=2)
     assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["cores"] >= 1
     assert cb["value"] > 0 and cb["value_1_thread"] > 0 and "sample" in cb
+    # the sample is a whole prompt of the workload, not a truncated one
+    assert f"({len(prompts[int(np.argmin(lens))])}-token prompt" in cb["sample"]
+
+
+def test_sub_line_keeps_only_measurement_keys():
+    d = {"metric": "m", "value": 1.0, "unit": "tokens/s", "n_gpus": 1, "roofline": {"frac": 0.5},
+         "e2e": {"value": 0.5}, "config": {"workload": "w"}, "vs_baseline": None}
+    sub = bench.sub_line(d, "other")
+    assert sub["metric"] == "other" and sub["value"] == 1.0 and sub["roofline"] == {"frac": 0.5}
+    assert "n_gpus" not in sub and "vs_baseline" not in sub

@@ -5,7 +5,14 @@ sampled outputs it can compute one by one, and two properties are checked at
 any size:
 
 * scoring (16 x 2048): causality makes logp[b, t] for t < T depend only on
-  tokens[b, :T+1], so the oracle scores a short prefix of one sequence;
+  tokens[b, :T+1], so the oracle scores a 130-position prefix of one
+  sequence (three 64-row query tiles of the attention kernel, the last one
+  ragged, over several 64-key tiles);
+* decode at B=1 (prompt 2048, the benchmark's launch configuration): the
+  oracle prefills the same 2048-token prompt, replays the first decode steps
+  teacher-forced (every stop decision checked against the device's own
+  router probabilities), and both caches are compared after the prefill and
+  after the flush, at least one layer in every exit block;
 * decode at B=64 (ragged prompts): the oracle replays the batch's shortest
   sequence alone (same Philox sequence index), teacher-forced, for a few
   steps, and its KV after the flush (deep bf16 caches: exceedances of the
@@ -53,7 +60,7 @@ def test_scoring_16x2048_prefix_matches_oracle(weights, oracle_model):
     assert abs(float(nll[0]) + float(logp.astype(np.float64).mean())) < 1e-3
     assert np.all(depth >= 12 / 48 - 1e-6) and np.all(depth <= 1 + 1e-6)
     assert abs(float(mean_depth[0]) - float(depth.astype(np.float64).mean())) < 1e-5
-    T = 40
+    T = 130
     ref, _, ref_depth, _ = O.score_mixture_with_depth(oracle_model, toks[5:6, : T + 1])
     np.testing.assert_allclose(logp[5, :T], ref[0], atol=tolerance(CFG), rtol=0)
     np.testing.assert_allclose(depth[5, :T], ref_depth[0], atol=tolerance(CFG), rtol=0)
@@ -76,7 +83,8 @@ def test_decode_b64_sampled_sequence_matches_oracle(weights, oracle_model):
     for s in range(steps):
         st.decode_step(seed + s, tok, ex, lp)
         rec = dec.step(seed + s, forced_exits=[int(ex[b])], forced_tokens=[int(tok[b])])
-        chk.check(rec, tok[b:b + 1], ex[b:b + 1], lp[b:b + 1])
+        chk.check(rec, tok[b:b + 1], ex[b:b + 1], lp[b:b + 1], st.router_probs()[:, b:b + 1])
+    chk.report("B=64 sequence %d" % b)
     st.flush()
     dec.flush()
     st.sync_status()
@@ -87,6 +95,44 @@ def test_decode_b64_sampled_sequence_matches_oracle(weights, oracle_model):
         # at most 1e-4 of the elements beyond the tolerance, none beyond twice it
         kv_close_counted(K, dec.caches[0].K[m][:n], CFG, f"K layer {m}", max_frac=1e-4, hard_factor=2.0)
         kv_close_counted(V, dec.caches[0].V[m][:n], CFG, f"V layer {m}", max_frac=1e-4, hard_factor=2.0)
+    st.close()
+    model.close()
+
+
+def test_decode_b1_prompt_2048_matches_oracle(weights, oracle_model):
+    wl = W.WORKLOADS["X1"]
+    prompt = W.make_prompts(wl)[0]
+    assert len(prompt) == 2048
+    steps, seed = 8, wl.philox_seed
+    max_seq = len(prompt) + wl.steps + 64
+    model = nv.Model(CFG, weights, max_batch=1, max_seq=max_seq, max_pending=256)
+    st = nv.State(model, 1)
+    st.prefill(prompt, [len(prompt)])
+    dec = O.OracleDecoder(oracle_model, [prompt], steps)
+    layers = (0, 11, 12, 23, 24, 35, 36, 47)
+    for m in (0, 23, 47):
+        K, V, n = gpu_kv(st, 0, m, max_seq, CFG)
+        assert n == len(prompt) - 1
+        kv_close_counted(K, dec.caches[0].K[m][:n], CFG, f"prefill K layer {m}", max_frac=1e-4, hard_factor=2.0)
+        kv_close_counted(V, dec.caches[0].V[m][:n], CFG, f"prefill V layer {m}", max_frac=1e-4, hard_factor=2.0)
+    chk = StepChecker(CFG)
+    tok, ex, lp = np.zeros(1, np.int32), np.zeros(1, np.int32), np.zeros(1, np.float32)
+    exits = []
+    for s in range(steps):
+        st.decode_step(seed + s, tok, ex, lp)
+        rec = dec.step(seed + s, forced_exits=ex, forced_tokens=tok)
+        chk.check(rec, tok, ex, lp, st.router_probs())
+        exits.append(int(ex[0]))
+    chk.report("B=1 prompt 2048")
+    st.flush()
+    dec.flush()
+    st.sync_status()
+    for m in layers:
+        K, V, n = gpu_kv(st, 0, m, max_seq, CFG)
+        assert n == dec.t[0] == len(prompt) - 1 + steps
+        kv_close_counted(K, dec.caches[0].K[m][:n], CFG, f"K layer {m}", max_frac=1e-4, hard_factor=2.0)
+        kv_close_counted(V, dec.caches[0].V[m][:n], CFG, f"V layer {m}", max_frac=1e-4, hard_factor=2.0)
+    print("B=1 exits", exits)
     st.close()
     model.close()
 

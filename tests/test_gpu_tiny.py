@@ -58,8 +58,10 @@ def test_decode_parity_prompt32_steps32(weights):
     prompts = W.make_prompts(W.WORKLOADS["T"])
     chk, state, dec, _ = run_decode_parity(nv, CFG, weights, prompts, 32)
     assert chk.steps == 32
-    # fp32: no near-ties expected
+    # fp32: no near-ties expected, and the device's router probabilities
+    # agree with the oracle's to fp32 rounding
     assert chk.exit_ties == 0 and chk.token_ties == 0
+    assert chk.junctions > 0 and chk.max_dw < 1e-5
     c = state.counters()
     assert c[nv.CTR["steps"]] == 32
     assert c[nv.CTR["exit0"]:nv.CTR["exit0"] + 4].sum() == 32

@@ -119,6 +119,45 @@ def test_rope_relative_position_and_identity():
     np.testing.assert_allclose(d1, d2, rtol=1e-10)
 
 
+@pytest.mark.parametrize("rows_per_block", [256, 7])
+def test_causal_attention_against_torch_sdpa(rows_per_block):
+    """The oracle's attention (per row, and as masked blocks of rows) against
+    torch's scaled_dot_product_attention with a causal mask in float64: rows
+    at positions 300..599 of one sequence attend to keys 0..their position."""
+    rng = np.random.default_rng(9)
+    H, hd, P = 3, 32, 600
+    q = rng.standard_normal((P, H, hd))
+    K = rng.standard_normal((P, H, hd))
+    V = rng.standard_normal((P, H, hd))
+    scale = 1.0 / np.sqrt(hd)
+    tq = torch.from_numpy(q.transpose(1, 0, 2))[None]
+    tk = torch.from_numpy(K.transpose(1, 0, 2))[None]
+    tv = torch.from_numpy(V.transpose(1, 0, 2))[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True)[0].numpy().transpose(1, 0, 2)
+    pos = np.arange(300, P)
+    blk = O.causal_attention_rows(q[pos], K, V, pos, scale, rows_per_block=rows_per_block)
+    np.testing.assert_allclose(blk, ref[pos], rtol=0, atol=1e-12)
+    for p in (300, 301, 450, 599):
+        np.testing.assert_allclose(O.attention_row(q[p], K, V, p, scale), ref[p], rtol=0, atol=1e-12)
+    # a ragged subset of positions (the deferred rows of a decode step)
+    sub = np.array([3, 4, 5, 77, 78, 599])
+    np.testing.assert_allclose(O.causal_attention_rows(q[sub], K, V, sub, scale, rows_per_block), ref[sub],
+                               rtol=0, atol=1e-12)
+
+
+def test_block_and_row_attention_give_the_same_forward():
+    """A full-depth forward with block attention equals the row-at-a-time one."""
+    om, _ = tiny_model()
+    toks = W.make_prompts(W.WORKLOADS["T"])[0]
+    h1, s1, c1 = om.forward_sequence(toks)
+    om.block_attention = False
+    h2, s2, c2 = om.forward_sequence(toks)
+    np.testing.assert_allclose(h1, h2, rtol=0, atol=1e-12)
+    for m in range(W.TINY.n_layers):
+        np.testing.assert_allclose(c1.K[m], c2.K[m], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(c1.V[m], c2.V[m], rtol=0, atol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # independent LLaMA (transformers, float64)
 # --------------------------------------------------------------------------
