@@ -66,6 +66,19 @@ template <> __device__ __forceinline__ float rnd<__nv_bfloat16>(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// per-element arithmetic shared by every kernel that performs the step, so
+// that two kernels doing the same step round identically
+// ---------------------------------------------------------------------------
+// rotate-half RoPE of the pair (y0, y1) by (cos, sin)
+__device__ __forceinline__ float2 rope_pair(float y0, float y1, float2 cs) {
+  return make_float2(y0 * cs.x - y1 * cs.y, y1 * cs.x + y0 * cs.y);
+}
+// SwiGLU: silu(g) * u
+__device__ __forceinline__ float swiglu(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// sum of squares of four values (one float4 of an RMSNorm row)
+__device__ __forceinline__ float sumsq4(float4 x) { return x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w; }
+
+// ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
 // Easy as 1, 2, 3", SC'11, section 3.2): ten rounds; each multiplies counter
 // words 0 and 2 by fixed odd constants, swaps in the high halves XORed with
@@ -176,6 +189,9 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // Which part of a fused weight a GEMM output column belongs to.
-enum EpiMode : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_STORE = 3, EPI_HEAD = 4 };
+// EPI_LSE: scoring head; per row and 128-token tile the max and the sum of
+// exp(logit - max), and the target token's logit (the logits never reach
+// global memory)
+enum EpiMode : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_STORE = 3, EPI_HEAD = 4, EPI_LSE = 5 };
 
 }  // namespace nv

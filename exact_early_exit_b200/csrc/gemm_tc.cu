@@ -38,26 +38,21 @@
 #include "gemm.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "tc_prims.cuh"
 
 namespace nv {
 namespace {
+using namespace tc;
 
-constexpr int BM = 128;      // features per tile (MMA M, TMEM lanes)
-constexpr int BK = 64;       // K per stage: one 128-byte swizzle row of bf16
-constexpr int BNMAX = 256;   // rows per tile (MMA N, TMEM columns)
-constexpr int BOXN = 32;     // rows per X TMA box
 constexpr int STAGES = 4;        // stages at the largest row tile (256 rows)
 constexpr int MAXST = 12;        // stages when the row tile is small
-constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNMAX * BK * 2;
-constexpr int BOX_BYTES = BOXN * BK * 2;
 constexpr int SMEM_TILES = STAGES * (A_BYTES + B_BYTES);
 constexpr int EPI_ROWS = 32;                    // rows per epilogue staging pass
 constexpr int EPI_BYTES = EPI_ROWS * BM * 4;    // fp32 staging tile [32 rows][128 features]
 constexpr int SMEM_BYTES = SMEM_TILES + 512 /*barriers*/ + EPI_BYTES + 1024 /*align*/;
 constexpr uint32_t TMEM_COLS = 512;  // two 256-column fp32 accumulators
 constexpr int THREADS = 192;
-constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on any single wait
 
 struct TcArgs {
   const int* nrows;
@@ -72,95 +67,6 @@ struct TcArgs {
   unsigned long long pf_bytes;
   EpiArgs epi;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait; false when `limit_ns` ran out (the CTA then aborts) or
-// another role aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                          unsigned long long limit_ns = WAIT_NS) {
-  if (mbar_try_wait(b, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((i & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
-          "r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (SBO), descriptor version 1 (sm_100).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
-__device__ __forceinline__ uint32_t idesc_bf16(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
-__device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 struct Item {
   int n0, r0, rows, nbox, kb0, kb1, split;
@@ -202,11 +108,9 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
       const int r = r0 + j;
       const int pos = e.rs.row_pos[r];
       if (part < 2) {
-        const float2 cs = e.rope[(size_t)pos * half + i];
-        const float u0 = y0 * cs.x - y1 * cs.y;
-        const float u1 = y1 * cs.x + y0 * cs.y;
-        y0 = u0;
-        y1 = u1;
+        const float2 u = rope_pair(y0, y1, e.rope[(size_t)pos * half + i]);
+        y0 = u.x;
+        y1 = u.y;
       }
       __nv_bfloat16* dst;
       if (part == 0) dst = (__nv_bfloat16*)e.q_out + (size_t)r * HQ + head * e.hd;
@@ -291,13 +195,41 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
       }
       epi_bar();
     }
+  } else if (e.mode == EPI_LSE) {
+    // scoring head: for each row of the tile, the max and the sum of
+    // exp(logit - max) over this tile's 128 tokens (lanes take 4 tokens
+    // each, then a fixed butterfly), and the target token's logit when the
+    // target falls in this tile
+    const int lane = tid & 31, w = tid >> 5;
+    for (int j = w; j < nrows; j += 4) {
+      const float* row = S + j * BM;
+      float x[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[i] = row[lane + 32 * i];
+      float M = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      float Ssum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Ssum += expf(x[i] - M);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
+        const float S2 = __shfl_xor_sync(0xffffffffu, Ssum, o);
+        const float Mn = fmaxf(M, M2);
+        Ssum = Ssum * expf(M - Mn) + S2 * expf(M2 - Mn);
+        M = Mn;
+      }
+      const int r = r0 + j;
+      if (lane == 0) e.lse_part[(size_t)r * e.nblk + n0 / BM] = make_float2(M, Ssum);
+      const int tg = e.lse_target[r] - n0;
+      if (tg >= 0 && tg < BM && (tg & 31) == lane) e.lse_tgt[r] = row[tg];
+    }
   } else if (e.mode == EPI_SWIGLU) {
 #pragma unroll 4
     for (int idx = tid; idx < nrows * (BM / 2); idx += 128) {
       const int j = idx / (BM / 2), jj = idx % (BM / 2);
       const float g = S[j * BM + jj], u = S[j * BM + BM / 2 + jj];
       ((__nv_bfloat16*)e.u_out)[(size_t)(r0 + j) * e.F + (n0 / BM) * (BM / 2) + jj] =
-          __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+          __float2bfloat16_rn(swiglu(g, u));
     }
   }
 }
@@ -624,6 +556,13 @@ static nv_status make_map(TcPlanCache* c, const void* ptr, uint64_t inner, uint6
   return NV_OK;
 }
 
+nv_status tc_map(TcPlanCache* c, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                 uint32_t box_rows, CUtensorMap* out) {
+  return make_map(c, ptr, inner, outer, ld_elems, box_rows, out);
+}
+
+int tc_sm_count() { return sm_count(); }
+
 nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int N, int K, const int* nrows,
                       int max_rows, float* Y, bool allow_split, const EpiArgs* epi, int* tile_counters,
                       const void* prefetch, size_t prefetch_bytes, cudaStream_t st, int* grid_out,
@@ -638,7 +577,7 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
       set_error("fused tcgen05 epilogue needs one K slice");
       return NV_ERR_UNSUPPORTED;
     }
-    const bool ok = epi->mode == EPI_RESID || epi->mode == EPI_HEAD ||
+    const bool ok = epi->mode == EPI_RESID || epi->mode == EPI_HEAD || epi->mode == EPI_LSE ||
                     (epi->mode == EPI_QKV && BM % epi->hd == 0 && (epi->H * epi->hd) % BM == 0) ||
                     (epi->mode == EPI_SWIGLU && epi->G == BM / 2);
     if (!ok) {

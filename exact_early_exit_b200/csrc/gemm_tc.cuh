@@ -23,4 +23,10 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
 nv_status encode_rows128_map(const void* base, uint64_t rows, uint32_t box_rows, CUtensorMap* out);
 // elements between split-K slices of an N-column output
 size_t tc_split_stride(size_t N);
+// Cached 2-D bf16 tensor map over [outer][inner] (row stride ld_elems), boxes
+// of 64 x box_rows, 128-byte swizzle (the GEMM operand layout).
+nv_status tc_map(TcPlanCache* c, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                 uint32_t box_rows, CUtensorMap* out);
+// SMs of the current device (the persistent grids' size)
+int tc_sm_count();
 }  // namespace nv

@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(512) k_resid_norm(RowSet rs, const float* __re
       x.w += ys.w;
       hp[j] = x;
     }
-    float ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+    float ss = sumsq4(x);
     ss = warp_sum(ss);
     if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
     __syncthreads();
@@ -500,11 +500,9 @@ __global__ void __launch_bounds__(256) k_epilogue(EpiArgs a) {
       float y0 = epi_sum(a, ns, r, c0), y1 = epi_sum(a, ns, r, c0 + half);
       const int pos = a.rs.row_pos[r];
       if (part < 2) {
-        const float2 cs = a.rope[(size_t)pos * half + i];
-        const float u0 = y0 * cs.x - y1 * cs.y;
-        const float u1 = y1 * cs.x + y0 * cs.y;
-        y0 = u0;
-        y1 = u1;
+        const float2 u = rope_pair(y0, y1, a.rope[(size_t)pos * half + i]);
+        y0 = u.x;
+        y1 = u.y;
       }
       if (part == 0) {
         T* q = (T*)a.q_out + (size_t)r * a.H * a.hd + head * a.hd;
@@ -527,7 +525,7 @@ __global__ void __launch_bounds__(256) k_epilogue(EpiArgs a) {
       const int blk = j / a.G, jj = j % a.G;
       const float g = epi_sum(a, ns, r, blk * 2 * a.G + jj);
       const float u = epi_sum(a, ns, r, blk * 2 * a.G + a.G + jj);
-      ((T*)a.u_out)[(size_t)r * a.F + j] = cvt<T>(g / (1.0f + expf(-g)) * u);
+      ((T*)a.u_out)[(size_t)r * a.F + j] = cvt<T>(swiglu(g, u));
     }
   } else {
     for (long long idx = tid0; idx < (long long)R * a.N; idx += stride) {
@@ -1464,6 +1462,42 @@ void launch_lse_target(const float* Y, int r_begin, int n, int V, const int* tar
   if (grid > 4096) grid = 4096;
   if (grid < 1) grid = 1;
   launch_k(k_lse_target, grid, 256, 0, st, Y, r_begin, n, V, target, logpi, k, n_exits);
+}
+
+// Combine the per-tile (max, sum exp) partials of one row in tile order,
+// one warp per row: each lane merges tiles lane, lane + 32, ... in order,
+// then the lanes merge in a fixed butterfly.
+__global__ void k_lse_combine(const float2* __restrict__ part, const float* __restrict__ tgt, int n, int nblk,
+                              float* __restrict__ logpi, int k, int n_exits) {
+  pdl_wait();
+  pdl_launch();
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
+    const float2* p = part + (size_t)r * nblk;
+    float M = -CUDART_INF_F, S = 0.f;
+    for (int b = lane; b < nblk; b += 32) {
+      const float2 v = p[b];
+      const float Mn = fmaxf(M, v.x);
+      S = S * expf(M - Mn) + v.y * expf(v.x - Mn);
+      M = Mn;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
+      const float S2 = __shfl_xor_sync(0xffffffffu, S, o);
+      const float Mn = fmaxf(M, M2);
+      S = (M == -CUDART_INF_F ? 0.f : S * expf(M - Mn)) + (M2 == -CUDART_INF_F ? 0.f : S2 * expf(M2 - Mn));
+      M = Mn;
+    }
+    if (lane == 0) logpi[(size_t)r * n_exits + k] = tgt[r] - (M + logf(S));
+  }
+}
+void launch_lse_combine(const float2* part, const float* tgt, int n, int nblk, float* logpi, int k, int n_exits,
+                        cudaStream_t st) {
+  int grid = (n + 7) / 8;
+  if (grid > 4096) grid = 4096;
+  if (grid < 1) grid = 1;
+  launch_k(k_lse_combine, grid, 256, 0, st, part, tgt, n, nblk, logpi, k, n_exits);
 }
 
 __device__ __forceinline__ float log_sigmoid(float z) {

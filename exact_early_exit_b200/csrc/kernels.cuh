@@ -76,6 +76,10 @@ struct EpiArgs {
   const unsigned long long* seed;  // Philox key
   float* head_part;                // [B][nblk][HEAD_PART]
   int nblk;
+  // EPI_LSE: rows r of the launch are scoring rows r_begin + r
+  const int* lse_target;           // [rows] target token of each scoring row (offset to the launch's first row)
+  float2* lse_part;                // [rows][nblk] (max, sum exp(logit - max)) per 128-token tile
+  float* lse_tgt;                  // [rows] logit of the target token
 };
 void launch_epilogue(bool bf16, const EpiArgs& a, int grid, cudaStream_t st);
 
@@ -211,6 +215,11 @@ void launch_exit_rows(bool bf16, RowSet rs, const ExitDev& e, int router_hidden,
                       float* z, int d, float eps, cudaStream_t st);
 void launch_lse_target(const float* Y, int r_begin, int n, int V, const int* target, float* logpi, int k,
                        int n_exits, cudaStream_t st);
+// log pi_k(target) of rows [0, n) from the fused head epilogue's per-tile
+// partials (EPI_LSE): LSE over the nblk tiles in tile order, minus nothing
+// else: logpi[r][k] = tgt[r] - (M + log S).
+void launch_lse_combine(const float2* part, const float* tgt, int n, int nblk, float* logpi, int k, int n_exits,
+                        cudaStream_t st);
 // Sets conditional `h` to (any active[b] or force[b]); when set, adds
 // *block_launches to counters[NV_CTR_LAUNCHES].
 void launch_set_cond(cudaGraphConditionalHandle h, const int* active, const int* force, int B, long long* counters,

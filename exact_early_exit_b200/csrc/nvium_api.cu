@@ -16,6 +16,7 @@
 #include "gemm.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "layer_tc.cuh"
 
 namespace nv {
 static thread_local std::string g_err;
@@ -47,6 +48,13 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool mma_attention_enabled() {
   const char* ev = std::getenv("NVIUM_ATTN");
   return !(ev && std::string(ev) == "simt");
+}
+
+// decode and flush layers run as one persistent kernel after attention
+// unless NVIUM_LAYER_KERNEL=0 selects the per-kernel path (kept for comparison)
+bool layer_kernel_enabled() {
+  const char* ev = std::getenv("NVIUM_LAYER_KERNEL");
+  return !(ev && ev[0] == '0');
 }
 
 constexpr int kTileCounters = 1024;  // >= N/128 of any split GEMM
@@ -88,10 +96,11 @@ struct nv_model {
   float2* rope = nullptr;
   long long layer_weight_bytes = 0;
   int gemm_kind = GEMM_SIMT;
+  bool layer_kernel = false;  // decode/flush layers on the persistent kernel (layer_tc.cu)
   GemmPlanCache* gemm_plans = nullptr;
   // scoring scratch
   Buf sc_h, sc_act, sc_u, sc_ctr, sc_q, sc_o, sc_Y, sc_kv, sc_part, sc_z, sc_logpi, sc_logp, sc_i32, sc_nll,
-      sc_depth, sc_mdepth;
+      sc_depth, sc_mdepth, sc_lse_part, sc_lse_tgt;
 };
 
 struct nv_state {
@@ -122,6 +131,8 @@ struct nv_state {
   int *row_b = nullptr, *row_pos = nullptr, *row_hrow = nullptr, *seq_start = nullptr, *nrows = nullptr;
   void *act = nullptr, *u = nullptr, *q = nullptr, *o = nullptr, *exit_act = nullptr;
   int* tile_counters = nullptr;
+  int* lt_sync = nullptr;      // [L][lt_sync_ints] counters of the persistent layer kernel
+  size_t lt_sync_ints = 0;
   float *Y = nullptr, *attn_part = nullptr, *head_part = nullptr;
   size_t Y_elems = 0;
   int head_nblk = 0, kv_splits = 1, row_groups = 1;
@@ -195,6 +206,8 @@ struct LayerIO {
   bool prefetch_next;  // the last GEMM of a layer prefetches the next layer's QKV weights
   bool split_k;        // few rows expected (decode, flush): let the GEMM split K
   int* status;
+  int* lt_sync;        // non-null: decode/flush layers on the persistent layer kernel
+  size_t lt_sync_ints;
 };
 
 // Per-kernel event timing for nv_decode_step_profiled (null when capturing).
@@ -249,8 +262,50 @@ void timed(Prof* prof, long long* launches, int nlaunch, int kind, long long byt
 // gate/up + SwiGLU, down + residual.  With `next_norm` (the next layer's
 // attention-norm gain, when it runs the same rows) the down projection's
 // residual is followed by that norm, so act is ready for the next layer.
+// The persistent decode-layer kernel's arguments for layer `layer`:
+// MLP part of this layer (when `mlp`), then the next layer's norm and QKV
+// when it runs the same rows (`next_norm`), or this layer's QKV alone.
+LayerTcRun layer_tc_args(nv_model* M, int layer, const LayerIO& io, bool mlp, const void* next_norm) {
+  const LayerDev& Lw = M->layers[layer];
+  LayerTcRun r{};
+  r.rs = io.rs;
+  r.kv = io.kv;
+  r.rope = M->rope;
+  r.o = io.o;
+  r.act = io.act;
+  r.u = io.u;
+  r.q = io.q;
+  r.Y = io.Y;
+  r.sync = io.lt_sync + (size_t)layer * io.lt_sync_ints;
+  r.status = io.status;
+  r.d = M->d;
+  r.HQ = M->HQ;
+  r.H = M->H;
+  r.hd = M->hd;
+  r.F = M->F;
+  r.eps = M->cfg.rms_eps;
+  if (mlp) {
+    r.w_o = Lw.w_o;
+    r.w_gu = Lw.w_gu;
+    r.w_d = Lw.w_d;
+    r.mlp_norm = Lw.mlp_norm;
+    r.flags = LT_MLP;
+    if (next_norm) {
+      r.flags |= LT_NORM2 | LT_QKV;
+      r.norm2 = next_norm;
+      r.w_qkv = M->layers[layer + 1].w_qkv;
+      r.kv_layer = layer + 1;
+    }
+  } else {
+    r.flags = LT_QKV;
+    r.w_qkv = Lw.w_qkv;
+    r.kv_layer = layer;
+  }
+  return r;
+}
+
 nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st, Prof* prof = nullptr,
-                     long long* launches = nullptr, const void* next_norm = nullptr) {
+                     long long* launches = nullptr, const void* next_norm = nullptr, bool qkv_ready = false) {
   const LayerDev& Lw = M->layers[layer];
   const bool bf = M->bf16;
   const long long es = (long long)M->esz;
@@ -290,8 +345,20 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
           });
     return gst;
   };
-  // QKV + RoPE + KV write (fused epilogue)
-  NV_TRY(gemm(EPI_QKV, io.act, d, Lw.w_qkv, 3 * HQ, d, R * 3 * HQ * es, Lw.w_o, d * HQ * es));
+  const bool persistent = io.lt_sync && io.split_k && M->layer_kernel;
+  const long long wq_bytes = 3 * HQ * d * es, wmlp_bytes = (d * HQ + 3 * F * d) * es;
+  if (persistent) {
+    // QKV + RoPE + KV write, unless the previous layer's launch did it
+    if (!qkv_ready) {
+      const LayerTcRun r = layer_tc_args(M, layer, io, false, nullptr);
+      timed(prof, launches, 1, NV_K_GEMM, wq_bytes + R * d * es + R * 3 * HQ * es, 2 * R * 3 * HQ * d,
+            [&] { gst = layer_tc_launch(gemm_tc_plans(M->gemm_plans), r, st); });
+      NV_TRY(gst);
+    }
+  } else {
+    // QKV + RoPE + KV write (fused epilogue)
+    NV_TRY(gemm(EPI_QKV, io.act, d, Lw.w_qkv, 3 * HQ, d, R * 3 * HQ * es, Lw.w_o, d * HQ * es));
+  }
   // attention
   AttnArgs a{};
   a.rs = io.rs;
@@ -317,6 +384,14 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
           if (io.dec_attn) launch_attention_decode(bf, a, st);
           else launch_attention(bf, a, st);
         });
+  if (persistent) {
+    // everything after attention, and the next layer's QKV when it runs the same rows
+    const LayerTcRun r = layer_tc_args(M, layer, io, true, next_norm);
+    const long long b = wmlp_bytes + (next_norm ? wq_bytes : 0) + R * HQ * es + R * d * 8;
+    const long long f = 2 * R * (d * HQ + 3 * F * d + (next_norm ? 3 * HQ * d : 0));
+    timed(prof, launches, 1, NV_K_GEMM, b, f, [&] { gst = layer_tc_launch(gemm_tc_plans(M->gemm_plans), r, st); });
+    return gst;
+  }
   // output projection + residual, MLP RMSNorm
   if (M->gemm_kind == GEMM_TC && io.split_k) {
     // split-K slices of the projection are summed into h by the norm kernel
@@ -397,6 +472,8 @@ LayerIO state_io(nv_state* s) {
   io.prefetch_next = true;
   io.split_k = true;
   io.status = s->status;
+  io.lt_sync = s->lt_sync;
+  io.lt_sync_ints = s->lt_sync_ints;
   return io;
 }
 
@@ -470,7 +547,8 @@ nv_status record_layers(nv_state* s, cudaStream_t st, Prof* prof, long long* lau
         prof->recs.back().bytes = (long long)prof->R * M->d * (4 + es);
       }
     }
-    NV_TRY(layer_body(M, layer, io, st, prof, launches, next_norm_in_block(M, layer)));
+    const bool block_start = layer == l0 || M->exit_at[layer - 1] >= 0;
+    NV_TRY(layer_body(M, layer, io, st, prof, launches, next_norm_in_block(M, layer), !block_start));
     const int k = M->exit_at[layer];
     if (k < 0) continue;
     JuncArgs j{};
@@ -940,9 +1018,12 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
   const bool tc_shapes = d % 128 == 0 && HQ % 128 == 0 && (2 * F) % 128 == 0 && F % 64 == 0 &&
                          V % 128 == 0 && cfg->adapter_hidden % 128 == 0;
   M->gemm_kind = (M->bf16 && tc_shapes) ? gemm_default_kind() : GEMM_SIMT;
+  M->layer_kernel = M->gemm_kind == GEMM_TC && layer_kernel_enabled() &&
+                    layer_tc_supported(M->d, M->HQ, M->hd, M->F, M->bf16) && M->G == 64;
   M->gemm_plans = gemm_plans_create();
   // kernels that need more than 48 KB of dynamic shared memory
   nv_status gs = gemm_prepare(M->gemm_kind, M->bf16);
+  if (gs == NV_OK && M->layer_kernel) gs = layer_tc_prepare();
   if (gs != NV_OK) {
     nv_destroy(M);
     return gs;
@@ -974,7 +1055,8 @@ nv_status nv_destroy(nv_model* M) {
   if (M->pool) cudaFree(M->pool);
   gemm_plans_destroy(M->gemm_plans);
   for (Buf* b : {&M->sc_h, &M->sc_act, &M->sc_u, &M->sc_ctr, &M->sc_q, &M->sc_o, &M->sc_Y, &M->sc_kv, &M->sc_part, &M->sc_z,
-                 &M->sc_logpi, &M->sc_logp, &M->sc_i32, &M->sc_nll, &M->sc_depth, &M->sc_mdepth})
+                 &M->sc_logpi, &M->sc_logp, &M->sc_i32, &M->sc_nll, &M->sc_depth, &M->sc_mdepth, &M->sc_lse_part,
+                 &M->sc_lse_tgt})
     b->release();
   delete M;
   return NV_OK;
@@ -1041,6 +1123,10 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   A(&s->act, (size_t)s->max_rows * wide * esz);
   A(&s->u, (size_t)s->max_rows * F * esz);
   A((void**)&s->tile_counters, (size_t)kTileCounters * 4);
+  if (M->layer_kernel) {
+    s->lt_sync_ints = layer_tc_sync_ints(s->max_rows, M->F);
+    A((void**)&s->lt_sync, (size_t)M->L * s->lt_sync_ints * 4);
+  }
   A(&s->q, (size_t)s->max_rows * HQ * esz);
   A(&s->o, (size_t)s->max_rows * HQ * esz);
   A(&s->exit_act, (size_t)B * d * esz);
@@ -1057,6 +1143,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   }
   cudaMemset(s->counters, 0, NV_CTR_COUNT * 8);
   cudaMemset(s->tile_counters, 0, (size_t)kTileCounters * 4);
+  if (s->lt_sync) cudaMemset(s->lt_sync, 0, (size_t)M->L * s->lt_sync_ints * 4);
   cudaMemset(s->nstop, 0, (size_t)NV_MAX_EXITS * 4);
   cudaMemcpy(s->d_B, &B, 4, cudaMemcpyHostToDevice);
   s->tc_head = M->bf16 && M->gemm_kind == GEMM_TC && B >= 16 && M->V % 128 == 0 && M->d % 64 == 0;
@@ -1223,6 +1310,7 @@ nv_status nv_prefill(nv_state* s, const int32_t* tokens, const int32_t* lens, vo
     }
     NV_CUDA_TRY(cudaStreamSynchronize(st));  // the host row arrays are reused by the next chunk
   }
+  if (s->lt_sync) NV_CUDA_TRY(cudaMemsetAsync(s->lt_sync, 0, (size_t)M->L * s->lt_sync_ints * 4, st));
   // decode state after the prompt
   std::vector<int> t0(B), tk(B), ln((size_t)B * M->L);
   for (int b = 0; b < B; ++b) {
@@ -1256,6 +1344,9 @@ nv_status nv_rewind(nv_state* s, void* stream) {
     t0[b] = s->h_prompt_len[b] - 1;
     for (int m = 0; m < L; ++m) ln[(size_t)b * L + m] = t0[b];
   }
+  // counters of the persistent layer kernel start from zero (they are zero
+  // after every completed launch; this also clears what an aborted one left)
+  if (s->lt_sync) NV_CUDA_TRY(cudaMemsetAsync(s->lt_sync, 0, (size_t)L * s->lt_sync_ints * 4, st));
   NV_CUDA_TRY(cudaMemcpyAsync(s->t, s->prompt_len, B * 4, cudaMemcpyDeviceToDevice, st));
   NV_CUDA_TRY(cudaMemcpyAsync(s->tok, s->prompt_last, B * 4, cudaMemcpyDeviceToDevice, st));
   // lens[b][m] = prompt_len[b] for all m
@@ -1404,7 +1495,8 @@ nv_status nv_flush_deferred(nv_state* s, void* stream) {
       launch_plan_norm(M->bf16, p, M->layers[layer].attn_norm, s->act, M->d, M->cfg.rms_eps, plan_grid(s), st);
       ++launches;
     }
-    NV_TRY(layer_body(M, layer, io, st, nullptr, &launches, next_norm_in_block(M, layer)));
+    const bool block_start = layer == M->cfg.exit_layers[0] || M->exit_at[layer - 1] >= 0;
+    NV_TRY(layer_body(M, layer, io, st, nullptr, &launches, next_norm_in_block(M, layer), !block_start));
   }
   s->launches_total += launches;
   NV_CUDA_TRY(cudaGetLastError());
@@ -1552,7 +1644,16 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
   const int AH = M->cfg.adapter_hidden;
   const size_t y_layers = gemm_workspace_elems(
       M->gemm_kind, R, std::max<size_t>(3 * M->HQ > 2 * M->F ? 3 * M->HQ : 2 * M->F, (size_t)AH));
-  const size_t y_head = gemm_workspace_elems(M->gemm_kind, head_chunk, M->V);
+  // tcgen05 engine: the head GEMM's epilogue reduces the logits of each
+  // 128-token tile to (max, sum exp) and picks the target logit, so logits
+  // never reach memory; the SIMT engine writes one chunk of logits at a time
+  const bool fused_lse = M->gemm_kind == GEMM_TC && M->V % 128 == 0;
+  const int lse_nblk = M->V / 128;
+  const size_t y_head = fused_lse ? 0 : gemm_workspace_elems(M->gemm_kind, head_chunk, M->V);
+  if (fused_lse) {
+    NV_TRY(M->sc_lse_part.need((size_t)R * lse_nblk * sizeof(float2)));
+    NV_TRY(M->sc_lse_tgt.need((size_t)R * 4));
+  }
   NV_TRY(M->sc_h.need((size_t)R * M->d * 4));
   NV_TRY(M->sc_act.need((size_t)R * wide * M->esz));
   NV_TRY(M->sc_u.need((size_t)R * std::max<size_t>(M->F, (size_t)AH) * M->esz));
@@ -1675,6 +1776,23 @@ nv_status score_impl(nv_model* M, const int32_t* tokens, int B, int S, float* lo
                                        st);
             });
       NV_TRY(ast);
+    }
+    if (fused_lse) {
+      EpiArgs le{};
+      le.mode = EPI_LSE;
+      le.lse_target = d_tgt;
+      le.lse_part = M->sc_lse_part.as<float2>();
+      le.lse_tgt = M->sc_lse_tgt.as<float>();
+      le.nblk = lse_nblk;
+      nv_status hst = NV_OK;
+      timed(prof, nullptr, 2, NV_K_HEAD, (long long)M->V * M->d * es + (long long)R * M->d * es,
+            2LL * R * M->V * M->d, [&] {
+              hst = gemm_run(M->gemm_plans, M->gemm_kind, M->bf16, io.act, M->d, M->exits[k].head, M->V, M->d,
+                             io.rs.nrows, io.rs.max_rows, io.Y, false, &le, nullptr, 0, nullptr, 0, st);
+              launch_lse_combine(le.lse_part, le.lse_tgt, R, lse_nblk, M->sc_logpi.as<float>(), k, NE, st);
+            });
+      NV_TRY(hst);
+      continue;
     }
     for (int c = 0; c < nchunks; ++c) {
       const int r0 = c * head_chunk;
