@@ -1,0 +1,345 @@
+// Causal attention for prefill and scoring on the 5th-generation tensor
+// cores (tcgen05, accumulators in TMEM), bf16 caches with head_dim 64.
+//
+// What it computes is the causal softmax attention of the LLaMA-2 backbone
+// ("N-vium: Mixture-of-Exits Transformer for Accelerated Exact Generation",
+// section 4): a row at position p gets o = sum_j softmax_j(q . k_j / sqrt(hd))
+// v_j over the keys j <= p of its sequence.
+//
+// CTA (128-row query tile, head, sequence); two CTAs per SM.  Roles:
+//   warps 0-3  one query row per thread (= its TMEM lane): read the row's
+//              64 scores of a key tile from TMEM, causal mask, online softmax
+//              (running max and sum), write P to shared memory as a bf16
+//              pair hi + lo (hi = bf16(P), lo = bf16(P - hi), ~16 significant
+//              bits), and fold each tile's P V into a register accumulator
+//              with the softmax correction factor;
+//   warp 4     TMA: the query tile once, then 64-key tiles of K and V
+//              through a 3-stage ring (128-byte swizzle);
+//   warp 5     issues the MMAs: S = Q K^T (M 128, N 64, K 16 x 4) into one
+//              of two TMEM score buffers, one tile ahead of the softmax, and
+//              O_tile = P_hi V + P_lo V (V read in place as an MN-major
+//              operand) into one of two TMEM output buffers.
+// The softmax of tile j+1 overlaps the P V product of tile j.  Every wait is
+// bounded (2 s); on expiry the CTA records DEV_ERR_TIMEOUT, lets its copies
+// and MMAs land and frees its TMEM.
+#include <math_constants.h>
+
+#include "kernels.cuh"
+#include "tc_prims.cuh"
+
+namespace nv {
+namespace {
+using namespace tc;
+
+constexpr int HD = 64;
+constexpr int TQ = 128;   // query rows per CTA (MMA M, TMEM lanes)
+constexpr int TK = 64;    // keys per tile (MMA N of S, K of P V)
+constexpr int KST = 3;    // K/V ring stages
+constexpr int FT_THREADS = 192;
+constexpr uint32_t FT_TMEM_COLS = 256;  // S[2] at columns 0 and 64, O[2] at 128 and 192
+constexpr int TILE_BYTES = TK * HD * 2;  // 8 KB
+
+struct FtSmem {
+  __nv_bfloat16 Q[TQ * HD];        // 16 KB, 1024-byte aligned (128-byte swizzle atoms)
+  __nv_bfloat16 K[KST][TK * HD];   // 8 KB each
+  __nv_bfloat16 V[KST][TK * HD];
+  __nv_bfloat16 Phi[TQ * TK];      // 16 KB
+  __nv_bfloat16 Plo[TQ * TK];
+  uint64_t q_full, kv_full[KST], kv_empty[KST], s_full[2], s_empty[2], p_full, o_full[2], o_empty[2], drain;
+  uint32_t tmem;
+  int abort, go;
+};
+constexpr size_t FT_SMEM_BYTES = sizeof(FtSmem) + 1024;
+
+__device__ __forceinline__ void tma_row_box(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int row) {
+  tma_load_2d(dst, map, bar, x, row);
+}
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+// The softmax warps wait together: one thread polls (bounded), a named
+// barrier over the four warps releases them.
+__device__ __forceinline__ void sm_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool sm_wait(FtSmem& S, uint64_t* bar, uint32_t parity) {
+  if (threadIdx.x == 0) S.go = mbar_wait(bar, parity, &S.abort) ? 1 : 0;
+  sm_bar();
+  const bool ok = S.go != 0;
+  sm_bar();
+  return ok;
+}
+
+__global__ void __launch_bounds__(FT_THREADS, 2)
+    k_attn_fa_tc(const __grid_constant__ CUtensorMap kvmap, const __grid_constant__ CUtensorMap qmap, AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
+  extern __shared__ unsigned char smem_raw[];
+  FtSmem& S = *reinterpret_cast<FtSmem*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  if (*a.rs.nrows == 0) return;
+  // grid (row tile, head, sequence), the latest row tiles (the most keys) first
+  const int b = blockIdx.z, head = blockIdx.y;
+  const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
+  const int nrt = (s1 - s0 + TQ - 1) / TQ;
+  const int rt = nrt - 1 - (int)blockIdx.x;
+  if (rt < 0) return;
+  const int g0 = s0 + rt * TQ, g1 = min(s1, g0 + TQ), nr = g1 - g0;
+  const int pos_last = a.rs.row_pos[g1 - 1];
+  const int ntk = pos_last / TK + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&S.q_full, 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&S.s_full[s], 1);
+      mbar_init(&S.s_empty[s], 128);
+      mbar_init(&S.o_full[s], 1);
+      mbar_init(&S.o_empty[s], 128);
+    }
+    mbar_init(&S.p_full, 128);
+    mbar_init(&S.drain, 1);
+    S.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem)),
+                 "r"(FT_TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem;
+  volatile int* abort_flag = &S.abort;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      bool ok = true;
+      int issued[KST];
+      for (int s = 0; s < KST; ++s) issued[s] = -1;
+      mbar_expect_tx(&S.q_full, (uint32_t)(TQ * HD * 2));
+      tma_row_box(S.Q, &qmap, &S.q_full, head * HD, g0);
+      for (int j = 0; j < ntk && ok; ++j) {
+        const int st = j % KST;
+        const uint32_t ph = (uint32_t)((j / KST) & 1);
+        if (!mbar_wait(&S.kv_empty[st], ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        issued[st] = (int)ph;
+        mbar_expect_tx(&S.kv_full[st], (uint32_t)(2 * TILE_BYTES));
+        const int pos = j * TK;
+        tma_row_box(S.K[st], &kvmap, &S.kv_full[st], 0, (int)(a.kv.offset(a.layer, b, pos, head, 0) / HD));
+        tma_row_box(S.V[st], &kvmap, &S.kv_full[st], 0, (int)(a.kv.offset(a.layer, b, pos, head, 1) / HD));
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        mbar_wait(&S.q_full, 0, &never, WAIT_NS / 4);
+        for (int s = 0; s < KST; ++s)
+          if (issued[s] >= 0) mbar_wait(&S.kv_full[s], (uint32_t)issued[s], &never, WAIT_NS / 4);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      bool ok = mbar_wait(&S.q_full, 0, abort_flag), issued_any = false;
+      const uint32_t idesc_s = idesc_bf16(TK);                  // M 128, N 64, K-major A and B
+      const uint32_t idesc_o = idesc_bf16(HD) | (1u << 16);     // B (V) MN-major
+      const uint64_t qd = sw128_desc(smem_u32(S.Q));
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % KST;
+        if (!mbar_wait(&S.kv_full[st], (uint32_t)((j / KST) & 1), abort_flag)) return false;
+        if (!mbar_wait(&S.s_empty[j & 1], (uint32_t)(((j >> 1) & 1) ^ 1), abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t kd = sw128_desc(smem_u32(S.K[st]));
+        const uint32_t d = tmem + (uint32_t)((j & 1) * TK);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) umma(d, qd + (uint64_t)(2 * kk), kd + (uint64_t)(2 * kk), idesc_s, kk > 0);
+        issued_any = true;
+        umma_commit(&S.s_full[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < ntk && ok; ++j) {
+        if (j + 1 < ntk && !issue_s(j + 1)) {
+          ok = false;
+          break;
+        }
+        // P of tile j is in shared memory; O buffer j&1 is free again
+        if (!mbar_wait(&S.p_full, (uint32_t)(j & 1), abort_flag) ||
+            !mbar_wait(&S.o_empty[j & 1], (uint32_t)(((j >> 1) & 1) ^ 1), abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int st = j % KST;
+        const uint64_t ph = sw128_desc(smem_u32(S.Phi)), pl = sw128_desc(smem_u32(S.Plo));
+        const uint64_t vd = sw128_desc(smem_u32(S.V[st]));
+        const uint32_t d = tmem + (uint32_t)(2 * TK + (j & 1) * HD);
+#pragma unroll
+        for (int kk = 0; kk < TK / 16; ++kk) {
+          // K step of 16 keys: 32 bytes along a P row, 16 rows (2048 bytes) of V
+          umma(d, ph + (uint64_t)(2 * kk), vd + (uint64_t)(128 * kk), idesc_o, kk > 0);
+          umma(d, pl + (uint64_t)(2 * kk), vd + (uint64_t)(128 * kk), idesc_o, 1u);
+        }
+        umma_commit(&S.o_full[j & 1]);
+        umma_commit(&S.kv_empty[st]);
+      }
+      if (!ok && issued_any) {
+        umma_commit(&S.drain);
+        volatile int never = 0;
+        mbar_wait(&S.drain, 0, &never, WAIT_NS / 4);
+      }
+    }
+  } else {
+    // softmax warps: thread t owns query row t of the tile (TMEM lane t)
+    const int t = threadIdx.x;
+    const int pos = t < nr ? a.rs.row_pos[g0 + t] : -1;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float m = -CUDART_INF_F, l = 0.f, c_prev = 0.f;
+    float acc[HD];
+#pragma unroll
+    for (int i = 0; i < HD; ++i) acc[i] = 0.f;
+    bool ok = true;
+    unsigned char* prow_hi = reinterpret_cast<unsigned char*>(S.Phi) + t * 128;
+    unsigned char* prow_lo = reinterpret_cast<unsigned char*>(S.Plo) + t * 128;
+    auto fold_o = [&](int jj) -> bool {
+      // O_tile of tile jj is complete: acc = acc * c(jj) + O_tile
+      uint32_t v0[32], v1[32];
+      const uint32_t oa = lane_base + (uint32_t)(2 * TK + (jj & 1) * HD);
+      tmem_ld32_nowait(oa, v0);
+      tmem_ld32_nowait(oa + 32, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&S.o_empty[jj & 1]);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        acc[i] = acc[i] * c_prev + __uint_as_float(v0[i]);
+        acc[32 + i] = acc[32 + i] * c_prev + __uint_as_float(v1[i]);
+      }
+      return true;
+    };
+    for (int j = 0; j < ntk; ++j) {
+      if (!sm_wait(S, &S.s_full[j & 1], (uint32_t)((j >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // the row's 64 scores of this key tile, turned into P in place
+      uint32_t r[TK];
+      const uint32_t sa = lane_base + (uint32_t)((j & 1) * TK);
+      tmem_ld32_nowait(sa, *reinterpret_cast<uint32_t(*)[32]>(r));
+      tmem_ld32_nowait(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&S.s_empty[j & 1]);
+      const int k0 = j * TK;
+      float tmax = -CUDART_INF_F;
+#pragma unroll
+      for (int i = 0; i < TK; ++i) {
+        const float v = k0 + i <= pos ? __uint_as_float(r[i]) * a.scale : -CUDART_INF_F;
+        r[i] = __float_as_uint(v);
+        tmax = fmaxf(tmax, v);
+      }
+      const float mn = fmaxf(m, tmax);
+      const float cj = mn == -CUDART_INF_F ? 1.f : expf(m - mn);
+      float rs = 0.f;
+#pragma unroll
+      for (int i = 0; i < TK; ++i) {
+        const float p = mn == -CUDART_INF_F ? 0.f : expf(__uint_as_float(r[i]) - mn);
+        r[i] = __float_as_uint(p);
+        rs += p;
+      }
+      l = l * cj + rs;
+      m = mn;
+      // the previous tile's P V must be done with P before P is rewritten
+      if (j > 0 && !sm_wait(S, &S.o_full[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      if (j == ntk - 1 && pos_last + 1 - k0 < TK) {
+        // V rows past the last key may hold stale values (P is 0 there, and
+        // 0 * NaN would poison the sums): zero them before the P V product
+        const int nk = pos_last + 1 - k0;
+        unsigned char* vb = reinterpret_cast<unsigned char*>(S.V[j % KST]);
+        for (int i = nk * 8 + t; i < TK * 8; i += 128)
+          *reinterpret_cast<uint4*>(vb + (i >> 3) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = __uint_as_float(r[8 * c + 2 * e]), x1 = __uint_as_float(r[8 * c + 2 * e + 1]);
+          const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
+          hi[e] = pack2(h0, h1);
+          lo[e] = pack2(x0 - h0, x1 - h1);
+        }
+        const int off = ((c ^ (t & 7)) << 4);
+        *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&S.p_full);
+      // fold the previous tile's P V (its correction factor is c_prev)
+      if (j > 0) {
+        tc_fence_after();
+        fold_o(j - 1);
+      }
+      c_prev = cj;
+    }
+    if (ok) {
+      if (sm_wait(S, &S.o_full[(ntk - 1) & 1], (uint32_t)(((ntk - 1) >> 1) & 1))) {
+        tc_fence_after();
+        fold_o(ntk - 1);
+      } else {
+        ok = false;
+      }
+    }
+    if (ok && t < nr) {
+      const float inv = 1.0f / l;
+      uint4* orow = reinterpret_cast<uint4*>((__nv_bfloat16*)a.o + (size_t)(g0 + t) * a.H * HD + head * HD);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        orow[c] = make_uint4(pack2(acc[8 * c] * inv, acc[8 * c + 1] * inv), pack2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
+                             pack2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv), pack2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(FT_TMEM_COLS) : "memory");
+  }
+  if (threadIdx.x == 0) {
+    if (S.abort) dev_fail(a.status, DEV_ERR_TIMEOUT);
+    else if (a.lens && head == 0 && g1 == s1) a.lens[b * a.L + a.layer] = pos_last + 1;
+  }
+}
+
+}  // namespace
+
+cudaError_t attn_tc_prepare() {
+  return cudaFuncSetAttribute(k_attn_fa_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FT_SMEM_BYTES);
+}
+
+void launch_attn_fa_tc(const CUtensorMap* kvmap, const CUtensorMap* qmap, const AttnArgs& a, cudaStream_t st) {
+  dim3 grid((a.row_groups * ATTN_RPC + TQ - 1) / TQ, a.H, a.rs.B);
+  launch_k(k_attn_fa_tc, grid, FT_THREADS, FT_SMEM_BYTES, st, *kvmap, *qmap, a);
+}
+
+}  // namespace nv

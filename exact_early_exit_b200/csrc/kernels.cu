@@ -945,7 +945,8 @@ static void attention_t(const AttnArgs& a, cudaStream_t st) {
 }
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st) {
   if (bf16 && a.hd == 64 && a.kv_map && a.kv_splits == 1 && a.rs.B <= 65535) {
-    launch_attn_fa_mma(a.kv_map, a, st);
+    if (a.q_map) launch_attn_fa_tc(a.kv_map, a.q_map, a, st);
+    else launch_attn_fa_mma(a.kv_map, a, st);
     return;
   }
   if (a.hd == 64) {

@@ -96,6 +96,7 @@ struct AttnArgs {
   int L;
   int* status;     // device status word (bounded-wait expiry)
   const CUtensorMap* kv_map;  // host copy of the KV pool's 128-byte-row map (bf16, hd 64), or null
+  const CUtensorMap* q_map;   // prefill / scoring: map of q (boxes of 64 x 128 rows) for the tcgen05 kernel, or null
   int dec_splits;             // MMA decode attention: key-range splits per (sequence, head)
   int* dec_ctr;               // [B][H] split arrival counters (zero between launches)
 };
@@ -118,6 +119,10 @@ int attention_decode_launches(bool bf16, const AttnArgs& a);
 cudaError_t attn_mma_prepare();
 void launch_attn_dec_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st);
 void launch_attn_fa_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_t st);
+// Prefill / scoring on tcgen05 (attn_tc.cu): 128-row query tiles, S and the
+// per-tile P V in TMEM; needs a.kv_map and a.q_map.
+cudaError_t attn_tc_prepare();
+void launch_attn_fa_tc(const CUtensorMap* kvmap, const CUtensorMap* qmap, const AttnArgs& a, cudaStream_t st);
 
 struct StepArgs {
   int B, L, cap, d, n_exits;

@@ -50,6 +50,13 @@ bool mma_attention_enabled() {
   return !(ev && std::string(ev) == "simt");
 }
 
+// prefill / scoring attention on tcgen05 unless NVIUM_ATTN=mma (the warp-MMA
+// kernel) or NVIUM_ATTN=simt selects another engine
+bool tc_attention_enabled() {
+  const char* ev = std::getenv("NVIUM_ATTN");
+  return !(ev && (std::string(ev) == "simt" || std::string(ev) == "mma"));
+}
+
 // decode and flush layers run as one persistent kernel after attention
 // unless NVIUM_LAYER_KERNEL=0 selects the per-kernel path (kept for comparison)
 bool layer_kernel_enabled() {
@@ -96,6 +103,7 @@ struct nv_model {
   float2* rope = nullptr;
   long long layer_weight_bytes = 0;
   int gemm_kind = GEMM_SIMT;
+  bool tc_attention = false;  // prefill/scoring attention on the tcgen05 kernel (attn_tc.cu)
   bool layer_kernel = false;  // decode/flush layers on the persistent kernel (layer_tc.cu)
   GemmPlanCache* gemm_plans = nullptr;
   // scoring scratch
@@ -376,6 +384,13 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   a.L = io.L;
   a.status = io.status;
   a.kv_map = io.kv_map;
+  CUtensorMap qmap;
+  if (!io.dec_attn && io.kv_map && M->tc_attention) {
+    gst = tc_map(gemm_tc_plans(M->gemm_plans), io.q, (uint64_t)HQ, (uint64_t)io.rs.max_rows, (uint64_t)HQ, 128,
+                 &qmap);
+    NV_TRY(gst);
+    a.q_map = &qmap;
+  }
   a.dec_splits = io.dec_splits;
   a.dec_ctr = io.dec_ctr;
   const int attn_launches = io.dec_attn ? attention_decode_launches(bf, a) : (io.kv_splits > 1 ? 2 : 1);
@@ -1018,6 +1033,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
   const bool tc_shapes = d % 128 == 0 && HQ % 128 == 0 && (2 * F) % 128 == 0 && F % 64 == 0 &&
                          V % 128 == 0 && cfg->adapter_hidden % 128 == 0;
   M->gemm_kind = (M->bf16 && tc_shapes) ? gemm_default_kind() : GEMM_SIMT;
+  M->tc_attention = M->gemm_kind == GEMM_TC && M->hd == 64 && M->HQ % 64 == 0 && tc_attention_enabled();
   M->layer_kernel = M->gemm_kind == GEMM_TC && layer_kernel_enabled() &&
                     layer_tc_supported(M->d, M->HQ, M->hd, M->F, M->bf16) && M->G == 64;
   M->gemm_plans = gemm_plans_create();
@@ -1032,6 +1048,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
     const size_t head_sm = (((size_t)cfg->max_batch * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * d * esz;
     cudaError_t e2 = kernels_set_smem_limits(head_sm, (size_t)(cfg->max_batch + 1) * 4);
     if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_mma_prepare();
+    if (e2 == cudaSuccess && M->tc_attention) e2 = attn_tc_prepare();
     if (e2 == cudaSuccess && cfg->adapter_hidden) e2 = exit_adapter_prepare(M->bf16, M->d, cfg->adapter_hidden);
     if (e2 != cudaSuccess) {
       set_error(std::string("shared memory limits: ") + cudaGetErrorString(e2));

@@ -230,3 +230,33 @@ def test_shared_head_with_adapters_bf16_matches_oracle(batch):
                                      np.random.default_rng(1).integers(1, 70, size=batch))]
     chk, *_ = run_decode_parity(nv, cfg, w, prompts, 8, check_kv=batch == 3)
     assert chk.steps == 8
+
+
+def test_tcgen05_and_mma_flash_attention_agree(weights):
+    """Scoring and prefill attention on the tcgen05 kernel (128-row query
+    tiles, scores and P V in TMEM) against the warp-MMA kernel, on sequences
+    of ragged lengths spanning several query and key tiles."""
+    toks = np.stack([W.make_prompts(W.WORKLOADS["S"], seed=s)[0][:300] for s in (7, 8)]).astype(np.int32)
+    out = {}
+    for eng in ("mma", "tc"):
+        if eng == "mma":
+            os.environ["NVIUM_ATTN"] = "mma"
+        try:
+            m = nv.Model(CFG, weights, max_batch=3, max_seq=320)
+        finally:
+            os.environ.pop("NVIUM_ATTN", None)
+        lp = np.zeros((2, 299), np.float32)
+        m.score_mixture(toks, lp)
+        # prefill of ragged prompts: every layer's KV depends on the attention outputs
+        lens = np.array([300, 129, 64], np.int32)
+        st = nv.State(m, 3)
+        st.prefill(np.concatenate([toks[0], toks[1][:129], toks[0][:64]]), lens)
+        kv = [st.read_kv(b, 11, 320) for b in range(3)]
+        out[eng] = (lp, kv)
+        st.close()
+        m.close()
+    np.testing.assert_allclose(out["mma"][0], out["tc"][0], atol=5e-3, rtol=0)
+    for (K1, V1, n1), (K2, V2, n2) in zip(out["mma"][1], out["tc"][1]):
+        assert n1 == n2
+        np.testing.assert_allclose(W.as_f32(K1), W.as_f32(K2), atol=2e-2, rtol=2 ** -7)
+        np.testing.assert_allclose(W.as_f32(V1), W.as_f32(V2), atol=2e-2, rtol=2 ** -7)
