@@ -270,6 +270,8 @@ void timed(Prof* prof, long long* launches, int nlaunch, int kind, long long byt
 // gate/up + SwiGLU, down + residual.  With `next_norm` (the next layer's
 // attention-norm gain, when it runs the same rows) the down projection's
 // residual is followed by that norm, so act is ready for the next layer.
+const void* next_norm_in_block(const nv_model* M, int layer);
+
 // The persistent decode-layer kernel's arguments for layer `layer`:
 // MLP part of this layer (when `mlp`), then the next layer's norm and QKV
 // when it runs the same rows (`next_norm`), or this layer's QKV alone.
@@ -303,6 +305,17 @@ LayerTcRun layer_tc_args(nv_model* M, int layer, const LayerIO& io, bool mlp, co
       r.norm2 = next_norm;
       r.w_qkv = M->layers[layer + 1].w_qkv;
       r.kv_layer = layer + 1;
+      // the next layer's launch runs the same rows: its weights can be
+      // pulled into L2 while this one finishes and the next attention runs
+      const LayerDev& Nw = M->layers[layer + 1];
+      r.next_w_o = Nw.w_o;
+      r.next_w_gu = Nw.w_gu;
+      r.next_w_d = Nw.w_d;
+      r.next_flags = LT_MLP;
+      if (next_norm_in_block(M, layer + 1)) {
+        r.next_flags |= LT_NORM2 | LT_QKV;
+        r.next_w_qkv = M->layers[layer + 2].w_qkv;
+      }
     }
   } else {
     r.flags = LT_QKV;
@@ -339,11 +352,12 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
                   const void* pf, long long pf_bytes) {
     e.mode = mode;
     e.N = (int)N;
-    // with 64 or more 128-feature tiles (gate/up of the 1.5B model) the GEMM
-    // nearly fills the GPU unsplit and its epilogue runs in the GEMM kernel,
-    // one launch fewer; with fewer tiles (QKV: 36) splitting K is faster
-    // (measured on B200: unsplit gate/up +1%, unsplit QKV -12% decode tokens/s)
-    const bool split = io.split_k && N / 128 < 64;
+    // gate/up is never split: its SwiGLU epilogue runs in the GEMM kernel (one
+    // launch fewer), and the persistent decode-layer kernel computes it the
+    // same way, so the two decode paths agree bit for bit; with fewer tiles
+    // (QKV: 36) splitting K is faster (measured on B200 with the 1.5B model:
+    // unsplit gate/up +1%, unsplit QKV -12% decode tokens/s)
+    const bool split = io.split_k && N / 128 < 64 && mode != EPI_SWIGLU;
     timed(prof, launches, gemm_launch_count(M->gemm_kind, bf, split, &e), NV_K_GEMM,
           N * K * es + R * K * es + out_bytes,
           2 * R * N * K, [&] {
