@@ -36,7 +36,7 @@ constexpr int TQ = 128;   // query rows per CTA (MMA M, TMEM lanes)
 constexpr int TK = 64;    // keys per tile (MMA N of S, K of P V)
 constexpr int KST = 3;    // K/V ring stages
 constexpr int FT_THREADS = 192;
-constexpr uint32_t FT_TMEM_COLS = 256;  // S[2] at columns 0 and 64, O[2] at 128 and 192
+constexpr uint32_t FT_TMEM_COLS = 256;  // S[2] at columns 0 and 64, O at 128
 constexpr int TILE_BYTES = TK * HD * 2;  // 8 KB
 
 struct FtSmem {
@@ -45,7 +45,7 @@ struct FtSmem {
   __nv_bfloat16 V[KST][TK * HD];
   __nv_bfloat16 Phi[TQ * TK];      // 16 KB
   __nv_bfloat16 Plo[TQ * TK];
-  uint64_t q_full, kv_full[KST], kv_empty[KST], s_full[2], s_empty[2], p_full, o_full[2], o_empty[2], drain;
+  uint64_t q_full, kv_full[KST], kv_empty[KST], s_full[2], s_empty[2], p_full, o_full, drain;
   uint32_t tmem;
   int abort, go;
 };
@@ -64,6 +64,25 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[3
         "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
         "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
+}
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32, relative error
+// about 2^-22): the softmax runs in base 2 with the scores pre-scaled by
+// log2(e), so exp(s - m) = 2^(s log2 e - m log2 e)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -107,9 +126,8 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&S.s_full[s], 1);
       mbar_init(&S.s_empty[s], 128);
-      mbar_init(&S.o_full[s], 1);
-      mbar_init(&S.o_empty[s], 128);
     }
+    mbar_init(&S.o_full, 1);
     mbar_init(&S.p_full, 128);
     mbar_init(&S.drain, 1);
     S.abort = 0;
@@ -179,9 +197,8 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
           ok = false;
           break;
         }
-        // P of tile j is in shared memory; O buffer j&1 is free again
-        if (!mbar_wait(&S.p_full, (uint32_t)(j & 1), abort_flag) ||
-            !mbar_wait(&S.o_empty[j & 1], (uint32_t)(((j >> 1) & 1) ^ 1), abort_flag)) {
+        // P of tile j is in shared memory and O has been rescaled for it
+        if (!mbar_wait(&S.p_full, (uint32_t)(j & 1), abort_flag)) {
           ok = false;
           break;
         }
@@ -189,14 +206,14 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
         const int st = j % KST;
         const uint64_t ph = sw128_desc(smem_u32(S.Phi)), pl = sw128_desc(smem_u32(S.Plo));
         const uint64_t vd = sw128_desc(smem_u32(S.V[st]));
-        const uint32_t d = tmem + (uint32_t)(2 * TK + (j & 1) * HD);
+        const uint32_t d = tmem + (uint32_t)(2 * TK);
 #pragma unroll
         for (int kk = 0; kk < TK / 16; ++kk) {
           // K step of 16 keys: 32 bytes along a P row, 16 rows (2048 bytes) of V
-          umma(d, ph + (uint64_t)(2 * kk), vd + (uint64_t)(128 * kk), idesc_o, kk > 0);
+          umma(d, ph + (uint64_t)(2 * kk), vd + (uint64_t)(128 * kk), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
           umma(d, pl + (uint64_t)(2 * kk), vd + (uint64_t)(128 * kk), idesc_o, 1u);
         }
-        umma_commit(&S.o_full[j & 1]);
+        umma_commit(&S.o_full);
         umma_commit(&S.kv_empty[st]);
       }
       if (!ok && issued_any) {
@@ -210,29 +227,12 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
     const int t = threadIdx.x;
     const int pos = t < nr ? a.rs.row_pos[g0 + t] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    float m = -CUDART_INF_F, l = 0.f, c_prev = 0.f;
-    float acc[HD];
-#pragma unroll
-    for (int i = 0; i < HD; ++i) acc[i] = 0.f;
-    bool ok = true;
+    float m = -CUDART_INF_F, l = 0.f;
+    const float scale2 = a.scale * 1.4426950408889634f;  // log2(e) / sqrt(hd)
     unsigned char* prow_hi = reinterpret_cast<unsigned char*>(S.Phi) + t * 128;
     unsigned char* prow_lo = reinterpret_cast<unsigned char*>(S.Plo) + t * 128;
-    auto fold_o = [&](int jj) -> bool {
-      // O_tile of tile jj is complete: acc = acc * c(jj) + O_tile
-      uint32_t v0[32], v1[32];
-      const uint32_t oa = lane_base + (uint32_t)(2 * TK + (jj & 1) * HD);
-      tmem_ld32_nowait(oa, v0);
-      tmem_ld32_nowait(oa + 32, v1);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&S.o_empty[jj & 1]);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        acc[i] = acc[i] * c_prev + __uint_as_float(v0[i]);
-        acc[32 + i] = acc[32 + i] * c_prev + __uint_as_float(v1[i]);
-      }
-      return true;
-    };
+    const uint32_t o_addr = lane_base + (uint32_t)(2 * TK);
+    bool ok = true;
     for (int j = 0; j < ntk; ++j) {
       if (!sm_wait(S, &S.s_full[j & 1], (uint32_t)((j >> 1) & 1))) {
         ok = false;
@@ -248,26 +248,43 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
       tc_fence_before();
       mbar_arrive(&S.s_empty[j & 1]);
       const int k0 = j * TK;
+      // scores in base 2 (scaled by log2 e / sqrt(hd)); keys past the row's
+      // position (only in the tiles that reach the diagonal) get -inf
       float tmax = -CUDART_INF_F;
+      if (k0 + TK - 1 <= pos) {
 #pragma unroll
-      for (int i = 0; i < TK; ++i) {
-        const float v = k0 + i <= pos ? __uint_as_float(r[i]) * a.scale : -CUDART_INF_F;
-        r[i] = __float_as_uint(v);
-        tmax = fmaxf(tmax, v);
+        for (int i = 0; i < TK; ++i) {
+          const float v = __uint_as_float(r[i]) * scale2;
+          r[i] = __float_as_uint(v);
+          tmax = fmaxf(tmax, v);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < TK; ++i) {
+          const float v = k0 + i <= pos ? __uint_as_float(r[i]) * scale2 : -CUDART_INF_F;
+          r[i] = __float_as_uint(v);
+          tmax = fmaxf(tmax, v);
+        }
       }
       const float mn = fmaxf(m, tmax);
-      const float cj = mn == -CUDART_INF_F ? 1.f : expf(m - mn);
+      const float cj = mn == -CUDART_INF_F ? 1.f : ex2(m - mn);
       float rs = 0.f;
+      if (mn == -CUDART_INF_F) {
 #pragma unroll
-      for (int i = 0; i < TK; ++i) {
-        const float p = mn == -CUDART_INF_F ? 0.f : expf(__uint_as_float(r[i]) - mn);
-        r[i] = __float_as_uint(p);
-        rs += p;
+        for (int i = 0; i < TK; ++i) r[i] = 0u;
+      } else {
+#pragma unroll
+        for (int i = 0; i < TK; ++i) {
+          const float p = ex2(__uint_as_float(r[i]) - mn);
+          r[i] = __float_as_uint(p);
+          rs += p;
+        }
       }
       l = l * cj + rs;
+      const bool grew = mn != m;
       m = mn;
-      // the previous tile's P V must be done with P before P is rewritten
-      if (j > 0 && !sm_wait(S, &S.o_full[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1))) {
+      // the previous tile's P V must be done with P (and with O) first
+      if (j > 0 && !sm_wait(S, &S.o_full, (uint32_t)((j - 1) & 1))) {
         ok = false;
         break;
       }
@@ -285,39 +302,52 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float x0 = __uint_as_float(r[8 * c + 2 * e]), x1 = __uint_as_float(r[8 * c + 2 * e + 1]);
-          const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
-          hi[e] = pack2(h0, h1);
-          lo[e] = pack2(x0 - h0, x1 - h1);
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+          hi[e] = *reinterpret_cast<const uint32_t*>(&hb);
+          lo[e] = pack2(x0 - __low2float(hb), x1 - __high2float(hb));
         }
         const int off = ((c ^ (t & 7)) << 4);
         *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
+      if (j > 0 && grew) {
+        // the row's max grew: O (the sum over the earlier tiles) is rescaled
+        // in TMEM by exp(m_old - m_new) before this tile's P V adds to it
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[32];
+          tmem_ld32_nowait(o_addr + 32 * h, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * cj);
+          tmem_st32(o_addr + 32 * h, v);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
       mbar_arrive(&S.p_full);
-      // fold the previous tile's P V (its correction factor is c_prev)
-      if (j > 0) {
-        tc_fence_after();
-        fold_o(j - 1);
-      }
-      c_prev = cj;
     }
+    if (ok && !sm_wait(S, &S.o_full, (uint32_t)((ntk - 1) & 1))) ok = false;
     if (ok) {
-      if (sm_wait(S, &S.o_full[(ntk - 1) & 1], (uint32_t)(((ntk - 1) >> 1) & 1))) {
-        tc_fence_after();
-        fold_o(ntk - 1);
-      } else {
-        ok = false;
-      }
-    }
-    if (ok && t < nr) {
+      tc_fence_after();
       const float inv = 1.0f / l;
       uint4* orow = reinterpret_cast<uint4*>((__nv_bfloat16*)a.o + (size_t)(g0 + t) * a.H * HD + head * HD);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        orow[c] = make_uint4(pack2(acc[8 * c] * inv, acc[8 * c + 1] * inv), pack2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
-                             pack2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv), pack2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        tmem_ld32_nowait(o_addr + 32 * h, v);
+        tmem_wait_ld();
+        if (t < nr) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float* o = reinterpret_cast<const float*>(v) + 8 * c;
+            orow[4 * h + c] = make_uint4(pack2(o[0] * inv, o[1] * inv), pack2(o[2] * inv, o[3] * inv),
+                                         pack2(o[4] * inv, o[5] * inv), pack2(o[6] * inv, o[7] * inv));
+          }
+        }
+      }
     }
   }
   __syncthreads();

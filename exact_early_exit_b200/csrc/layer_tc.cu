@@ -77,6 +77,7 @@ struct LtArgs {
   __nv_bfloat16* u;
   __nv_bfloat16* q;
   float* Y;
+  float* Ygu;  // gate/up split slices [split][256][2F] (separate: D writes Y while gate/up tiles are reduced)
   int* sync;
   int* status;
   int d, HQ, H, hd, F, kv_layer, flags;
@@ -110,9 +111,10 @@ __device__ __forceinline__ Item item_of(const Ph& p, int it, int R) {
   return t;
 }
 
-// The four GEMM parts of this launch and the CTAs that run each.  With fewer
-// gate/up tiles than CTAs, gate/up takes the last CTAs and D and QKV the
-// others, so that the weight bytes per CTA stay close.
+// The four GEMM parts of this launch: every part is spread over all CTAs,
+// K split as the per-kernel path splits it (tc_split_count), so that each
+// CTA's share of a part's weights is a few tiles that its ring can hold
+// before the part's activations are ready.
 __device__ __forceinline__ void make_phases(const LtArgs& a, int R, int G, Ph* ph, int flags) {
   const int NK[NPH][2] = {{a.d, a.HQ}, {2 * a.F, a.d}, {a.d, a.F}, {3 * a.HQ, a.d}};
   const bool mlp = flags & LT_MLP, qkv = flags & LT_QKV;
@@ -125,17 +127,10 @@ __device__ __forceinline__ void make_phases(const LtArgs& a, int R, int G, Ph* p
     q.ntn = q.N / BM;
     q.kblocks = q.K / BK;
     q.nrt = (R + BNMAX - 1) / BNMAX;
-    q.splits = p == PH_GU ? 1 : tc_split_count(R, q.N, q.K, a.sgrid[p], TC_MAX_SPLIT);
+    q.splits = tc_split_count(R, q.N, q.K, a.sgrid[p], TC_MAX_SPLIT);
     q.items = q.ntn * q.nrt * q.splits;
     q.lo = 0;
     q.cnt = G;
-  }
-  const int ngu = ph[PH_GU].items;
-  if (mlp && ngu < G && G - ngu >= G / 4) {
-    ph[PH_GU].lo = G - ngu;
-    ph[PH_GU].cnt = ngu;
-    ph[PH_D].cnt = G - ngu;
-    ph[PH_QKV].cnt = G - ngu;
   }
 }
 __device__ __forceinline__ bool mine(const Ph& p, int c) { return p.on && c >= p.lo && c < p.lo + p.cnt; }
@@ -155,6 +150,11 @@ __device__ __forceinline__ void store4_bf16(__nv_bfloat16* p, float a, float b, 
 __device__ __forceinline__ float4 add4(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
+
+// k_epilogue's sum of the split slices adds all TC_MAX_SPLIT terms from 0,
+// the ones past the split count being +0; adding +0 once after the real
+// terms gives the same value (it only turns a -0 into +0).
+__device__ __forceinline__ float pad_zero(float y, int ns) { return ns < TC_MAX_SPLIT ? y + 0.f : y; }
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
@@ -209,20 +209,28 @@ __device__ void rows_norm(const LtArgs& a, int R, int ns, int K, const __nv_bflo
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     float4* hp = reinterpret_cast<float4*>(a.rs.h + (size_t)a.rs.row_hrow[r] * d);
     const float4* yp = reinterpret_cast<const float4*>(a.Y + (size_t)r * d);
-    float4 x[NORM_SLOTS];
+    // all slots' slice loads of one split are issued together
+    float4 x[NORM_SLOTS], ys[NORM_SLOTS];
+#pragma unroll
+    for (int c = 0; c < NORM_SLOTS; ++c) ys[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < ns; ++sp) {
+      float4 v[NORM_SLOTS];
+#pragma unroll
+      for (int c = 0; c < NORM_SLOTS; ++c) {
+        const int j = t + 128 * c;
+        v[c] = j < nv ? __ldcg(yp + sp * sstride4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int c = 0; c < NORM_SLOTS; ++c) ys[c] = add4(ys[c], v[c]);
+    }
 #pragma unroll
     for (int c = 0; c < NORM_SLOTS; ++c) {
       const int j = t + 128 * c;
       x[c] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < nv) {
-        float4 v[TC_MAX_SPLIT];
-#pragma unroll
-        for (int sp = 0; sp < TC_MAX_SPLIT; ++sp)
-          v[sp] = sp < ns ? __ldcg(yp + sp * sstride4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 ys = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int sp = 0; sp < TC_MAX_SPLIT; ++sp) ys = add4(ys, v[sp]);
-        x[c] = add4(__ldcg(hp + j), ys);
+        const float4 y4 = make_float4(pad_zero(ys[c].x, ns), pad_zero(ys[c].y, ns), pad_zero(ys[c].z, ns),
+                                      pad_zero(ys[c].w, ns));
+        x[c] = add4(__ldcg(hp + j), y4);
         hp[j] = x[c];
       }
       const float ss = warp_sum(sumsq4(x[c]));
@@ -250,53 +258,92 @@ __device__ void rows_norm(const LtArgs& a, int R, int ns, int K, const __nv_bflo
   }
 }
 
-// Sum of the split slices of output (r, n), in slice order (k_epilogue's).
-__device__ __forceinline__ float slice_sum(const float* Y, size_t sstride, int N, int ns, int r, int n) {
-  const float* p = Y + (size_t)r * N + n;
-  float v[TC_MAX_SPLIT];
-#pragma unroll
-  for (int s = 0; s < TC_MAX_SPLIT; ++s) v[s] = s < ns ? __ldcg(p + s * sstride) : 0.f;
-  float y = 0.f;
-#pragma unroll
-  for (int s = 0; s < TC_MAX_SPLIT; ++s) y += v[s];
-  return y;
-}
 
-// h += slices (the last layer before an exit: no norm follows here)
+// h += slices (the last layer before an exit: no norm follows here).  Each
+// thread takes four elements at a time and issues their slice loads together.
 __device__ void rows_resid(const LtArgs& a, int R, int ns) {
   const long long stride = (long long)gridDim.x * 128;
   const size_t sstride = (size_t)BNMAX * a.d;
-  for (long long idx = blockIdx.x * 128LL + threadIdx.x; idx < (long long)R * a.d; idx += stride) {
-    const int r = (int)(idx / a.d), n = (int)(idx % a.d);
-    float* hp = a.rs.h + (size_t)a.rs.row_hrow[r] * a.d + n;
-    *hp = __ldcg(hp) + slice_sum(a.Y, sstride, a.d, ns, r, n);
+  const long long n_el = (long long)R * a.d;
+  for (long long i0 = blockIdx.x * 128LL + threadIdx.x; i0 < n_el; i0 += 4 * stride) {
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* src[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const long long idx = i0 + e * stride;
+      src[e] = idx < n_el ? a.Y + idx : nullptr;  // Y[0][r][n] with N = d: element idx
+    }
+    for (int sp = 0; sp < ns; ++sp) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = src[e] ? __ldcg(src[e] + sp * sstride) : 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) y[e] += v[e];
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (!src[e]) continue;
+      const long long idx = i0 + e * stride;
+      const int r = (int)(idx / a.d), n = (int)(idx % a.d);
+      float* hp = a.rs.h + (size_t)a.rs.row_hrow[r] * a.d + n;
+      *hp = __ldcg(hp) + pad_zero(y[e], ns);
+    }
   }
 }
 
-// E: q, k, v from the slices, RoPE, stores (k_epilogue's EPI_QKV per element)
+// E: q, k, v from the slices, RoPE, stores (k_epilogue's EPI_QKV per
+// element); each thread takes two rotation pairs at a time.
 __device__ void qkv_epilogue(const LtArgs& a, int R, int ns) {
   const int half = a.hd / 2, N = 3 * a.HQ;
   const long long per_row = 3LL * a.H * half;
   const long long stride = (long long)gridDim.x * 128;
   const size_t sstride = (size_t)BNMAX * N;
-  for (long long idx = blockIdx.x * 128LL + threadIdx.x; idx < (long long)R * per_row; idx += stride) {
-    const int r = (int)(idx / per_row);
-    const int rem = (int)(idx % per_row);
-    const int h3 = rem / half, i = rem % half;
-    const int part = h3 / a.H, head = h3 % a.H;
-    const int c0 = h3 * a.hd + i;
-    float y0 = slice_sum(a.Y, sstride, N, ns, r, c0), y1 = slice_sum(a.Y, sstride, N, ns, r, c0 + half);
-    const int pos = a.rs.row_pos[r];
-    if (part < 2) {
-      const float2 u = rope_pair(y0, y1, a.rope[(size_t)pos * half + i]);
-      y0 = u.x;
-      y1 = u.y;
+  const long long n_el = (long long)R * per_row;
+  for (long long i0 = blockIdx.x * 128LL + threadIdx.x; i0 < n_el; i0 += 2 * stride) {
+    int r[2], c0[2];
+    bool on[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const long long idx = i0 + e * stride;
+      on[e] = idx < n_el;
+      const long long id = on[e] ? idx : i0;
+      r[e] = (int)(id / per_row);
+      const int rem = (int)(id % per_row);
+      c0[e] = (rem / half) * a.hd + rem % half;
     }
-    __nv_bfloat16* dst;
-    if (part == 0) dst = a.q + (size_t)r * a.HQ + head * a.hd;
-    else dst = (__nv_bfloat16*)a.kv.base + a.kv.offset(a.kv_layer, a.rs.row_b[r], pos, head, part - 1);
-    dst[i] = __float2bfloat16_rn(y0);
-    dst[i + half] = __float2bfloat16_rn(y1);
+    float y0[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f};
+    for (int sp = 0; sp < ns; ++sp) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float* p = a.Y + sp * sstride + (size_t)r[e] * N + c0[e];
+        v[2 * e] = __ldcg(p);
+        v[2 * e + 1] = __ldcg(p + half);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        y0[e] += v[2 * e];
+        y1[e] += v[2 * e + 1];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      if (!on[e]) continue;
+      const int h3 = c0[e] / a.hd, i = c0[e] % a.hd;
+      const int part = h3 / a.H, head = h3 % a.H;
+      float z0 = pad_zero(y0[e], ns), z1 = pad_zero(y1[e], ns);
+      const int pos = a.rs.row_pos[r[e]];
+      if (part < 2) {
+        const float2 u = rope_pair(z0, z1, a.rope[(size_t)pos * half + i]);
+        z0 = u.x;
+        z1 = u.y;
+      }
+      __nv_bfloat16* dst;
+      if (part == 0) dst = a.q + (size_t)r[e] * a.HQ + head * a.hd;
+      else dst = (__nv_bfloat16*)a.kv.base + a.kv.offset(a.kv_layer, a.rs.row_b[r[e]], pos, head, part - 1);
+      dst[i] = __float2bfloat16_rn(z0);
+      dst[i + half] = __float2bfloat16_rn(z1);
+    }
   }
 }
 
@@ -529,22 +576,59 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * BNMAX);
+          bool publish = true;
           if (p == PH_GU) {
-            // SwiGLU: the tile holds 64 gate features, then the 64 matching up features
-            for (int c0 = 0; c0 < t.nbox * BOXN; c0 += 32) {
-              uint32_t v[32];
-              tmem_ld32(tbase + (uint32_t)c0, v);
+            // SwiGLU over the tile's 64 gate and 64 matching up features, from
+            // the sum of its K splits: every split but the last to finish
+            // leaves its partial sums in memory; the last one adds them in
+            // split order to its own (still in TMEM), as k_epilogue does
+            const int ns = ph[p].splits, gn = 2 * a.F;
+            const int col = t.n0 + warp * 32 + lane;
+            const int tile_idx = t.rt * ph[PH_GU].ntn + t.tn;
+            const size_t gstride = (size_t)BNMAX * gn;
+            if (ns > 1) {
+              float* Ys = a.Ygu + (size_t)t.split * gstride;
+              for (int c0 = 0; c0 < t.nbox * BOXN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tbase + (uint32_t)c0, v);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) stile[j * BM + warp * 32 + lane] = __uint_as_float(v[j]);
-              epi_bar();
-              const int nrows = min(32, R - (t.r0 + c0));
-#pragma unroll 4
-              for (int idx = threadIdx.x; idx < nrows * (BM / 2); idx += 128) {
-                const int j = idx / (BM / 2), jj = idx % (BM / 2);
-                const float gv = stile[j * BM + jj], uv = stile[j * BM + BM / 2 + jj];
-                a.u[(size_t)(t.r0 + c0 + j) * a.F + (t.n0 / BM) * (BM / 2) + jj] = __float2bfloat16_rn(swiglu(gv, uv));
+                for (int j = 0; j < 32; ++j) {
+                  const int r = t.r0 + c0 + j;
+                  if (r < R) Ys[(size_t)r * gn + col] = __uint_as_float(v[j]);
+                }
               }
+              __threadfence();
               epi_bar();
+              if (threadIdx.x == 0)
+                s_go = atomicAdd(sync + SY_GU + ph[PH_GU].nrt * ph[PH_GU].ntn + tile_idx, 1) == ns - 1 ? 1 : 0;
+              epi_bar();
+              publish = s_go != 0;
+              if (publish) __threadfence();
+            }
+            if (publish) {
+              for (int c0 = 0; c0 < t.nbox * BOXN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tbase + (uint32_t)c0, v);
+#pragma unroll 4
+                for (int j = 0; j < 32; ++j) {
+                  const int r = t.r0 + c0 + j;
+                  float y = 0.f;
+                  for (int sp = 0; sp < ns; ++sp)
+                    y += sp == t.split ? __uint_as_float(v[j])
+                                       : (r < R ? __ldcg(a.Ygu + sp * gstride + (size_t)r * gn + col) : 0.f);
+                  stile[j * BM + warp * 32 + lane] = pad_zero(y, ns);
+                }
+                epi_bar();
+                const int nrows = min(32, R - (t.r0 + c0));
+#pragma unroll 4
+                for (int idx = threadIdx.x; idx < nrows * (BM / 2); idx += 128) {
+                  const int j = idx / (BM / 2), jj = idx % (BM / 2);
+                  const float gv = stile[j * BM + jj], uv = stile[j * BM + BM / 2 + jj];
+                  a.u[(size_t)(t.r0 + c0 + j) * a.F + (t.n0 / BM) * (BM / 2) + jj] =
+                      __float2bfloat16_rn(swiglu(gv, uv));
+                }
+                epi_bar();
+              }
             }
           } else {
             const int n = t.n0 + warp * 32 + lane;
@@ -563,13 +647,16 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
           mbar_arrive(tempty + acc);
           acc ^= 1;
           if (acc == 0) aphase ^= 1u;
-          // publish: this item's outputs, then its counter or ready flag
-          if (p == PH_GU) fence_proxy_async_global();
-          __threadfence();
-          epi_bar();
-          if (threadIdx.x == 0) {
-            if (p == PH_GU) red_release_add(sync + SY_GU + t.rt * ph[PH_GU].ntn + t.tn, 1);
-            else red_release_add(sync + (p == PH_O ? SY_O : p == PH_D ? SY_D : SY_QKV), 1);
+          // publish: this item's outputs, then its counter or (the split that
+          // finished a gate/up tile) the tile's ready flag
+          if (publish) {
+            if (p == PH_GU) fence_proxy_async_global();
+            __threadfence();
+            epi_bar();
+            if (threadIdx.x == 0) {
+              if (p == PH_GU) red_release_add(sync + SY_GU + t.rt * ph[PH_GU].ntn + t.tn, 1);
+              else red_release_add(sync + (p == PH_O ? SY_O : p == PH_D ? SY_D : SY_QKV), 1);
+            }
           }
         }
         if (!ok) break;
@@ -618,8 +705,9 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
   if (s_last) {
     // every CTA is past its last use of the sync words: zero them for the next launch
     __threadfence();
+    // gate/up ready flags, then the gate/up split arrival counters
     const int nflags = ph[PH_GU].nrt * ph[PH_GU].ntn;
-    for (int i = threadIdx.x; i < SY_GU + nflags; i += blockDim.x) sync[i] = 0;
+    for (int i = threadIdx.x; i < SY_GU + 2 * nflags; i += blockDim.x) sync[i] = 0;
   }
 }
 
@@ -627,8 +715,10 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
 
 size_t layer_tc_sync_ints(int max_rows, int F) {
   const size_t nrt = ((size_t)max_rows + BNMAX - 1) / BNMAX;
-  return SY_GU + nrt * (size_t)(2 * F / BM);
+  return SY_GU + 2 * nrt * (size_t)(2 * F / BM);
 }
+
+size_t layer_tc_gu_floats(int F) { return (size_t)TC_MAX_SPLIT * BNMAX * 2 * F; }
 
 bool layer_tc_supported(int d, int HQ, int hd, int F, bool bf16) {
   return bf16 && hd == 64 && d % BM == 0 && HQ % BM == 0 && F % 64 == 0 && (2 * F) % BM == 0 && d <= 2048 &&
@@ -689,6 +779,7 @@ nv_status layer_tc_launch(TcPlanCache* plans, const LayerTcRun& r, cudaStream_t 
   a.u = (__nv_bfloat16*)r.u;
   a.q = (__nv_bfloat16*)r.q;
   a.Y = r.Y;
+  a.Ygu = r.Ygu;
   a.sync = r.sync;
   a.status = r.status;
   a.d = d;

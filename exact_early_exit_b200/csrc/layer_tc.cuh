@@ -18,6 +18,9 @@ enum LayerTcFlags : int {
 // Integers of device scratch one launch site needs (counters and per-tile
 // ready flags); zero between launches.
 size_t layer_tc_sync_ints(int max_rows, int F);
+// floats of the gate/up split-slice buffer (gate/up splits only when all
+// rows fit one 256-row tile)
+size_t layer_tc_gu_floats(int F);
 
 struct LayerTcRun {
   // weights (bf16): this layer's O, gate/up, down and norm gains; the QKV
@@ -31,6 +34,7 @@ struct LayerTcRun {
   const float2* rope;
   void *o, *act, *u, *q;
   float* Y;
+  float* Ygu;  // gate/up split slices: layer_tc_gu_floats(F) floats
   int* sync;
   int* status;
   int d, HQ, H, hd, F;

@@ -141,6 +141,7 @@ struct nv_state {
   int* tile_counters = nullptr;
   int* lt_sync = nullptr;      // [L][lt_sync_ints] counters of the persistent layer kernel
   size_t lt_sync_ints = 0;
+  float* lt_ygu = nullptr;     // its gate/up split slices
   float *Y = nullptr, *attn_part = nullptr, *head_part = nullptr;
   size_t Y_elems = 0;
   int head_nblk = 0, kv_splits = 1, row_groups = 1;
@@ -216,6 +217,7 @@ struct LayerIO {
   int* status;
   int* lt_sync;        // non-null: decode/flush layers on the persistent layer kernel
   size_t lt_sync_ints;
+  float* lt_ygu;
 };
 
 // Per-kernel event timing for nv_decode_step_profiled (null when capturing).
@@ -286,6 +288,7 @@ LayerTcRun layer_tc_args(nv_model* M, int layer, const LayerIO& io, bool mlp, co
   r.u = io.u;
   r.q = io.q;
   r.Y = io.Y;
+  r.Ygu = io.lt_ygu;
   r.sync = io.lt_sync + (size_t)layer * io.lt_sync_ints;
   r.status = io.status;
   r.d = M->d;
@@ -352,12 +355,11 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
                   const void* pf, long long pf_bytes) {
     e.mode = mode;
     e.N = (int)N;
-    // gate/up is never split: its SwiGLU epilogue runs in the GEMM kernel (one
-    // launch fewer), and the persistent decode-layer kernel computes it the
-    // same way, so the two decode paths agree bit for bit; with fewer tiles
-    // (QKV: 36) splitting K is faster (measured on B200 with the 1.5B model:
-    // unsplit gate/up +1%, unsplit QKV -12% decode tokens/s)
-    const bool split = io.split_k && N / 128 < 64 && mode != EPI_SWIGLU;
+    // decode and flush may split K when the rows fit one tile and the feature
+    // tiles cannot fill the GPU (tc_split_count); the persistent decode-layer
+    // kernel splits every part the same way, so the two decode paths agree
+    // bit for bit
+    const bool split = io.split_k;
     timed(prof, launches, gemm_launch_count(M->gemm_kind, bf, split, &e), NV_K_GEMM,
           N * K * es + R * K * es + out_bytes,
           2 * R * N * K, [&] {
@@ -503,6 +505,7 @@ LayerIO state_io(nv_state* s) {
   io.status = s->status;
   io.lt_sync = s->lt_sync;
   io.lt_sync_ints = s->lt_sync_ints;
+  io.lt_ygu = s->lt_ygu;
   return io;
 }
 
@@ -1157,6 +1160,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   if (M->layer_kernel) {
     s->lt_sync_ints = layer_tc_sync_ints(s->max_rows, M->F);
     A((void**)&s->lt_sync, (size_t)M->L * s->lt_sync_ints * 4);
+    A((void**)&s->lt_ygu, layer_tc_gu_floats(M->F) * 4);
   }
   A(&s->q, (size_t)s->max_rows * HQ * esz);
   A(&s->o, (size_t)s->max_rows * HQ * esz);
