@@ -69,14 +69,20 @@ template <> __device__ __forceinline__ float rnd<__nv_bfloat16>(float x) {
 // per-element arithmetic shared by every kernel that performs the step, so
 // that two kernels doing the same step round identically
 // ---------------------------------------------------------------------------
+// (each written with explicit rounding intrinsics, so the compiler cannot
+// contract or reorder it differently in different kernels)
 // rotate-half RoPE of the pair (y0, y1) by (cos, sin)
 __device__ __forceinline__ float2 rope_pair(float y0, float y1, float2 cs) {
-  return make_float2(y0 * cs.x - y1 * cs.y, y1 * cs.x + y0 * cs.y);
+  return make_float2(__fmaf_rn(y0, cs.x, -__fmul_rn(y1, cs.y)), __fmaf_rn(y1, cs.x, __fmul_rn(y0, cs.y)));
 }
 // SwiGLU: silu(g) * u
-__device__ __forceinline__ float swiglu(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+__device__ __forceinline__ float swiglu(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
 // sum of squares of four values (one float4 of an RMSNorm row)
-__device__ __forceinline__ float sumsq4(float4 x) { return x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w; }
+__device__ __forceinline__ float sumsq4(float4 x) {
+  return __fmaf_rn(x.w, x.w, __fmaf_rn(x.z, x.z, __fmaf_rn(x.y, x.y, __fmul_rn(x.x, x.x))));
+}
 
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
