@@ -54,9 +54,13 @@ using namespace tc;
 
 constexpr int LT_THREADS = 224;
 constexpr int W_WARP = 4, MMA_WARP = 5, X_WARP = 6;
-constexpr int STAGES = 4;   // stages at the largest row tile (256 rows)
-constexpr int MAXST = 12;   // stages when the row tile is small
-constexpr int SMEM_TILES = STAGES * (A_BYTES + BNMAX * BK * 2);
+// Separate rings for weight tiles (16 KB each) and activation tiles (the
+// row tile's boxes): the activations come from L2 right after their producer
+// finishes, so three stages hide them, and the rest of the shared memory goes
+// to the weight ring, which keeps streaming while a part waits for its input.
+constexpr int SMEM_TILES = 4 * (A_BYTES + BNMAX * BK * 2);  // 192 KB for both rings
+constexpr int XST = 3;      // activation stages
+constexpr int MAXST = 16;   // weight stages at most (used for small row tiles)
 constexpr int EPI_BYTES = 32 * BM * 4;  // fp32 staging tile [32 rows][128 features]
 constexpr int BAR_BYTES = 512;
 constexpr int SMEM_BYTES = SMEM_TILES + BAR_BYTES + EPI_BYTES + 1024;
@@ -209,19 +213,26 @@ __device__ void rows_norm(const LtArgs& a, int R, int ns, int K, const __nv_bflo
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     float4* hp = reinterpret_cast<float4*>(a.rs.h + (size_t)a.rs.row_hrow[r] * d);
     const float4* yp = reinterpret_cast<const float4*>(a.Y + (size_t)r * d);
-    // all slots' slice loads of one split are issued together
+    // the slice loads of four splits and every slot are issued together,
+    // then added in split order
     float4 x[NORM_SLOTS], ys[NORM_SLOTS];
 #pragma unroll
     for (int c = 0; c < NORM_SLOTS; ++c) ys[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < ns; ++sp) {
-      float4 v[NORM_SLOTS];
+    for (int s0 = 0; s0 < ns; s0 += 4) {
+      float4 v[4][NORM_SLOTS];
 #pragma unroll
-      for (int c = 0; c < NORM_SLOTS; ++c) {
-        const int j = t + 128 * c;
-        v[c] = j < nv ? __ldcg(yp + sp * sstride4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-      for (int c = 0; c < NORM_SLOTS; ++c) ys[c] = add4(ys[c], v[c]);
+        for (int c = 0; c < NORM_SLOTS; ++c) {
+          const int j = t + 128 * c;
+          v[q][c] = (s0 + q < ns && j < nv) ? __ldcg(yp + (s0 + q) * sstride4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (s0 + q < ns) {
+#pragma unroll
+          for (int c = 0; c < NORM_SLOTS; ++c) ys[c] = add4(ys[c], v[q][c]);
+        }
     }
 #pragma unroll
     for (int c = 0; c < NORM_SLOTS; ++c) {
@@ -273,12 +284,18 @@ __device__ void rows_resid(const LtArgs& a, int R, int ns) {
       const long long idx = i0 + e * stride;
       src[e] = idx < n_el ? a.Y + idx : nullptr;  // Y[0][r][n] with N = d: element idx
     }
-    for (int sp = 0; sp < ns; ++sp) {
-      float v[4];
+    for (int s0 = 0; s0 < ns; s0 += 8) {
+      float v[8][4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = src[e] ? __ldcg(src[e] + sp * sstride) : 0.f;
+      for (int q = 0; q < 8; ++q)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) y[e] += v[e];
+        for (int e = 0; e < 4; ++e) v[q][e] = (s0 + q < ns && src[e]) ? __ldcg(src[e] + (s0 + q) * sstride) : 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (s0 + q < ns) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) y[e] += v[q][e];
+        }
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -312,19 +329,26 @@ __device__ void qkv_epilogue(const LtArgs& a, int R, int ns) {
       c0[e] = (rem / half) * a.hd + rem % half;
     }
     float y0[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f};
-    for (int sp = 0; sp < ns; ++sp) {
-      float v[4];
+    for (int s0 = 0; s0 < ns; s0 += 8) {
+      float v[8][4];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float* p = a.Y + sp * sstride + (size_t)r[e] * N + c0[e];
-        v[2 * e] = __ldcg(p);
-        v[2 * e + 1] = __ldcg(p + half);
-      }
+      for (int q = 0; q < 8; ++q)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        y0[e] += v[2 * e];
-        y1[e] += v[2 * e + 1];
-      }
+        for (int e = 0; e < 2; ++e) {
+          const float* p = a.Y + (s0 + q) * sstride + (size_t)r[e] * N + c0[e];
+          const bool ld = s0 + q < ns && on[e];
+          v[q][2 * e] = ld ? __ldcg(p) : 0.f;
+          v[q][2 * e + 1] = ld ? __ldcg(p + half) : 0.f;
+        }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (s0 + q < ns) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            y0[e] += v[q][2 * e];
+            y1[e] += v[q][2 * e + 1];
+          }
+        }
     }
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -393,21 +417,26 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
 
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int nbmax = (min(R, BNMAX) + BOXN - 1) / BOXN;
-  const int stage_bytes = A_BYTES + nbmax * BOX_BYTES;
-  const int nst = min(MAXST, SMEM_TILES / stage_bytes);
+  const int xstage_bytes = nbmax * BOX_BYTES;
+  const int nwst = min(MAXST, (SMEM_TILES - XST * xstage_bytes) / A_BYTES);
+  unsigned char* xring = smem + nwst * A_BYTES;
   uint64_t* fullw = (uint64_t*)(smem + SMEM_TILES);
-  uint64_t* fullx = fullw + MAXST;
-  uint64_t* empty = fullx + MAXST;
-  uint64_t* tfull = empty + MAXST;
+  uint64_t* emptyw = fullw + MAXST;
+  uint64_t* fullx = emptyw + MAXST;
+  uint64_t* emptyx = fullx + XST;
+  uint64_t* tfull = emptyx + XST;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   float* stile = (float*)(smem + SMEM_TILES + BAR_BYTES);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < nst; ++s) {
+    for (int s = 0; s < nwst; ++s) {
       mbar_init(fullw + s, 1);
+      mbar_init(emptyw + s, 1);
+    }
+    for (int s = 0; s < XST; ++s) {
       mbar_init(fullx + s, 1);
-      mbar_init(empty + s, 1);
+      mbar_init(emptyx + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(tfull + s, 1);
@@ -430,11 +459,13 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
   volatile int* abort_flag = &s_abort;
 
   if (warp == W_WARP || warp == X_WARP) {
-    // producers: the same walk over (part, item, K block) stages; warp 4
-    // fills the weight half of each stage, warp 6 the activation half
+    // producers: the same walk over (part, item, K block); warp 4 fills the
+    // weight ring, warp 6 the activation ring
     if (lane == 0) {
       const bool isw = warp == W_WARP;
       uint64_t* full = isw ? fullw : fullx;
+      uint64_t* empty = isw ? emptyw : emptyx;
+      const int nst = isw ? nwst : XST;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -464,14 +495,14 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
               break;
             }
             issued[stage] = (int)phase;
-            unsigned char* sa = smem + stage * stage_bytes;
             if (isw) {
               mbar_expect_tx(full + stage, (uint32_t)A_BYTES);
-              tma_load_2d(sa, wmap[p], full + stage, kb * BK, t.n0);
+              tma_load_2d(smem + stage * A_BYTES, wmap[p], full + stage, kb * BK, t.n0);
             } else {
+              unsigned char* sx = xring + stage * xstage_bytes;
               mbar_expect_tx(full + stage, (uint32_t)(t.nbox * BOX_BYTES));
               for (int j = 0; j < t.nbox; ++j)
-                tma_load_2d(sa + A_BYTES + j * BOX_BYTES, xmap[p], full + stage, kb * BK, t.r0 + j * BOXN);
+                tma_load_2d(sx + j * BOX_BYTES, xmap[p], full + stage, kb * BK, t.r0 + j * BOXN);
             }
             if (++stage == nst) {
               stage = 0;
@@ -513,8 +544,8 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
     }
   } else if (warp == MMA_WARP) {
     if (lane == 0) {
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, aphase = 0;
+      int ws = 0, xs = 0, acc = 0;
+      uint32_t wphase = 0, xphase = 0, aphase = 0;
       bool ok = true, issued_any = false;
       for (int p = 0; p < NPH && ok; ++p) {
         if (!mine(ph[p], c)) continue;
@@ -528,21 +559,26 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
           tc_fence_after();
           const uint32_t dt = tmem + (uint32_t)(acc * BNMAX);
           for (int kb = t.kb0; kb < t.kb1; ++kb) {
-            if (!mbar_wait(fullw + stage, phase, abort_flag) || !mbar_wait(fullx + stage, phase, abort_flag)) {
+            if (!mbar_wait(fullw + ws, wphase, abort_flag) || !mbar_wait(fullx + xs, xphase, abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t ad = sw128_desc(smem_u32(smem + stage * stage_bytes));
-            const uint64_t bd = sw128_desc(smem_u32(smem + stage * stage_bytes + A_BYTES));
+            const uint64_t ad = sw128_desc(smem_u32(smem + ws * A_BYTES));
+            const uint64_t bd = sw128_desc(smem_u32(xring + xs * xstage_bytes));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
               umma(dt, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (kb > t.kb0 || kk > 0) ? 1u : 0u);
             issued_any = true;
-            umma_commit(empty + stage);
-            if (++stage == nst) {
-              stage = 0;
-              phase ^= 1u;
+            umma_commit(emptyw + ws);
+            umma_commit(emptyx + xs);
+            if (++ws == nwst) {
+              ws = 0;
+              wphase ^= 1u;
+            }
+            if (++xs == XST) {
+              xs = 0;
+              xphase ^= 1u;
             }
           }
           if (!ok) break;
