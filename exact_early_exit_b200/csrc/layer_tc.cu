@@ -639,6 +639,8 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
                 s_go = atomicAdd(sync + SY_GU + ph[PH_GU].nrt * ph[PH_GU].ntn + tile_idx, 1) == ns - 1 ? 1 : 0;
               epi_bar();
               publish = s_go != 0;
+              // every thread has read the decision before thread 0 reuses s_go
+              epi_bar();
               if (publish) __threadfence();
             }
             if (publish) {
