@@ -310,9 +310,12 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
         *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      if (j > 0 && grew) {
-        // the row's max grew: O (the sum over the earlier tiles) is rescaled
-        // in TMEM by exp(m_old - m_new) before this tile's P V adds to it
+      // a row whose max grew: O (the sum over the earlier tiles) is rescaled
+      // in TMEM by exp(m_old - m_new) before this tile's P V adds to it.  The
+      // TMEM loads and stores are warp-collective: a warp with any such row
+      // rescales all its rows, the others by exactly 1.
+      if (__any_sync(0xffffffffu, j > 0 && grew)) {
+        const float f = grew ? cj : 1.0f;
         tc_fence_after();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -320,7 +323,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
           tmem_ld32_nowait(o_addr + 32 * h, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * cj);
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
           tmem_st32(o_addr + 32 * h, v);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
