@@ -75,9 +75,14 @@ template <> __device__ __forceinline__ float rnd<__nv_bfloat16>(float x) {
 __device__ __forceinline__ float2 rope_pair(float y0, float y1, float2 cs) {
   return make_float2(__fmaf_rn(y0, cs.x, -__fmul_rn(y1, cs.y)), __fmaf_rn(y1, cs.x, __fmul_rn(y0, cs.y)));
 }
-// SwiGLU: silu(g) * u
+// SwiGLU: silu(g) * u = g / (1 + 2^(-g log2 e)) * u, with the hardware's
+// base-2 exponential and reciprocal (PTX ex2.approx / rcp.approx, relative
+// errors near 2^-22; the product is rounded to bf16 afterwards)
 __device__ __forceinline__ float swiglu(float g, float u) {
-  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(__fmul_rn(g, -1.4426950408889634f)));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(__fadd_rn(1.0f, e)));
+  return __fmul_rn(__fmul_rn(g, r), u);
 }
 // sum of squares of four values (one float4 of an RMSNorm row)
 __device__ __forceinline__ float sumsq4(float4 x) {

@@ -193,7 +193,7 @@ __device__ __noinline__ bool wait_geq(const int* p, int target, int* gabort, vol
         return false;
       }
     }
-    __nanosleep(32);
+    if (i >= 512) __nanosleep(64);  // a tight poll first: most waits end within a few microseconds
   }
 }
 
@@ -213,11 +213,15 @@ __device__ void rows_norm(const LtArgs& a, int R, int ns, int K, const __nv_bflo
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     float4* hp = reinterpret_cast<float4*>(a.rs.h + (size_t)a.rs.row_hrow[r] * d);
     const float4* yp = reinterpret_cast<const float4*>(a.Y + (size_t)r * d);
-    // the slice loads of four splits and every slot are issued together,
-    // then added in split order
-    float4 x[NORM_SLOTS], ys[NORM_SLOTS];
+    // the row's residual and the slices of four splits for every slot are
+    // loaded together, then added in split order
+    float4 x[NORM_SLOTS], ys[NORM_SLOTS], hv[NORM_SLOTS];
 #pragma unroll
-    for (int c = 0; c < NORM_SLOTS; ++c) ys[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < NORM_SLOTS; ++c) {
+      const int j = t + 128 * c;
+      ys[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      hv[c] = j < nv ? __ldcg(hp + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     for (int s0 = 0; s0 < ns; s0 += 4) {
       float4 v[4][NORM_SLOTS];
 #pragma unroll
@@ -241,7 +245,7 @@ __device__ void rows_norm(const LtArgs& a, int R, int ns, int K, const __nv_bflo
       if (j < nv) {
         const float4 y4 = make_float4(pad_zero(ys[c].x, ns), pad_zero(ys[c].y, ns), pad_zero(ys[c].z, ns),
                                       pad_zero(ys[c].w, ns));
-        x[c] = add4(__ldcg(hp + j), y4);
+        x[c] = add4(hv[c], y4);
         hp[j] = x[c];
       }
       const float ss = warp_sum(sumsq4(x[c]));
@@ -309,64 +313,86 @@ __device__ void rows_resid(const LtArgs& a, int R, int ns) {
 }
 
 // E: q, k, v from the slices, RoPE, stores (k_epilogue's EPI_QKV per
-// element); each thread takes two rotation pairs at a time.
+// element).  A thread takes four consecutive rotation pairs of one head (16
+// bytes of each half), two such quads at a time: every slice load and the
+// row indices are issued first, the RoPE table (which needs the position)
+// second.
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, float a, float b, float c, float d) {
+  store4_bf16(p, a, b, c, d);
+}
 __device__ void qkv_epilogue(const LtArgs& a, int R, int ns) {
-  const int half = a.hd / 2, N = 3 * a.HQ;
-  const long long per_row = 3LL * a.H * half;
+  const int half = a.hd / 2, N = 3 * a.HQ, qph = half / 4;  // quads per head
+  const int per_row = 3 * a.H * qph;
   const long long stride = (long long)gridDim.x * 128;
-  const size_t sstride = (size_t)BNMAX * N;
-  const long long n_el = (long long)R * per_row;
-  for (long long i0 = blockIdx.x * 128LL + threadIdx.x; i0 < n_el; i0 += 2 * stride) {
-    int r[2], c0[2];
+  const size_t sstride4 = (size_t)BNMAX * N / 4;
+  const long long n_q = (long long)R * per_row;
+  const float4* Y4 = reinterpret_cast<const float4*>(a.Y);
+  for (long long q0 = blockIdx.x * 128LL + threadIdx.x; q0 < n_q; q0 += 2 * stride) {
+    int r[2], c0[2], h3[2];
     bool on[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const long long idx = i0 + e * stride;
-      on[e] = idx < n_el;
-      const long long id = on[e] ? idx : i0;
+      const long long qd = q0 + e * stride;
+      on[e] = qd < n_q;
+      const long long id = on[e] ? qd : q0;
       r[e] = (int)(id / per_row);
       const int rem = (int)(id % per_row);
-      c0[e] = (rem / half) * a.hd + rem % half;
+      h3[e] = rem / qph;
+      c0[e] = h3[e] * a.hd + (rem % qph) * 4;
     }
-    float y0[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f};
-    for (int s0 = 0; s0 < ns; s0 += 8) {
-      float v[8][4];
+    int pos[2], rb[2];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+    for (int e = 0; e < 2; ++e) {
+      pos[e] = a.rs.row_pos[r[e]];
+      rb[e] = a.rs.row_b[r[e]];
+    }
+    float4 y0[2], y1[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) y0[e] = y1[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < ns; s0 += 4) {
+      float4 v[4][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float* p = a.Y + (s0 + q) * sstride + (size_t)r[e] * N + c0[e];
+          const float4* p = Y4 + (s0 + q) * sstride4 + ((size_t)r[e] * N + c0[e]) / 4;
           const bool ld = s0 + q < ns && on[e];
-          v[q][2 * e] = ld ? __ldcg(p) : 0.f;
-          v[q][2 * e + 1] = ld ? __ldcg(p + half) : 0.f;
+          v[q][2 * e] = ld ? __ldcg(p) : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[q][2 * e + 1] = ld ? __ldcg(p + half / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+      for (int q = 0; q < 4; ++q)
         if (s0 + q < ns) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            y0[e] += v[q][2 * e];
-            y1[e] += v[q][2 * e + 1];
+            y0[e] = add4(y0[e], v[q][2 * e]);
+            y1[e] = add4(y1[e], v[q][2 * e + 1]);
           }
         }
     }
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       if (!on[e]) continue;
-      const int h3 = c0[e] / a.hd, i = c0[e] % a.hd;
-      const int part = h3 / a.H, head = h3 % a.H;
-      float z0 = pad_zero(y0[e], ns), z1 = pad_zero(y1[e], ns);
-      const int pos = a.rs.row_pos[r[e]];
+      const int part = h3[e] / a.H, head = h3[e] % a.H, i = c0[e] % a.hd;
+      float z0[4] = {pad_zero(y0[e].x, ns), pad_zero(y0[e].y, ns), pad_zero(y0[e].z, ns), pad_zero(y0[e].w, ns)};
+      float z1[4] = {pad_zero(y1[e].x, ns), pad_zero(y1[e].y, ns), pad_zero(y1[e].z, ns), pad_zero(y1[e].w, ns)};
       if (part < 2) {
-        const float2 u = rope_pair(z0, z1, a.rope[(size_t)pos * half + i]);
-        z0 = u.x;
-        z1 = u.y;
+        const float4* cs4 = reinterpret_cast<const float4*>(a.rope + (size_t)pos[e] * half + i);
+        const float4 ca = cs4[0], cb = cs4[1];
+        const float2 cs[4] = {make_float2(ca.x, ca.y), make_float2(ca.z, ca.w), make_float2(cb.x, cb.y),
+                              make_float2(cb.z, cb.w)};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 u = rope_pair(z0[k], z1[k], cs[k]);
+          z0[k] = u.x;
+          z1[k] = u.y;
+        }
       }
       __nv_bfloat16* dst;
       if (part == 0) dst = a.q + (size_t)r[e] * a.HQ + head * a.hd;
-      else dst = (__nv_bfloat16*)a.kv.base + a.kv.offset(a.kv_layer, a.rs.row_b[r[e]], pos, head, part - 1);
-      dst[i] = __float2bfloat16_rn(z0);
-      dst[i + half] = __float2bfloat16_rn(z1);
+      else dst = (__nv_bfloat16*)a.kv.base + a.kv.offset(a.kv_layer, rb[e], pos[e], head, part - 1);
+      store_bf16x4(dst + i, z0[0], z0[1], z0[2], z0[3]);
+      store_bf16x4(dst + i + half, z1[0], z1[1], z1[2], z1[3]);
     }
   }
 }
@@ -647,15 +673,23 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
               for (int c0 = 0; c0 < t.nbox * BOXN; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(tbase + (uint32_t)c0, v);
-#pragma unroll 4
-                for (int j = 0; j < 32; ++j) {
-                  const int r = t.r0 + c0 + j;
-                  float y = 0.f;
-                  for (int sp = 0; sp < ns; ++sp)
-                    y += sp == t.split ? __uint_as_float(v[j])
-                                       : (r < R ? __ldcg(a.Ygu + sp * gstride + (size_t)r * gn + col) : 0.f);
-                  stile[j * BM + warp * 32 + lane] = pad_zero(y, ns);
+                // y = 0 + slice 0 + slice 1 + ..., each other split's 32 rows
+                // loaded together; v (this split, from TMEM) enters at its turn
+                float y[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[j] = 0.f;
+                for (int sp = 0; sp < ns; ++sp) {
+                  if (sp == t.split) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(v[j]);
+                  } else {
+                    const float* src = a.Ygu + sp * gstride + (size_t)(t.r0 + c0) * gn + col;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] += t.r0 + c0 + j < R ? __ldcg(src + (size_t)j * gn) : 0.f;
+                  }
                 }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) stile[j * BM + warp * 32 + lane] = pad_zero(y[j], ns);
                 epi_bar();
                 const int nrows = min(32, R - (t.r0 + c0));
 #pragma unroll 4
@@ -688,8 +722,9 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
           // publish: this item's outputs, then its counter or (the split that
           // finished a gate/up tile) the tile's ready flag
           if (publish) {
+            // the barrier orders every thread's stores before thread 0's
+            // release; TMA (the async proxy) reads the gate/up output
             if (p == PH_GU) fence_proxy_async_global();
-            __threadfence();
             epi_bar();
             if (threadIdx.x == 0) {
               if (p == PH_GU) red_release_add(sync + SY_GU + t.rt * ph[PH_GU].ntn + t.tn, 1);
@@ -717,7 +752,6 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
           rows_norm(a, R, ph[p].splits, ph[p].K, g, s_red);
           // publish the normed rows (TMA reads them in other CTAs)
           fence_proxy_async_global();
-          __threadfence();
           epi_bar();
           int mine_rows = 0;
           for (int r = blockIdx.x; r < R; r += gridDim.x) ++mine_rows;
