@@ -15,7 +15,8 @@ from typing import Optional, Sequence
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libnvium.so")
+# NVIUM_LIB points the binding at another build of the library (the same ABI)
+LIB_PATH = os.environ.get("NVIUM_LIB") or os.path.join(_HERE, "libnvium.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "nvium.h")
 
 NV_OK = 0

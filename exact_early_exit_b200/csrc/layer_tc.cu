@@ -87,10 +87,6 @@ struct LtArgs {
   int d, HQ, H, hd, F, kv_layer, flags;
   float eps;
   int sgrid[NPH];  // grid whose split count a phase reproduces (the per-kernel path's GEMM grid)
-  // the next layer's launch (same rows): its flags, and whether to pull its
-  // weight tiles into L2 once this launch's own loads are issued
-  int next_flags, pf_next;
-  long long pf_kv_limit;  // prefetch only while the next attention reads fewer K/V bytes than this
 };
 
 struct Ph {
@@ -401,9 +397,7 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
     k_layer_tc(const __grid_constant__ CUtensorMap m_wo, const __grid_constant__ CUtensorMap m_wgu,
                const __grid_constant__ CUtensorMap m_wd, const __grid_constant__ CUtensorMap m_wqkv,
                const __grid_constant__ CUtensorMap m_xo, const __grid_constant__ CUtensorMap m_xact,
-               const __grid_constant__ CUtensorMap m_xu, const __grid_constant__ CUtensorMap n_wo,
-               const __grid_constant__ CUtensorMap n_wgu, const __grid_constant__ CUtensorMap n_wd,
-               const __grid_constant__ CUtensorMap n_wqkv, LtArgs a) {
+               const __grid_constant__ CUtensorMap m_xu, LtArgs a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort, s_go, s_last;
@@ -533,30 +527,6 @@ __global__ void __launch_bounds__(LT_THREADS, 1)
             if (++stage == nst) {
               stage = 0;
               phase ^= 1u;
-            }
-          }
-        }
-      }
-      if (ok && isw && a.pf_next) {
-        // every weight tile of this launch is requested: pull the tiles this
-        // CTA will stream in the next layer's launch (same rows, same
-        // schedule) into L2, unless the next attention's K/V reads would
-        // evict them first
-        long long kv = 0;
-        const long long per_pos = 4LL * a.HQ;
-        for (int b = 0; b < a.rs.B && kv < a.pf_kv_limit; ++b) {
-          const int s0 = a.rs.seq_start[b], s1 = a.rs.seq_start[b + 1];
-          if (s1 > s0) kv += (long long)(a.rs.row_pos[s1 - 1] + 1) * per_pos;
-        }
-        if (kv < a.pf_kv_limit) {
-          const CUtensorMap* nmap[NPH] = {&n_wo, &n_wgu, &n_wd, &n_wqkv};
-          Ph nx[NPH];
-          make_phases(a, R, G, nx, a.next_flags);
-          for (int p = 0; p < NPH; ++p) {
-            if (!mine(nx[p], c)) continue;
-            for (int it = c - nx[p].lo; it < nx[p].items; it += nx[p].cnt) {
-              const Item t = item_of(nx[p], it, R);
-              for (int kb = t.kb0; kb < t.kb1; ++kb) tma_prefetch_l2_2d(nmap[p], kb * BK, t.n0);
             }
           }
         }
@@ -828,17 +798,6 @@ nv_status layer_tc_launch(TcPlanCache* plans, const LayerTcRun& r, cudaStream_t 
   NV_TRY(tc_map(plans, r.act, (uint64_t)d, (uint64_t)max_rows, (uint64_t)d, BOXN, &m[5]));
   if (!mlp) m[0] = m[1] = m[2] = m[3], m[4] = m[6] = m[5];
   if (!qkv) m[3] = m[0];
-  // the next layer's weights (prefetched into L2 only)
-  CUtensorMap nm[4] = {m[0], m[1], m[2], m[3]};
-  const bool pf = r.next_w_o && (r.flags & LT_NORM2);
-  if (pf) {
-    NV_TRY(tc_map(plans, r.next_w_o, (uint64_t)HQ, (uint64_t)d, (uint64_t)HQ, BM, &nm[0]));
-    NV_TRY(tc_map(plans, r.next_w_gu, (uint64_t)d, (uint64_t)(2 * F), (uint64_t)d, BM, &nm[1]));
-    NV_TRY(tc_map(plans, r.next_w_d, (uint64_t)F, (uint64_t)d, (uint64_t)F, BM, &nm[2]));
-    if (r.next_flags & LT_QKV)
-      NV_TRY(tc_map(plans, r.next_w_qkv, (uint64_t)d, (uint64_t)(3 * HQ), (uint64_t)d, BM, &nm[3]));
-    else nm[3] = nm[0];
-  }
 
   const int G = tc_sm_count();
   LtArgs a{};
@@ -862,9 +821,6 @@ nv_status layer_tc_launch(TcPlanCache* plans, const LayerTcRun& r, cudaStream_t 
   a.kv_layer = r.kv_layer;
   a.flags = r.flags;
   a.eps = r.eps;
-  a.next_flags = pf ? r.next_flags : 0;
-  a.pf_next = pf ? 1 : 0;
-  a.pf_kv_limit = 48LL << 20;
   // the split counts of the per-kernel path: its GEMM grid is the SM count,
   // capped by the work items it could have (feature tiles x row tiles x 16)
   const int nrt_max = (max_rows + BNMAX - 1) / BNMAX;
@@ -874,7 +830,7 @@ nv_status layer_tc_launch(TcPlanCache* plans, const LayerTcRun& r, cudaStream_t 
     a.sgrid[p] = most < G ? (int)most : G;
   }
   cudaError_t e = launch_k(k_layer_tc, dim3(G), dim3(LT_THREADS), SMEM_BYTES, st, m[0], m[1], m[2], m[3], m[4], m[5],
-                           m[6], nm[0], nm[1], nm[2], nm[3], a);
+                           m[6], a);
   if (e != cudaSuccess) {
     set_error(std::string("decode-layer kernel launch: ") + cudaGetErrorString(e));
     return NV_ERR_CUDA;

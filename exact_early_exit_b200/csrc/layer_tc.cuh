@@ -40,10 +40,6 @@ struct LayerTcRun {
   int d, HQ, H, hd, F;
   float eps;
   int flags;
-  // with LT_NORM2: the next layer's launch (same rows), whose weight tiles
-  // this launch pulls into L2 after its own (null: no prefetch)
-  const void *next_w_o, *next_w_gu, *next_w_d, *next_w_qkv;
-  int next_flags;
 };
 
 // True when the model's shapes fit the kernel (bf16, head_dim 64, d and

@@ -57,11 +57,15 @@ bool tc_attention_enabled() {
   return !(ev && (std::string(ev) == "simt" || std::string(ev) == "mma"));
 }
 
-// decode and flush layers run as one persistent kernel after attention
-// unless NVIUM_LAYER_KERNEL=0 selects the per-kernel path (kept for comparison)
+// NVIUM_LAYER_KERNEL=1: decode and flush layers run as one persistent kernel
+// after attention (layer_tc.cu), which gives the same bits as the default
+// per-kernel path; measured on B200 it is slower (its seven cross-CTA
+// hand-offs per layer cost more than the per-kernel path's launches, which
+// overlap through programmatic dependent launch and pull the next GEMM's
+// weights into L2), so it is an option, not the default
 bool layer_kernel_enabled() {
   const char* ev = std::getenv("NVIUM_LAYER_KERNEL");
-  return !(ev && ev[0] == '0');
+  return ev && ev[0] == '1';
 }
 
 constexpr int kTileCounters = 1024;  // >= N/128 of any split GEMM
@@ -272,8 +276,6 @@ void timed(Prof* prof, long long* launches, int nlaunch, int kind, long long byt
 // gate/up + SwiGLU, down + residual.  With `next_norm` (the next layer's
 // attention-norm gain, when it runs the same rows) the down projection's
 // residual is followed by that norm, so act is ready for the next layer.
-const void* next_norm_in_block(const nv_model* M, int layer);
-
 // The persistent decode-layer kernel's arguments for layer `layer`:
 // MLP part of this layer (when `mlp`), then the next layer's norm and QKV
 // when it runs the same rows (`next_norm`), or this layer's QKV alone.
@@ -308,17 +310,6 @@ LayerTcRun layer_tc_args(nv_model* M, int layer, const LayerIO& io, bool mlp, co
       r.norm2 = next_norm;
       r.w_qkv = M->layers[layer + 1].w_qkv;
       r.kv_layer = layer + 1;
-      // the next layer's launch runs the same rows: its weights can be
-      // pulled into L2 while this one finishes and the next attention runs
-      const LayerDev& Nw = M->layers[layer + 1];
-      r.next_w_o = Nw.w_o;
-      r.next_w_gu = Nw.w_gu;
-      r.next_w_d = Nw.w_d;
-      r.next_flags = LT_MLP;
-      if (next_norm_in_block(M, layer + 1)) {
-        r.next_flags |= LT_NORM2 | LT_QKV;
-        r.next_w_qkv = M->layers[layer + 2].w_qkv;
-      }
     }
   } else {
     r.flags = LT_QKV;
