@@ -50,7 +50,10 @@ constexpr int B_BYTES = BNMAX * BK * 2;
 constexpr int SMEM_TILES = STAGES * (A_BYTES + B_BYTES);
 constexpr int EPI_ROWS = 32;                    // rows per epilogue staging pass
 constexpr int EPI_BYTES = EPI_ROWS * BM * 4;    // fp32 staging tile [32 rows][128 features]
-constexpr int SMEM_BYTES = SMEM_TILES + 512 /*barriers*/ + EPI_BYTES + 1024 /*align*/;
+// per-row data of the fused epilogue, two tiles deep: [2][BNMAX] offsets + [2][BNMAX] ints
+constexpr int META_BYTES = 2 * BNMAX * (8 + 4);
+constexpr int SMEM_BYTES = SMEM_TILES + 512 /*barriers*/ + EPI_BYTES + META_BYTES + 1024 /*align*/;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 constexpr uint32_t TMEM_COLS = 512;  // two 256-column fp32 accumulators
 constexpr int THREADS = 192;
 
@@ -86,18 +89,56 @@ __device__ __forceinline__ Item decode_item(int it, int ntn, int splits, int R, 
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Per-row data of a fused epilogue, gathered into shared memory by the
+// epilogue threads before they wait for the tile's accumulator, so these
+// loads overlap the tile's MMAs instead of sitting inside the per-element
+// loops.  off[j] / iv[j] for row r0 + j of the tile:
+//   EPI_QKV:   iv = position; off = element offset of the row in q (part q),
+//              or of its slot in the KV page with head 0 and the K half
+//              (parts k, v: the head and half add (half*H + head)*page*hd)
+//   EPI_RESID: off = element offset of the row's residual in h
+//   EPI_HEAD:  iv = the token position t[b] when sequence b stopped here, else -1
+//   EPI_LSE:   iv = the row's target token
+__device__ __forceinline__ void load_row_meta(const EpiArgs& e, int n0, int r0, int rows, long long* off, int* iv) {
+  for (int j = threadIdx.x; j < rows; j += 128) {
+    const int r = r0 + j;
+    if (e.mode == EPI_QKV) {
+      const int pos = e.rs.row_pos[r];
+      iv[j] = pos;
+      off[j] = n0 < e.H * e.hd ? (long long)r * (e.H * e.hd)
+                               : (long long)e.kv.offset(e.layer, e.rs.row_b[r], pos, 0, 0);
+    } else if (e.mode == EPI_RESID) {
+      off[j] = (long long)e.rs.row_hrow[r] * e.d;
+    } else if (e.mode == EPI_HEAD) {
+      iv[j] = e.stop[r] ? e.t[r] : -1;
+    } else if (e.mode == EPI_LSE) {
+      iv[j] = e.lse_target[r];
+    }
+  }
+}
+
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Apply the layer epilogue to a staged tile: S[j][f] = y for row r0 + j and
-// feature n0 + f (f < 128).  Run by the 128 epilogue threads.
+// feature n0 + f (f < 128); off / iv are the rows' entries of load_row_meta.
+// Run by the 128 epilogue threads.
 //   EPI_QKV:    the tile holds whole heads of one of q/k/v (n0 % 128 == 0,
 //               head_dim | 128, H*head_dim % 128 == 0): rotate-half RoPE on q
 //               and k pairs, q -> q_out, k and v -> the paged KV cache.
-//   EPI_RESID:  h[row] += y.
 //   EPI_SWIGLU: the tile holds 64 gate rows then the 64 matching up rows.
-__device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, int n0, int r0, int nrows) {
+//   EPI_HEAD / EPI_LSE: per-row reductions over the tile's 128 tokens.
+// (EPI_RESID runs from the accumulator registers, without staging.)
+__device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, int n0, int r0, int nrows,
+                                              const long long* off, const int* iv) {
   const int tid = threadIdx.x;
   if (e.mode == EPI_QKV) {
     const int half = e.hd / 2, HQ = e.H * e.hd;
     const int part = n0 / HQ;
+    const size_t hstride = (size_t)e.kv.page_size * e.hd;
 #pragma unroll 4
     for (int idx = tid; idx < nrows * (BM / 2); idx += 128) {
       const int j = idx / (BM / 2), pr = idx % (BM / 2);
@@ -105,31 +146,17 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
       const int nl = n0 % HQ + f0;  // feature within q, k or v
       const int head = nl / e.hd, i = nl % e.hd;
       float y0 = S[j * BM + f0], y1 = S[j * BM + f0 + half];
-      const int r = r0 + j;
-      const int pos = e.rs.row_pos[r];
       if (part < 2) {
-        const float2 u = rope_pair(y0, y1, e.rope[(size_t)pos * half + i]);
+        const float2 u = rope_pair(y0, y1, __ldg(e.rope + (size_t)iv[j] * half + i));
         y0 = u.x;
         y1 = u.y;
       }
       __nv_bfloat16* dst;
-      if (part == 0) dst = (__nv_bfloat16*)e.q_out + (size_t)r * HQ + head * e.hd;
-      else dst = (__nv_bfloat16*)e.kv.base + e.kv.offset(e.layer, e.rs.row_b[r], pos, head, part - 1);
+      if (part == 0) dst = (__nv_bfloat16*)e.q_out + off[j] + head * e.hd;
+      else dst = (__nv_bfloat16*)e.kv.base + off[j] + (size_t)((part - 1) * e.H + head) * hstride;
       dst[i] = __float2bfloat16_rn(y0);
       dst[i + half] = __float2bfloat16_rn(y1);
     }
-  } else if (e.mode == EPI_RESID) {
-    // all row addresses and old values first (independent loads in flight)
-    float* hp[EPI_ROWS];
-    float hv[EPI_ROWS];
-#pragma unroll
-    for (int j = 0; j < EPI_ROWS; ++j)
-      hp[j] = j < nrows ? e.rs.h + (size_t)e.rs.row_hrow[r0 + j] * e.d + n0 + tid : nullptr;
-#pragma unroll
-    for (int j = 0; j < EPI_ROWS; ++j) hv[j] = hp[j] ? *hp[j] : 0.f;
-#pragma unroll
-    for (int j = 0; j < EPI_ROWS; ++j)
-      if (hp[j]) *hp[j] = hv[j] + S[j * BM + tid];
   } else if (e.mode == EPI_HEAD) {
     // exact sampling at this exit: score_v = logit_v + Gumbel(U_v), U_v from
     // Philox counter (b, t, 1, v/4) lane v%4; argmax with ties to the lowest
@@ -138,11 +165,11 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
     const unsigned long long seed = *e.seed;
     const int lane = tid & 31, w = tid >> 5;
     for (int j = 0; j < nrows; ++j) {
-      const int b = r0 + j;
-      if (!e.stop[b]) continue;  // same b for every thread: uniform
+      const int b = r0 + j, tb = iv[j];
+      if (tb < 0) continue;  // same b for every thread: uniform
       const int v = n0 + tid;
       const float logit = S[j * BM + tid];
-      const uint4 rb = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)e.t[b], STREAM_GUMBEL, (uint32_t)(v >> 2)),
+      const uint4 rb = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)tb, STREAM_GUMBEL, (uint32_t)(v >> 2)),
                                      (uint32_t)seed, (uint32_t)(seed >> 32));
       float bs = logit - logf(-logf(uniform01(lane_of(rb, v & 3))));
       int bv = v;
@@ -196,31 +223,29 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
       epi_bar();
     }
   } else if (e.mode == EPI_LSE) {
-    // scoring head: for each row of the tile, the max and the sum of
-    // exp(logit - max) over this tile's 128 tokens (lanes take 4 tokens
-    // each, then a fixed butterfly), and the target token's logit when the
-    // target falls in this tile
+    // scoring head: for each row of the tile, the max of this tile's 128
+    // logits (lanes take 4 tokens each, then a butterfly), then the sum of
+    // exp(logit - max) as 2^((logit - max) log2 e) with the hardware's
+    // base-2 exponential (relative error near 2^-22 per term), and the
+    // target token's logit when the target falls in this tile
     const int lane = tid & 31, w = tid >> 5;
+    constexpr float LOG2E = 1.4426950408889634f;
     for (int j = w; j < nrows; j += 4) {
       const float* row = S + j * BM;
       float x[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) x[i] = row[lane + 32 * i];
       float M = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
       float Ssum = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) Ssum += expf(x[i] - M);
+      for (int i = 0; i < 4; ++i) Ssum += exp2_approx(__fmul_rn(x[i] - M, LOG2E));
 #pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
-        const float S2 = __shfl_xor_sync(0xffffffffu, Ssum, o);
-        const float Mn = fmaxf(M, M2);
-        Ssum = Ssum * expf(M - Mn) + S2 * expf(M2 - Mn);
-        M = Mn;
-      }
+      for (int o = 16; o; o >>= 1) Ssum += __shfl_xor_sync(0xffffffffu, Ssum, o);
       const int r = r0 + j;
       if (lane == 0) e.lse_part[(size_t)r * e.nblk + n0 / BM] = make_float2(M, Ssum);
-      const int tg = e.lse_target[r] - n0;
+      const int tg = iv[j] - n0;
       if (tg >= 0 && tg < BM && (tg & 31) == lane) e.lse_tgt[r] = row[tg];
     }
   } else if (e.mode == EPI_SWIGLU) {
@@ -239,7 +264,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_go;
+  __shared__ int s_go[2];
   const int ntn = a.N / BM, kblocks = a.K / BK;
   // Before waiting for the previous kernel: nothing here reads what it
   // writes.  Pull the weight tiles this CTA will stream when all rows fit
@@ -290,6 +315,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* tfull = empty + MAXST;
   uint64_t* tempty = tfull + 2;
   float* stile = (float*)(smem + SMEM_TILES + 512);  // epilogue staging [EPI_ROWS][BM]
+  long long* meta_off = (long long*)(smem + SMEM_TILES + 512 + EPI_BYTES);  // [2][BNMAX]
+  int* meta_iv = (int*)(meta_off + 2 * BNMAX);                              // [2][BNMAX]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -386,29 +413,45 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // epilogue warps 0..3: TMEM lanes 32*warp .. 32*warp+31
-    int acc = 0;
+    int acc = 0, ipar = 0;
     uint32_t aphase = 0;
-    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+    const bool direct = a.fused != 0;  // fused launches never split
+    for (int it = blockIdx.x; it < items; it += gridDim.x, ipar ^= 1) {
       const Item t = decode_item(it, ntn, splits, R, kblocks);
+      long long* moff = meta_off + ipar * BNMAX;
+      int* miv = meta_iv + ipar * BNMAX;
+      // the tile's per-row data first (the previous tile's copy is the other
+      // buffer: every thread passed this tile's predecessor's barrier, so
+      // none still reads the buffer written here)
+      if (direct) load_row_meta(a.epi, t.n0, t.r0, t.rows, moff, miv);
       // one thread waits, the named barrier releases all four warps together,
       // so an expired wait makes every epilogue warp leave at the same point
-      if (threadIdx.x == 0) s_go = mbar_wait(tfull + acc, aphase, abort_flag) ? 1 : 0;
+      if (threadIdx.x == 0) s_go[ipar] = mbar_wait(tfull + acc, aphase, abort_flag) ? 1 : 0;
       epi_bar();
-      if (!s_go) break;
+      if (!s_go[ipar]) break;
       tc_fence_after();
       const int n = t.n0 + warp * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * BNMAX);
-      const bool direct = a.fused != 0;  // fused launches never split
       float* Ys = a.Y + (size_t)t.split * a.split_stride;
       for (int c0 = 0; c0 < t.nbox * BOXN; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tbase + (uint32_t)c0, v);
-        if (direct) {
+        const int nr = min(32, R - (t.r0 + c0));
+        if (direct && a.epi.mode == EPI_RESID) {
+          // h[row][n] += y straight from the accumulator: for each row the
+          // warp's 32 features are 128 contiguous bytes; all loads first
+          float hv[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) hv[j] = j < nr ? a.epi.rs.h[moff[c0 + j] + n] : 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nr) a.epi.rs.h[moff[c0 + j] + n] = hv[j] + __uint_as_float(v[j]);
+        } else if (direct) {
           // stage [32 rows][128 features], then the layer epilogue
 #pragma unroll
           for (int j = 0; j < 32; ++j) stile[j * BM + warp * 32 + lane] = __uint_as_float(v[j]);
           epi_bar();
-          tile_epilogue(a.epi, stile, t.n0, t.r0 + c0, min(32, R - (t.r0 + c0)));
+          tile_epilogue(a.epi, stile, t.n0, t.r0 + c0, nr, moff + c0, miv + c0);
           epi_bar();
         } else {
 #pragma unroll
