@@ -48,14 +48,24 @@ constexpr int STAGES = 4;        // stages at the largest row tile (256 rows)
 constexpr int MAXST = 12;        // stages when the row tile is small
 constexpr int B_BYTES = BNMAX * BK * 2;
 constexpr int SMEM_TILES = STAGES * (A_BYTES + B_BYTES);
-constexpr int EPI_ROWS = 32;                    // rows per epilogue staging pass
-constexpr int EPI_BYTES = EPI_ROWS * BM * 4;    // fp32 staging tile [32 rows][128 features]
+// Epilogue: two groups of four warps (warp w reads TMEM lanes 32*(w%4)..+31);
+// group g takes the 16-column accumulator chunks 2k+g of a tile, so two
+// chunks are in flight at once
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int WARP_TMA = EPI_WARPS, WARP_MMA = EPI_WARPS + 1;
+constexpr int EPI_ROWS = 16;                        // rows per staged chunk (one 32x32b.x16 TMEM load)
+constexpr int EPI_BYTES = 2 * EPI_ROWS * BM * 4;    // fp32 staging tile [16 rows][128 features] per group
 // per-row data of the fused epilogue, two tiles deep: [2][BNMAX] offsets + [2][BNMAX] ints
 constexpr int META_BYTES = 2 * BNMAX * (8 + 4);
 constexpr int SMEM_BYTES = SMEM_TILES + 512 /*barriers*/ + EPI_BYTES + META_BYTES + 1024 /*align*/;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 constexpr uint32_t TMEM_COLS = 512;  // two 256-column fp32 accumulators
-constexpr int THREADS = 192;
+constexpr int THREADS = EPI_THREADS + 64;  // + the TMA warp and the MMA warp
+// row tiles per band of the tile order: within a band the row tile changes
+// fastest, so each weight tile is read once per band and the band's rows
+// (16 x 256 rows) stay in L2 while the feature tiles sweep past
+constexpr int RBAND = 16;
 
 struct TcArgs {
   const int* nrows;
@@ -78,8 +88,11 @@ __device__ __forceinline__ Item decode_item(int it, int ntn, int splits, int R, 
   Item t;
   t.split = it % splits;
   const int tile = it / splits;
-  t.n0 = (tile % ntn) * BM;
-  t.r0 = (tile / ntn) * BNMAX;
+  const int nrt = (R + BNMAX - 1) / BNMAX;
+  const int band = tile / (ntn * RBAND), rt0 = band * RBAND, gb = min(RBAND, nrt - rt0);
+  const int local = tile - band * ntn * RBAND;
+  t.n0 = (local / gb) * BM;
+  t.r0 = (rt0 + local % gb) * BNMAX;
   t.rows = min(BNMAX, R - t.r0);
   t.nbox = (t.rows + BOXN - 1) / BOXN;
   t.kb0 = (int)((long long)t.split * kblocks / splits);
@@ -87,7 +100,9 @@ __device__ __forceinline__ Item decode_item(int it, int ntn, int splits, int R, 
   return t;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// all epilogue warps; the four warps of group g
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory"); }
+__device__ __forceinline__ void grp_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
 
 // Per-row data of a fused epilogue, gathered into shared memory by the
 // epilogue threads before they wait for the tile's accumulator, so these
@@ -100,7 +115,7 @@ __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: 
 //   EPI_HEAD:  iv = the token position t[b] when sequence b stopped here, else -1
 //   EPI_LSE:   iv = the row's target token
 __device__ __forceinline__ void load_row_meta(const EpiArgs& e, int n0, int r0, int rows, long long* off, int* iv) {
-  for (int j = threadIdx.x; j < rows; j += 128) {
+  for (int j = threadIdx.x; j < rows; j += EPI_THREADS) {
     const int r = r0 + j;
     if (e.mode == EPI_QKV) {
       const int pos = e.rs.row_pos[r];
@@ -109,6 +124,10 @@ __device__ __forceinline__ void load_row_meta(const EpiArgs& e, int n0, int r0, 
                                : (long long)e.kv.offset(e.layer, e.rs.row_b[r], pos, 0, 0);
     } else if (e.mode == EPI_RESID) {
       off[j] = (long long)e.rs.row_hrow[r] * e.d;
+      // the tile's 128 residual values of the row (512 bytes) into L2
+      const float* hp = e.rs.h + off[j] + n0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) asm volatile("prefetch.global.L2 [%0];" ::"l"(hp + 32 * q));
     } else if (e.mode == EPI_HEAD) {
       iv[j] = e.stop[r] ? e.t[r] : -1;
     } else if (e.mode == EPI_LSE) {
@@ -123,45 +142,66 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
-// Apply the layer epilogue to a staged tile: S[j][f] = y for row r0 + j and
-// feature n0 + f (f < 128); off / iv are the rows' entries of load_row_meta.
-// Run by the 128 epilogue threads.
-//   EPI_QKV:    the tile holds whole heads of one of q/k/v (n0 % 128 == 0,
-//               head_dim | 128, H*head_dim % 128 == 0): rotate-half RoPE on q
-//               and k pairs, q -> q_out, k and v -> the paged KV cache.
-//   EPI_SWIGLU: the tile holds 64 gate rows then the 64 matching up rows.
-//   EPI_HEAD / EPI_LSE: per-row reductions over the tile's 128 tokens.
-// (EPI_RESID runs from the accumulator registers, without staging.)
-__device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, int n0, int r0, int nrows,
-                                              const long long* off, const int* iv) {
-  const int tid = threadIdx.x;
-  if (e.mode == EPI_QKV) {
-    const int half = e.hd / 2, HQ = e.H * e.hd;
-    const int part = n0 / HQ;
-    const size_t hstride = (size_t)e.kv.page_size * e.hd;
-#pragma unroll 4
-    for (int idx = tid; idx < nrows * (BM / 2); idx += 128) {
-      const int j = idx / (BM / 2), pr = idx % (BM / 2);
-      const int f0 = (pr / half) * e.hd + pr % half;
-      const int nl = n0 % HQ + f0;  // feature within q, k or v
-      const int head = nl / e.hd, i = nl % e.hd;
+// EPI_QKV in two steps around the staging barrier.  Thread gt of a group
+// (0..127) takes rotary pair p = gt % 64 of the tile's 128 features (feature
+// f0 of its head half and f0 + hd/2) in rows gt / 64, gt / 64 + 2, ... of the
+// group's staged chunk: first it loads the
+// (cos, sin) entries of its rows, all independent loads, then (tile staged)
+// it rotates q and k, and writes q rows or the paged K / V cache.
+constexpr int QKV_RPT = EPI_ROWS / 2;  // rows per thread of a staged chunk
+__device__ __forceinline__ void qkv_load_rope(const EpiArgs& e, int n0, int nrows, const int* iv, int gt,
+                                              float2 (&cs)[QKV_RPT]) {
+  const int half = e.hd / 2, pr = gt & 63, j0 = gt >> 6, i = pr % half;
+  const bool rot = n0 < 2 * e.H * e.hd;  // q or k
+#pragma unroll
+  for (int k = 0; k < QKV_RPT; ++k) {
+    const int j = j0 + 2 * k;
+    cs[k] = rot && j < nrows ? __ldg(e.rope + (size_t)iv[j] * half + i) : make_float2(1.f, 0.f);
+  }
+}
+__device__ __forceinline__ void qkv_store(const EpiArgs& e, const float* S, int n0, int nrows, const long long* off,
+                                          int gt, const float2 (&cs)[QKV_RPT]) {
+  const int half = e.hd / 2, HQ = e.H * e.hd, part = n0 / HQ;
+  const int pr = gt & 63, j0 = gt >> 6;
+  const int f0 = (pr / half) * e.hd + pr % half;
+  const int nl = n0 % HQ + f0;  // feature within q, k or v
+  const int head = nl / e.hd, i = nl % e.hd;
+  const size_t fo = part == 0 ? (size_t)head * e.hd + i
+                              : (size_t)((part - 1) * e.H + head) * e.kv.page_size * e.hd + i;
+  __nv_bfloat16* base = part == 0 ? (__nv_bfloat16*)e.q_out : (__nv_bfloat16*)e.kv.base;
+#pragma unroll
+  for (int k = 0; k < QKV_RPT; ++k) {
+    const int j = j0 + 2 * k;
+    if (j < nrows) {
       float y0 = S[j * BM + f0], y1 = S[j * BM + f0 + half];
       if (part < 2) {
-        const float2 u = rope_pair(y0, y1, __ldg(e.rope + (size_t)iv[j] * half + i));
+        const float2 u = rope_pair(y0, y1, cs[k]);
         y0 = u.x;
         y1 = u.y;
       }
-      __nv_bfloat16* dst;
-      if (part == 0) dst = (__nv_bfloat16*)e.q_out + off[j] + head * e.hd;
-      else dst = (__nv_bfloat16*)e.kv.base + off[j] + (size_t)((part - 1) * e.H + head) * hstride;
-      dst[i] = __float2bfloat16_rn(y0);
-      dst[i + half] = __float2bfloat16_rn(y1);
+      __nv_bfloat16* dst = base + off[j] + fo;
+      dst[0] = __float2bfloat16_rn(y0);
+      dst[half] = __float2bfloat16_rn(y1);
     }
-  } else if (e.mode == EPI_HEAD) {
+  }
+}
+
+// Apply the layer epilogue to a staged tile: S[j][f] = y for row r0 + j and
+// feature n0 + f (f < 128); off / iv are the rows' entries of load_row_meta.
+// Run by the 128 threads of epilogue group g (gt = 0..127).
+//   EPI_SWIGLU: the tile holds 64 gate rows then the 64 matching up rows.
+//   EPI_HEAD / EPI_LSE: per-row reductions over the tile's 128 tokens.
+// (EPI_RESID runs from the accumulator registers, without staging; EPI_QKV
+// is qkv_load_rope / qkv_store above.)
+__device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, int n0, int r0, int nrows,
+                                              const long long* off, const int* iv, int gt, int g) {
+  const int tid = gt;
+  if (e.mode == EPI_HEAD) {
     // exact sampling at this exit: score_v = logit_v + Gumbel(U_v), U_v from
     // Philox counter (b, t, 1, v/4) lane v%4; argmax with ties to the lowest
     // v, and the log-sum-exp of the logits, over this tile's 128 v
-    __shared__ float red[4][HEAD_PART];
+    __shared__ float reds[2][4][HEAD_PART];
+    float(*red)[HEAD_PART] = reds[g];
     const unsigned long long seed = *e.seed;
     const int lane = tid & 31, w = tid >> 5;
     for (int j = 0; j < nrows; ++j) {
@@ -197,7 +237,7 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
         red[w][3] = M;
         red[w][4] = Ssum;
       }
-      epi_bar();
+      grp_bar(g);
       if (tid == 0) {
         float fs = red[0][0], fl = red[0][2], fM = red[0][3], fS = red[0][4];
         int fv = __float_as_int(red[0][1]);
@@ -220,7 +260,7 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
         out[3] = fM;
         out[4] = fS;
       }
-      epi_bar();
+      grp_bar(g);
     }
   } else if (e.mode == EPI_LSE) {
     // scoring head: for each row of the tile, the max of this tile's 128
@@ -269,7 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // Before waiting for the previous kernel: nothing here reads what it
   // writes.  Pull the weight tiles this CTA will stream when all rows fit
   // one tile (the decode case), and the next GEMM's share, into L2.
-  if (threadIdx.x == 160) {
+  if (threadIdx.x == WARP_MMA * 32) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tx)) : "memory");
     const int s1 = tc_split_count(1, a.N, a.K, gridDim.x, a.max_split);
@@ -314,7 +354,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* empty = full + MAXST;
   uint64_t* tfull = empty + MAXST;
   uint64_t* tempty = tfull + 2;
-  float* stile = (float*)(smem + SMEM_TILES + 512);  // epilogue staging [EPI_ROWS][BM]
+  float* stile = (float*)(smem + SMEM_TILES + 512);  // epilogue staging [2 groups][EPI_ROWS][BM]
   long long* meta_off = (long long*)(smem + SMEM_TILES + 512 + EPI_BYTES);  // [2][BNMAX]
   int* meta_iv = (int*)(meta_off + 2 * BNMAX);                              // [2][BNMAX]
 
@@ -326,7 +366,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(tfull + s, 1);
-      mbar_init(tempty + s, 128);
+      mbar_init(tempty + s, EPI_THREADS);
     }
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -343,7 +383,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 4) {
+  if (warp == WARP_TMA) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -377,7 +417,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (issued[s] >= 0) mbar_wait(full + s, (uint32_t)issued[s], &never, WAIT_NS / 4);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == WARP_MMA) {
     if (lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, aphase = 0;
@@ -412,7 +452,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
-    // epilogue warps 0..3: TMEM lanes 32*warp .. 32*warp+31
+    // epilogue warps 0..7: warp w reads TMEM lanes 32*(w%4) .. +31 (features
+    // n0 + 32*(w%4) ..), group w/4 takes the tile's 16-column chunks 2k + w/4
+    const int g = warp >> 2, qw = warp & 3, gt = threadIdx.x & 127;
+    float* sg = stile + g * EPI_ROWS * BM;
     int acc = 0, ipar = 0;
     uint32_t aphase = 0;
     const bool direct = a.fused != 0;  // fused launches never split
@@ -424,38 +467,47 @@ __global__ void __launch_bounds__(THREADS, 1)
       // buffer: every thread passed this tile's predecessor's barrier, so
       // none still reads the buffer written here)
       if (direct) load_row_meta(a.epi, t.n0, t.r0, t.rows, moff, miv);
-      // one thread waits, the named barrier releases all four warps together,
-      // so an expired wait makes every epilogue warp leave at the same point
+      // one thread waits, the named barrier releases all epilogue warps
+      // together, so an expired wait makes them all leave at the same point
       if (threadIdx.x == 0) s_go[ipar] = mbar_wait(tfull + acc, aphase, abort_flag) ? 1 : 0;
       epi_bar();
       if (!s_go[ipar]) break;
       tc_fence_after();
-      const int n = t.n0 + warp * 32 + lane;
-      const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * BNMAX);
+      const int n = t.n0 + qw * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(qw * 32) << 16) + (uint32_t)(acc * BNMAX);
       float* Ys = a.Y + (size_t)t.split * a.split_stride;
-      for (int c0 = 0; c0 < t.nbox * BOXN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tbase + (uint32_t)c0, v);
-        const int nr = min(32, R - (t.r0 + c0));
+      for (int c0 = g * EPI_ROWS; c0 < t.nbox * BOXN; c0 += 2 * EPI_ROWS) {
+        uint32_t v[EPI_ROWS];
+        tmem_ld16(tbase + (uint32_t)c0, v);
+        const int nr = min(EPI_ROWS, R - (t.r0 + c0));  // may be <= 0 in a ragged last chunk
         if (direct && a.epi.mode == EPI_RESID) {
           // h[row][n] += y straight from the accumulator: for each row the
           // warp's 32 features are 128 contiguous bytes; all loads first
-          float hv[32];
+          float hv[EPI_ROWS];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) hv[j] = j < nr ? a.epi.rs.h[moff[c0 + j] + n] : 0.f;
+          for (int j = 0; j < EPI_ROWS; ++j) hv[j] = j < nr ? a.epi.rs.h[moff[c0 + j] + n] : 0.f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
+          for (int j = 0; j < EPI_ROWS; ++j)
             if (j < nr) a.epi.rs.h[moff[c0 + j] + n] = hv[j] + __uint_as_float(v[j]);
-        } else if (direct) {
-          // stage [32 rows][128 features], then the layer epilogue
+        } else if (direct && a.epi.mode == EPI_QKV) {
+          // the rotary table loads go out before the staging barrier
+          float2 cs[QKV_RPT];
+          qkv_load_rope(a.epi, t.n0, nr, miv + c0, gt, cs);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) stile[j * BM + warp * 32 + lane] = __uint_as_float(v[j]);
-          epi_bar();
-          tile_epilogue(a.epi, stile, t.n0, t.r0 + c0, nr, moff + c0, miv + c0);
-          epi_bar();
+          for (int j = 0; j < EPI_ROWS; ++j) sg[j * BM + qw * 32 + lane] = __uint_as_float(v[j]);
+          grp_bar(g);
+          qkv_store(a.epi, sg, t.n0, nr, moff + c0, gt, cs);
+          grp_bar(g);
+        } else if (direct) {
+          // stage [16 rows][128 features], then the layer epilogue
+#pragma unroll
+          for (int j = 0; j < EPI_ROWS; ++j) sg[j * BM + qw * 32 + lane] = __uint_as_float(v[j]);
+          grp_bar(g);
+          tile_epilogue(a.epi, sg, t.n0, t.r0 + c0, nr, moff + c0, miv + c0, gt, g);
+          grp_bar(g);
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < EPI_ROWS; ++j) {
             const int r = t.r0 + c0 + j;
             if (r < R) Ys[(size_t)r * a.N + n] = __uint_as_float(v[j]);
           }
