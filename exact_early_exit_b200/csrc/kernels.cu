@@ -914,6 +914,10 @@ template <typename T, int HD>
 static void attention_dec_t(const AttnArgs& a, cudaStream_t st) {
   int g = (a.rs.max_rows * a.H + 7) / 8;
   if (g > 4096) g = 4096;
+  if (sizeof(T) == 2 && HD == 64 && attn_dec_pc_fits(a)) {
+    launch_attn_dec_pc(a, st);
+    return;
+  }
   if (a.kv_map && sizeof(T) == 2 && HD == 64) {
     AttnArgs m = a;
     m.kv_splits = a.dec_splits;

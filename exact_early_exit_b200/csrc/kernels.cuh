@@ -98,7 +98,8 @@ struct AttnArgs {
   const CUtensorMap* kv_map;  // host copy of the KV pool's 128-byte-row map (bf16, hd 64), or null
   const CUtensorMap* q_map;   // prefill / scoring: map of q (boxes of 64 x 128 rows) for the tcgen05 kernel, or null
   int dec_splits;             // MMA decode attention: key-range splits per (sequence, head)
-  int* dec_ctr;               // [B][H] split arrival counters (zero between launches)
+  int* dec_ctr;               // [B][H] split arrival counters + 2 item counters (zero between launches)
+  const CUtensorMap* kv_map32;  // decode / flush: the pool's map with 32-row boxes for k_attn_dec_pc, or null
 };
 void launch_attention(bool bf16, const AttnArgs& a, cudaStream_t st);
 // Decode / flush attention.  bf16 with head_dim 64 and a KV tensor map: the
@@ -122,6 +123,13 @@ void launch_attn_fa_mma(const CUtensorMap* kvmap, const AttnArgs& a, cudaStream_
 // Prefill / scoring on tcgen05 (attn_tc.cu): 128-row query tiles, S and the
 // per-tile P V in TMEM; needs a.kv_map and a.q_map.
 cudaError_t attn_tc_prepare();
+// Decode / flush on persistent warps (attn_dec.cu): items of (sequence,
+// head, 16-row pass, key chunk) taken from a counter in a.dec_ctr[B*H], each
+// warp streaming 32-key tiles through its own TMA ring; needs a.kv_map32,
+// a.part with a.kv_splits 128-key slots per (row, head), and B <= 512.
+cudaError_t attn_dec_pc_prepare();
+bool attn_dec_pc_fits(const AttnArgs& a);
+void launch_attn_dec_pc(const AttnArgs& a, cudaStream_t st);
 void launch_attn_fa_tc(const CUtensorMap* kvmap, const CUtensorMap* qmap, const AttnArgs& a, cudaStream_t st);
 
 struct StepArgs {

@@ -57,6 +57,16 @@ bool tc_attention_enabled() {
   return !(ev && (std::string(ev) == "simt" || std::string(ev) == "mma"));
 }
 
+// NVIUM_DEC_ATTN=pc: decode / flush attention on persistent warps
+// (k_attn_dec_pc) instead of one CTA per (sequence, head, key split)
+// (k_attn_dec_mma).  Both give the path's results; measured on B200 the
+// persistent one is slower (B=64 decode 9.4k against 12.3k tokens/s, B=1
+// 562 against 614), so it is an option, not the default
+bool dec_pc_attention_enabled() {
+  const char* ev = std::getenv("NVIUM_DEC_ATTN");
+  return mma_attention_enabled() && ev && std::string(ev) == "pc";
+}
+
 // NVIUM_LAYER_KERNEL=1: decode and flush layers run as one persistent kernel
 // after attention (layer_tc.cu), which gives the same bits as the default
 // per-kernel path; measured on B200 it is slower (its seven cross-CTA
@@ -123,8 +133,10 @@ struct nv_state {
   size_t kv_layer_stride = 0;
   CUtensorMap kv_map;        // the pool as rows of 128 bytes (bf16, head_dim 64)
   bool kv_map_ok = false;
+  CUtensorMap kv_map32;      // the same with boxes of 32 rows (persistent decode attention)
+  bool kv_map32_ok = false;
   int dec_splits = 1;        // key-range splits per (sequence, head) of the MMA decode attention
-  int* dec_ctr = nullptr;    // [B][H] split arrival counters of that kernel
+  int* dec_ctr = nullptr;    // [B][H] split arrival counters of the decode attention, + 2 item counters
   int n_pages = 0;
   int* page_table = nullptr;
   std::vector<int> h_page_table;
@@ -214,6 +226,7 @@ struct LayerIO {
   int epi_grid;
   bool dec_attn;       // chunked decode attention (else row-group attention)
   const CUtensorMap* kv_map;  // nullable: TMA view of the KV pool for the MMA attention kernels
+  const CUtensorMap* kv_map32;  // nullable: the same with 32-row boxes (persistent decode attention)
   int dec_splits;             // key-range splits of the MMA decode attention
   int* dec_ctr;               // its per-(sequence, head) split arrival counters
   bool prefetch_next;  // the last GEMM of a layer prefetches the next layer's QKV weights
@@ -400,6 +413,7 @@ nv_status layer_body(nv_model* M, int layer, const LayerIO& io, cudaStream_t st,
   }
   a.dec_splits = io.dec_splits;
   a.dec_ctr = io.dec_ctr;
+  a.kv_map32 = io.dec_attn ? io.kv_map32 : nullptr;
   const int attn_launches = io.dec_attn ? attention_decode_launches(bf, a) : (io.kv_splits > 1 ? 2 : 1);
   timed(prof, launches, attn_launches, NV_K_ATTENTION,
         (prof ? prof->kv_read : 0) + 2 * R * HQ * es, 0, [&] {
@@ -489,6 +503,7 @@ LayerIO state_io(nv_state* s) {
   io.epi_grid = 1184;
   io.dec_attn = s->dec_attn;
   io.kv_map = s->kv_map_ok ? &s->kv_map : nullptr;
+  io.kv_map32 = s->kv_map32_ok ? &s->kv_map32 : nullptr;
   io.dec_splits = s->dec_splits;
   io.dec_ctr = s->dec_ctr;
   io.prefetch_next = true;
@@ -1056,6 +1071,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
     const size_t head_sm = (((size_t)cfg->max_batch * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * d * esz;
     cudaError_t e2 = kernels_set_smem_limits(head_sm, (size_t)(cfg->max_batch + 1) * 4);
     if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_mma_prepare();
+    if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_dec_pc_prepare();
     if (e2 == cudaSuccess && M->tc_attention) e2 = attn_tc_prepare();
     if (e2 == cudaSuccess && cfg->adapter_hidden) e2 = exit_adapter_prepare(M->bf16, M->d, cfg->adapter_hidden);
     if (e2 != cudaSuccess) {
@@ -1162,7 +1178,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   A((void**)&s->seed_dev, 8);
   A((void**)&s->counters, NV_CTR_COUNT * 8);
   A((void**)&s->status, 4);
-  A((void**)&s->dec_ctr, (size_t)B * M->H * 4);
+  A((void**)&s->dec_ctr, ((size_t)B * M->H + 2) * 4);
   if (st != NV_OK) {
     nv_state_destroy(s);
     return st;
@@ -1179,6 +1195,8 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
     const uint64_t rows = (uint64_t)M->L * s->kv_layer_stride / 64;
     if (mma_attention_enabled() && s->dec_attn && M->bf16 && M->hd == 64 && rows < (1ull << 31))
       s->kv_map_ok = encode_rows128_map(s->kv, rows, 64, &s->kv_map) == NV_OK;
+    if (s->kv_map_ok && dec_pc_attention_enabled())
+      s->kv_map32_ok = encode_rows128_map(s->kv, rows, 32, &s->kv_map32) == NV_OK;
     // enough (sequence, head, split) CTAs for two waves of three per SM, each
     // split keeping at least two 64-key tiles
     const int pairs = B * M->H, target = 2 * 3 * 148;
@@ -1188,7 +1206,7 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
     s->dec_splits = std::max(1, sp);
   }
   cudaMemset(s->status, 0, 4);
-  cudaMemset(s->dec_ctr, 0, (size_t)B * M->H * 4);
+  cudaMemset(s->dec_ctr, 0, ((size_t)B * M->H + 2) * 4);
   cudaMemset(s->nrows, 0, 4);
   cudaMemset(s->lens, 0, (size_t)B * M->L * 4);
   cudaMemset(s->t, 0, (size_t)B * 4);

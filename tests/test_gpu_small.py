@@ -160,6 +160,76 @@ def test_mma_and_simt_decode_attention_agree(weights):
     np.testing.assert_allclose(l0[same], l1[same], atol=tolerance(CFG), rtol=0)
 
 
+def _decode_run(cfg, w, prompts, steps, max_seq, env):
+    """Decode `steps` steps and flush with the environment `env` set while the
+    model is built; returns tokens, exits, log-probs and every layer's KV."""
+    for k, v in env.items():
+        os.environ[k] = v
+    try:
+        m = nv.Model(cfg, w, max_batch=len(prompts), max_seq=max_seq)
+        st = nv.State(m, len(prompts))
+    finally:
+        for k in env:
+            os.environ.pop(k, None)
+    B = len(prompts)
+    st.prefill(np.concatenate(prompts).astype(np.int32), np.array([len(p) for p in prompts], np.int32))
+    toks, exs, lps = [], [], []
+    tok, ex, lp = np.zeros(B, np.int32), np.zeros(B, np.int32), np.zeros(B, np.float32)
+    for s in range(steps):
+        st.decode_step(1000 + s, tok, ex, lp)
+        toks.append(tok.copy()); exs.append(ex.copy()); lps.append(lp.copy())
+    st.flush()
+    st.sync_status()
+    kv = {(b, l): st.read_kv(b, l, max_seq) for b in range(B) for l in range(cfg.n_layers)}
+    st.close()
+    m.close()
+    return np.array(toks), np.array(exs), np.array(lps), kv
+
+
+def test_persistent_and_per_head_decode_attention_agree(weights):
+    """Decode attention on persistent warps (items of 16 rows x a key chunk,
+    taken from a counter, chunks merged by the last arrival) against one CTA
+    per (sequence, head): ragged prompts spanning several chunks, 64 sequences
+    (several items per warp), then a flush
+    whose sequences owe 40 deferred rows each (three 16-row passes), every
+    token having stopped at the first exit."""
+    wl = W.WORKLOADS["S"]
+    lens = np.array([300, 129, 64, 517], np.int64)
+    prompts = [p[:n] for p, n in zip(W.make_prompts(wl, lengths=[600] * 4), lens)]
+    a = _decode_run(CFG, weights, prompts, 24, 640, {})
+    b = _decode_run(CFG, weights, prompts, 24, 640, {"NVIUM_DEC_ATTN": "pc"})
+    same = np.cumprod((a[0] == b[0]) & (a[1] == b[1]), axis=0).astype(bool)
+    assert same.mean() >= 0.9, same.mean()
+    np.testing.assert_allclose(a[2][same], b[2][same], atol=tolerance(CFG), rtol=0)
+
+    # 64 sequences: several items per warp, so each warp's ring streams
+    # across item boundaries
+    lens = np.random.default_rng(4).integers(200, 600, size=64)
+    prompts = W.make_prompts(wl, lengths=lens)
+    a = _decode_run(CFG, weights, prompts, 6, 640, {})
+    b = _decode_run(CFG, weights, prompts, 6, 640, {"NVIUM_DEC_ATTN": "pc"})
+    same = np.cumprod((a[0] == b[0]) & (a[1] == b[1]), axis=0).astype(bool)
+    assert same.mean() >= 0.9, same.mean()
+    np.testing.assert_allclose(a[2][same], b[2][same], atol=tolerance(CFG), rtol=0)
+
+    w30 = W.make_weights(CFG, seed=0, router_bias=[30.0, 0.0, 0.0])
+    prompts = [p[:n] for p, n in zip(W.make_prompts(wl, seed=2), (20, 5, 33, 64))]
+    a = _decode_run(CFG, w30, prompts, 40, 128, {})
+    b = _decode_run(CFG, w30, prompts, 40, 128, {"NVIUM_DEC_ATTN": "pc"})
+    assert (a[1] == 1).all() and (b[1] == 1).all()
+    # a near tie may flip a draw (different summation orders): compare each
+    # sequence's cache up to its first differing token
+    diff = a[0] != b[0]
+    assert diff.mean() <= 0.05, diff.mean()
+    first = np.where(diff.any(0), diff.argmax(0), 40)
+    for (bq, layer), (K1, V1, n1) in a[3].items():
+        K2, V2, n2 = b[3][bq, layer]
+        assert n1 == n2, (bq, layer)
+        n = n1 if first[bq] == 40 else len(prompts[bq]) + first[bq] - 1
+        np.testing.assert_allclose(W.as_f32(K1[:n]), W.as_f32(K2[:n]), atol=2e-2, rtol=2 ** -7, err_msg=str((bq, layer)))
+        np.testing.assert_allclose(W.as_f32(V1[:n]), W.as_f32(V2[:n]), atol=2e-2, rtol=2 ** -7, err_msg=str((bq, layer)))
+
+
 def test_mma_and_simt_scoring_attention_agree(weights):
     """Flash-style MMA attention (64-row query tiles, 64-key tiles, online
     softmax) and the SIMT row-group kernel score the same sequences alike:
