@@ -501,7 +501,8 @@ def measure_scoring(wl, n_steps, n_warmup, dev, rank, world):
                    "h2d_bytes_per_step": int(toks.nbytes), "d2h_bytes_per_step": int(B * (S - 1) * 4 + 4)},
            "gpu_launches": sum(v["kernels"] for v in kern.values()) * n_steps,
            "roofline": {"bound": "tensor", "kernel": "gemm (layers + exit heads)", "achieved": round(achieved, 1),
-                        "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                        "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                        "traffic": ncu_traffic("gemm", wl.name),
                         "peak_source": src, "kernel_share": {k: round(v["ms"] / total_k, 4) for k, v in kern.items()},
                         "gemm_tflop_per_step": round(gemm_flops / 1e12, 2)},
            "mean_nll": float(nll_d.item()),
