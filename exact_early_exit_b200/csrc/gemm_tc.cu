@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -84,14 +85,15 @@ struct TcArgs {
 struct Item {
   int n0, r0, rows, nbox, kb0, kb1, split;
 };
-__device__ __forceinline__ Item decode_item(int it, int ntn, int splits, int R, int kblocks) {
+// fw: features per tile (128, or 256 for a CTA pair)
+__device__ __forceinline__ Item decode_item(int it, int ntn, int splits, int R, int kblocks, int fw = BM) {
   Item t;
   t.split = it % splits;
   const int tile = it / splits;
   const int nrt = (R + BNMAX - 1) / BNMAX;
   const int band = tile / (ntn * RBAND), rt0 = band * RBAND, gb = min(RBAND, nrt - rt0);
   const int local = tile - band * ntn * RBAND;
-  t.n0 = (local / gb) * BM;
+  t.n0 = (local / gb) * fw;
   t.r0 = (rt0 + local % gb) * BNMAX;
   t.rows = min(BNMAX, R - t.r0);
   t.nbox = (t.rows + BOXN - 1) / BOXN;
@@ -299,6 +301,99 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
   }
 }
 
+// Epilogue warps 0..7 of both GEMM kernels: warp w reads TMEM lanes
+// 32*(w%4) .. +31 (features n0 + 32*(w%4) ..), group w/4 takes the tile's
+// 16-column chunks 2k + w/4.  PAIR: this CTA holds rows 128*rank .. of a CTA
+// pair's M = 256 accumulator (features n0 + 128*rank ..), and each warp
+// signals the end of a tile on the leader CTA's barrier.
+struct EpiCtx {
+  float* stile;
+  long long* meta_off;
+  int* meta_iv;
+  int* s_go;
+  uint64_t* tfull;
+  uint64_t* tempty;      // one CTA: this CTA's tile-empty barriers
+  uint32_t tempty_lead;  // pair: cluster address of the leader's tile-empty barriers
+  uint32_t tmem;
+  volatile int* abort_flag;
+};
+template <bool PAIR>
+__device__ __forceinline__ void epilogue_warps(const TcArgs& a, const EpiCtx& c, int ntn, int splits, int R,
+                                               int kblocks, int items, int first, int stride, uint32_t rank) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = warp >> 2, qw = warp & 3, gt = threadIdx.x & 127;
+  float* sg = c.stile + g * EPI_ROWS * BM;
+  int acc = 0, ipar = 0;
+  uint32_t aphase = 0;
+  const bool direct = a.fused != 0;  // fused launches never split
+  for (int it = first; it < items; it += stride, ipar ^= 1) {
+    const Item t = decode_item(it, ntn, splits, R, kblocks, PAIR ? 2 * BM : BM);
+    const int n0 = t.n0 + (int)rank * BM;  // this CTA's 128 features
+    long long* moff = c.meta_off + ipar * BNMAX;
+    int* miv = c.meta_iv + ipar * BNMAX;
+    // the tile's per-row data first (the previous tile's copy is the other
+    // buffer: every thread passed this tile's predecessor's barrier, so
+    // none still reads the buffer written here)
+    if (direct) load_row_meta(a.epi, n0, t.r0, t.rows, moff, miv);
+    // one thread waits, the named barrier releases all epilogue warps
+    // together, so an expired wait makes them all leave at the same point
+    if (threadIdx.x == 0) c.s_go[ipar] = mbar_wait(c.tfull + acc, aphase, c.abort_flag) ? 1 : 0;
+    epi_bar();
+    if (!c.s_go[ipar]) break;
+    tc_fence_after();
+    const int n = n0 + qw * 32 + lane;
+    const uint32_t tbase = c.tmem + ((uint32_t)(qw * 32) << 16) + (uint32_t)(acc * BNMAX);
+    float* Ys = a.Y + (size_t)t.split * a.split_stride;
+    for (int c0 = g * EPI_ROWS; c0 < t.nbox * BOXN; c0 += 2 * EPI_ROWS) {
+      uint32_t v[EPI_ROWS];
+      tmem_ld16(tbase + (uint32_t)c0, v);
+      const int nr = min(EPI_ROWS, R - (t.r0 + c0));  // may be <= 0 in a ragged last chunk
+      if (direct && a.epi.mode == EPI_RESID) {
+        // h[row][n] += y straight from the accumulator: for each row the
+        // warp's 32 features are 128 contiguous bytes; all loads first
+        float hv[EPI_ROWS];
+#pragma unroll
+        for (int j = 0; j < EPI_ROWS; ++j) hv[j] = j < nr ? a.epi.rs.h[moff[c0 + j] + n] : 0.f;
+#pragma unroll
+        for (int j = 0; j < EPI_ROWS; ++j)
+          if (j < nr) a.epi.rs.h[moff[c0 + j] + n] = hv[j] + __uint_as_float(v[j]);
+      } else if (direct && a.epi.mode == EPI_QKV) {
+        // the rotary table loads go out before the staging barrier
+        float2 cs[QKV_RPT];
+        qkv_load_rope(a.epi, n0, nr, miv + c0, gt, cs);
+#pragma unroll
+        for (int j = 0; j < EPI_ROWS; ++j) sg[j * BM + qw * 32 + lane] = __uint_as_float(v[j]);
+        grp_bar(g);
+        qkv_store(a.epi, sg, n0, nr, moff + c0, gt, cs);
+        grp_bar(g);
+      } else if (direct) {
+        // stage [16 rows][128 features], then the layer epilogue
+#pragma unroll
+        for (int j = 0; j < EPI_ROWS; ++j) sg[j * BM + qw * 32 + lane] = __uint_as_float(v[j]);
+        grp_bar(g);
+        tile_epilogue(a.epi, sg, n0, t.r0 + c0, nr, moff + c0, miv + c0, gt, g);
+        grp_bar(g);
+      } else {
+#pragma unroll
+        for (int j = 0; j < EPI_ROWS; ++j) {
+          const int r = t.r0 + c0 + j;
+          if (r < R) Ys[(size_t)r * a.N + n] = __uint_as_float(v[j]);
+        }
+      }
+    }
+    tc_fence_before();
+    if (PAIR) {
+      // one arrival per warp on the leader CTA's barrier
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(c.tempty_lead + 8u * (uint32_t)acc);
+    } else {
+      mbar_arrive(c.tempty + acc);
+    }
+    acc ^= 1;
+    if (acc == 0) aphase ^= 1u;
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, TcArgs a) {
   extern __shared__ unsigned char smem_raw[];
@@ -452,78 +547,173 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
-    // epilogue warps 0..7: warp w reads TMEM lanes 32*(w%4) .. +31 (features
-    // n0 + 32*(w%4) ..), group w/4 takes the tile's 16-column chunks 2k + w/4
-    const int g = warp >> 2, qw = warp & 3, gt = threadIdx.x & 127;
-    float* sg = stile + g * EPI_ROWS * BM;
-    int acc = 0, ipar = 0;
-    uint32_t aphase = 0;
-    const bool direct = a.fused != 0;  // fused launches never split
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ipar ^= 1) {
-      const Item t = decode_item(it, ntn, splits, R, kblocks);
-      long long* moff = meta_off + ipar * BNMAX;
-      int* miv = meta_iv + ipar * BNMAX;
-      // the tile's per-row data first (the previous tile's copy is the other
-      // buffer: every thread passed this tile's predecessor's barrier, so
-      // none still reads the buffer written here)
-      if (direct) load_row_meta(a.epi, t.n0, t.r0, t.rows, moff, miv);
-      // one thread waits, the named barrier releases all epilogue warps
-      // together, so an expired wait makes them all leave at the same point
-      if (threadIdx.x == 0) s_go[ipar] = mbar_wait(tfull + acc, aphase, abort_flag) ? 1 : 0;
-      epi_bar();
-      if (!s_go[ipar]) break;
-      tc_fence_after();
-      const int n = t.n0 + qw * 32 + lane;
-      const uint32_t tbase = tmem + ((uint32_t)(qw * 32) << 16) + (uint32_t)(acc * BNMAX);
-      float* Ys = a.Y + (size_t)t.split * a.split_stride;
-      for (int c0 = g * EPI_ROWS; c0 < t.nbox * BOXN; c0 += 2 * EPI_ROWS) {
-        uint32_t v[EPI_ROWS];
-        tmem_ld16(tbase + (uint32_t)c0, v);
-        const int nr = min(EPI_ROWS, R - (t.r0 + c0));  // may be <= 0 in a ragged last chunk
-        if (direct && a.epi.mode == EPI_RESID) {
-          // h[row][n] += y straight from the accumulator: for each row the
-          // warp's 32 features are 128 contiguous bytes; all loads first
-          float hv[EPI_ROWS];
-#pragma unroll
-          for (int j = 0; j < EPI_ROWS; ++j) hv[j] = j < nr ? a.epi.rs.h[moff[c0 + j] + n] : 0.f;
-#pragma unroll
-          for (int j = 0; j < EPI_ROWS; ++j)
-            if (j < nr) a.epi.rs.h[moff[c0 + j] + n] = hv[j] + __uint_as_float(v[j]);
-        } else if (direct && a.epi.mode == EPI_QKV) {
-          // the rotary table loads go out before the staging barrier
-          float2 cs[QKV_RPT];
-          qkv_load_rope(a.epi, t.n0, nr, miv + c0, gt, cs);
-#pragma unroll
-          for (int j = 0; j < EPI_ROWS; ++j) sg[j * BM + qw * 32 + lane] = __uint_as_float(v[j]);
-          grp_bar(g);
-          qkv_store(a.epi, sg, t.n0, nr, moff + c0, gt, cs);
-          grp_bar(g);
-        } else if (direct) {
-          // stage [16 rows][128 features], then the layer epilogue
-#pragma unroll
-          for (int j = 0; j < EPI_ROWS; ++j) sg[j * BM + qw * 32 + lane] = __uint_as_float(v[j]);
-          grp_bar(g);
-          tile_epilogue(a.epi, sg, t.n0, t.r0 + c0, nr, moff + c0, miv + c0, gt, g);
-          grp_bar(g);
-        } else {
-#pragma unroll
-          for (int j = 0; j < EPI_ROWS; ++j) {
-            const int r = t.r0 + c0 + j;
-            if (r < R) Ys[(size_t)r * a.N + n] = __uint_as_float(v[j]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(tempty + acc);
-      acc ^= 1;
-      if (acc == 0) aphase ^= 1u;
-    }
+    EpiCtx c{stile, meta_off, meta_iv, s_go, tfull, tempty, 0u, tmem, abort_flag};
+    epilogue_warps<false>(a, c, ntn, splits, R, kblocks, items, blockIdx.x, gridDim.x, 0u);
   }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
+  if (threadIdx.x == 0 && s_abort) dev_fail(a.status, DEV_ERR_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair GEMM (prefill and scoring: many rows, one K slice).  A cluster of
+// two CTAs computes a 256-feature x 256-row tile with tcgen05.mma
+// cta_group::2 (M = 256): each CTA stages its own 128 weight rows and 128 of
+// the tile's X rows, so a CTA moves 32 KB of operands per 64-deep K step
+// instead of 48 KB, and holds its 128 features x 256 rows of the accumulator
+// in its own TMEM.  The leader CTA (rank 0) issues the MMAs; both CTAs' TMA
+// loads count on the leader's stage barrier, and the leader's commits
+// arrive on the stage and tile barriers of both CTAs.  Epilogue as in the
+// one-CTA kernel, on this CTA's 128 features.
+// ---------------------------------------------------------------------------
+constexpr int PAIR_ROWS = BNMAX / 2;  // X rows a CTA stages per tile
+constexpr int PAIR_STAGE = A_BYTES + (PAIR_ROWS / BOXN) * BOX_BYTES;
+constexpr int PAIR_NST = SMEM_TILES / PAIR_STAGE;
+static_assert(PAIR_NST <= MAXST, "pair stages fit the barrier array");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_gemm_tc2(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, TcArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_go[2];
+  const int ntn2 = a.N / (2 * BM), kblocks = a.K / BK;
+  const uint32_t rank = cluster_ctarank();
+  if (threadIdx.x == WARP_MMA * 32) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tx)) : "memory");
+  }
+  pdl_wait();
+  pdl_launch();
+  // both CTAs of a pair read the same values, so they leave together
+  const int R = *a.nrows;
+  if (R <= 0 || (a.skip_if_zero && *a.skip_if_zero == 0)) return;
+  const int items = ntn2 * ((R + BNMAX - 1) / BNMAX);
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+  if (pair >= items) return;
+
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + SMEM_TILES);
+  uint64_t* empty = full + MAXST;
+  uint64_t* tfull = empty + MAXST;
+  uint64_t* tempty = tfull + 2;
+  float* stile = (float*)(smem + SMEM_TILES + 512);
+  long long* meta_off = (long long*)(smem + SMEM_TILES + 512 + EPI_BYTES);
+  int* meta_iv = (int*)(meta_off + 2 * BNMAX);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_NST; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(tfull + s, 1);
+      mbar_init(tempty + s, 2 * EPI_WARPS);  // the leader's: one arrival per epilogue warp of both CTAs
+    }
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers are initialised before either uses the other's
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == WARP_TMA) {
+    if (lane == 0) {
+      const uint32_t full_lead = mapa_shared(smem_u32(full), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int issued[MAXST];  // leader: parity of the last phase it armed in each stage, -1 if none
+#pragma unroll
+      for (int s = 0; s < MAXST; ++s) issued[s] = -1;
+      for (int it = pair; it < items && ok; it += npairs) {
+        const Item t = decode_item(it, ntn2, 1, R, kblocks, 2 * BM);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          unsigned char* sa = smem + stage * PAIR_STAGE;
+          if (rank == 0) {
+            issued[stage] = (int)phase;
+            mbar_expect_tx(full + stage, (uint32_t)(2 * PAIR_STAGE));  // both CTAs' bytes
+          }
+          const uint32_t fb = full_lead + 8u * (uint32_t)stage;
+          tma_load_2d_pair(sa, &tw, fb, kb * BK, t.n0 + (int)rank * BM);
+          for (int j = 0; j < PAIR_ROWS / BOXN; ++j)
+            tma_load_2d_pair(sa + A_BYTES + j * BOX_BYTES, &tx, fb, kb * BK, t.r0 + (int)rank * PAIR_ROWS + j * BOXN);
+          if (++stage == PAIR_NST) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag && rank == 0) {
+        // let the copies already issued land before the pair leaves (bounded;
+        // the leader's stage barriers count both CTAs' bytes)
+        volatile int never = 0;
+        for (int s = 0; s < PAIR_NST; ++s)
+          if (issued[s] >= 0) mbar_wait(full + s, (uint32_t)issued[s], &never, WAIT_NS / 4);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t empty_own = mapa_shared(smem_u32(empty), 0), empty_peer = mapa_shared(smem_u32(empty), 1);
+      const uint32_t tfull_own = mapa_shared(smem_u32(tfull), 0), tfull_peer = mapa_shared(smem_u32(tfull), 1);
+      const uint32_t idesc = idesc_bf16_m256(BNMAX);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, aphase = 0;
+      bool ok = true;
+      for (int it = pair; it < items && ok; it += npairs) {
+        if (!mbar_wait(tempty + acc, aphase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BNMAX);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full + stage, phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(smem_u32(smem + stage * PAIR_STAGE));
+          const uint64_t bd = sw128_desc(smem_u32(smem + stage * PAIR_STAGE + A_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_pair(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair(empty_own + 8u * (uint32_t)stage);
+          umma_commit_pair(empty_peer + 8u * (uint32_t)stage);
+          if (++stage == PAIR_NST) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(tfull_own + 8u * (uint32_t)acc);
+        umma_commit_pair(tfull_peer + 8u * (uint32_t)acc);
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1u;
+      }
+    }
+  } else {
+    EpiCtx c{stile, meta_off, meta_iv, s_go, tfull, tempty, mapa_shared(smem_u32(tempty), 0), tmem, abort_flag};
+    epilogue_warps<true>(a, c, ntn2, 1, R, kblocks, items, pair, npairs, rank);
+  }
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync();  // neither CTA leaves while the other may still signal its barriers or read its tiles
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   if (threadIdx.x == 0 && s_abort) dev_fail(a.status, DEV_ERR_TIMEOUT);
 }
 
@@ -575,8 +765,21 @@ void tc_plans_destroy(TcPlanCache* c) {
 
 int* tc_status_ptr(TcPlanCache* c) { return c ? c->status : nullptr; }
 
+// CTA-pair kernel for launches with many rows and one K slice, unless
+// NVIUM_GEMM_PAIR=0 keeps every launch on the one-CTA kernel
+static bool pair_gemm_enabled() {
+  static const bool on = [] {
+    const char* ev = std::getenv("NVIUM_GEMM_PAIR");
+    return !(ev && ev[0] == '0');
+  }();
+  return on;
+}
+constexpr int PAIR_MIN_ROWS = 1024;
+
 nv_status tc_prepare() {
   cudaError_t e = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) {
     set_error(std::string("tcgen05 GEMM shared memory: ") + cudaGetErrorString(e));
     return NV_ERR_UNSUPPORTED;
@@ -683,6 +886,34 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
   CUtensorMap tw, tx;
   NV_TRY(make_map(c, W, (uint64_t)K, (uint64_t)N, (uint64_t)K, BM, &tw));
   NV_TRY(make_map(c, X, (uint64_t)K, (uint64_t)max_rows, (uint64_t)ldx, BOXN, &tx));
+  if (!allow_split && N % (2 * BM) == 0 && max_rows >= PAIR_MIN_ROWS && pair_gemm_enabled() &&
+      !(epi && epi->mode == EPI_HEAD)) {
+    // CTA pairs: an even grid of at most one pair per 256 x 256 tile
+    const long long tiles = (long long)(N / (2 * BM)) * ((max_rows + BNMAX - 1) / BNMAX);
+    int grid = sm_count() & ~1;
+    if (2 * tiles < grid) grid = (int)(2 * tiles);
+    TcArgs a;
+    a.nrows = nrows;
+    a.Y = Y;
+    a.N = N;
+    a.K = K;
+    a.max_split = 1;
+    a.split_stride = (size_t)BNMAX * N;
+    a.status = c->status;
+    a.fused = (epi && epi->mode != EPI_STORE) ? 1 : 0;
+    a.skip_if_zero = skip_if_zero;
+    a.pf_ptr = nullptr;
+    a.pf_bytes = 0;
+    if (epi) a.epi = *epi;
+    else std::memset(&a.epi, 0, sizeof(a.epi));
+    cudaError_t le = launch_k(k_gemm_tc2, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tw, tx, a);
+    if (le != cudaSuccess) {
+      set_error(std::string("tcgen05 pair GEMM launch: ") + cudaGetErrorString(le));
+      return NV_ERR_CUDA;
+    }
+    if (grid_out) *grid_out = grid;
+    return NV_OK;
+  }
   // persistent grid: never more CTAs than there can be work items
   const int ntn = N / BM;
   const int nrt_max = (max_rows + BNMAX - 1) / BNMAX;

@@ -302,6 +302,39 @@ def test_shared_head_with_adapters_bf16_matches_oracle(batch):
     assert chk.steps == 8
 
 
+def test_cta_pair_and_single_cta_gemm_agree(weights):
+    """The CTA-pair GEMM (tcgen05.mma cta_group::2, 256 x 256 tiles; launches
+    with 1024 rows or more and one K slice) against the one-CTA kernel, on
+    scoring rows whose last pair tile is ragged (5 x 257 = 1285 rows) and on a
+    ragged prefill: every epilogue (RoPE + KV write, residual, SwiGLU, exit
+    log-sum-exp) runs on both."""
+    toks = np.stack([W.make_prompts(W.WORKLOADS["S"], seed=s)[0][:257] for s in range(5)]).astype(np.int32)
+    lens = np.array([300, 257, 129, 64, 517], np.int32)
+    prompts = [p[:n] for p, n in zip(W.make_prompts(W.WORKLOADS["S"], lengths=[600] * 5), lens)]
+    out = {}
+    for eng in ("single", "pair"):
+        if eng == "single":
+            os.environ["NVIUM_GEMM_PAIR"] = "0"
+        try:
+            m = nv.Model(CFG, weights, max_batch=5, max_seq=640)
+        finally:
+            os.environ.pop("NVIUM_GEMM_PAIR", None)
+        lp = np.zeros((5, 256), np.float32)
+        m.score_mixture(toks, lp)
+        st = nv.State(m, 5)
+        st.prefill(np.concatenate(prompts), lens)
+        st.sync_status()
+        kv = [st.read_kv(b, l, 640) for b in range(5) for l in (0, 11)]
+        out[eng] = (lp, kv)
+        st.close()
+        m.close()
+    np.testing.assert_allclose(out["single"][0], out["pair"][0], atol=5e-3, rtol=0)
+    for (K1, V1, n1), (K2, V2, n2) in zip(out["single"][1], out["pair"][1]):
+        assert n1 == n2
+        np.testing.assert_allclose(W.as_f32(K1), W.as_f32(K2), atol=2e-2, rtol=2 ** -7)
+        np.testing.assert_allclose(W.as_f32(V1), W.as_f32(V2), atol=2e-2, rtol=2 ** -7)
+
+
 def test_tcgen05_and_mma_flash_attention_agree(weights):
     """Scoring and prefill attention on the tcgen05 kernel (128-row query
     tiles, scores and P V in TMEM) against the warp-MMA kernel, on sequences
