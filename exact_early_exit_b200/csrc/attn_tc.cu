@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
     const int t = threadIdx.x;
     const int pos = t < nr ? a.rs.row_pos[g0 + t] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    float m = -CUDART_INF_F, l = 0.f;
+    float mref = -CUDART_INF_F, l = 0.f;
     const float scale2 = a.scale * 1.4426950408889634f;  // log2(e) / sqrt(hd)
     unsigned char* prow_hi = reinterpret_cast<unsigned char*>(S.Phi) + t * 128;
     unsigned char* prow_lo = reinterpret_cast<unsigned char*>(S.Plo) + t * 128;
@@ -248,41 +248,57 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
       tc_fence_before();
       mbar_arrive(&S.s_empty[j & 1]);
       const int k0 = j * TK;
-      // scores in base 2 (scaled by log2 e / sqrt(hd)); keys past the row's
-      // position (only in the tiles that reach the diagonal) get -inf
+      // raw scores; keys past the row's position (only in the tiles that
+      // reach the diagonal) get -inf
       float tmax = -CUDART_INF_F;
       if (k0 + TK - 1 <= pos) {
 #pragma unroll
-        for (int i = 0; i < TK; ++i) {
-          const float v = __uint_as_float(r[i]) * scale2;
-          r[i] = __float_as_uint(v);
-          tmax = fmaxf(tmax, v);
-        }
+        for (int i = 0; i < TK; ++i) tmax = fmaxf(tmax, __uint_as_float(r[i]));
       } else {
 #pragma unroll
         for (int i = 0; i < TK; ++i) {
-          const float v = k0 + i <= pos ? __uint_as_float(r[i]) * scale2 : -CUDART_INF_F;
-          r[i] = __float_as_uint(v);
-          tmax = fmaxf(tmax, v);
+          if (k0 + i > pos) r[i] = __float_as_uint(-CUDART_INF_F);
+          tmax = fmaxf(tmax, __uint_as_float(r[i]));
         }
       }
-      const float mn = fmaxf(m, tmax);
-      const float cj = mn == -CUDART_INF_F ? 1.f : ex2(m - mn);
+      // Softmax in base 2 against a reference max mref (scores scaled by
+      // log2(e) / sqrt(hd)): P = 2^(s scale2 - mref).  mref moves only when a
+      // score exceeds it by more than 8, so P <= 256 and O is rescaled in TMEM
+      // only then, not at every growth of the running max; numerator and
+      // denominator share the reference, so O / l is unchanged.
+      const float tm2 = tmax * scale2;
+      float cj = 1.f;
+      bool resc = false;
+      if (tm2 > mref + 8.f) {
+        if (mref != -CUDART_INF_F) {
+          cj = ex2(mref - tm2);
+          resc = true;
+        }
+        mref = tm2;
+      }
       float rs = 0.f;
-      if (mn == -CUDART_INF_F) {
+      if (mref == -CUDART_INF_F) {
 #pragma unroll
         for (int i = 0; i < TK; ++i) r[i] = 0u;
       } else {
 #pragma unroll
         for (int i = 0; i < TK; ++i) {
-          const float p = ex2(__uint_as_float(r[i]) - mn);
+          const float p = ex2(__fmaf_rn(__uint_as_float(r[i]), scale2, -mref));
           r[i] = __float_as_uint(p);
           rs += p;
         }
       }
       l = l * cj + rs;
-      const bool grew = mn != m;
-      m = mn;
+      // P as bf16 pairs, hi = bf16(P) and lo = bf16(P - hi), packed
+      // (pk[0..31]: hi, pk[32..63]: lo) before waiting for the previous P V
+      uint32_t pk[TK];
+#pragma unroll
+      for (int e = 0; e < TK / 2; ++e) {
+        const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+        pk[e] = *reinterpret_cast<const uint32_t*>(&hb);
+        pk[TK / 2 + e] = pack2(x0 - __low2float(hb), x1 - __high2float(hb));
+      }
       // the previous tile's P V must be done with P (and with O) first
       if (j > 0 && !sm_wait(S, &S.o_full, (uint32_t)((j - 1) & 1))) {
         ok = false;
@@ -298,24 +314,17 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = __uint_as_float(r[8 * c + 2 * e]), x1 = __uint_as_float(r[8 * c + 2 * e + 1]);
-          const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&hb);
-          lo[e] = pack2(x0 - __low2float(hb), x1 - __high2float(hb));
-        }
         const int off = ((c ^ (t & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow_lo + off) =
+            make_uint4(pk[TK / 2 + 4 * c], pk[TK / 2 + 4 * c + 1], pk[TK / 2 + 4 * c + 2], pk[TK / 2 + 4 * c + 3]);
       }
-      // a row whose max grew: O (the sum over the earlier tiles) is rescaled
-      // in TMEM by exp(m_old - m_new) before this tile's P V adds to it.  The
-      // TMEM loads and stores are warp-collective: a warp with any such row
-      // rescales all its rows, the others by exactly 1.
-      if (__any_sync(0xffffffffu, j > 0 && grew)) {
-        const float f = grew ? cj : 1.0f;
+      // a row whose reference moved: O (the sum over the earlier tiles) is
+      // rescaled in TMEM by 2^(mref_old - mref_new) before this tile's P V
+      // adds to it.  The TMEM loads and stores are warp-collective: a warp
+      // with any such row rescales all its rows, the others by exactly 1.
+      if (__any_sync(0xffffffffu, resc)) {
+        const float f = resc ? cj : 1.0f;
         tc_fence_after();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
