@@ -201,21 +201,34 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
   if (e.mode == EPI_HEAD) {
     // exact sampling at this exit: score_v = logit_v + Gumbel(U_v), U_v from
     // Philox counter (b, t, 1, v/4) lane v%4; argmax with ties to the lowest
-    // v, and the log-sum-exp of the logits, over this tile's 128 v
-    __shared__ float reds[2][4][HEAD_PART];
-    float(*red)[HEAD_PART] = reds[g];
+    // v, and the log-sum-exp of the logits, over this tile's 128 v.  A warp
+    // takes whole rows (rows w, w+4, ...), a lane the 4 tokens of one Philox
+    // block (v = n0 + 4 lane + i), then a butterfly over the warp.
     const unsigned long long seed = *e.seed;
     const int lane = tid & 31, w = tid >> 5;
-    for (int j = 0; j < nrows; ++j) {
+    for (int j = w; j < nrows; j += 4) {
       const int b = r0 + j, tb = iv[j];
-      if (tb < 0) continue;  // same b for every thread: uniform
-      const int v = n0 + tid;
-      const float logit = S[j * BM + tid];
-      const uint4 rb = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)tb, STREAM_GUMBEL, (uint32_t)(v >> 2)),
+      if (tb < 0) continue;  // same row for the whole warp: uniform
+      const int v0 = n0 + 4 * lane;
+      const uint4 rb = philox4x32_10(make_uint4((uint32_t)b, (uint32_t)tb, STREAM_GUMBEL, (uint32_t)(v0 >> 2)),
                                      (uint32_t)seed, (uint32_t)(seed >> 32));
-      float bs = logit - logf(-logf(uniform01(lane_of(rb, v & 3))));
-      int bv = v;
-      float bl = logit, M = logit, Ssum = 1.0f;
+      const float* row = S + j * BM + 4 * lane;
+      float bs = -INFINITY, bl = 0.f, M = -INFINITY;
+      int bv = v0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float logit = row[i];
+        const float sc = logit - logf(-logf(uniform01(lane_of(rb, i))));
+        if (sc > bs) {  // ascending v: ties keep the lowest
+          bs = sc;
+          bv = v0 + i;
+          bl = logit;
+        }
+        M = fmaxf(M, logit);
+      }
+      float Ssum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Ssum += expf(row[i] - M);
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
         const float s2 = __shfl_xor_sync(0xffffffffu, bs, o);
@@ -233,36 +246,13 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
         M = Mn;
       }
       if (lane == 0) {
-        red[w][0] = bs;
-        red[w][1] = __int_as_float(bv);
-        red[w][2] = bl;
-        red[w][3] = M;
-        red[w][4] = Ssum;
-      }
-      grp_bar(g);
-      if (tid == 0) {
-        float fs = red[0][0], fl = red[0][2], fM = red[0][3], fS = red[0][4];
-        int fv = __float_as_int(red[0][1]);
-        for (int q = 1; q < 4; ++q) {
-          const float s2 = red[q][0];
-          const int v2 = __float_as_int(red[q][1]);
-          if (s2 > fs || (s2 == fs && v2 < fv)) {
-            fs = s2;
-            fv = v2;
-            fl = red[q][2];
-          }
-          const float Mn = fmaxf(fM, red[q][3]);
-          fS = fS * expf(fM - Mn) + red[q][4] * expf(red[q][3] - Mn);
-          fM = Mn;
-        }
         float* out = e.head_part + ((size_t)b * e.nblk + n0 / BM) * HEAD_PART;
-        out[0] = fs;
-        out[1] = __int_as_float(fv);
-        out[2] = fl;
-        out[3] = fM;
-        out[4] = fS;
+        out[0] = bs;
+        out[1] = __int_as_float(bv);
+        out[2] = bl;
+        out[3] = M;
+        out[4] = Ssum;
       }
-      grp_bar(g);
     }
   } else if (e.mode == EPI_LSE) {
     // scoring head: for each row of the tile, the max of this tile's 128
