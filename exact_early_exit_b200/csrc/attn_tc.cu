@@ -47,7 +47,7 @@ struct FtSmem {
   __nv_bfloat16 Plo[TQ * TK];
   uint64_t q_full, kv_full[KST], kv_empty[KST], s_full[2], s_empty[2], p_full, o_full, drain;
   uint32_t tmem;
-  int abort, go;
+  int abort;
 };
 constexpr size_t FT_SMEM_BYTES = sizeof(FtSmem) + 1024;
 
@@ -89,15 +89,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-// The softmax warps wait together: one thread polls (bounded), a named
-// barrier over the four warps releases them.
-__device__ __forceinline__ void sm_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Each softmax warp waits on its own: lane 0 polls (bounded), the warp
+// follows.  No barrier across the four warps, so a warp starts on a tile as
+// soon as the tile is ready, not when the slowest warp has finished the last.
 __device__ __forceinline__ bool sm_wait(FtSmem& S, uint64_t* bar, uint32_t parity) {
-  if (threadIdx.x == 0) S.go = mbar_wait(bar, parity, &S.abort) ? 1 : 0;
-  sm_bar();
-  const bool ok = S.go != 0;
-  sm_bar();
-  return ok;
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, &S.abort) ? 1 : 0;
+  __syncwarp();
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 __global__ void __launch_bounds__(FT_THREADS, 2)
