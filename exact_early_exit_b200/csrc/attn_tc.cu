@@ -249,17 +249,20 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
       const int k0 = j * TK;
       // raw scores; keys past the row's position (only in the tiles that
       // reach the diagonal) get -inf
-      float tmax = -CUDART_INF_F;
-      if (k0 + TK - 1 <= pos) {
+      if (k0 + TK - 1 > pos) {
 #pragma unroll
-        for (int i = 0; i < TK; ++i) tmax = fmaxf(tmax, __uint_as_float(r[i]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < TK; ++i) {
+        for (int i = 0; i < TK; ++i)
           if (k0 + i > pos) r[i] = __float_as_uint(-CUDART_INF_F);
-          tmax = fmaxf(tmax, __uint_as_float(r[i]));
-        }
       }
+      // the row max as eight independent chains, then a tree (a single
+      // 64-long dependent chain would leave the pipe waiting on itself)
+      float pm[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) pm[c] = __uint_as_float(r[c]);
+#pragma unroll
+      for (int i = 8; i < TK; ++i) pm[i & 7] = fmaxf(pm[i & 7], __uint_as_float(r[i]));
+      const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       // Softmax in base 2 against a reference max mref (scores scaled by
       // log2(e) / sqrt(hd)): P = 2^(s scale2 - mref).  mref moves only when a
       // score exceeds it by more than 8, so P <= 256 and O is rescaled in TMEM
@@ -280,12 +283,17 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
 #pragma unroll
         for (int i = 0; i < TK; ++i) r[i] = 0u;
       } else {
+        // the row sum as eight partial sums added in a fixed tree
+        float ps[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) ps[c] = 0.f;
 #pragma unroll
         for (int i = 0; i < TK; ++i) {
           const float p = ex2(__fmaf_rn(__uint_as_float(r[i]), scale2, -mref));
           r[i] = __float_as_uint(p);
-          rs += p;
+          ps[i & 7] += p;
         }
+        rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       }
       l = l * cj + rs;
       // P as bf16 pairs, hi = bf16(P) and lo = bf16(P - hi), packed
