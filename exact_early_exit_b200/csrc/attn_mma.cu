@@ -193,20 +193,36 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) k_attn_dec_mma(const __grid_co
 #pragma unroll
       for (int e = 0; e < 4; ++e) oc[nt8][e] = 0.f;
     if (w == 4) {
-      if (lane == 0) {
-        for (int i = 0; i < nt; ++i) {
-          const int q = q_base + i, st = q % DS;
+      // the whole warp walks the tiles: lanes hold the page ids of the next
+      // 32 pages (loaded ahead, off the per-tile path), lane 0 waits and issues
+      const int ps = a.kv.page_size;
+      const size_t hstride = (size_t)ps * HD, lbase = (size_t)a.layer * a.kv.layer_stride;
+      const int* pt = a.kv.page_table + (size_t)b * a.kv.pages_per_seq;
+      const int plast = pos_last / ps;
+      int chunk = -1, pg = 0;
+      for (int i = 0; i < nt; ++i) {
+        const int q = q_base + i, st = q % DS;
+        const int pos = (t_beg + i) * BOX, pi = pos / ps;
+        if (pi >= chunk + 32 || chunk < 0) {
+          chunk = pi;
+          pg = chunk + lane <= plast ? pt[chunk + lane] : 0;
+        }
+        const int page = __shfl_sync(0xffffffffu, pg, pi - chunk);
+        int ok = 1;
+        if (lane == 0) {
           if (q >= DS && !fa_wait(&S.empty[st], (uint32_t)((q / DS - 1) & 1))) {
             S.abort = 1;
-            break;
+            ok = 0;
+          } else {
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(&S.full[st])),
+                         "r"((uint32_t)(2 * BOX_BYTES))
+                         : "memory");
+            const size_t off = lbase + ((size_t)page * 2 * a.H + head) * hstride + (size_t)(pos % ps) * HD;
+            tma_box(S.K[st], &kvmap, &S.full[st], (int)(off / HD));
+            tma_box(S.V[st], &kvmap, &S.full[st], (int)((off + (size_t)a.H * hstride) / HD));
           }
-          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(&S.full[st])),
-                       "r"((uint32_t)(2 * BOX_BYTES))
-                       : "memory");
-          const int pos = (t_beg + i) * BOX;
-          tma_box(S.K[st], &kvmap, &S.full[st], (int)(a.kv.offset(a.layer, b, pos, head, 0) / HD));
-          tma_box(S.V[st], &kvmap, &S.full[st], (int)(a.kv.offset(a.layer, b, pos, head, 1) / HD));
         }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
     } else {
       {  // this pass's query rows (16 rows x 8 chunks: one chunk per consumer thread)

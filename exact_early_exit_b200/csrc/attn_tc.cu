@@ -145,25 +145,44 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
   volatile int* abort_flag = &S.abort;
 
   if (warp == 4) {
+    // the whole warp walks the key tiles: lanes hold the page ids of the next
+    // 32 pages (loaded ahead, off the per-tile path), lane 0 waits and issues
+    const int ps = a.kv.page_size;
+    const size_t hstride = (size_t)ps * HD, lbase = (size_t)a.layer * a.kv.layer_stride;
+    const int* pt = a.kv.page_table + (size_t)b * a.kv.pages_per_seq;
+    const int plast = pos_last / ps;
+    int chunk = -1, pg = 0;
+    bool ok = true;
+    int issued[KST];
+    for (int s = 0; s < KST; ++s) issued[s] = -1;
     if (lane == 0) {
-      bool ok = true;
-      int issued[KST];
-      for (int s = 0; s < KST; ++s) issued[s] = -1;
       mbar_expect_tx(&S.q_full, (uint32_t)(TQ * HD * 2));
       tma_row_box(S.Q, &qmap, &S.q_full, head * HD, g0);
-      for (int j = 0; j < ntk && ok; ++j) {
-        const int st = j % KST;
-        const uint32_t ph = (uint32_t)((j / KST) & 1);
-        if (!mbar_wait(&S.kv_empty[st], ph ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        issued[st] = (int)ph;
-        mbar_expect_tx(&S.kv_full[st], (uint32_t)(2 * TILE_BYTES));
-        const int pos = j * TK;
-        tma_row_box(S.K[st], &kvmap, &S.kv_full[st], 0, (int)(a.kv.offset(a.layer, b, pos, head, 0) / HD));
-        tma_row_box(S.V[st], &kvmap, &S.kv_full[st], 0, (int)(a.kv.offset(a.layer, b, pos, head, 1) / HD));
+    }
+    for (int j = 0; j < ntk && ok; ++j) {
+      const int st = j % KST;
+      const uint32_t ph = (uint32_t)((j / KST) & 1);
+      const int pos = j * TK, pi = pos / ps;
+      if (pi >= chunk + 32 || chunk < 0) {
+        chunk = pi;
+        pg = chunk + lane <= plast ? pt[chunk + lane] : 0;
       }
+      const int page = __shfl_sync(0xffffffffu, pg, pi - chunk);
+      int go = 1;
+      if (lane == 0) {
+        if (!mbar_wait(&S.kv_empty[st], ph ^ 1u, abort_flag)) {
+          go = 0;
+        } else {
+          issued[st] = (int)ph;
+          mbar_expect_tx(&S.kv_full[st], (uint32_t)(2 * TILE_BYTES));
+          const size_t off = lbase + ((size_t)page * 2 * a.H + head) * hstride + (size_t)(pos % ps) * HD;
+          tma_row_box(S.K[st], &kvmap, &S.kv_full[st], 0, (int)(off / HD));
+          tma_row_box(S.V[st], &kvmap, &S.kv_full[st], 0, (int)((off + (size_t)a.H * hstride) / HD));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, go, 0) != 0;
+    }
+    if (lane == 0) {
       if (*abort_flag) {
         volatile int never = 0;
         mbar_wait(&S.q_full, 0, &never, WAIT_NS / 4);
