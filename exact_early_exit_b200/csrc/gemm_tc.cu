@@ -49,12 +49,14 @@ constexpr int STAGES = 4;        // stages at the largest row tile (256 rows)
 constexpr int MAXST = 12;        // stages when the row tile is small
 constexpr int B_BYTES = BNMAX * BK * 2;
 constexpr int SMEM_TILES = STAGES * (A_BYTES + B_BYTES);
-// Epilogue: two groups of four warps (warp w reads TMEM lanes 32*(w%4)..+31);
-// group g takes the 16-column accumulator chunks 2k+g of a tile, so two
-// chunks are in flight at once
-constexpr int EPI_WARPS = 8;
+// Epilogue: one or two groups of four warps (warp w reads TMEM lanes
+// 32*(w%4)..+31); with two, group g takes the 16-column accumulator chunks
+// 2k+g of a tile, so two chunks are in flight at once.  Launches that may
+// split K (decode: a few rows, fp32 slices) run one group; the others two.
+// The TMA and MMA warps follow the epilogue warps.
+constexpr int EPI_WARPS = 8;  // at most
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-constexpr int WARP_TMA = EPI_WARPS, WARP_MMA = EPI_WARPS + 1;
+constexpr int WARP_TMA = EPI_WARPS, WARP_MMA = EPI_WARPS + 1;  // with two groups
 constexpr int EPI_ROWS = 16;                        // rows per staged chunk (one 32x32b.x16 TMEM load)
 constexpr int EPI_BYTES = 2 * EPI_ROWS * BM * 4;    // fp32 staging tile [16 rows][128 features] per group
 // per-row data of the fused epilogue, two tiles deep: [2][BNMAX] offsets + [2][BNMAX] ints
@@ -62,7 +64,8 @@ constexpr int META_BYTES = 2 * BNMAX * (8 + 4);
 constexpr int SMEM_BYTES = SMEM_TILES + 512 /*barriers*/ + EPI_BYTES + META_BYTES + 1024 /*align*/;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 constexpr uint32_t TMEM_COLS = 512;  // two 256-column fp32 accumulators
-constexpr int THREADS = EPI_THREADS + 64;  // + the TMA warp and the MMA warp
+constexpr int THREADS = EPI_THREADS + 64;  // + the TMA warp and the MMA warp (two groups)
+constexpr int THREADS_1G = 128 + 64;        // one epilogue group
 // row tiles per band of the tile order: within a band the row tile changes
 // fastest, so each weight tile is read once per band and the band's rows
 // (16 x 256 rows) stay in L2 while the feature tiles sweep past
@@ -102,8 +105,8 @@ __device__ __forceinline__ Item decode_item(int it, int ntn, int splits, int R, 
   return t;
 }
 
-// all epilogue warps; the four warps of group g
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory"); }
+// all epilogue warps (ng groups); the four warps of group g
+__device__ __forceinline__ void epi_bar(int ng) { asm volatile("bar.sync 1, %0;" ::"r"(ng * 128) : "memory"); }
 __device__ __forceinline__ void grp_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
 
 // Per-row data of a fused epilogue, gathered into shared memory by the
@@ -116,8 +119,9 @@ __device__ __forceinline__ void grp_bar(int g) { asm volatile("bar.sync %0, 128;
 //   EPI_RESID: off = element offset of the row's residual in h
 //   EPI_HEAD:  iv = the token position t[b] when sequence b stopped here, else -1
 //   EPI_LSE:   iv = the row's target token
-__device__ __forceinline__ void load_row_meta(const EpiArgs& e, int n0, int r0, int rows, long long* off, int* iv) {
-  for (int j = threadIdx.x; j < rows; j += EPI_THREADS) {
+__device__ __forceinline__ void load_row_meta(const EpiArgs& e, int n0, int r0, int rows, long long* off, int* iv,
+                                              int nthreads) {
+  for (int j = threadIdx.x; j < rows; j += nthreads) {
     const int r = r0 + j;
     if (e.mode == EPI_QKV) {
       const int pos = e.rs.row_pos[r];
@@ -309,7 +313,8 @@ struct EpiCtx {
 };
 template <bool PAIR>
 __device__ __forceinline__ void epilogue_warps(const TcArgs& a, const EpiCtx& c, int ntn, int splits, int R,
-                                               int kblocks, int items, int first, int stride, uint32_t rank) {
+                                               int kblocks, int items, int first, int stride, uint32_t rank,
+                                               int ng) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = warp >> 2, qw = warp & 3, gt = threadIdx.x & 127;
   float* sg = c.stile + g * EPI_ROWS * BM;
@@ -324,17 +329,17 @@ __device__ __forceinline__ void epilogue_warps(const TcArgs& a, const EpiCtx& c,
     // the tile's per-row data first (the previous tile's copy is the other
     // buffer: every thread passed this tile's predecessor's barrier, so
     // none still reads the buffer written here)
-    if (direct) load_row_meta(a.epi, n0, t.r0, t.rows, moff, miv);
+    if (direct) load_row_meta(a.epi, n0, t.r0, t.rows, moff, miv, ng * 128);
     // one thread waits, the named barrier releases all epilogue warps
     // together, so an expired wait makes them all leave at the same point
     if (threadIdx.x == 0) c.s_go[ipar] = mbar_wait(c.tfull + acc, aphase, c.abort_flag) ? 1 : 0;
-    epi_bar();
+    epi_bar(ng);
     if (!c.s_go[ipar]) break;
     tc_fence_after();
     const int n = n0 + qw * 32 + lane;
     const uint32_t tbase = c.tmem + ((uint32_t)(qw * 32) << 16) + (uint32_t)(acc * BNMAX);
     float* Ys = a.Y + (size_t)t.split * a.split_stride;
-    for (int c0 = g * EPI_ROWS; c0 < t.nbox * BOXN; c0 += 2 * EPI_ROWS) {
+    for (int c0 = g * EPI_ROWS; c0 < t.nbox * BOXN; c0 += ng * EPI_ROWS) {
       uint32_t v[EPI_ROWS];
       tmem_ld16(tbase + (uint32_t)c0, v);
       const int nr = min(EPI_ROWS, R - (t.r0 + c0));  // may be <= 0 in a ragged last chunk
@@ -386,6 +391,8 @@ __device__ __forceinline__ void epilogue_warps(const TcArgs& a, const EpiCtx& c,
 
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, TcArgs a) {
+  const int ng = ((int)blockDim.x - 64) >> 7;  // epilogue groups: 1 or 2
+  const int warp_tma = 4 * ng, warp_mma = 4 * ng + 1;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -394,7 +401,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // Before waiting for the previous kernel: nothing here reads what it
   // writes.  Pull the weight tiles this CTA will stream when all rows fit
   // one tile (the decode case), and the next GEMM's share, into L2.
-  if (threadIdx.x == WARP_MMA * 32) {
+  if (threadIdx.x == warp_mma * 32) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tw)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tx)) : "memory");
     const int s1 = tc_split_count(1, a.N, a.K, gridDim.x, a.max_split);
@@ -451,7 +458,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(tfull + s, 1);
-      mbar_init(tempty + s, EPI_THREADS);
+      mbar_init(tempty + s, ng * 128);
     }
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -468,7 +475,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == WARP_TMA) {
+  if (warp == warp_tma) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -502,7 +509,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (issued[s] >= 0) mbar_wait(full + s, (uint32_t)issued[s], &never, WAIT_NS / 4);
       }
     }
-  } else if (warp == WARP_MMA) {
+  } else if (warp == warp_mma) {
     if (lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, aphase = 0;
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     EpiCtx c{stile, meta_off, meta_iv, s_go, tfull, tempty, 0u, tmem, abort_flag};
-    epilogue_warps<false>(a, c, ntn, splits, R, kblocks, items, blockIdx.x, gridDim.x, 0u);
+    epilogue_warps<false>(a, c, ntn, splits, R, kblocks, items, blockIdx.x, gridDim.x, 0u, ng);
   }
   __syncthreads();
   if (warp == 0) {
@@ -696,7 +703,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   } else {
     EpiCtx c{stile, meta_off, meta_iv, s_go, tfull, tempty, mapa_shared(smem_u32(tempty), 0), tmem, abort_flag};
-    epilogue_warps<true>(a, c, ntn2, 1, R, kblocks, items, pair, npairs, rank);
+    epilogue_warps<true>(a, c, ntn2, 1, R, kblocks, items, pair, npairs, rank, 2);
   }
   __syncthreads();
   tc_fence_before();
@@ -924,7 +931,7 @@ nv_status tc_gemm_run(TcPlanCache* c, const void* X, int ldx, const void* W, int
   a.pf_bytes = ((uintptr_t)prefetch & 15) ? 0ull : (unsigned long long)prefetch_bytes;
   if (epi) a.epi = *epi;
   else std::memset(&a.epi, 0, sizeof(a.epi));
-  cudaError_t le = launch_k(k_gemm_tc, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tw, tx, a);
+  cudaError_t le = launch_k(k_gemm_tc, dim3(grid), dim3(allow_split ? THREADS_1G : THREADS), SMEM_BYTES, st, tw, tx, a);
   if (le != cudaSuccess) {
     set_error(std::string("tcgen05 GEMM launch: ") + cudaGetErrorString(le));
     return NV_ERR_CUDA;
