@@ -257,13 +257,13 @@ nv_status nv_philox4x32_10(uint64_t seed, const uint32_t *ctr, int n,
  * ctr, out: n x 4 uint32 (host or device); 1 <= n <= NV_PHILOX_NOALLOC_MAX,
  * larger n returns NV_ERR_INVALID_ARG with a message.  The first call on a
  * device looks up the array's device address once, with that device
- * current, and keeps it for the life of the process; make that first call
- * before any stream capture.  A cudaDeviceReset (or any reset of the primary
- * context) unloads the array, so the kept address is no longer valid: do
- * not call this entry point on that device again after such a reset.  All calls share
- * the array and it keeps the last call's contents, so calls that overlap on
- * the GPU (other streams, other host threads) race; serialise them.
- * Synchronous. */
+ * current, and keeps it for the life of the process.  A cudaDeviceReset (or
+ * any reset of the primary context) unloads the array, so the kept address
+ * is no longer valid: do not call this entry point on that device again
+ * after such a reset.  All calls share the array and it keeps the last
+ * call's contents, so calls that overlap on the GPU (other streams, other
+ * host threads) race; serialise them.  Synchronous: the call waits for its
+ * stream, so it cannot be recorded into a stream capture. */
 #define NV_PHILOX_NOALLOC_MAX 32768
 nv_status nv_philox4x32_10_noalloc(uint64_t seed, const uint32_t *ctr, int n,
                                    uint32_t *out, void *stream);
