@@ -84,6 +84,25 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
+// packed pairs of fp32 (sm_100 f32x2 instructions: each lane of the pair is
+// an ordinary IEEE fp32 operation, rounded to nearest)
+__device__ __forceinline__ uint64_t as_u64(float2 v) { return *reinterpret_cast<const uint64_t*>(&v); }
+__device__ __forceinline__ float2 as_f2(uint64_t v) { return *reinterpret_cast<const float2*>(&v); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)), "l"(as_u64(c)));
+  return as_f2(r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
+  return as_f2(r);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
+  return as_f2(r);
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -302,17 +321,21 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
 #pragma unroll
         for (int i = 0; i < TK; ++i) r[i] = 0u;
       } else {
-        // the row sum as eight partial sums added in a fixed tree
-        float ps[8];
+        // the row sum as eight partial sums (element i into sum i % 8, as
+        // pairs) added in a fixed tree
+        const float2 sc2 = make_float2(scale2, scale2), nm2 = make_float2(-mref, -mref);
+        float2 ps[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) ps[c] = 0.f;
+        for (int c = 0; c < 4; ++c) ps[c] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < TK; ++i) {
-          const float p = ex2(__fmaf_rn(__uint_as_float(r[i]), scale2, -mref));
-          r[i] = __float_as_uint(p);
-          ps[i & 7] += p;
+        for (int e = 0; e < TK / 2; ++e) {
+          const float2 y = fma2(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), sc2, nm2);
+          const float2 p = make_float2(ex2(y.x), ex2(y.y));
+          r[2 * e] = __float_as_uint(p.x);
+          r[2 * e + 1] = __float_as_uint(p.y);
+          ps[e & 3] = add2(ps[e & 3], p);
         }
-        rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        rs = ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) + ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
       }
       l = l * cj + rs;
       // P as bf16 pairs, hi = bf16(P) and lo = bf16(P - hi), packed
@@ -323,7 +346,8 @@ __global__ void __launch_bounds__(FT_THREADS, 2)
         const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
         const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
         pk[e] = *reinterpret_cast<const uint32_t*>(&hb);
-        pk[TK / 2 + e] = pack2(x0 - __low2float(hb), x1 - __high2float(hb));
+        const float2 lo = sub2(make_float2(x0, x1), make_float2(__low2float(hb), __high2float(hb)));
+        pk[TK / 2 + e] = pack2(lo.x, lo.y);
       }
       // the previous tile's P V must be done with P (and with O) first
       if (j > 0 && !sm_wait(S, &S.o_full, (uint32_t)((j - 1) & 1))) {
