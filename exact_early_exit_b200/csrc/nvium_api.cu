@@ -1452,8 +1452,15 @@ nv_status decode_step_impl(nv_state* s, uint64_t seed, int32_t* tokens_out, int3
   } else {
     if (!s->graph) {
       cudaGraph_t g = nullptr;
+      // Conditional blocks pay off when a step may leave an exit block
+      // unreached; with 32 or more sequences every block runs in practice
+      // (the chance that no token passes an exit is the product of the
+      // sequences' stop probabilities), so the step is one flat graph, which
+      // saves the conditional nodes' launch latency.  NVIUM_COND_GRAPH=1 / 0
+      // forces either form.
       const char* cg = std::getenv("NVIUM_COND_GRAPH");
-      const bool try_cond = !(cg && cg[0] == '0') && M->NE > 1;
+      const bool want_cond = cg ? cg[0] != '0' : s->B < 32;
+      const bool try_cond = want_cond && M->NE > 1;
       if (!try_cond || build_conditional_step_graph(s, &g) != NV_OK) {
         // one flat graph of every layer (conditional nodes unavailable or disabled)
         g = nullptr;
