@@ -266,23 +266,39 @@ __device__ __forceinline__ void tile_epilogue(const EpiArgs& e, const float* S, 
     // target token's logit when the target falls in this tile
     const int lane = tid & 31, w = tid >> 5;
     constexpr float LOG2E = 1.4426950408889634f;
-    for (int j = w; j < nrows; j += 4) {
-      const float* row = S + j * BM;
-      float x[4];
+    // a warp takes rows w, w+4, w+8, w+12 of the staged chunk together, so
+    // the four rows' butterflies interleave instead of running one by one
+    constexpr int RPW = EPI_ROWS / 4;
+    float x[RPW][4], M[RPW], Ssum[RPW];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) x[i] = row[lane + 32 * i];
-      float M = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    for (int k = 0; k < RPW; ++k) {
+      const int j = w + 4 * k;
 #pragma unroll
-      for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      float Ssum = 0.f;
+      for (int i = 0; i < 4; ++i) x[k][i] = j < nrows ? S[j * BM + lane + 32 * i] : 0.f;
+      M[k] = fmaxf(fmaxf(x[k][0], x[k][1]), fmaxf(x[k][2], x[k][3]));
+    }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) Ssum += exp2_approx(__fmul_rn(x[i] - M, LOG2E));
+    for (int o = 16; o; o >>= 1)
 #pragma unroll
-      for (int o = 16; o; o >>= 1) Ssum += __shfl_xor_sync(0xffffffffu, Ssum, o);
+      for (int k = 0; k < RPW; ++k) M[k] = fmaxf(M[k], __shfl_xor_sync(0xffffffffu, M[k], o));
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+      Ssum[k] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Ssum[k] += exp2_approx(__fmul_rn(x[k][i] - M[k], LOG2E));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int k = 0; k < RPW; ++k) Ssum[k] += __shfl_xor_sync(0xffffffffu, Ssum[k], o);
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+      const int j = w + 4 * k;
+      if (j >= nrows) break;
       const int r = r0 + j;
-      if (lane == 0) e.lse_part[(size_t)r * e.nblk + n0 / BM] = make_float2(M, Ssum);
+      if (lane == 0) e.lse_part[(size_t)r * e.nblk + n0 / BM] = make_float2(M[k], Ssum[k]);
       const int tg = iv[j] - n0;
-      if (tg >= 0 && tg < BM && (tg & 31) == lane) e.lse_tgt[r] = row[tg];
+      if (tg >= 0 && tg < BM && (tg & 31) == lane) e.lse_tgt[r] = S[j * BM + tg];
     }
   } else if (e.mode == EPI_SWIGLU) {
 #pragma unroll 4
