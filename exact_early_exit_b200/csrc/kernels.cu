@@ -1198,98 +1198,294 @@ void launch_adapter_norm_rows(bool bf16, RowSet rs, const float* Y, const void* 
 }
 
 // ---------------------------------------------------------------------------
-// Fused exit-head sampler (exact sampling, section 3; Gumbel-max reading).
-// For the rows that stopped at exit k: logit_v = W_k[v] . n_k with 16-byte
-// coalesced loads of each head row, score_v = logit_v + Gumbel(U_v) with U_v
-// from counter (b, t, 1, v/4) lane v%4, running argmax (ties to the lowest v)
-// and online log-sum-exp of the logits.  Logits never leave the chip; each CTA
-// writes one partial per row, merged by k_head_reduce in CTA order.
+// Fused exit-head sampler (exact sampling, section 3; Gumbel-max reading),
+// for the batches the tensor-core head does not take.  For the rows that
+// stopped at exit k: logit_v = W_k[v] . n_k, score_v = logit_v + Gumbel(U_v)
+// with U_v from counter (b, t, 1, v/4) lane v%4, running argmax (ties to the
+// lowest v) and online log-sum-exp of the logits.  Logits never leave the
+// chip; each CTA writes one partial per row, merged by k_head_reduce in CTA
+// order.
+//
+// One CTA per SM streams a contiguous range of head rows (a multiple of four,
+// the rows of one Philox draw) through a shared-memory ring: a producer
+// thread copies HS_ROWS rows per stage with one bulk copy (cp.async.bulk,
+// completion counted on the stage's mbarrier).  The consumer warps form two
+// teams that take alternate stages; in a stage, warp q of the team takes the
+// q-th group of four rows: one Philox draw serves the group, the four dot
+// products share each activation chunk and run as independent chains, and
+// the stage goes back to the producer as soon as the rows are in registers.
+// Stopped rows beyond one pass (rp rows, at most HEAD_RMAX, the lanes of a
+// warp) are taken in further passes over the same range.
 // ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
+constexpr int HS_TEAM = 4;                       // warps per team: the groups of a stage
+constexpr int HS_WARPS = 2 * HS_TEAM;            // consumer warps
+constexpr int HS_THREADS = 32 * (HS_WARPS + 1);  // + one producer warp
+constexpr int HS_ROWS = 4 * HS_TEAM;             // head rows per stage
+constexpr int HS_MAX_STAGES = 8;
+constexpr int HS_MAXC = 8;                       // 16-byte chunks of a row per lane (d * size <= 4096 bytes)
+constexpr size_t HS_DYN_MAX = 208 * 1024;        // dynamic shared memory of one CTA
+
+struct HeadPlan {
+  int rp = 0, stages = 0;
+  size_t act_off = 0, ring_off = 0, bytes = 0;
+};
+// list of stopped rows [B] | rp activation rows | ring of `stages` x HS_ROWS head rows
+static HeadPlan head_plan(int B, int d, size_t esz) {
+  HeadPlan p;
+  const size_t rowb = (size_t)d * esz, stage = HS_ROWS * rowb;
+  auto al = [](size_t x) { return (x + 127) / 128 * 128; };
+  p.act_off = al((size_t)B * 4);
+  if (rowb % 16 || rowb > 16 * 32 * HS_MAXC || p.act_off + rowb + 2 * stage > HS_DYN_MAX) return HeadPlan{};
+  size_t rp = (size_t)(B < HEAD_RMAX ? B : HEAD_RMAX);
+  const size_t rp_fit = (HS_DYN_MAX - p.act_off - 2 * stage) / rowb;
+  if (rp > rp_fit) rp = rp_fit;
+  p.rp = (int)rp;
+  p.ring_off = al(p.act_off + rp * rowb);
+  size_t ns = (HS_DYN_MAX - p.ring_off) / stage;
+  if (ns > HS_MAX_STAGES) ns = HS_MAX_STAGES;
+  p.stages = (int)ns;
+  p.bytes = p.ring_off + ns * stage;
+  return p;
+}
+bool head_sample_fits(int B, int d, size_t esz) { return head_plan(B, d, esz).stages >= 2; }
+
+__device__ __forceinline__ void hs_bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool hs_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait of one thread on an mbarrier phase: false when 2 s passed
+// (the thread raises `abort` and the device error word) or another thread
+// raised `abort`.
+__device__ __forceinline__ bool hs_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                        unsigned long long limit_ns = 2000000000ull) {
+  if (hs_try_wait(bar, parity)) return true;
+  unsigned long long t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t i = 1;; ++i) {
+    if (hs_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0u) {
+      if (*abort) return false;
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > limit_ns) {
+        *abort = 1;
+        dev_fail(status, DEV_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// c + w.lo * a.lo, then + w.hi * a.hi for two packed bf16 pairs: each step
+// one fused multiply-add of two bf16 values into fp32 (their product is exact
+// in fp32), so the result equals fmaf on the converted values
+__device__ __forceinline__ float fma_bf16x2_seq(uint32_t w, uint32_t a, float c) {
+  asm("{\n\t.reg .b16 wl, wh, al, ah;\n\tmov.b32 {wl, wh}, %1;\n\tmov.b32 {al, ah}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, wl, al, %0;\n\tfma.rn.f32.bf16 %0, wh, ah, %0;\n\t}"
+      : "+f"(c)
+      : "r"(w), "r"(a));
+  return c;
+}
+// barrier of the consumer warps only (the producer warp keeps streaming)
+__device__ __forceinline__ void hs_cbar() { asm volatile("bar.sync 1, %0;" ::"r"(HS_WARPS * 32) : "memory"); }
+__device__ __forceinline__ bool hs_cbar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(HS_WARPS * 32)
+      : "memory");
+  return r != 0;
+}
+
+// MAXC: 16-byte chunks of a head row per lane (a row is 32 * MAXC chunks at most)
+template <typename T, int MAXC>
+__global__ void __launch_bounds__(HS_THREADS, 1) k_head_sample(HeadArgs a) {
   pdl_wait();
   pdl_launch();
-  constexpr int NW = 8, EPC = 16 / sizeof(T), MAXC = 8;
-  extern __shared__ __align__(16) unsigned char smem[];
-  int* s_list = (int*)smem;                                   // [B]
-  T* s_act = (T*)(smem + (((size_t)a.B * 4 + 15) / 16) * 16);  // [HEAD_RMAX][d]
-  __shared__ float s_part[NW][HEAD_RMAX][HEAD_PART];
+  constexpr int EPC = 16 / sizeof(T);
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ float s_part[HS_WARPS][HEAD_RMAX][HEAD_PART];
+  __shared__ float s_gm[HS_WARPS][HEAD_RMAX][4];  // Gumbel noise of a warp's group
   __shared__ int s_b[HEAD_RMAX], s_t[HEAD_RMAX];
+  __shared__ __align__(8) uint64_t s_full[HS_MAX_STAGES], s_empty[HS_MAX_STAGES];
+  __shared__ int s_n;
+  __shared__ volatile int s_abort;
+  int* s_list = (int*)smem;                          // [B]
+  T* s_act = (T*)(smem + a.act_off);                 // [rp][d]
+  T* ring = (T*)(smem + a.ring_off);                 // [stages][HS_ROWS][d]
   const int B = a.B, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int d = a.d, V = a.V, NS = a.stages, RP = a.rp;
   // compact the rows that stopped here, in sequence order
-  const int ipt = (B + 255) / 256;
-  int local = 0;
-  for (int i = 0; i < ipt; ++i) {
-    const int b = tid * ipt + i;
-    if (b < B) local += a.stop[b] ? 1 : 0;
-  }
-  int n;
-  int off = block_exclusive_scan<256>(local, &n);
-  for (int i = 0; i < ipt; ++i) {
-    const int b = tid * ipt + i;
-    if (b < B && a.stop[b]) s_list[off++] = b;
+  if (w == 0) {
+    int n = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + lane;
+      const bool st = b < B && a.stop[b] != 0;
+      const unsigned m = __ballot_sync(0xffffffffu, st);
+      if (st) s_list[n + __popc(m & ((1u << lane) - 1u))] = b;
+      n += __popc(m);
+    }
+    if (lane == 0) {
+      s_n = n;
+      s_abort = 0;
+      for (int s = 0; s < NS; ++s) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&s_full[s])) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&s_empty[s])), "r"(HS_TEAM)
+                     : "memory");
+      }
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
   }
   __syncthreads();
+  const int n = s_n;
   if (n == 0) return;
-  const unsigned long long seed = *a.seed;
-  const int d = a.d, V = a.V;
-  const int nchunk = d / EPC;  // 16-byte chunks per row
-  // this CTA's vocab range, a multiple of 4 rows
+  // this CTA's head rows [rbeg, rend): whole groups of four
   const int groups = (V + 3) / 4;
   const int gpc = (groups + gridDim.x - 1) / gridDim.x;
-  const int gbeg = blockIdx.x * gpc, gend = min(groups, gbeg + gpc);
-  for (int p0 = 0; p0 < n; p0 += HEAD_RMAX) {
-    const int nr = min(HEAD_RMAX, n - p0);
-    __syncthreads();
-    for (int i = tid; i < nr * nchunk; i += 256) {
-      const int r = i / nchunk, c = i % nchunk;
-      ((uint4*)s_act)[(size_t)r * nchunk + c] =
-          ((const uint4*)((const T*)a.exit_act + (size_t)s_list[p0 + r] * d))[c];
+  const int rbeg = min(V, (int)blockIdx.x * gpc * 4), rend = min(V, rbeg + gpc * 4);
+  const int nst = (rend - rbeg + HS_ROWS - 1) / HS_ROWS;  // stages per pass
+  const int passes = (n + RP - 1) / RP;
+  if (w == HS_WARPS) {
+    // producer: the same stage sequence, pass after pass
+    if (lane != 0) return;
+    const T* head = (const T*)a.head;
+    int i = 0;
+    bool ok = true;
+    for (int p = 0; p < passes && ok; ++p) {
+      for (int s = 0; s < nst; ++s, ++i) {
+        const int slot = i % NS;
+        if (i >= NS && !hs_wait(&s_empty[slot], (uint32_t)((i / NS - 1) & 1), &s_abort, a.status)) {
+          ok = false;
+          break;
+        }
+        const int r0 = rbeg + s * HS_ROWS, nr = min(HS_ROWS, rend - r0);
+        const uint32_t bytes = (uint32_t)((size_t)nr * d * sizeof(T));
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&s_full[slot])),
+                     "r"(bytes)
+                     : "memory");
+        hs_bulk_load(ring + (size_t)slot * HS_ROWS * d, head + (size_t)r0 * d, bytes, &s_full[slot]);
+      }
+    }
+    // no copy may still be landing when the CTA's shared memory goes: wait
+    // (bounded) for the last stages issued; after a normal run the consumers
+    // have already seen them complete
+    int never = 0;
+    for (int j = max(0, i - NS); j < i; ++j)
+      hs_wait(&s_full[j % NS], (uint32_t)((j / NS) & 1), &never, nullptr, 100000000ull);
+    return;
+  }
+  // consumers
+  const int nchunk = d / EPC;  // 16-byte chunks per row
+  const unsigned long long seed = *a.seed;
+  int i = 0;  // stage sequence number, as the producer counts it
+  for (int p0 = 0; p0 < n; p0 += RP) {
+    const int nr = min(RP, n - p0);
+    hs_cbar();  // the previous pass's rows and partials are no longer read
+    for (int x = tid; x < nr * nchunk; x += HS_WARPS * 32) {
+      const int r = x / nchunk, c = x % nchunk;
+      ((uint4*)s_act)[(size_t)r * nchunk + c] = ((const uint4*)((const T*)a.exit_act + (size_t)s_list[p0 + r] * d))[c];
     }
     if (tid < nr) {
       s_b[tid] = s_list[p0 + tid];
       s_t[tid] = a.t[s_list[p0 + tid]];
     }
-    __syncthreads();
+    hs_cbar();
     // lane r keeps row r's running state
     float best_s = -CUDART_INF_F, best_l = 0.f, mx = -CUDART_INF_F, se = 0.f;
     int best_v = 0x7fffffff;
-    const int myb = lane < nr ? s_b[lane] : 0, myt = lane < nr ? s_t[lane] : 0;
-    for (int g = gbeg + w; g < gend; g += NW) {
-      uint4 rb = make_uint4(0, 0, 0, 0);
-      if (lane < nr)
-        rb = philox4x32_10(make_uint4((uint32_t)myb, (uint32_t)myt, STREAM_GUMBEL, (uint32_t)g), (uint32_t)seed,
-                           (uint32_t)(seed >> 32));
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        const int v = 4 * g + q;
-        if (v >= V) break;
-        uint4 wv[MAXC];
-        const uint4* wrow = (const uint4*)((const T*)a.head + (size_t)v * d);
+    bool ok = true;
+    const int team = w / HS_TEAM, q = w % HS_TEAM;
+    for (int s = 0; s < nst; ++s, ++i) {
+      if ((i & 1) != team) continue;
+      const int slot = i % NS;
+      const int v0 = rbeg + s * HS_ROWS + 4 * q;  // this warp's group: rows v0 .. v0 + nv - 1
+      const int nv = min(4, rend - v0);
+      // Gumbel noise of the group: one Philox draw per stopped row gives its
+      // four lanes; entry (r, j) is computed by lane 4r + j (+ 32 per round)
+      __syncwarp();  // the previous group's noise has been read
+      if (nv > 0) {
+        for (int x = lane; x < 4 * nr; x += 32) {
+          const int r = x >> 2, j = x & 3;
+          float g = 0.f;
+          if (j < nv) {
+            const uint4 rb = philox4x32_10(
+                make_uint4((uint32_t)s_b[r], (uint32_t)s_t[r], STREAM_GUMBEL, (uint32_t)(v0 >> 2)), (uint32_t)seed,
+                (uint32_t)(seed >> 32));
+            g = -logf(-logf(uniform01(lane_of(rb, j))));
+          }
+          s_gm[w][r][j] = g;
+        }
+      }
+      // lane 0 waits, the warp follows its verdict
+      int got = 1;
+      if (lane == 0) got = hs_wait(&s_full[slot], (uint32_t)((i / NS) & 1), &s_abort, a.status) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        ok = false;
+        break;
+      }
+      uint4 wv[4][MAXC];
+      if (nv > 0) {
+        const uint4* wrow = (const uint4*)(ring + ((size_t)slot * HS_ROWS + 4 * q) * d);
 #pragma unroll
-        for (int c = 0; c < MAXC; ++c)
-          if (lane + 32 * c < nchunk) wv[c] = __ldg(wrow + lane + 32 * c);
-        float gm = 0.f;
-        if (lane < nr) gm = -logf(-logf(uniform01(lane_of(rb, q))));
-        for (int r = 0; r < nr; ++r) {
-          const uint4* arow = (const uint4*)s_act + (size_t)r * nchunk;
-          float part = 0.f;
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int c = 0; c < MAXC; ++c) {
-            if (lane + 32 * c < nchunk) {
-              const uint4 av = arow[lane + 32 * c];
-              const T* wp = (const T*)&wv[c];
+          for (int c = 0; c < MAXC; ++c)
+            if (j < nv && lane + 32 * c < nchunk) wv[j][c] = wrow[(size_t)j * nchunk + lane + 32 * c];
+      }
+      // the rows are in registers: hand the stage back
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&s_empty[slot])) : "memory");
+      if (nv <= 0) continue;
+      for (int r = 0; r < nr; ++r) {
+        const uint4* arow = (const uint4*)s_act + (size_t)r * nchunk;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < MAXC; ++c) {
+          if (lane + 32 * c < nchunk) {
+            const uint4 av = arow[lane + 32 * c];
+            if constexpr (sizeof(T) == 2) {
+              const uint32_t* aw = (const uint32_t*)&av;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) part[j] = fma_bf16x2_seq(((const uint32_t*)&wv[j][c])[k], aw[k], part[j]);
+            } else {
               const T* ap = (const T*)&av;
 #pragma unroll
-              for (int e = 0; e < EPC; ++e) part = fmaf(ld(wp + e), ld(ap + e), part);
+              for (int e = 0; e < EPC; ++e) {
+                const float x = ld(ap + e);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) part[j] = fmaf(ld((const T*)&wv[j][c] + e), x, part[j]);
+              }
             }
           }
-          const float logit = warp_sum(part);
-          if (lane == r) {
-            const float s = logit + gm;
-            if (s > best_s) {
-              best_s = s;
-              best_v = v;
+        }
+        // four butterflies, interleaved
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+        if (lane == r) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j >= nv) break;
+            const float logit = part[j];
+            const float sc = logit + s_gm[w][r][j];
+            if (sc > best_s) {
+              best_s = sc;
+              best_v = v0 + j;
               best_l = logit;
             }
             if (logit > mx) {
@@ -1302,6 +1498,8 @@ __global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
         }
       }
     }
+    // every consumer leaves together when any of them gave up
+    if (hs_cbar_or(!ok || s_abort)) return;
     if (lane < nr) {
       s_part[w][lane][0] = best_s;
       s_part[w][lane][1] = __int_as_float(best_v);
@@ -1309,15 +1507,15 @@ __global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
       s_part[w][lane][3] = mx;
       s_part[w][lane][4] = se;
     }
-    __syncthreads();
+    hs_cbar();
     if (tid < nr) {
       float bs = -CUDART_INF_F, bl = 0.f, M = -CUDART_INF_F, S = 0.f;
       int bv = 0x7fffffff;
-      for (int ww = 0; ww < NW; ++ww) {
-        const float s = s_part[ww][tid][0];
+      for (int ww = 0; ww < HS_WARPS; ++ww) {
+        const float sc = s_part[ww][tid][0];
         const int v = __float_as_int(s_part[ww][tid][1]);
-        if (s > bs || (s == bs && v < bv)) {
-          bs = s;
+        if (sc > bs || (sc == bs && v < bv)) {
+          bs = sc;
           bv = v;
           bl = s_part[ww][tid][2];
         }
@@ -1339,11 +1537,25 @@ __global__ void __launch_bounds__(256) k_head_sample(HeadArgs a) {
     }
   }
 }
+template <int MAXC>
+static void launch_head_sample_c(bool bf16, const HeadArgs& b, size_t bytes, cudaStream_t st) {
+  if (bf16) launch_k(k_head_sample<__nv_bfloat16, MAXC>, b.nblk, HS_THREADS, bytes, st, b);
+  else launch_k(k_head_sample<float, MAXC>, b.nblk, HS_THREADS, bytes, st, b);
+}
 void launch_head_sample(bool bf16, const HeadArgs& a, cudaStream_t st) {
   const size_t esz = bf16 ? 2 : 4;
-  const size_t sm = (((size_t)a.B * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * a.d * esz;
-  if (bf16) launch_k(k_head_sample<__nv_bfloat16>, a.nblk, 256, sm, st, a);
-  else launch_k(k_head_sample<float>, a.nblk, 256, sm, st, a);
+  const HeadPlan p = head_plan(a.B, a.d, esz);  // the state checked head_sample_fits
+  HeadArgs b = a;
+  b.rp = p.rp;
+  b.stages = p.stages;
+  b.act_off = (int)p.act_off;
+  b.ring_off = (int)p.ring_off;
+  // the register tile of four rows fits the row length
+  const int per_lane = ((int)(a.d * esz / 16) + 31) / 32;
+  if (per_lane <= 2) launch_head_sample_c<2>(bf16, b, p.bytes, st);
+  else if (per_lane <= 4) launch_head_sample_c<4>(bf16, b, p.bytes, st);
+  else if (per_lane <= 6) launch_head_sample_c<6>(bf16, b, p.bytes, st);
+  else launch_head_sample_c<HS_MAXC>(bf16, b, p.bytes, st);
 }
 
 __global__ void k_head_reduce(HeadArgs a) {
@@ -1590,13 +1802,19 @@ void launch_set_cond(cudaGraphConditionalHandle h, const int* active, const int*
   launch_k(k_set_cond, 1, 256, 0, st, h, active, force, B, counters, block_launches);
 }
 
-cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes) {
-  cudaError_t e = cudaSuccess;
-  if (head_bytes > 48 * 1024) {
-    e = cudaFuncSetAttribute(k_head_sample<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)head_bytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_head_sample<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)head_bytes);
-  }
+template <int MAXC>
+static cudaError_t head_sample_smem_limit() {
+  cudaError_t e = cudaFuncSetAttribute(k_head_sample<__nv_bfloat16, MAXC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)HS_DYN_MAX);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_head_sample<float, MAXC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HS_DYN_MAX);
+  return e;
+}
+cudaError_t kernels_set_smem_limits(size_t plan_bytes) {
+  cudaError_t e = head_sample_smem_limit<2>();
+  if (e == cudaSuccess) e = head_sample_smem_limit<4>();
+  if (e == cudaSuccess) e = head_sample_smem_limit<6>();
+  if (e == cudaSuccess) e = head_sample_smem_limit<HS_MAXC>();
   if (e == cudaSuccess && plan_bytes > 48 * 1024) {
     e = cudaFuncSetAttribute(k_plan_norm<__nv_bfloat16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)plan_bytes);

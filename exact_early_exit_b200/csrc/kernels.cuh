@@ -214,10 +214,17 @@ struct HeadArgs {
   int nblk;
   long long* counters;
   long long head_bytes;
+  int* status;           // device error word (a bounded wait that ran out)
+  // shared-memory plan of the sampler, filled by launch_head_sample
+  int rp, stages, act_off, ring_off;
   // reduce
   int* sampled;
   float* logp;
 };
+// The small-batch sampler runs one CTA per SM (nblk = the SM count) and
+// needs its stopped-row list, one pass of rows and a ring of at least two
+// stages in shared memory; false when B and d leave no such plan.
+bool head_sample_fits(int B, int d, size_t esz);
 void launch_head_sample(bool bf16, const HeadArgs& a, cudaStream_t st);
 void launch_head_reduce(const HeadArgs& a, cudaStream_t st);
 
@@ -240,7 +247,7 @@ void launch_set_cond(cudaGraphConditionalHandle h, const int* active, const int*
 void launch_philox(unsigned long long seed, const void* ctr, int n, void* out, cudaStream_t st);
 
 // Opt-in shared memory for the head sampler and the planner.
-cudaError_t kernels_set_smem_limits(size_t head_bytes, size_t plan_bytes);
+cudaError_t kernels_set_smem_limits(size_t plan_bytes);
 
 // Normalised depth of each exit: exit_layers[k] / n_layers.
 struct ExitFrac {

@@ -648,6 +648,7 @@ nv_status record_layers(nv_state* s, cudaStream_t st, Prof* prof, long long* lau
     h.part = s->head_part;
     h.nblk = s->head_nblk;
     h.counters = s->counters;
+    h.status = s->status;
     h.head_bytes = (long long)M->V * M->d * es;
     h.sampled = s->sampled;
     h.logp = s->logp;
@@ -1068,8 +1069,7 @@ nv_status nv_create(const nv_config* cfg, const nv_weights* w, nv_model** out) {
     return gs;
   }
   {
-    const size_t head_sm = (((size_t)cfg->max_batch * 4 + 15) / 16) * 16 + (size_t)HEAD_RMAX * d * esz;
-    cudaError_t e2 = kernels_set_smem_limits(head_sm, (size_t)(cfg->max_batch + 1) * 4);
+    cudaError_t e2 = kernels_set_smem_limits((size_t)(cfg->max_batch + 1) * 4);
     if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_mma_prepare();
     if (e2 == cudaSuccess && M->bf16 && M->hd == 64) e2 = attn_dec_pc_prepare();
     if (e2 == cudaSuccess && M->tc_attention) e2 = attn_tc_prepare();
@@ -1136,7 +1136,8 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
     s->kv_splits = ks < 1 ? 1 : (ks > 16 ? 16 : ks);
   }
   s->row_groups = (s->cap + 1 + ATTN_RPC - 1) / ATTN_RPC;
-  s->head_nblk = 296;
+  // the small-batch sampler runs one CTA per SM
+  s->head_nblk = tc_sm_count();
   const size_t wide = d > F ? d : F;
   s->Y_elems = gemm_workspace_elems(M->gemm_kind, (size_t)s->max_rows, (size_t)(3 * HQ > 2 * F ? 3 * HQ : 2 * F));
   nv_status st = NV_OK;
@@ -1174,7 +1175,8 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   A(&s->exit_act, (size_t)B * d * esz);
   A((void**)&s->Y, s->Y_elems * 4);
   A((void**)&s->attn_part, (size_t)s->max_rows * M->H * s->kv_splits * (M->hd + 2) * 4);
-  A((void**)&s->head_part, (size_t)B * s->head_nblk * HEAD_PART * 4);
+  // partials of the sampler (one per CTA) or of the tensor-core head (one per 128 vocab rows)
+  A((void**)&s->head_part, (size_t)B * std::max(s->head_nblk, (M->V + 127) / 128) * HEAD_PART * 4);
   A((void**)&s->seed_dev, 8);
   A((void**)&s->counters, NV_CTR_COUNT * 8);
   A((void**)&s->status, 4);
@@ -1189,6 +1191,11 @@ nv_status nv_state_create(nv_model* M, int B, nv_state** out) {
   cudaMemset(s->nstop, 0, (size_t)NV_MAX_EXITS * 4);
   cudaMemcpy(s->d_B, &B, 4, cudaMemcpyHostToDevice);
   s->tc_head = M->bf16 && M->gemm_kind == GEMM_TC && B >= 16 && M->V % 128 == 0 && M->d % 64 == 0;
+  if (!s->tc_head && !head_sample_fits(B, M->d, M->esz)) {
+    set_error("nv_state_create: the exit-head sampler has no shared-memory plan for this batch and d_model");
+    nv_state_destroy(s);
+    return NV_ERR_UNSUPPORTED;
+  }
   {
     // the MMA decode attention reads the pool through a tensor map: rows of
     // 128 bytes, boxes of 64 positions, row coordinates within int32
