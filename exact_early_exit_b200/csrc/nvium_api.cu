@@ -500,7 +500,9 @@ LayerIO state_io(nv_state* s) {
   io.row_groups = s->row_groups;
   io.lens = s->lens;
   io.L = s->m->L;
-  io.epi_grid = 1184;
+  // split-K epilogues: a few rows per sequence at small batch, where a
+  // smaller grid starts sooner; 8 CTAs per SM otherwise
+  io.epi_grid = s->B <= 8 ? 296 : 1184;
   io.dec_attn = s->dec_attn;
   io.kv_map = s->kv_map_ok ? &s->kv_map : nullptr;
   io.kv_map32 = s->kv_map32_ok ? &s->kv_map32 : nullptr;
