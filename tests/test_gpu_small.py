@@ -251,6 +251,19 @@ def test_mma_and_simt_scoring_attention_agree(weights):
     np.testing.assert_allclose(out["mma"], out["simt"], atol=tolerance(CFG), rtol=0)
 
 
+def test_sampler_many_rows_at_one_exit_bf16():
+    """Twelve sequences that all stop at the first exit (router bias +30): the
+    small-batch sampler takes twelve stopped rows in one pass, its Gumbel
+    draws in two rounds over a warp's lanes (four lanes per row).  Tokens,
+    exits and log-probs against the oracle, then every cache after the flush."""
+    w = W.make_weights(CFG, seed=0, router_bias=[30.0, 0.0, 0.0])
+    wl = W.WORKLOADS["S"]
+    prompts = [p[:n] for p, n in zip(W.make_prompts(wl, seed=5, lengths=[40] * 12), range(5, 41, 3))]
+    chk, state, dec, _ = run_decode_parity(nv, CFG, w, prompts, 6, max_pending=8)
+    chk.report("B=12, every row at exit 1")
+    assert chk.steps == 6
+
+
 def test_decode_parity_bf16_degenerate_and_ragged_prompts(weights):
     """A one-token prompt (no prefill rows), one ending a 64-row query tile
     plus one row, and one spanning several key tiles, through the MMA
