@@ -1214,8 +1214,11 @@ void launch_adapter_norm_rows(bool bf16, RowSet rs, const float* Y, const void* 
 // q-th group of four rows: one Philox draw serves the group, the four dot
 // products share each activation chunk and run as independent chains, and
 // the stage goes back to the producer as soon as the rows are in registers.
-// Stopped rows beyond one pass (rp rows, at most HEAD_RMAX, the lanes of a
-// warp) are taken in further passes over the same range.
+// A warp draws the Gumbel noise of its next groups together (one lane per
+// stopped row, group and row of the group), and the four lanes 4r'+j keep
+// stopped row r's running argmax and log-sum-exp over the rows v = j mod 4,
+// merged once at the end.  Stopped rows beyond one pass (rp rows, at most
+// HS_RP) are taken in further passes over the same range.
 // ---------------------------------------------------------------------------
 constexpr int HS_TEAM = 4;                       // warps per team: the groups of a stage
 constexpr int HS_WARPS = 2 * HS_TEAM;            // consumer warps
@@ -1223,6 +1226,8 @@ constexpr int HS_THREADS = 32 * (HS_WARPS + 1);  // + one producer warp
 constexpr int HS_ROWS = 4 * HS_TEAM;             // head rows per stage
 constexpr int HS_MAX_STAGES = 8;
 constexpr int HS_MAXC = 8;                       // 16-byte chunks of a row per lane (d * size <= 4096 bytes)
+constexpr int HS_RP = 16;                        // stopped rows per pass
+constexpr int HS_SLOTS = HS_RP / 8;              // running states per lane (8 rows x 4 lanes per slot)
 constexpr size_t HS_DYN_MAX = 208 * 1024;        // dynamic shared memory of one CTA
 
 struct HeadPlan {
@@ -1236,7 +1241,7 @@ static HeadPlan head_plan(int B, int d, size_t esz) {
   auto al = [](size_t x) { return (x + 127) / 128 * 128; };
   p.act_off = al((size_t)B * 4);
   if (rowb % 16 || rowb > 16 * 32 * HS_MAXC || p.act_off + rowb + 2 * stage > HS_DYN_MAX) return HeadPlan{};
-  size_t rp = (size_t)(B < HEAD_RMAX ? B : HEAD_RMAX);
+  size_t rp = (size_t)(B < HS_RP ? B : HS_RP);
   const size_t rp_fit = (HS_DYN_MAX - p.act_off - 2 * stage) / rowb;
   if (rp > rp_fit) rp = rp_fit;
   p.rp = (int)rp;
@@ -1296,6 +1301,23 @@ __device__ __forceinline__ float fma_bf16x2_seq(uint32_t w, uint32_t a, float c)
       : "r"(w), "r"(a));
   return c;
 }
+// one head row into a stopped row's running state: argmax of the Gumbel
+// score (rows arrive in increasing v, so the first maximum is kept) and the
+// online log-sum-exp of the logits
+__device__ __forceinline__ void hs_update(float sc, float logit, int v, float& best_s, int& best_v, float& best_l,
+                                          float& mx, float& se) {
+  if (sc > best_s) {
+    best_s = sc;
+    best_v = v;
+    best_l = logit;
+  }
+  if (logit > mx) {
+    se = se * expf(mx - logit) + 1.0f;
+    mx = logit;
+  } else {
+    se += expf(logit - mx);
+  }
+}
 // barrier of the consumer warps only (the producer warp keeps streaming)
 __device__ __forceinline__ void hs_cbar() { asm volatile("bar.sync 1, %0;" ::"r"(HS_WARPS * 32) : "memory"); }
 __device__ __forceinline__ bool hs_cbar_or(bool v) {
@@ -1315,9 +1337,9 @@ __global__ void __launch_bounds__(HS_THREADS, 1) k_head_sample(HeadArgs a) {
   pdl_launch();
   constexpr int EPC = 16 / sizeof(T);
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ float s_part[HS_WARPS][HEAD_RMAX][HEAD_PART];
-  __shared__ float s_gm[HS_WARPS][HEAD_RMAX][4];  // Gumbel noise of a warp's group
-  __shared__ int s_b[HEAD_RMAX], s_t[HEAD_RMAX];
+  __shared__ float s_part[HS_WARPS][HS_RP][HEAD_PART];
+  __shared__ float s_gm[HS_WARPS][4 * HS_RP];  // Gumbel noise of a warp's next groups
+  __shared__ int s_b[HS_RP], s_t[HS_RP];
   __shared__ __align__(8) uint64_t s_full[HS_MAX_STAGES], s_empty[HS_MAX_STAGES];
   __shared__ int s_n;
   __shared__ volatile int s_abort;
@@ -1401,31 +1423,48 @@ __global__ void __launch_bounds__(HS_THREADS, 1) k_head_sample(HeadArgs a) {
       s_t[tid] = a.t[s_list[p0 + tid]];
     }
     hs_cbar();
-    // lane r keeps row r's running state
-    float best_s = -CUDART_INF_F, best_l = 0.f, mx = -CUDART_INF_F, se = 0.f;
-    int best_v = 0x7fffffff;
+    // Lane 4r' + j keeps the running state of stopped row r = 8t + r' (slot t)
+    // over this warp's rows v with v % 4 == j.
+    float best_s[HS_SLOTS], best_l[HS_SLOTS], mx[HS_SLOTS], se[HS_SLOTS];
+    int best_v[HS_SLOTS];
+#pragma unroll
+    for (int t = 0; t < HS_SLOTS; ++t) {
+      best_s[t] = -CUDART_INF_F;
+      best_l[t] = 0.f;
+      mx[t] = -CUDART_INF_F;
+      se[t] = 0.f;
+      best_v[t] = 0x7fffffff;
+    }
     bool ok = true;
     const int team = w / HS_TEAM, q = w % HS_TEAM;
+    const int jl = lane & 3, rl = lane >> 2;
+    // Gumbel noise is drawn for G of this warp's groups at a time (its stages
+    // s, s + 2, ...): entry (k, r, j), one Philox draw per (stopped row,
+    // group), is computed by lane (k nr + r) 4 + j (+ 32 per round)
+    const int G = nr <= 8 ? 8 / nr : 1;
+    int kg = 0;  // this warp's groups so far in the pass
     for (int s = 0; s < nst; ++s, ++i) {
       if ((i & 1) != team) continue;
       const int slot = i % NS;
       const int v0 = rbeg + s * HS_ROWS + 4 * q;  // this warp's group: rows v0 .. v0 + nv - 1
       const int nv = min(4, rend - v0);
-      // Gumbel noise of the group: one Philox draw per stopped row gives its
-      // four lanes; entry (r, j) is computed by lane 4r + j (+ 32 per round)
-      __syncwarp();  // the previous group's noise has been read
-      if (nv > 0) {
-        for (int x = lane; x < 4 * nr; x += 32) {
-          const int r = x >> 2, j = x & 3;
+      const int kb = kg % G;
+      ++kg;
+      if (kb == 0) {
+        __syncwarp();  // the previous batch has been read
+        for (int x = lane; x < 4 * nr * G; x += 32) {
+          const int k = x / (4 * nr), r = (x >> 2) % nr, j = x & 3;
+          const int s2 = s + 2 * k, v = rbeg + s2 * HS_ROWS + 4 * q + j;
           float g = 0.f;
-          if (j < nv) {
+          if (s2 < nst && v < rend) {
             const uint4 rb = philox4x32_10(
-                make_uint4((uint32_t)s_b[r], (uint32_t)s_t[r], STREAM_GUMBEL, (uint32_t)(v0 >> 2)), (uint32_t)seed,
+                make_uint4((uint32_t)s_b[r], (uint32_t)s_t[r], STREAM_GUMBEL, (uint32_t)(v >> 2)), (uint32_t)seed,
                 (uint32_t)(seed >> 32));
             g = -logf(-logf(uniform01(lane_of(rb, j))));
           }
-          s_gm[w][r][j] = g;
+          s_gm[w][x] = g;
         }
+        __syncwarp();
       }
       // lane 0 waits, the warp follows its verdict
       int got = 1;
@@ -1472,40 +1511,52 @@ __global__ void __launch_bounds__(HS_THREADS, 1) k_head_sample(HeadArgs a) {
             }
           }
         }
-        // four butterflies, interleaved
+        // four butterflies, interleaved: every lane ends with the four sums
 #pragma unroll
         for (int o = 16; o; o >>= 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
-        if (lane == r) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j >= nv) break;
-            const float logit = part[j];
-            const float sc = logit + s_gm[w][r][j];
-            if (sc > best_s) {
-              best_s = sc;
-              best_v = v0 + j;
-              best_l = logit;
-            }
-            if (logit > mx) {
-              se = se * expf(mx - logit) + 1.0f;
-              mx = logit;
-            } else {
-              se += expf(logit - mx);
-            }
-          }
+        if (rl == (r & 7) && jl < nv) {
+          const float logit = jl == 0 ? part[0] : jl == 1 ? part[1] : jl == 2 ? part[2] : part[3];
+          const float sc = logit + s_gm[w][(kb * nr + r) * 4 + jl];
+          static_assert(HS_SLOTS == 2, "two state slots");
+          if (r < 8) hs_update(sc, logit, v0 + jl, best_s[0], best_v[0], best_l[0], mx[0], se[0]);
+          else hs_update(sc, logit, v0 + jl, best_s[1], best_v[1], best_l[1], mx[1], se[1]);
         }
       }
     }
     // every consumer leaves together when any of them gave up
     if (hs_cbar_or(!ok || s_abort)) return;
-    if (lane < nr) {
-      s_part[w][lane][0] = best_s;
-      s_part[w][lane][1] = __int_as_float(best_v);
-      s_part[w][lane][2] = best_l;
-      s_part[w][lane][3] = mx;
-      s_part[w][lane][4] = se;
+    // the four lanes of a stopped row merge (argmax ties to the lowest v)
+#pragma unroll
+    for (int t = 0; t < HS_SLOTS; ++t) {
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        const float bs2 = __shfl_xor_sync(0xffffffffu, best_s[t], o);
+        const int bv2 = __shfl_xor_sync(0xffffffffu, best_v[t], o);
+        const float bl2 = __shfl_xor_sync(0xffffffffu, best_l[t], o);
+        const float m2 = __shfl_xor_sync(0xffffffffu, mx[t], o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, se[t], o);
+        if (bs2 > best_s[t] || (bs2 == best_s[t] && bv2 < best_v[t])) {
+          best_s[t] = bs2;
+          best_v[t] = bv2;
+          best_l[t] = bl2;
+        }
+        const float mn = fmaxf(mx[t], m2);
+        if (mn != -CUDART_INF_F) {
+          se[t] = (mx[t] == -CUDART_INF_F ? 0.f : se[t] * expf(mx[t] - mn)) +
+                  (m2 == -CUDART_INF_F ? 0.f : s2 * expf(m2 - mn));
+          mx[t] = mn;
+        }
+      }
+      const int r = 8 * t + rl;
+      if (jl == 0 && r < nr) {
+        s_part[w][r][0] = best_s[t];
+        s_part[w][r][1] = __int_as_float(best_v[t]);
+        s_part[w][r][2] = best_l[t];
+        s_part[w][r][3] = mx[t];
+        s_part[w][r][4] = se[t];
+      }
     }
     hs_cbar();
     if (tid < nr) {
