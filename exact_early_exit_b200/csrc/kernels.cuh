@@ -11,7 +11,6 @@ namespace nv {
 
 constexpr int ATTN_KT = 64;    // keys per attention tile; page_size must be a multiple
 constexpr int ATTN_RPC = 32;   // rows per attention CTA (row group)
-constexpr int HEAD_RMAX = 32;  // rows per pass of the exit-head sampler
 constexpr int HEAD_PART = 5;   // floats per head partial: score, id, logit, max, sumexp
 
 void launch_rope_table(float2* cs, int max_seq, int hd, double theta, cudaStream_t st);
