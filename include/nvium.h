@@ -162,7 +162,13 @@ nv_status nv_score_mixture_ex(nv_model *m, const int32_t *tokens, int B, int S,
                               float *mean_depth, void *stream);
 
 /* A decode state for B sequences (B <= max_batch): paged KV cache with its own
- * length per (sequence, layer), deferred-row store, work lists, CUDA graph. */
+ * length per (sequence, layer), deferred-row store, work lists, CUDA graph.
+ * *out (host) receives the state, owned by the caller until nv_state_destroy.
+ * NV_ERR_INVALID_ARG for a null argument or B outside [1, max_batch];
+ * NV_ERR_OOM / NV_ERR_CUDA when device memory or a CUDA call fails;
+ * NV_ERR_UNSUPPORTED when the small-batch exit-head sampler has no
+ * shared-memory plan for B and d_model (not reached by any configuration
+ * nv_create accepts).  On error *out is NULL. */
 nv_status nv_state_create(nv_model *m, int B, nv_state **out);
 nv_status nv_state_destroy(nv_state *s);
 
